@@ -1,0 +1,289 @@
+/*
+ * metis.h -- C ABI of the B200-native spectral-split W4A4G4 linear layer
+ * (Metis) and the Averis mean/residual split.
+ *
+ * What the library computes (sources cited by page title and section):
+ *   - "Metis: Training LLMs with FP4 Quantization" (arXiv 2509.00404v4),
+ *     abstract and technical framework: the anisotropic spectrum of a weight,
+ *     activation or gradient matrix is split into a dominant part and a long
+ *     tail that are quantized to FP4 independently (W4A4G4); the split uses
+ *     random projection and sparse random sampling to stay cheap.
+ *   - SII open-source-week release on Metis, section 2.4 item 1: spectral
+ *     decomposition A = U_k S_k V_k^T + R with randomized dimension reduction;
+ *     section 2.3 / Fig. 3 and the feature list: block-wise FP4 quantization
+ *     (MXFP4, NVFP4) where every block's scale follows the block maximum.
+ *   - Retelling of arXiv 2603.10444 (mean bias in FP4 training), Averis
+ *     paragraphs: X = 1 mu^T + R with mu the mean over all rows; mean and
+ *     residual are quantized separately, in forward and backward.
+ *
+ * Conventions shared by every entry point
+ *   - Memory: the caller owns all memory.  Pointers named "device" must be
+ *     device memory of the current CUDA device; "host" pointers are read on the
+ *     host before any launch.  The library never allocates, frees, prints or
+ *     synchronises the stream; every call only enqueues work on `stream`
+ *     (a cudaStream_t; NULL means the legacy default stream).
+ *   - Workspace: each call that needs scratch takes `workspace` (device) and
+ *     `workspace_bytes` (host, in/out).  With workspace == NULL the call writes
+ *     the required size to *workspace_bytes, launches nothing and returns
+ *     METIS_OK.  Otherwise *workspace_bytes must be at least that size
+ *     (METIS_ERR_WORKSPACE) and the workspace must be 256-byte aligned.  The
+ *     workspace is used only during the enqueued work; calls that share one
+ *     workspace must be ordered on one stream.
+ *   - Errors: argument problems are returned before anything is launched.
+ *     Problems found on the device (numerical breakdown, a bounded wait that
+ *     expired) are OR-ed into the caller's device word *dev_status as
+ *     METIS_DEV_* bits; the caller reads it after synchronising.  dev_status
+ *     may be NULL where an entry point says so.
+ *   - Layouts: all dense matrices are row-major with a leading dimension in
+ *     elements.  FP4 matrices use metis_fp4_tensor below.
+ *   - Determinism: identical inputs, sizes and seed give bit-identical outputs
+ *     (no atomics on floating-point sums; fixed reduction orders).
+ *   - Requires an sm_100 device (B200); METIS_ERR_UNSUPPORTED otherwise.
+ */
+#ifndef METIS_H
+#define METIS_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  METIS_OK = 0,
+  METIS_ERR_NULL = 1,        /* a required pointer is NULL                       */
+  METIS_ERR_SHAPE = 2,       /* a size is out of range or not a block multiple   */
+  METIS_ERR_ALIGN = 3,       /* a pointer or leading dimension is misaligned     */
+  METIS_ERR_UNSUPPORTED = 4, /* not an sm_100 device, or an unsupported option   */
+  METIS_ERR_WORKSPACE = 5,   /* workspace too small or misaligned                */
+  METIS_ERR_CUDA = 6,        /* a CUDA runtime/driver call failed                */
+  METIS_ERR_ARG = 7          /* any other invalid argument (enum value, k, ...)  */
+} metis_status;
+
+/* bits OR-ed into *dev_status by kernels */
+#define METIS_DEV_NUMERIC 1  /* Jacobi did not converge within max sweeps       */
+#define METIS_DEV_TIMEOUT 2  /* a bounded device wait expired; outputs invalid   */
+#define METIS_DEV_SAMPLING 4 /* a sparse-sign row could not draw its columns     */
+
+typedef enum { METIS_BF16 = 0, METIS_F32 = 1 } metis_dtype;
+typedef enum { METIS_MXFP4 = 0, METIS_NVFP4 = 1 } metis_fp4_fmt;
+typedef enum { METIS_SKETCH_GAUSSIAN = 0, METIS_SKETCH_SPARSE_SIGN = 1 } metis_sketch;
+
+/*
+ * One FP4 matrix, "outer x inner", blocks of 32 (MXFP4) or 16 (NVFP4)
+ * consecutive elements along `inner`.  A GEMM operand is stored with `inner`
+ * equal to the contraction dimension ("K-major").
+ *
+ *   codes          device, outer * inner / 2 bytes, row-major [outer][inner/2];
+ *                  element 2j in the low nibble of byte j.  E2M1 code
+ *                  s|e1 e0|m: magnitudes {0,.5,1,1.5,2,3,4,6}.
+ *   scales         device, metis_fp4_scales_bytes(fmt, outer, inner) bytes:
+ *                  the tensor-core layout.  Rows are padded to 128 and scale
+ *                  columns to a whole 256-element K tile; scale (r, c) sits at
+ *                  byte ((r/128)*(C/4) + c/4)*512 + (r%32)*16 + ((r%128)/32)*4
+ *                  + c%4 where C is the padded scale-column count.  Padding is
+ *                  zero.  MXFP4: E8M0 codes (2^(code-127)).  NVFP4: E4M3 codes.
+ *   scales_linear  device, optional (may be NULL): [outer][inner/bs] codes.
+ *   tensor_scale   device, one float: NVFP4 decode scale s_t (value =
+ *                  e2m1 * e4m3 * s_t).  Written by the quantizer.  Ignored for
+ *                  MXFP4 (may be NULL).
+ *   inner_sum      device, optional (may be NULL): one float per outer index,
+ *                  the sum over `inner` of the dequantized values (float32,
+ *                  fixed summation order).
+ */
+typedef struct {
+  int32_t fmt;          /* metis_fp4_fmt */
+  int64_t outer;
+  int64_t inner;
+  uint8_t* codes;
+  uint8_t* scales;
+  uint8_t* scales_linear;
+  float* tensor_scale;
+  float* inner_sum;
+} metis_fp4_tensor;
+
+/* Host-only helpers (no device work): buffer sizes for a metis_fp4_tensor. */
+size_t metis_fp4_codes_bytes(int64_t outer, int64_t inner);
+size_t metis_fp4_scales_bytes(int32_t fmt, int64_t outer, int64_t inner);
+
+/* Host-only: short description of a status code (static string). */
+const char* metis_status_string(int32_t status);
+
+/* Host-only: 1 if a device of compute capability 10.x is current, else 0. */
+int32_t metis_device_supported(void);
+
+/*
+ * metis_quantize_fp4 -- block-quantize a dense matrix to FP4.
+ * Source: SII release section 2.3 / Fig. 3 (one scale per block, set by the
+ * block maximum) and the feature list (MXFP4 / NVFP4).  Bit-level rules
+ * (OCP MX v1.0 for MXFP4; two-level NVFP4):
+ *   MXFP4 (block 32): a = max|x|; a == 0 -> scale code 0, codes 0; else
+ *     se = clamp(floor(log2 a) - 2, -127, 127), scale code se + 127,
+ *     code = E2M1(x * 2^-se).
+ *   NVFP4 (block 16): alpha = max|x| over the tensor; s_t = alpha / 2688
+ *     (1 if alpha == 0); t = (a / s_t) / 6; d = E4M3(t) round-to-nearest-even,
+ *     saturating at 448; d == 0 -> codes 0; else code = E2M1(x * (1/(d*s_t))).
+ *   E2M1 rounds to nearest, ties to the even code, saturates at 6; the sign bit
+ *   is the sign of the scaled value.  All arithmetic is IEEE float32 in this
+ *   order (bit-exact against the CPU oracle).
+ *
+ *   X            device, rows x cols, leading dimension ld (elements),
+ *                dtype METIS_BF16 or METIS_F32.  16-byte aligned rows.
+ *   block_axis   1: blocks along cols (out->outer = rows, out->inner = cols);
+ *                0: blocks along rows (out->outer = cols, out->inner = rows).
+ *   sub_col      device, optional: cols floats; the quantized value is
+ *                fl32(x_ij - sub_col[j]) (the Averis residual).  May be NULL.
+ *   out          host struct with device buffers; out->fmt selects the format;
+ *                outer/inner must match.  The blocked dimension must be a
+ *                multiple of 32 (METIS_ERR_SHAPE).
+ * Workspace: NVFP4 needs a few bytes for the tensor maximum.
+ */
+metis_status metis_quantize_fp4(const void* X, int32_t dtype, int64_t rows, int64_t cols,
+                                int64_t ld, int32_t block_axis, const float* sub_col,
+                                metis_fp4_tensor* out, void* workspace,
+                                size_t* workspace_bytes, void* stream);
+
+/*
+ * Parameters of the randomized split (host struct).
+ *   k, p          rank kept and oversampling; l = k + p <= 128, l <= min(m, n)
+ *                 (or <= sample_rows), l a multiple of 16 is not required.
+ *   power_iters   q >= 0 subspace iterations.
+ *   seed          Philox4x32-10 key for the sketch and the row sample.
+ *   sketch        METIS_SKETCH_GAUSSIAN or METIS_SKETCH_SPARSE_SIGN.
+ *   sparse_nnz    nonzeros per input coordinate of the sparse-sign sketch.
+ *   sample_rows   0, or the number of rows sampled to find the right singular
+ *                 subspace (then power_iters applies to the sample).
+ *   fmt           metis_fp4_fmt of every quantized output.
+ *   max_jacobi_sweeps  cap on Jacobi sweeps of the core (e.g. 30).
+ */
+typedef struct {
+  int32_t k;
+  int32_t p;
+  int32_t power_iters;
+  uint64_t seed;
+  int32_t sketch;
+  int32_t sparse_nnz;
+  int64_t sample_rows;
+  int32_t fmt;
+  int32_t max_jacobi_sweeps;
+} metis_split_params;
+
+/*
+ * metis_split -- spectral split A = U diag(S) V^T + R and FP4 quantization of
+ * U, V and R.
+ * Source: SII release section 2.4 item 1 (dominant + long-tail split with
+ * randomized dimension reduction); "Metis: Training LLMs with FP4
+ * Quantization" abstract (random projection and sparse random sampling);
+ * older Metis abstract item (i) (random embedding).
+ * Steps: [sample rows] -> Omega (Philox Gaussian / sparse sign, bf16) ->
+ * Y = A Omega -> CholeskyQR2 -> q x (A^T Q, QR, A Q, QR) -> B^T = A^T Q ->
+ * one-sided Jacobi on the l-wide core (via its l x l Gram, float64) -> top k,
+ * U = Q U~, V = B^T U~ S^-1, signs (largest-|.| entry of each U column made
+ * positive) -> R = A - U S V^T fused with FP4 quantization.
+ * With sample_rows > 0: V_s from the sampled rows, P = A V_s, CholeskyQR2 of
+ * P, SVD of its triangular factor; U = Q_P W1, V = V_s W2.
+ *
+ *   A, dtype, m, n, lda   device input (bf16 or f32), row-major, 16-byte rows.
+ *   U       device m x k float (row-major), S device k floats (descending),
+ *   V       device n x k float.
+ *   U_q     optional FP4 of U quantized along m (outer = k, inner = m).
+ *   V_q     optional FP4 of V quantized along n (outer = k, inner = n).
+ *   R_rows  optional FP4 of R with blocks along n (outer = m, inner = n).
+ *   R_cols  optional FP4 of R with blocks along m (outer = n, inner = m).
+ *   R_f32   optional device m x n float tap of the residual the quantizer saw.
+ *   sample_idx  optional device int32[sample_rows]: the sampled rows.
+ *   dev_status  device int32 (required).
+ * Quantized outputs need m and n multiples of 32 along their blocked axis.
+ */
+metis_status metis_split(const void* A, int32_t dtype, int64_t m, int64_t n, int64_t lda,
+                         const metis_split_params* prm, float* U, float* S, float* V,
+                         metis_fp4_tensor* U_q, metis_fp4_tensor* V_q,
+                         metis_fp4_tensor* R_rows, metis_fp4_tensor* R_cols, float* R_f32,
+                         int32_t* sample_idx, void* workspace, size_t* workspace_bytes,
+                         int32_t* dev_status, void* stream);
+
+/*
+ * One operand of an FP4 product C = A B (host struct):
+ *   left  operand A (M x K) = R + F diag(S) P^T
+ *   right operand B (K x N) = R + P diag(S) F^T
+ *   R  FP4, quantized along the contraction axis: outer = M (left) or N
+ *      (right), inner = K.  Required.
+ *   k  rank of the low-rank term (0 = plain FP4 operand; then P, F, S unused).
+ *   P  FP4, the factor along the contraction axis: outer = k, inner = K.
+ *      NULL means the all-ones vector (k must be 1).
+ *   F  FP4, the factor along the free axis: outer = k, inner = M or N.
+ *      NULL means the all-ones vector (k must be 1).
+ *   S  device k floats (NULL = all ones).
+ * Averis operands are rank 1 with one factor all-ones; the product then needs
+ * R->inner_sum of the other operand's residual where the ones-vector is
+ * contracted against it.  Both operands must share one FP4 format.
+ */
+typedef struct {
+  const metis_fp4_tensor* R;
+  int32_t k;
+  const metis_fp4_tensor* P;
+  const metis_fp4_tensor* F;
+  const float* S;
+} metis_operand;
+
+/*
+ * metis_linear_fwd -- Y = X W on FP4 operands (W4A4 forward).
+ * Source: "Metis: Training LLMs with FP4 Quantization" abstract (W4A4G4);
+ * SII release section 2.4 item 1 (both parts of the split take part).
+ * Computes Y = R_X R_W (block-scaled tcgen05 FP4 MMA, fp32 accumulation) plus
+ * the low-rank terms T1 F_W^T + F_X T2 accumulated into the same tensor-memory
+ * accumulator (T1 = (R_X P_W + F_X S_X P_X^T P_W) S_W, T2 = S_X P_X^T R_W).
+ *   X  left operand (M x K), W right operand (K x N).
+ *   Y  device M x N, y_dtype METIS_F32 or METIS_BF16, leading dimension ldy.
+ * K must be a multiple of 32.
+ */
+metis_status metis_linear_fwd(const metis_operand* X, const metis_operand* W, int64_t M,
+                              int64_t N, int64_t K, void* Y, int32_t y_dtype, int64_t ldy,
+                              void* workspace, size_t* workspace_bytes, int32_t* dev_status,
+                              void* stream);
+
+/*
+ * metis_linear_bwd -- the two backward products of Y = X W on FP4 operands:
+ *   dX = dY W^T  (left operand dY_n: dY quantized along N;
+ *                 right operand Wt:  W quantized along N, P = V_W, F = U_W)
+ *   dW = X^T dY  (left operand Xt:   X quantized along M, P = U_X, F = V_X;
+ *                 right operand dY_m: dY quantized along M)
+ * Source: "Metis: Training LLMs with FP4 Quantization" abstract (FP4
+ * gradients, G4); Averis paragraphs (the output gradient is split too).
+ *   dX  device M x K (or NULL to skip), dW device K x N (or NULL to skip),
+ *   out_dtype METIS_F32 or METIS_BF16; ld_dx, ld_dw leading dimensions.
+ * N must be a multiple of 32 for dX and M a multiple of 32 for dW.
+ */
+metis_status metis_linear_bwd(const metis_operand* dY_n, const metis_operand* Wt,
+                              const metis_operand* Xt, const metis_operand* dY_m, int64_t M,
+                              int64_t N, int64_t K, void* dX, int64_t ld_dx, void* dW,
+                              int64_t ld_dw, int32_t out_dtype, void* workspace,
+                              size_t* workspace_bytes, int32_t* dev_status, void* stream);
+
+/*
+ * averis_split -- X = 1 mu^T + R with mu the mean over all rows, then FP4 of
+ * mu and R.
+ * Source: retelling of arXiv 2603.10444, Averis paragraphs (mean over all
+ * rows, broadcast subtraction, separate quantization of mean and residual;
+ * the same split is applied to the output gradient in the backward pass).
+ *   X, dtype, m, n, ld  device input.
+ *   mean     device n floats: mu_j = (sum_i x_ij) / m (float32, fixed order).
+ *   mean_q   optional FP4 of mu (outer = 1, inner = n).
+ *   R_rows   optional FP4 of fl32(x_ij - mu_j), blocks along n (outer m).
+ *   R_cols   optional FP4 of the same residual, blocks along m (outer n).
+ *   R_f32    optional device m x n float tap.
+ * NVFP4 takes the residual's tensor maximum from the column minima and maxima
+ * (exact: rounding is monotonic), so X is read twice in total.
+ */
+metis_status averis_split(const void* X, int32_t dtype, int64_t m, int64_t n, int64_t ld,
+                          int32_t fmt, float* mean, metis_fp4_tensor* mean_q,
+                          metis_fp4_tensor* R_rows, metis_fp4_tensor* R_cols, float* R_f32,
+                          void* workspace, size_t* workspace_bytes, int32_t* dev_status,
+                          void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* METIS_H */

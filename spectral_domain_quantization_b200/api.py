@@ -1,0 +1,273 @@
+"""Python binding of the C ABI in include/metis.h (ctypes).
+
+Argument marshalling only: torch tensors provide device memory and the current
+CUDA stream; every arithmetic step runs in the CUDA kernels of
+``libmetis_b200.so``.  There is no fallback: if the library is missing or the
+device is not sm_100, calls raise.
+"""
+import ctypes
+import os
+import re
+
+import torch
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(HERE, "libmetis_b200.so")
+HEADER = os.path.join(os.path.dirname(HERE), "include", "metis.h")
+
+OK = 0
+BF16, F32 = 0, 1
+MXFP4, NVFP4 = 0, 1
+SKETCH_GAUSSIAN, SKETCH_SPARSE_SIGN = 0, 1
+DEV_NUMERIC, DEV_TIMEOUT, DEV_SAMPLING = 1, 2, 4
+
+FMT = {"mx": MXFP4, "nv": NVFP4, MXFP4: MXFP4, NVFP4: NVFP4}
+FMT_NAME = {MXFP4: "mx", NVFP4: "nv"}
+
+
+class MetisError(RuntimeError):
+    def __init__(self, status, what):
+        self.status = status
+        super().__init__(f"{what}: {status_string(status)} (status {status})")
+
+
+class FP4Struct(ctypes.Structure):
+    _fields_ = [("fmt", ctypes.c_int32), ("outer", ctypes.c_int64), ("inner", ctypes.c_int64),
+                ("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("scales_linear", ctypes.c_void_p), ("tensor_scale", ctypes.c_void_p),
+                ("inner_sum", ctypes.c_void_p)]
+
+
+class SplitParams(ctypes.Structure):
+    _fields_ = [("k", ctypes.c_int32), ("p", ctypes.c_int32), ("power_iters", ctypes.c_int32),
+                ("seed", ctypes.c_uint64), ("sketch", ctypes.c_int32),
+                ("sparse_nnz", ctypes.c_int32), ("sample_rows", ctypes.c_int64),
+                ("fmt", ctypes.c_int32), ("max_jacobi_sweeps", ctypes.c_int32)]
+
+
+class OperandStruct(ctypes.Structure):
+    _fields_ = [("R", ctypes.POINTER(FP4Struct)), ("k", ctypes.c_int32),
+                ("P", ctypes.POINTER(FP4Struct)), ("F", ctypes.POINTER(FP4Struct)),
+                ("S", ctypes.c_void_p)]
+
+
+_lib = None
+
+_VP, _I32, _I64, _SZP = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.POINTER(ctypes.c_size_t)
+_FP = ctypes.POINTER(FP4Struct)
+_OP = ctypes.POINTER(OperandStruct)
+
+_SIGS = {
+    "metis_fp4_codes_bytes": (ctypes.c_size_t, [_I64, _I64]),
+    "metis_fp4_scales_bytes": (ctypes.c_size_t, [_I32, _I64, _I64]),
+    "metis_status_string": (ctypes.c_char_p, [_I32]),
+    "metis_device_supported": (_I32, []),
+    "metis_quantize_fp4": (_I32, [_VP, _I32, _I64, _I64, _I64, _I32, _VP, _FP, _VP, _SZP, _VP]),
+    "metis_split": (_I32, [_VP, _I32, _I64, _I64, _I64, ctypes.POINTER(SplitParams), _VP, _VP, _VP,
+                           _FP, _FP, _FP, _FP, _VP, _VP, _VP, _SZP, _VP, _VP]),
+    "metis_linear_fwd": (_I32, [_OP, _OP, _I64, _I64, _I64, _VP, _I32, _I64, _VP, _SZP, _VP, _VP]),
+    "metis_linear_bwd": (_I32, [_OP, _OP, _OP, _OP, _I64, _I64, _I64, _VP, _I64, _VP, _I64, _I32,
+                                _VP, _SZP, _VP, _VP]),
+    "averis_split": (_I32, [_VP, _I32, _I64, _I64, _I64, _I32, _VP, _FP, _FP, _FP, _VP, _VP, _SZP,
+                            _VP, _VP]),
+}
+
+
+def lib():
+    """Load libmetis_b200.so (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError("libmetis_b200.so is not built: run __graft_entry__.build() "
+                               "or python spectral_domain_quantization_b200/build.py")
+        L = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def header_functions():
+    """Names of the functions declared in include/metis.h."""
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\**\s+\**(\w+)\s*\(", src, flags=re.M)))
+
+
+def status_string(status):
+    try:
+        return lib().metis_status_string(int(status)).decode()
+    except Exception:  # pragma: no cover - only when the library is absent
+        return "status"
+
+
+def _check(status, what):
+    if status != OK:
+        raise MetisError(status, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream():
+    return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+
+
+def _dtype_code(t):
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError("only bfloat16 and float32 inputs are supported")
+
+
+class _Workspace:
+    """Grow-only workspace per device (allocated by torch, the caller side)."""
+
+    def __init__(self):
+        self.buf = {}
+
+    def get(self, nbytes, device):
+        key = torch.device(device).index
+        cur = self.buf.get(key)
+        if cur is None or cur.numel() < nbytes:
+            cur = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+            self.buf[key] = cur
+        return cur
+
+
+_ws = _Workspace()
+
+
+def _call_with_workspace(fn, args_before_ws, args_after_ws, device, what):
+    """Query the workspace size, provide it, then run the call."""
+    size = ctypes.c_size_t(0)
+    _check(fn(*args_before_ws, None, ctypes.byref(size), *args_after_ws), what + " (workspace query)")
+    ws = _ws.get(size.value, device)
+    size2 = ctypes.c_size_t(ws.numel())
+    _check(fn(*args_before_ws, _ptr(ws), ctypes.byref(size2), *args_after_ws), what)
+
+
+# --------------------------------------------------------------------------
+# FP4 tensors
+# --------------------------------------------------------------------------
+
+class QTensor:
+    """An FP4 matrix (outer x inner, blocks along inner) held in torch buffers."""
+
+    def __init__(self, fmt, outer, inner, device="cuda", linear=False, inner_sum=False):
+        L = lib()
+        self.fmt = FMT[fmt]
+        self.outer, self.inner = int(outer), int(inner)
+        self.block = 32 if self.fmt == MXFP4 else 16
+        self.codes = torch.empty(L.metis_fp4_codes_bytes(self.outer, self.inner), dtype=torch.uint8,
+                                 device=device)
+        self.scales = torch.empty(L.metis_fp4_scales_bytes(self.fmt, self.outer, self.inner),
+                                  dtype=torch.uint8, device=device)
+        self.scales_linear = (torch.empty(self.outer * (self.inner // self.block), dtype=torch.uint8,
+                                          device=device) if linear else None)
+        self.tensor_scale = torch.ones(1, dtype=torch.float32, device=device)
+        self.inner_sum = torch.empty(self.outer, dtype=torch.float32, device=device) if inner_sum else None
+
+    def struct(self):
+        s = FP4Struct()
+        s.fmt, s.outer, s.inner = self.fmt, self.outer, self.inner
+        s.codes = self.codes.data_ptr()
+        s.scales = self.scales.data_ptr()
+        s.scales_linear = self.scales_linear.data_ptr() if self.scales_linear is not None else None
+        s.tensor_scale = self.tensor_scale.data_ptr()
+        s.inner_sum = self.inner_sum.data_ptr() if self.inner_sum is not None else None
+        self._s = s          # keep alive while pointers are in use
+        return s
+
+
+def quantize_fp4(X, fmt, axis=1, sub_col=None, linear=False, inner_sum=False, out=None):
+    """FP4 block quantization of a 2-D bf16/f32 CUDA tensor (metis_quantize_fp4)."""
+    if X.dim() != 2 or X.stride(1) != 1:
+        raise ValueError("X must be a row-major 2-D tensor")
+    rows, cols = X.shape
+    outer, inner = (rows, cols) if axis == 1 else (cols, rows)
+    if out is None:
+        out = QTensor(fmt, outer, inner, X.device, linear=linear, inner_sum=inner_sum)
+    s = out.struct()
+    L = lib()
+    _call_with_workspace(
+        L.metis_quantize_fp4,
+        (_ptr(X), _dtype_code(X), rows, cols, X.stride(0), axis, _ptr(sub_col), ctypes.byref(s)),
+        (_stream(),), X.device, "metis_quantize_fp4")
+    return out
+
+
+# --------------------------------------------------------------------------
+# split-linear products
+# --------------------------------------------------------------------------
+
+class Operand:
+    """One operand of an FP4 product (see metis_operand in metis.h).
+
+    left operand  A (M x K) = R + F diag(S) P^T
+    right operand B (K x N) = R + P diag(S) F^T
+    R: QTensor quantized along K; P: QTensor (outer k, inner K) or None for
+    the all-ones vector; F: QTensor (outer k, inner M or N) or None for ones;
+    S: CUDA float tensor of k values or None (ones)."""
+
+    def __init__(self, R, k=0, P=None, F=None, S=None):
+        self.R, self.k, self.P, self.F, self.S = R, int(k), P, F, S
+
+    def struct(self):
+        o = OperandStruct()
+        self._r = self.R.struct()
+        o.R = ctypes.pointer(self._r)
+        o.k = self.k
+        self._p = self.P.struct() if self.P is not None else None
+        self._f = self.F.struct() if self.F is not None else None
+        o.P = ctypes.pointer(self._p) if self._p is not None else None
+        o.F = ctypes.pointer(self._f) if self._f is not None else None
+        o.S = self.S.data_ptr() if self.S is not None else None
+        self._o = o
+        return o
+
+
+def _out_dtype(dt):
+    return F32 if dt == torch.float32 else BF16
+
+
+def linear_fwd(X, W, M, N, K, out_dtype=torch.float32, Y=None, dev_status=None):
+    """Y = X W on FP4 operands (metis_linear_fwd).  X, W: Operand."""
+    dev = X.R.codes.device
+    if Y is None:
+        Y = torch.empty((M, N), dtype=out_dtype, device=dev)
+    if dev_status is None:
+        dev_status = torch.zeros(1, dtype=torch.int32, device=dev)
+    xs, ws_ = X.struct(), W.struct()
+    _call_with_workspace(
+        lib().metis_linear_fwd,
+        (ctypes.byref(xs), ctypes.byref(ws_), M, N, K, _ptr(Y), _out_dtype(Y.dtype), Y.stride(0)),
+        (_ptr(dev_status), _stream()), dev, "metis_linear_fwd")
+    return Y
+
+
+def linear_bwd(dY_n, Wt, Xt, dY_m, M, N, K, out_dtype=torch.float32, dX=None, dW=None,
+               want_dx=True, want_dw=True, dev_status=None):
+    """dX = dY W^T and dW = X^T dY on FP4 operands (metis_linear_bwd)."""
+    dev = (dY_n or Xt).R.codes.device
+    if want_dx and dX is None:
+        dX = torch.empty((M, K), dtype=out_dtype, device=dev)
+    if want_dw and dW is None:
+        dW = torch.empty((K, N), dtype=out_dtype, device=dev)
+    if dev_status is None:
+        dev_status = torch.zeros(1, dtype=torch.int32, device=dev)
+    a = ctypes.byref(dY_n.struct()) if want_dx else None
+    b = ctypes.byref(Wt.struct()) if want_dx else None
+    c = ctypes.byref(Xt.struct()) if want_dw else None
+    d = ctypes.byref(dY_m.struct()) if want_dw else None
+    dt = _out_dtype(out_dtype)
+    _call_with_workspace(
+        lib().metis_linear_bwd,
+        (a, b, c, d, M, N, K, _ptr(dX) if want_dx else None, dX.stride(0) if want_dx else 0,
+         _ptr(dW) if want_dw else None, dW.stride(0) if want_dw else 0, dt),
+        (_ptr(dev_status), _stream()), dev, "metis_linear_bwd")
+    return dX, dW

@@ -1,0 +1,117 @@
+// Host-side helpers of the C ABI and the entry points that need no kernels.
+#include <mutex>
+
+#include "abi_common.h"
+#include "common.cuh"
+
+namespace metis {
+
+namespace {
+constexpr int kMaxDevices = 64;
+int g_sm_count[kMaxDevices] = {0};
+int g_major[kMaxDevices] = {0};
+std::once_flag g_driver_once;
+// signature of cuTensorMapEncodeTiled (driver API, CUDA 12.0+)
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+int current_device() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return -1;
+  return dev;
+}
+
+void fill_props(int dev) {
+  if (dev < 0 || dev >= kMaxDevices || g_sm_count[dev] != 0) return;
+  int sms = 0, major = 0;
+  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  g_major[dev] = major;
+  g_sm_count[dev] = sms;
+}
+}  // namespace
+
+int device_sm_count() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return 148;
+  fill_props(dev);
+  return g_sm_count[dev] > 0 ? g_sm_count[dev] : 148;
+}
+
+bool device_is_sm100() {
+  const int dev = current_device();
+  if (dev < 0 || dev >= kMaxDevices) return false;
+  fill_props(dev);
+  return g_major[dev] == 10;
+}
+
+CUresult encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank,
+                           const void* gaddr, const uint64_t* dims, const uint64_t* strides_bytes,
+                           const uint32_t* box, CUtensorMapSwizzle swizzle) {
+  std::call_once(g_driver_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+  });
+  if (!g_encode) return CUDA_ERROR_NOT_SUPPORTED;
+  uint32_t elem_strides[5] = {1, 1, 1, 1, 1};
+  return g_encode(map, dtype, static_cast<cuuint32_t>(rank), const_cast<void*>(gaddr),
+                  reinterpret_cast<const cuuint64_t*>(dims),
+                  reinterpret_cast<const cuuint64_t*>(strides_bytes), box, elem_strides,
+                  CU_TENSOR_MAP_INTERLEAVE_NONE, swizzle, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                  CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
+metis_status check_fp4(const metis_fp4_tensor* t, int64_t outer, int64_t inner, int fmt) {
+  if (!t || !t->codes || !t->scales) return METIS_ERR_NULL;
+  if (!valid_fmt(t->fmt) || t->fmt != fmt) return METIS_ERR_ARG;
+  if (t->outer != outer || t->inner != inner) return METIS_ERR_SHAPE;
+  if (outer <= 0 || inner <= 0 || inner % 32 != 0) return METIS_ERR_SHAPE;
+  if (t->fmt == METIS_NVFP4 && !t->tensor_scale) return METIS_ERR_NULL;
+  if (!aligned16(t->codes) || !aligned16(t->scales)) return METIS_ERR_ALIGN;
+  return METIS_OK;
+}
+
+metis_status launch_status() {
+  const cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? METIS_OK : METIS_ERR_CUDA;
+}
+
+}  // namespace metis
+
+extern "C" {
+
+size_t metis_fp4_codes_bytes(int64_t outer, int64_t inner) {
+  if (outer <= 0 || inner <= 0) return 0;
+  return static_cast<size_t>(outer) * static_cast<size_t>((inner + 1) / 2);
+}
+
+size_t metis_fp4_scales_bytes(int32_t fmt, int64_t outer, int64_t inner) {
+  if (outer <= 0 || inner <= 0 || !metis::valid_fmt(fmt)) return 0;
+  return static_cast<size_t>(metis::tc_scale_rows(outer)) *
+         static_cast<size_t>(metis::tc_scale_cols(fmt, inner));
+}
+
+const char* metis_status_string(int32_t status) {
+  switch (status) {
+    case METIS_OK: return "ok";
+    case METIS_ERR_NULL: return "a required pointer is NULL";
+    case METIS_ERR_SHAPE: return "invalid shape";
+    case METIS_ERR_ALIGN: return "misaligned pointer or leading dimension";
+    case METIS_ERR_UNSUPPORTED: return "unsupported device or option";
+    case METIS_ERR_WORKSPACE: return "workspace too small or misaligned";
+    case METIS_ERR_CUDA: return "CUDA error";
+    case METIS_ERR_ARG: return "invalid argument";
+    default: return "unknown status";
+  }
+}
+
+int32_t metis_device_supported(void) { return metis::device_is_sm100() ? 1 : 0; }
+
+}  // extern "C"

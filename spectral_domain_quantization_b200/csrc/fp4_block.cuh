@@ -1,0 +1,63 @@
+// One FP4 block: amax -> scale -> E2M1 codes, in the float32 op order of
+// metis.h (MXFP4: OCP MX v1.0 scale rule; NVFP4: two-level scale).  Shared by
+// the plain quantizer, the fused residual quantizer and the Averis quantizer.
+#pragma once
+
+#include "common.cuh"
+
+namespace metis {
+
+// NVFP4 tensor scale s_t = alpha / 2688 (1 when alpha == 0).
+MDEV float nv_tensor_scale(float alpha) {
+  return alpha == 0.f ? 1.f : __fdiv_rn(alpha, 2688.f);
+}
+
+// NVFP4 block of 16.  Returns the E4M3 scale code; writes 16 nibbles to
+// `packed` (element i in bits 4i..4i+3) and the sum of the dequantized
+// values to `dsum`.
+MDEV uint32_t quant_block_nv(const float* v, float s_t, uint64_t& packed, float& dsum) {
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[i]));
+  const float t = __fdiv_rn(__fdiv_rn(a, s_t), 6.f);
+  const uint32_t dc = e4m3_code(t);
+  const float d = e4m3_value(dc);
+  packed = 0;
+  dsum = 0.f;
+  if (d == 0.f) return dc;
+  const float enc = __fdiv_rn(1.f, __fmul_rn(d, s_t));
+  float csum = 0.f;  // exact: at most 16 values that are multiples of 0.5
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t c = e2m1_code(__fmul_rn(v[i], enc));
+    packed |= static_cast<uint64_t>(c) << (4 * i);
+    csum += e2m1_value(c);
+  }
+  dsum = __fmul_rn(csum * d, s_t);  // csum * d is exact in float32
+  return dc;
+}
+
+// MXFP4 block of 32.  Returns the E8M0 scale code; writes 32 nibbles to
+// packed[0..1] and the sum of dequantized values to `dsum`.
+MDEV uint32_t quant_block_mx(const float* v, uint64_t* packed, float& dsum) {
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) a = fmaxf(a, fabsf(v[i]));
+  packed[0] = packed[1] = 0;
+  dsum = 0.f;
+  if (a == 0.f) return 0u;
+  int se = floor_log2(a) - 2;
+  se = se < -127 ? -127 : (se > 127 ? 127 : se);
+  const float inv = pow2f(-se);  // -se in [-125, 127]: a normal float
+  float csum = 0.f;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const uint32_t c = e2m1_code(__fmul_rn(v[i], inv));
+    packed[i >> 4] |= static_cast<uint64_t>(c) << (4 * (i & 15));
+    csum += e2m1_value(c);
+  }
+  dsum = ldexpf(csum, se);
+  return static_cast<uint32_t>(se + 127);
+}
+
+}  // namespace metis

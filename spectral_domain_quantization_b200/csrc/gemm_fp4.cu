@@ -1,0 +1,441 @@
+// Block-scaled FP4 GEMM on the sm_100a tensor cores (tcgen05), with an
+// optional low-rank update accumulated into the same TMEM accumulator.
+//
+// Source: "Metis: Training LLMs with FP4 Quantization" abstract (W4A4G4: the
+// forward and both backward products run on FP4 operands); SII release
+// section 2.4 item 1 (the dominant low-rank part and the long-tail residual
+// both enter the product).
+//
+//   C[M x N] = alpha * ( sum_k A_q[m,k] B_q[n,k]  (FP4, block scales applied
+//                                                  by the MMA)
+//                        + sum_j LA[m,j] LB[n,j] ) (bf16 low-rank chunks)
+//
+// A_q, B_q: FP4 codes, K-major ([rows][K/2] bytes) with the tensor-core scale
+// layout; alpha = product of the NVFP4 tensor scales (1 for MXFP4).
+//
+// Design (one persistent CTA per SM, 320 threads, warp-specialized):
+//   warp 0      TMA producer: per 256-element K tile loads the A tile
+//               (128 rows x 128 B) and B tile (BN rows x 128 B) with 128-byte
+//               swizzle, and the matching 512-byte scale chunks with bulk
+//               copies, into a 4-stage shared-memory ring.
+//   warp 1      TMEM allocator + MMA issuer: copies each stage's scale chunks
+//               into that stage's own TMEM columns (tcgen05.cp 32x128b.warpx4),
+//               issues four K=64 block-scaled MMAs (kind::mxf4 / mxf4nvf4),
+//               then kind::f16 MMAs for the low-rank chunks, and commits.
+//   warps 2-9   epilogue: drain the 128 x BN fp32 accumulator from TMEM into
+//               registers, release it, scale and store (fp32 or bf16), or
+//               store raw partial sums for split-K.
+// Every wait is bounded (METIS_DEV_TIMEOUT) and the kernel always frees its
+// TMEM.  Shared memory per stage: A 16 KB + B BN*128 B + scales 6 KB.
+#include "abi_common.h"
+#include "common.cuh"
+#include "gemm_fp4.h"
+
+namespace metis {
+
+namespace {
+
+constexpr int kStages = 4;
+constexpr int kThreads = 320;
+constexpr int kEpiWarps = 8;
+
+template <int BN>
+struct Smem {
+  static constexpr int kA = 128 * 128;
+  static constexpr int kB = BN * 128;
+  static constexpr int kSFA = 2048;
+  static constexpr int kSFB = 4096;
+  static constexpr int kStage = kA + kB + kSFA + kSFB;
+  static constexpr int kBytes = kStages * kStage + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+MDEV bool wait_ns(uint64_t* bar, uint32_t parity, uint64_t ns) {
+  const uint64_t t0 = global_timer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (global_timer_ns() - t0 > ns) return false;
+  }
+  return true;
+}
+
+template <int BN>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_fp4_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmA,
+                    const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmLA,
+                    const __grid_constant__ CUtensorMap tmLB) {
+  using S = Smem<BN>;
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * S::kStage);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_sh + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const bool nv = p.fmt == METIS_NVFP4;
+  const int atoms_per_kt = nv ? 4 : 2;           // 512-byte scale chunks per 128 rows per K tile
+  const int sfa_cols = 4 * atoms_per_kt;          // TMEM columns for A scales per stage
+  constexpr int kBHalves = BN > 128 ? 2 : 1;      // 128-row scale chunk groups of B
+  const int sfb_cols = 4 * atoms_per_kt * kBHalves;
+  const int sf_stage_cols = sfa_cols + sfb_cols;
+  constexpr uint32_t kTmemCols = 512;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kEpiWarps);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+    if (p.lr_chunks) {
+      prefetch_tensormap(&tmLA);
+      prefetch_tensormap(&tmLB);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_sh, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_sh;
+
+  const int tiles_m = (p.M + 127) / 128;
+  const int tiles_n = (p.N + BN - 1) / BN;
+  const int num_tiles = tiles_m * tiles_n * p.splits;
+  const int kt_per_split = (p.num_kt + p.splits - 1) / p.splits;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int issued = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int split = t % p.splits;
+        const int tt = t / p.splits;
+        const int tm = tt % tiles_m;
+        const int tn = tt / tiles_m;
+        const int kt0 = split * kt_per_split;
+        const int kt1 = min(p.num_kt, kt0 + kt_per_split);
+        const int nlr = (split == p.splits - 1) ? p.lr_chunks : 0;
+        for (int it = kt0; it < kt1 + nlr; ++it) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* sA = smem + stage * S::kStage;
+          uint8_t* sB = sA + S::kA;
+          uint8_t* sSFA = sB + S::kB;
+          uint8_t* sSFB = sSFA + S::kSFA;
+          if (it < kt1) {
+            const int kt = it;
+            const uint32_t sf_bytes = 512u * atoms_per_kt;
+            const bool second = kBHalves == 2 && (2 * tn + 1) * 128 < p.sfb_rows;
+            const uint32_t bytes = S::kA + S::kB + sf_bytes * (1 + (kBHalves == 2 ? (second ? 2 : 1) : 1));
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            tma_load_2d(sA, &tmA, &full[stage], kt * 128, tm * 128);
+            tma_load_2d(sB, &tmB, &full[stage], kt * 128, tn * BN);
+            bulk_load(sSFA, p.sfa + (static_cast<int64_t>(tm) * p.sfa_chunks + kt * atoms_per_kt) * 512,
+                      sf_bytes, &full[stage]);
+            const int nb0 = kBHalves == 2 ? 2 * tn : tn * BN / 128;
+            bulk_load(sSFB, p.sfb + (static_cast<int64_t>(nb0) * p.sfb_chunks + kt * atoms_per_kt) * 512,
+                      sf_bytes, &full[stage]);
+            if (kBHalves == 2 && second)
+              bulk_load(sSFB + 2048, p.sfb + (static_cast<int64_t>(nb0 + 1) * p.sfb_chunks + kt * atoms_per_kt) * 512,
+                        sf_bytes, &full[stage]);
+          } else {
+            const int c = it - kt1;
+            mbar_arrive_expect_tx(&full[stage], S::kA + S::kB);
+            tma_load_2d(sA, &tmLA, &full[stage], c * 64, tm * 128);
+            tma_load_2d(sB, &tmLB, &full[stage], c * 64, tn * BN);
+          }
+          ++issued;
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (*abort_flag) {
+        // let copies already in flight land before the CTA exits
+        int s = stage;
+        uint32_t ph = phase;
+        for (int i = 0; i < min(issued, kStages); ++i) {
+          if (--s < 0) { s = kStages - 1; ph ^= 1u; }
+          wait_ns(&full[s], ph, 100000000ull);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int split = t % p.splits;
+        const int tn = (t / p.splits) / tiles_m;
+        // with BN = 64 a tile covers half of a 128-row scale chunk: the upper
+        // half's scales sit two TMEM columns further
+        const uint32_t sfb_off = BN == 64 ? 2u * (tn & 1) : 0u;
+        const int kt0 = split * kt_per_split;
+        const int kt1 = min(p.num_kt, kt0 + kt_per_split);
+        const int nlr = (split == p.splits - 1) ? p.lr_chunks : 0;
+        if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t accumulate = 0;
+        for (int it = kt0; it < kt1 + nlr; ++it) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          uint8_t* sA = smem + stage * S::kStage;
+          uint8_t* sB = sA + S::kA;
+          const uint64_t adesc = make_sdesc(smem_u32(sA), 16, 1024, kSwizzle128B);
+          const uint64_t bdesc = make_sdesc(smem_u32(sB), 16, 1024, kSwizzle128B);
+          if (it < kt1) {
+            uint8_t* sSFA = sB + S::kB;
+            uint8_t* sSFB = sSFA + S::kSFA;
+            const uint32_t sfa_t = tmem + 256 + stage * sf_stage_cols;
+            const uint32_t sfb_t = sfa_t + sfa_cols + sfb_off;
+            for (int a = 0; a < atoms_per_kt; ++a) {
+              tc_cp_32x128b_warpx4(sfa_t + 4 * a, make_sdesc(smem_u32(sSFA + 512 * a), 0, 128, kSwizzleNone));
+              for (int h = 0; h < kBHalves; ++h)
+                tc_cp_32x128b_warpx4(sfb_t - sfb_off + 4 * kBHalves * a + 4 * h,
+                                     make_sdesc(smem_u32(sSFB + 2048 * h + 512 * a), 0, 128, kSwizzleNone));
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint64_t koff = static_cast<uint64_t>((j * 32) >> 4);
+              if (nv) {
+                mma_nvf4(tmem, adesc + koff, bdesc + koff, idesc_fp4(128, BN, false, 0, 0),
+                         sfa_t + 4 * j, sfb_t + 4 * kBHalves * j, accumulate);
+              } else {
+                const uint32_t id = 2u * (j & 1);
+                mma_mxf4(tmem, adesc + koff, bdesc + koff, idesc_fp4(128, BN, true, id, id),
+                         (sfa_t + 4 * (j >> 1)) | (id << 30), (sfb_t + 4 * kBHalves * (j >> 1)) | (id << 30),
+                         accumulate);
+              }
+              accumulate = 1;
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint64_t koff = static_cast<uint64_t>((j * 32) >> 4);
+              mma_bf16(tmem, adesc + koff, bdesc + koff, idesc_bf16(128, BN, false, false), accumulate);
+              accumulate = 1;
+            }
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+        acc_phase ^= 1u;
+      }
+      if (*abort_flag) {
+        // wait for MMAs already issued before the TMEM is freed
+        tc_commit(acc_full);
+        wait_ns(acc_full, acc_phase, 100000000ull);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;                 // TMEM lane quadrant of this warp
+    const int half = (warp - 2) >> 2;       // which BN/2 columns
+    constexpr int kCols = BN / 2;           // columns per thread
+    float alpha = 1.f;
+    if (p.ts_a) alpha = __fmul_rn(alpha, *p.ts_a);
+    if (p.ts_b) alpha = __fmul_rn(alpha, *p.ts_b);
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      const int split = t % p.splits;
+      const int tt = t / p.splits;
+      const int tm = tt % tiles_m;
+      const int tn = tt / tiles_m;
+      if (!mbar_wait(acc_full, acc_phase, abort_flag)) break;
+      tc_fence_after();
+      uint32_t v[kCols];
+#pragma unroll
+      for (int c = 0; c < kCols / 16; ++c)
+        tmem_ld16(tmem + (static_cast<uint32_t>(32 * q) << 16) + half * kCols + 16 * c, v + 16 * c);
+      tmem_ld_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      acc_phase ^= 1u;
+      const int64_t row = static_cast<int64_t>(tm) * 128 + 32 * q + lane;
+      const int64_t col0 = static_cast<int64_t>(tn) * BN + half * kCols;
+      if (row >= p.M) continue;
+      if (p.partial) {
+        float* dst = p.partial + (static_cast<int64_t>(split) * p.M + row) * p.N;
+#pragma unroll
+        for (int c = 0; c < kCols; c += 4) {
+          const int64_t col = col0 + c;
+          if (col + 3 < p.N && (p.N & 3) == 0) {
+            *reinterpret_cast<float4*>(dst + col) = make_float4(__uint_as_float(v[c]), __uint_as_float(v[c + 1]),
+                                                                __uint_as_float(v[c + 2]), __uint_as_float(v[c + 3]));
+          } else {
+            for (int e = 0; e < 4; ++e)
+              if (col + e < p.N) dst[col + e] = __uint_as_float(v[c + e]);
+          }
+        }
+      } else if (p.c_dtype == METIS_F32) {
+        float* dst = reinterpret_cast<float*>(p.C) + row * p.ldc;
+#pragma unroll
+        for (int c = 0; c < kCols; c += 4) {
+          const int64_t col = col0 + c;
+          const float4 f = make_float4(__fmul_rn(alpha, __uint_as_float(v[c])), __fmul_rn(alpha, __uint_as_float(v[c + 1])),
+                                       __fmul_rn(alpha, __uint_as_float(v[c + 2])), __fmul_rn(alpha, __uint_as_float(v[c + 3])));
+          if (col + 3 < p.N && p.vec_ok) {
+            *reinterpret_cast<float4*>(dst + col) = f;
+          } else {
+            const float fe[4] = {f.x, f.y, f.z, f.w};
+            for (int e = 0; e < 4; ++e)
+              if (col + e < p.N) dst[col + e] = fe[e];
+          }
+        }
+      } else {
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.C) + row * p.ldc;
+#pragma unroll
+        for (int c = 0; c < kCols; c += 4) {
+          const int64_t col = col0 + c;
+          __nv_bfloat16 b[4];
+          for (int e = 0; e < 4; ++e) b[e] = __float2bfloat16_rn(__fmul_rn(alpha, __uint_as_float(v[c + e])));
+          if (col + 3 < p.N && p.vec_ok) {
+            uint2 u;
+            u.x = static_cast<uint32_t>(__bfloat16_as_ushort(b[0])) | (static_cast<uint32_t>(__bfloat16_as_ushort(b[1])) << 16);
+            u.y = static_cast<uint32_t>(__bfloat16_as_ushort(b[2])) | (static_cast<uint32_t>(__bfloat16_as_ushort(b[3])) << 16);
+            *reinterpret_cast<uint2*>(dst + col) = u;
+          } else {
+            for (int e = 0; e < 4; ++e)
+              if (col + e < p.N) dst[col + e] = b[e];
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+  if (threadIdx.x == 0 && *abort_flag) report(p.dev_status, METIS_DEV_TIMEOUT);
+}
+
+// Deterministic split-K reduction: C = alpha * sum_s partial[s] (+ nothing).
+__global__ void splitk_reduce_kernel(const float* partial, int splits, int64_t M, int64_t N, const float* ts_a,
+                                     const float* ts_b, void* C, int c_dtype, int64_t ldc) {
+  const int64_t total = M * N;
+  float alpha = 1.f;
+  if (ts_a) alpha = __fmul_rn(alpha, *ts_a);
+  if (ts_b) alpha = __fmul_rn(alpha, *ts_b);
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float s = 0.f;
+    for (int k = 0; k < splits; ++k) s += partial[k * total + i];
+    const int64_t r = i / N, c = i - r * N;
+    const float v = __fmul_rn(alpha, s);
+    if (c_dtype == METIS_F32)
+      reinterpret_cast<float*>(C)[r * ldc + c] = v;
+    else
+      reinterpret_cast<__nv_bfloat16*>(C)[r * ldc + c] = __float2bfloat16_rn(v);
+  }
+}
+
+template <int BN>
+cudaError_t launch_bn(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& la,
+                      const CUtensorMap& lb, int grid, cudaStream_t s) {
+  const int bytes = Smem<BN>::kBytes;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(gemm_fp4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  gemm_fp4_kernel<BN><<<grid, kThreads, bytes, s>>>(p, a, b, la, lb);
+  return cudaGetLastError();
+}
+
+CUresult fp4_map(CUtensorMap* m, const uint8_t* codes, int64_t rows, int64_t inner, uint32_t box_rows) {
+  const uint64_t dims[2] = {static_cast<uint64_t>(inner / 2), static_cast<uint64_t>(rows)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(inner / 2)};
+  const uint32_t box[2] = {128, box_rows};
+  return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, codes, dims, strides, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+CUresult bf16_map(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, uint32_t box_rows) {
+  const uint64_t dims[2] = {static_cast<uint64_t>(cols), static_cast<uint64_t>(rows)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(cols) * 2};
+  const uint32_t box[2] = {64, box_rows};
+  return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box,
+                           CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+}  // namespace
+
+metis_status run_gemm_fp4(const GemmCall& g, cudaStream_t s) {
+  GemmParams p{};
+  p.fmt = g.fmt;
+  p.M = static_cast<int>(g.M);
+  p.N = static_cast<int>(g.N);
+  p.num_kt = static_cast<int>((g.K + 255) / 256);
+  const int64_t sc_cols = tc_scale_cols(g.fmt, g.K);
+  p.sfa = g.a_scales;
+  p.sfb = g.b_scales;
+  p.sfa_chunks = sc_cols / 4;
+  p.sfb_chunks = sc_cols / 4;
+  p.sfb_rows = tc_scale_rows(g.N);
+  p.ts_a = g.fmt == METIS_NVFP4 ? g.a_tensor_scale : nullptr;
+  p.ts_b = g.fmt == METIS_NVFP4 ? g.b_tensor_scale : nullptr;
+  p.lr_chunks = g.lr_k / 64;
+  p.C = g.C;
+  p.c_dtype = g.c_dtype;
+  p.ldc = g.ldc;
+  p.vec_ok = (g.ldc % 4 == 0) && ((reinterpret_cast<uintptr_t>(g.C) & 15u) == 0);
+  p.dev_status = g.dev_status;
+  p.splits = g.splits < 1 ? 1 : g.splits;
+  p.partial = g.partial;
+  if (p.splits > 1 && !p.partial) return METIS_ERR_ARG;
+  if (p.splits > 1 && p.lr_chunks) return METIS_ERR_ARG;
+  const int bn = g.bn;
+  CUtensorMap ma, mb, mla, mlb;
+  if (fp4_map(&ma, g.a_codes, g.M, g.K, 128) != CUDA_SUCCESS) return METIS_ERR_CUDA;
+  if (fp4_map(&mb, g.b_codes, g.N, g.K, static_cast<uint32_t>(bn)) != CUDA_SUCCESS) return METIS_ERR_CUDA;
+  if (p.lr_chunks) {
+    if (bf16_map(&mla, g.lr_a, g.M, g.lr_k, 128) != CUDA_SUCCESS) return METIS_ERR_CUDA;
+    if (bf16_map(&mlb, g.lr_b, g.N, g.lr_k, static_cast<uint32_t>(bn)) != CUDA_SUCCESS) return METIS_ERR_CUDA;
+  } else {
+    mla = ma;
+    mlb = mb;
+  }
+  const int tiles = static_cast<int>(((g.M + 127) / 128) * ((g.N + bn - 1) / bn)) * p.splits;
+  const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
+  cudaError_t e;
+  if (bn == 256)
+    e = launch_bn<256>(p, ma, mb, mla, mlb, grid, s);
+  else if (bn == 128)
+    e = launch_bn<128>(p, ma, mb, mla, mlb, grid, s);
+  else if (bn == 64)
+    e = launch_bn<64>(p, ma, mb, mla, mlb, grid, s);
+  else
+    return METIS_ERR_ARG;
+  if (e != cudaSuccess) return METIS_ERR_CUDA;
+  if (p.splits > 1 && g.C) {
+    const int64_t total = g.M * g.N;
+    int blocks = static_cast<int>((total + 255) / 256);
+    if (blocks > device_sm_count() * 8) blocks = device_sm_count() * 8;
+    splitk_reduce_kernel<<<blocks, 256, 0, s>>>(p.partial, p.splits, g.M, g.N, p.ts_a, p.ts_b, g.C, g.c_dtype, g.ldc);
+  }
+  return launch_status();
+}
+
+}  // namespace metis

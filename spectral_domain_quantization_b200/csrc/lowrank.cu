@@ -1,0 +1,156 @@
+// Low-rank terms of the split-operand product, assembled into the bf16
+// operands that the FP4 GEMM accumulates into its TMEM accumulator.
+//
+// Source: SII release on Metis, section 2.4 item 1 (the dominant rank-k part is
+// quantized on its own and still enters the product); Averis paragraphs of
+// the arXiv 2603.10444 retelling (mean and residual recombine in the output).
+//
+// For C = A B with A = R_A + F_A S_A P_A^T and B = R_B + P_B S_B F_B^T:
+//   C = R_A R_B + T1 F_B^T + F_A T2,
+//   T1 = (R_A P_B + F_A S_A (P_A^T P_B)) S_B     (M x kB)
+//   T2 = S_A (P_A^T R_B)                          (kA x N)
+// The GEMM accumulates alpha_main * (R_A R_B) with alpha_main the product of
+// the residuals' tensor scales, so the low-rank operands are pre-divided by
+// it.  Dequantized factors divided by their own tensor scale are exact in
+// bf16 (<= 6 significant bits); fp32 T1/T2 enter as a bf16 hi/lo pair:
+//   LA[m] = [hi(T1') | lo(T1') | F~_A | F~_A | 0...]
+//   LB[n] = [F~_B    | F~_B    | hi(T2') | lo(T2') | 0...]
+#include "common.cuh"
+#include "lowrank.h"
+
+namespace metis {
+
+namespace {
+
+// Dequantized value of factor element (row i of `outer`, position l of
+// `inner`) without the NVFP4 tensor scale.
+MDEV float factor_value(const FactorView& f, int64_t i, int64_t l) {
+  if (f.ones) return 1.f;
+  const uint8_t byte = f.codes[i * (f.inner / 2) + (l >> 1)];
+  const uint32_t code = (l & 1) ? (byte >> 4) : (byte & 15u);
+  const int bs = f.fmt == METIS_MXFP4 ? 32 : 16;
+  const uint8_t sc = f.scales[tc_scale_offset(i, l / bs, f.scale_cols)];
+  const float s = f.fmt == METIS_MXFP4 ? ldexpf(1.f, static_cast<int>(sc) - 127) : e4m3_value(sc);
+  return e2m1_value(code) * s;  // exact
+}
+
+MDEV float tscale(const FactorView& f) {
+  return (f.ones || f.fmt != METIS_NVFP4 || !f.tensor_scale) ? 1.f : *f.tensor_scale;
+}
+
+// Cab[i][j] = sum_l P^_A[i][l] P^_B[j][l] (with tensor scales), one block per (i, j).
+__global__ void cab_kernel(FactorView pa, FactorView pb, int64_t K, int kb, float* cab) {
+  const int i = blockIdx.y, j = blockIdx.x;
+  float s = 0.f;
+  for (int64_t l = threadIdx.x; l < K; l += blockDim.x) s += factor_value(pa, i, l) * factor_value(pb, j, l);
+  __shared__ float red[256];
+  red[threadIdx.x] = s;
+  __syncthreads();
+  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
+    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) cab[i * kb + j] = red[0] * tscale(pa) * tscale(pb);
+}
+
+MDEV void split_hi_lo(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
+  hi = __float2bfloat16_rn(x);
+  lo = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(hi)));
+}
+
+MDEV float alpha_main(const LowRankArgs& a) {
+  float v = 1.f;
+  if (a.ts_ra) v = __fmul_rn(v, *a.ts_ra);
+  if (a.ts_rb) v = __fmul_rn(v, *a.ts_rb);
+  return v;
+}
+
+// LA rows: one thread per (m, column of LA).
+__global__ void build_la_kernel(LowRankArgs a) {
+  const int64_t total = a.M * a.lr_k;
+  const float inv_alpha = 1.f / alpha_main(a);
+  const float s_fb = tscale(a.fb);
+  const float s_fa = tscale(a.fa);
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t m = t / a.lr_k;
+    const int c = static_cast<int>(t - m * a.lr_k);
+    __nv_bfloat16 out = __float2bfloat16_rn(0.f);
+    if (c < 2 * a.kb) {
+      const int j = c % a.kb;
+      float v = a.t1raw ? a.t1raw[m * a.t1_ld + j] : 0.f;
+      if (a.ka > 0 && a.cab) {
+        float acc = 0.f;
+        for (int i = 0; i < a.ka; ++i) {
+          const float sa = a.s_a ? a.s_a[i] : 1.f;
+          acc += factor_value(a.fa, i, m) * s_fa * sa * a.cab[i * a.kb + j];
+        }
+        v += acc;
+      }
+      const float sb = a.s_b ? a.s_b[j] : 1.f;
+      v = v * sb * s_fb * inv_alpha;
+      __nv_bfloat16 hi, lo;
+      split_hi_lo(v, hi, lo);
+      out = c < a.kb ? hi : lo;
+    } else if (c < 2 * a.kb + 2 * a.ka) {
+      const int i = (c - 2 * a.kb) % a.ka;
+      out = __float2bfloat16_rn(factor_value(a.fa, i, m));
+    }
+    a.la[m * a.lr_k + c] = out;
+  }
+}
+
+// LB rows: one thread per (n, column of LB).
+__global__ void build_lb_kernel(LowRankArgs a) {
+  const int64_t total = a.N * a.lr_k;
+  const float inv_alpha = 1.f / alpha_main(a);
+  const float s_fa = tscale(a.fa);
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t n = t / a.lr_k;
+    const int c = static_cast<int>(t - n * a.lr_k);
+    __nv_bfloat16 out = __float2bfloat16_rn(0.f);
+    if (c < 2 * a.kb) {
+      out = __float2bfloat16_rn(factor_value(a.fb, c % a.kb, n));
+    } else if (c < 2 * a.kb + 2 * a.ka) {
+      const int cc = c - 2 * a.kb;
+      const int i = cc % a.ka;
+      const float sa = a.s_a ? a.s_a[i] : 1.f;
+      const float v = a.t2raw[i * a.t2_ld + n] * sa * s_fa * inv_alpha;
+      __nv_bfloat16 hi, lo;
+      split_hi_lo(v, hi, lo);
+      out = cc < a.ka ? hi : lo;
+    }
+    a.lb[n * a.lr_k + c] = out;
+  }
+}
+
+__global__ void copy_rows_kernel(const float* src, float* dst, int64_t n) {
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    dst[i] = src[i];
+}
+
+int blocks_for(int64_t n, int sms) {
+  int64_t b = (n + 255) / 256;
+  if (b > sms * 8) b = sms * 8;
+  return static_cast<int>(b < 1 ? 1 : b);
+}
+
+}  // namespace
+
+void launch_cab(const FactorView& pa, const FactorView& pb, int64_t K, int ka, int kb, float* cab,
+                cudaStream_t s) {
+  cab_kernel<<<dim3(kb, ka), 256, 0, s>>>(pa, pb, K, kb, cab);
+}
+
+void launch_build_lowrank(const LowRankArgs& a, int sms, cudaStream_t s) {
+  build_la_kernel<<<blocks_for(a.M * a.lr_k, sms), 256, 0, s>>>(a);
+  build_lb_kernel<<<blocks_for(a.N * a.lr_k, sms), 256, 0, s>>>(a);
+}
+
+void launch_copy(const float* src, float* dst, int64_t n, int sms, cudaStream_t s) {
+  copy_rows_kernel<<<blocks_for(n, sms), 256, 0, s>>>(src, dst, n);
+}
+
+}  // namespace metis

@@ -1,0 +1,48 @@
+// Interface of the low-rank operand builders (lowrank.cu).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/metis.h"
+
+namespace metis {
+
+// Read-only view of one FP4 factor (outer = k, inner = length), or the
+// all-ones vector.
+struct FactorView {
+  int ones;
+  int fmt;
+  int64_t inner;
+  int64_t scale_cols;
+  const uint8_t* codes;
+  const uint8_t* scales;
+  const float* tensor_scale;
+};
+
+struct LowRankArgs {
+  int64_t M, N;
+  int ka, kb;
+  int64_t lr_k;             // padded width of LA / LB (multiple of 64)
+  FactorView fa;            // F_A (outer ka, inner M)
+  FactorView fb;            // F_B (outer kb, inner N)
+  const float* s_a;         // S_A (ka) or NULL
+  const float* s_b;         // S_B (kb) or NULL
+  const float* t1raw;       // R_A P_B, M x kb (row stride t1_ld), or NULL
+  int64_t t1_ld;
+  const float* t2raw;       // P_A^T R_B, ka x N (row stride t2_ld)
+  int64_t t2_ld;
+  const float* cab;         // P_A^T P_B, ka x kb, or NULL
+  const float* ts_ra;       // tensor scales of the residuals (NVFP4) or NULL
+  const float* ts_rb;
+  __nv_bfloat16* la;        // out: M x lr_k
+  __nv_bfloat16* lb;        // out: N x lr_k
+};
+
+void launch_cab(const FactorView& pa, const FactorView& pb, int64_t K, int ka, int kb, float* cab,
+                cudaStream_t s);
+void launch_build_lowrank(const LowRankArgs& a, int sms, cudaStream_t s);
+void launch_copy(const float* src, float* dst, int64_t n, int sms, cudaStream_t s);
+
+}  // namespace metis

@@ -21,3 +21,13 @@ def pytest_configure(config):
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")
+
+
+@pytest.fixture(autouse=True)
+def _gpu_guard(request):
+    """GPU tests need CUDA; without it they are skipped (they are deselected by
+    ``-m "not gpu"`` anyway).  With CUDA present, a missing library fails."""
+    if request.node.get_closest_marker("gpu") is not None:
+        import torch
+        if not torch.cuda.is_available():
+            pytest.skip("no CUDA device")
