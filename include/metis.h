@@ -113,6 +113,11 @@ const char* metis_status_string(int32_t status);
 /* Host-only: 1 if a device of compute capability 10.x is current, else 0. */
 int32_t metis_device_supported(void);
 
+/* Host-only: description of the last METIS_ERR_CUDA reported on this thread
+ * (which step failed and the CUDA error string); "" if none.  The string is
+ * owned by the library and overwritten by the next failure on the thread. */
+const char* metis_last_error(void);
+
 /*
  * metis_quantize_fp4 -- block-quantize a dense matrix to FP4.
  * Source: SII release section 2.3 / Fig. 3 (one scale per block, set by the

@@ -28,7 +28,13 @@ FMT_NAME = {MXFP4: "mx", NVFP4: "nv"}
 class MetisError(RuntimeError):
     def __init__(self, status, what):
         self.status = status
-        super().__init__(f"{what}: {status_string(status)} (status {status})")
+        detail = ""
+        if status == 6:
+            try:
+                detail = " [" + lib().metis_last_error().decode() + "]"
+            except Exception:  # pragma: no cover
+                pass
+        super().__init__(f"{what}: {status_string(status)} (status {status}){detail}")
 
 
 class FP4Struct(ctypes.Structure):
@@ -62,6 +68,7 @@ _SIGS = {
     "metis_fp4_scales_bytes": (ctypes.c_size_t, [_I32, _I64, _I64]),
     "metis_status_string": (ctypes.c_char_p, [_I32]),
     "metis_device_supported": (_I32, []),
+    "metis_last_error": (ctypes.c_char_p, []),
     "metis_quantize_fp4": (_I32, [_VP, _I32, _I64, _I64, _I64, _I32, _VP, _FP, _VP, _SZP, _VP]),
     "metis_split": (_I32, [_VP, _I32, _I64, _I64, _I64, ctypes.POINTER(SplitParams), _VP, _VP, _VP,
                            _FP, _FP, _FP, _FP, _VP, _VP, _VP, _SZP, _VP, _VP]),
@@ -271,3 +278,106 @@ def linear_bwd(dY_n, Wt, Xt, dY_m, M, N, K, out_dtype=torch.float32, dX=None, dW
          _ptr(dW) if want_dw else None, dW.stride(0) if want_dw else 0, dt),
         (_ptr(dev_status), _stream()), dev, "metis_linear_bwd")
     return dX, dW
+
+
+# --------------------------------------------------------------------------
+# spectral split
+# --------------------------------------------------------------------------
+
+SKETCH = {"gaussian": SKETCH_GAUSSIAN, "sparse_sign": SKETCH_SPARSE_SIGN}
+
+
+class Split:
+    """Outputs of metis_split: U (m x k), S (k), V (n x k) float32; FP4 U_q
+    (k x m), V_q (k x n), R_rows (m x n, blocks along n), R_cols (n x m,
+    blocks along m); optional float32 residual tap and sample indices."""
+
+    def __init__(self, **kw):
+        self.__dict__.update(kw)
+
+    def operand(self, side, axis_rows=True):
+        """Operand of a product: side "right" for W in X W (residual quantized
+        along K = rows of W), "left" for X in X W (residual along its columns)."""
+        if side == "right":
+            return Operand(self.R_cols if axis_rows else self.R_rows, self.k, self.U_q, self.V_q, self.S)
+        return Operand(self.R_rows, self.k, self.V_q, self.U_q, self.S)
+
+
+def split(A, k, p, q=1, seed=0, fmt="nv", sketch="gaussian", nnz=4, sample_rows=0, max_sweeps=40,
+          rows=True, cols=True, factors=True, tap=False, dev_status=None):
+    """Spectral split A = U diag(S) V^T + R with FP4 outputs (metis_split)."""
+    if A.dim() != 2 or A.stride(1) != 1:
+        raise ValueError("A must be a row-major 2-D tensor")
+    m, n = A.shape
+    dev = A.device
+    f = FMT[fmt]
+    U = torch.empty((m, k), dtype=torch.float32, device=dev)
+    S = torch.empty(k, dtype=torch.float32, device=dev)
+    V = torch.empty((n, k), dtype=torch.float32, device=dev)
+    U_q = QTensor(f, k, m, dev) if factors else None
+    V_q = QTensor(f, k, n, dev) if factors else None
+    R_rows = QTensor(f, m, n, dev) if rows else None
+    R_cols = QTensor(f, n, m, dev) if cols else None
+    R_f32 = torch.empty((m, n), dtype=torch.float32, device=dev) if tap else None
+    idx = torch.empty(sample_rows, dtype=torch.int32, device=dev) if sample_rows else None
+    if dev_status is None:
+        dev_status = torch.zeros(1, dtype=torch.int32, device=dev)
+    prm = SplitParams(k=k, p=p, power_iters=q, seed=seed, sketch=SKETCH[sketch], sparse_nnz=nnz,
+                      sample_rows=sample_rows, fmt=f, max_jacobi_sweeps=max_sweeps)
+    st = [t.struct() if t is not None else None for t in (U_q, V_q, R_rows, R_cols)]
+    refs = [ctypes.byref(s) if s is not None else None for s in st]
+    _call_with_workspace(
+        lib().metis_split,
+        (_ptr(A), _dtype_code(A), m, n, A.stride(0), ctypes.byref(prm), _ptr(U), _ptr(S), _ptr(V), *refs,
+         _ptr(R_f32), _ptr(idx)),
+        (_ptr(dev_status), _stream()), dev, "metis_split")
+    return Split(U=U, S=S, V=V, U_q=U_q, V_q=V_q, R_rows=R_rows, R_cols=R_cols, R_f32=R_f32, idx=idx,
+                 dev_status=dev_status, k=k, fmt=f)
+
+
+# --------------------------------------------------------------------------
+# Averis
+# --------------------------------------------------------------------------
+
+class AverisSplit:
+    """Outputs of averis_split: mean (n), mean_q (1 x n), R_rows (m x n,
+    blocks along n), R_cols (n x m, blocks along m, with inner sums), tap."""
+
+    def __init__(self, **kw):
+        self.__dict__.update(kw)
+
+    def left(self):
+        """X as the left operand of X W (contraction over n): 1 mu^T + R."""
+        return Operand(self.R_rows, 1, self.mean_q, None, None)
+
+    def left_t(self):
+        """X^T as the left operand of X^T dY (contraction over m): mu 1^T + R^T."""
+        return Operand(self.R_cols, 1, None, self.mean_q, None)
+
+    def right_m(self):
+        """dY as the right operand of X^T dY (contraction over m): 1 nu^T + R."""
+        return Operand(self.R_cols, 1, None, self.mean_q, None)
+
+
+def averis_split(X, fmt="nv", rows=True, cols=True, tap=False, dev_status=None):
+    """Mean / residual split with FP4 outputs (averis_split)."""
+    if X.dim() != 2 or X.stride(1) != 1:
+        raise ValueError("X must be a row-major 2-D tensor")
+    m, n = X.shape
+    dev = X.device
+    f = FMT[fmt]
+    mean = torch.empty(n, dtype=torch.float32, device=dev)
+    mean_q = QTensor(f, 1, n, dev)
+    R_rows = QTensor(f, m, n, dev, inner_sum=True) if rows else None
+    R_cols = QTensor(f, n, m, dev, inner_sum=True) if cols else None
+    R_f32 = torch.empty((m, n), dtype=torch.float32, device=dev) if tap else None
+    if dev_status is None:
+        dev_status = torch.zeros(1, dtype=torch.int32, device=dev)
+    st = [t.struct() if t is not None else None for t in (mean_q, R_rows, R_cols)]
+    refs = [ctypes.byref(s) if s is not None else None for s in st]
+    _call_with_workspace(
+        lib().averis_split,
+        (_ptr(X), _dtype_code(X), m, n, X.stride(0), f, _ptr(mean), *refs, _ptr(R_f32)),
+        (_ptr(dev_status), _stream()), dev, "averis_split")
+    return AverisSplit(mean=mean, mean_q=mean_q, R_rows=R_rows, R_cols=R_cols, R_f32=R_f32,
+                       dev_status=dev_status, fmt=f)

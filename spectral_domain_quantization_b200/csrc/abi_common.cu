@@ -1,4 +1,5 @@
 // Host-side helpers of the C ABI and the entry points that need no kernels.
+#include <cstdio>
 #include <mutex>
 
 #include "abi_common.h"
@@ -78,9 +79,47 @@ metis_status check_fp4(const metis_fp4_tensor* t, int64_t outer, int64_t inner, 
   return METIS_OK;
 }
 
+namespace {
+thread_local char g_last_error[256] = "";
+}
+
+metis_status fail(metis_status st, const char* where, const char* detail) {
+  snprintf(g_last_error, sizeof(g_last_error), "%s%s%s", where ? where : "", detail ? ": " : "",
+           detail ? detail : "");
+  return st;
+}
+
+bool ensure_smem(const void* kernel, size_t bytes) {
+  static std::mutex mu;
+  static const void* keys[64];
+  static size_t vals[64];
+  static int count = 0;
+  std::lock_guard<std::mutex> lock(mu);
+  int slot = -1;
+  for (int i = 0; i < count; ++i)
+    if (keys[i] == kernel) slot = i;
+  if (slot >= 0 && vals[slot] >= bytes) return true;
+  if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
+      cudaSuccess)
+    return false;
+  if (slot < 0 && count < 64) {
+    slot = count++;
+    keys[slot] = kernel;
+  }
+  if (slot >= 0) vals[slot] = bytes;
+  return true;
+}
+
+metis_status step_status(const char* where) {
+  const cudaError_t e = cudaGetLastError();
+  if (e == cudaSuccess) return METIS_OK;
+  return fail(METIS_ERR_CUDA, where, cudaGetErrorString(e));
+}
+
 metis_status launch_status() {
   const cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? METIS_OK : METIS_ERR_CUDA;
+  if (e == cudaSuccess) return METIS_OK;
+  return fail(METIS_ERR_CUDA, "kernel launch", cudaGetErrorString(e));
 }
 
 }  // namespace metis
@@ -113,5 +152,7 @@ const char* metis_status_string(int32_t status) {
 }
 
 int32_t metis_device_supported(void) { return metis::device_is_sm100() ? 1 : 0; }
+
+const char* metis_last_error(void) { return metis::g_last_error; }
 
 }  // extern "C"

@@ -47,6 +47,14 @@ metis_status check_fp4(const metis_fp4_tensor* t, int64_t outer, int64_t inner, 
 
 // Finish a launch sequence: map a pending CUDA error to METIS_ERR_CUDA.
 metis_status launch_status();
+// METIS_OK, or METIS_ERR_CUDA naming `where` if a launch or call before it
+// failed (a synchronous error such as an invalid launch configuration).
+metis_status step_status(const char* where);
+// Raise a kernel's dynamic shared-memory limit to at least `bytes` (cached
+// per kernel); false if the runtime refuses.
+bool ensure_smem(const void* kernel, size_t bytes);
+// Record a failure description for metis_last_error(); returns `st`.
+metis_status fail(metis_status st, const char* where, const char* detail = nullptr);
 
 }  // namespace metis
 

@@ -354,12 +354,7 @@ template <int BN>
 cudaError_t launch_bn(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& la,
                       const CUtensorMap& lb, int grid, cudaStream_t s) {
   const int bytes = Smem<BN>::kBytes;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(gemm_fp4_kernel<BN>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
+  if (!ensure_smem(reinterpret_cast<const void*>(gemm_fp4_kernel<BN>), bytes)) return cudaErrorInvalidValue;
   gemm_fp4_kernel<BN><<<grid, kThreads, bytes, s>>>(p, a, b, la, lb);
   return cudaGetLastError();
 }
@@ -408,11 +403,11 @@ metis_status run_gemm_fp4(const GemmCall& g, cudaStream_t s) {
   if (p.splits > 1 && p.lr_chunks) return METIS_ERR_ARG;
   const int bn = g.bn;
   CUtensorMap ma, mb, mla, mlb;
-  if (fp4_map(&ma, g.a_codes, g.M, g.K, 128) != CUDA_SUCCESS) return METIS_ERR_CUDA;
-  if (fp4_map(&mb, g.b_codes, g.N, g.K, static_cast<uint32_t>(bn)) != CUDA_SUCCESS) return METIS_ERR_CUDA;
+  if (fp4_map(&ma, g.a_codes, g.M, g.K, 128) != CUDA_SUCCESS) return fail(METIS_ERR_CUDA, "gemm_fp4 tensor map");
+  if (fp4_map(&mb, g.b_codes, g.N, g.K, static_cast<uint32_t>(bn)) != CUDA_SUCCESS) return fail(METIS_ERR_CUDA, "gemm_fp4 tensor map");
   if (p.lr_chunks) {
-    if (bf16_map(&mla, g.lr_a, g.M, g.lr_k, 128) != CUDA_SUCCESS) return METIS_ERR_CUDA;
-    if (bf16_map(&mlb, g.lr_b, g.N, g.lr_k, static_cast<uint32_t>(bn)) != CUDA_SUCCESS) return METIS_ERR_CUDA;
+    if (bf16_map(&mla, g.lr_a, g.M, g.lr_k, 128) != CUDA_SUCCESS) return fail(METIS_ERR_CUDA, "gemm_fp4 tensor map");
+    if (bf16_map(&mlb, g.lr_b, g.N, g.lr_k, static_cast<uint32_t>(bn)) != CUDA_SUCCESS) return fail(METIS_ERR_CUDA, "gemm_fp4 tensor map");
   } else {
     mla = ma;
     mlb = mb;
@@ -428,7 +423,7 @@ metis_status run_gemm_fp4(const GemmCall& g, cudaStream_t s) {
     e = launch_bn<64>(p, ma, mb, mla, mlb, grid, s);
   else
     return METIS_ERR_ARG;
-  if (e != cudaSuccess) return METIS_ERR_CUDA;
+  if (e != cudaSuccess) return fail(METIS_ERR_CUDA, "gemm_fp4 launch", cudaGetErrorString(e));
   if (p.splits > 1 && g.C) {
     const int64_t total = g.M * g.N;
     int blocks = static_cast<int>((total + 255) / 256);

@@ -1,0 +1,46 @@
+// Interface of the small dense linear algebra kernels (small_linalg.cu).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace metis {
+
+struct ApplyArgs {
+  const float* in;         // rows x kin, row stride in_ld
+  int64_t rows;
+  int kin;
+  int64_t in_ld;
+  const float* M;          // kin x kout, row-major
+  int kout;
+  int upper;               // M upper triangular (only j <= c terms)
+  float* out;              // optional rows x kout, row stride out_ld
+  int64_t out_ld;
+  __nv_bfloat16* outT;     // optional [2*lpT][ldx]: hi rows 0..kout-1, lo rows lpT..
+  int lpT;
+  int64_t ldx;
+  double* gpart;           // optional [blocks][kout][kout]
+};
+
+int64_t gram_blocks(int64_t rows);
+// Y (optional) = sum of split partials; G = Y^T Y (float64, lp x lp).
+// gpart: gram_blocks(rows) * lp * lp doubles of scratch.
+void launch_gram(const float* partial, int splits, int64_t rows, int lp, float* Y, double* gpart, double* G,
+                 cudaStream_t s);
+void launch_gram_reduce(const double* gpart, int nblocks, int lp, double* G, cudaStream_t s);
+// Rinv (lp x lp float, upper triangular) with G = R^T R, dropped pivots -> 0.
+void launch_cholesky_inv(const double* G, int lp, float* Rinv, cudaStream_t s);
+void launch_apply(const ApplyArgs& a, cudaStream_t s);
+// Symmetric eigen-decomposition, eigenvalues descending; evec column j.
+void launch_jacobi(const double* C, int n, int max_sweeps, double* eval, float* evec, int32_t* dev_status,
+                   cudaStream_t s);
+void launch_factor_mats(const double* eval, const float* evec, int lp, int k, float* Mu, float* Mv, float* S,
+                        cudaStream_t s);
+int64_t sign_blocks(int64_t rows);
+// Make the largest-|.| entry (lowest row on ties) of each U column positive,
+// flipping the matching V column.
+void launch_signs(float* U, int64_t m, float* V, int64_t n, int k, float* bmax, int64_t* bidx, float* sign, int sms,
+                  cudaStream_t s);
+
+}  // namespace metis

@@ -1,0 +1,114 @@
+"""GPU parity of metis_split against the oracle's randomized split.
+
+Checks (reading R8): singular values S, the rank-k part L = U S V^T and the
+residual R within relative Frobenius 1e-3; U, V column by column where the
+singular values are well separated; FP4 outputs (U_q, V_q, R along both axes)
+bit-exact against the oracle quantizer fed the GPU's own float32 U, V and R."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import fp4, sketch, split
+from spectral_domain_quantization_b200 import api, inputs
+
+from gpu_helpers import assert_fp4_equal, rel_fro, to_device
+
+pytestmark = pytest.mark.gpu
+
+TOL = 1e-3
+
+
+def _check(A64, res, ref, fmt, check_vectors=True, r_tol=TOL):
+    U = res.U.cpu().numpy().astype(np.float64)
+    S = res.S.cpu().numpy().astype(np.float64)
+    V = res.V.cpu().numpy().astype(np.float64)
+    assert int(res.dev_status.cpu()[0]) == 0
+    assert rel_fro(S, ref["S"]) < TOL
+    L = (U * S) @ V.T
+    Lref = (ref["U"] * ref["S"]) @ ref["V"].T
+    assert rel_fro(L, Lref) < TOL
+    R = res.R_f32.cpu().numpy()
+    assert rel_fro(R, ref["R"]) < r_tol
+    assert rel_fro(R.astype(np.float64), A64 - L) < 1e-5      # tap is A - U S V^T
+    if check_vectors:
+        s = ref["S"]
+        gap = np.minimum(np.abs(np.diff(np.r_[np.inf, s])), np.abs(np.diff(np.r_[s, -np.inf])))
+        sep = gap / s > 0.05
+        for j in np.flatnonzero(sep):
+            assert rel_fro(U[:, j], ref["U"][:, j]) < 1e-2, j
+            assert rel_fro(V[:, j], ref["V"][:, j]) < 1e-2, j
+    # FP4 outputs: bit-exact on the GPU's own float32 values
+    k = U.shape[1]
+    assert_fp4_equal(res.U_q, fp4.quantize(res.U.cpu().numpy(), fmt, 0), check_linear=False)
+    assert_fp4_equal(res.V_q, fp4.quantize(res.V.cpu().numpy(), fmt, 0), check_linear=False)
+    assert_fp4_equal(res.R_rows, fp4.quantize(R, fmt, 1), check_linear=False)
+    assert_fp4_equal(res.R_cols, fp4.quantize(R, fmt, 0), check_linear=False)
+
+
+def test_split_tiny_workload():
+    d = inputs.make("tiny_256")
+    c = d["cfg"]
+    A = to_device(d["W"])
+    res = api.split(A, c["k"], c["p"], c["q"], c["sketch_seed"], c["fmt"], tap=True)
+    torch.cuda.synchronize()
+    A64 = d["W"].f64()
+    ref = split.split(A64, c["k"], c["p"], c["q"], c["sketch_seed"])
+    _check(A64, res, ref, c["fmt"])
+
+
+def test_split_exact_rank_recovered():
+    rng = np.random.default_rng(3)
+    A = (rng.standard_normal((192, 6)) @ rng.standard_normal((6, 160))).astype(np.float32)
+    res = api.split(torch.from_numpy(A).cuda(), 8, 8, 1, 7, "mx", tap=True)
+    torch.cuda.synchronize()
+    R = res.R_f32.cpu().numpy()
+    assert np.linalg.norm(R) / np.linalg.norm(A) < 1e-5
+    ref = split.split(A.astype(np.float64), 8, 8, 1, 7)
+    L = (res.U.cpu().numpy().astype(np.float64) * res.S.cpu().numpy()) @ res.V.cpu().numpy().T
+    assert rel_fro(L, (ref["U"] * ref["S"]) @ ref["V"].T) < TOL
+
+
+@pytest.mark.parametrize("fmt", ["nv", "mx"])
+def test_split_layer_shape_reduced(fmt):
+    # the single-layer recipe at 512 x 768 (several tiles), k=64, p=16, q=1
+    d = inputs.make("layer_4096", scale=dict(K=512, N=768, M=128))
+    A = to_device(d["W"])
+    res = api.split(A, 64, 16, 1, 0, fmt, tap=True)
+    torch.cuda.synchronize()
+    A64 = d["W"].f64()
+    ref = split.split(A64, 64, 16, 1, 0)
+    _check(A64, res, ref, fmt)
+
+
+@pytest.mark.parametrize("q", [0, 2])
+def test_split_power_iterations(q):
+    d = inputs.make("layer_4096", scale=dict(K=384, N=256, M=128))
+    A = to_device(d["W"])
+    res = api.split(A, 16, 16, q, 5, "nv", tap=True)
+    torch.cuda.synchronize()
+    A64 = d["W"].f64()
+    _check(A64, res, split.split(A64, 16, 16, q, 5), "nv")
+
+
+def test_split_sampled_sparse_sign():
+    # the sampled-activation recipe at 4096 x 512: 256 rows, sparse sign (4), k=32, p=16
+    d = inputs.make("sampled_65536", scale=dict(M=4096, K=512))
+    A = to_device(d["A"])
+    res = api.split(A, 32, 16, 0, 0, "mx", sketch="sparse_sign", nnz=4, sample_rows=256, tap=True)
+    torch.cuda.synchronize()
+    assert np.array_equal(res.idx.cpu().numpy(), sketch.sample_rows(4096, 256, 0))
+    A64 = d["A"].f64()
+    ref = split.split(A64, 32, 16, 0, 0, kind="sparse_sign", nnz=4, sample_rows=256)
+    _check(A64, res, ref, "mx", check_vectors=False)
+
+
+def test_split_full_size_layer_weight():
+    # W 4096 x 4096 of the single-layer workload, NVFP4, k=64, p=16, q=1
+    d = inputs.make("layer_4096")
+    c = d["cfg"]
+    A = to_device(d["W"])
+    res = api.split(A, c["k"], c["p"], c["q"], c["sketch_seed"], "nv", tap=True)
+    torch.cuda.synchronize()
+    A64 = d["W"].f64()
+    ref = split.split(A64, c["k"], c["p"], c["q"], c["sketch_seed"])
+    _check(A64, res, ref, "nv", check_vectors=False)
