@@ -1,0 +1,385 @@
+#!/usr/bin/env python
+"""Benchmark of the spectral-split W4A4 linear layer on one B200 per rank.
+
+Workload (``layer_4096``): W bf16 4096 x 4096 with a planted spectrum
+sigma_i = 8/i (i <= 256) + N(0, 0.02^2) noise, X bf16 8192 x 4096 N(0, 1);
+one step = metis_split of W (k=64, p=16, one power iteration, Gaussian
+sketch, NVFP4 residual along K, FP4 factors) + metis_quantize_fp4 of X along K
+(NVFP4) + metis_linear_fwd Y = X W (FP4 GEMM with the rank-64 update fused,
+bf16 output).  Inputs are synthetic and seeded (no dataset).
+
+Metric: effective FP4 split-linear TFLOPS = 2 M N K (the dense product the
+layer replaces) / step time, plus the split + quantize time per layer.
+Timing: CUDA events on the launching stream around a CUDA-graph replay of the
+step, L2 (126 MB) flushed with a 512 MB write before every timed step, W >= 3
+warm-up steps, max over ranks.  With torchrun and N GPUs every rank runs the
+same layer independently (replicas: the path has no cross-GPU exchange), and
+``value`` is the work of all ranks over the slowest rank's time.
+
+``--impl reference`` times the CPU oracle (numpy) on a bounded sample of the
+same workload instead: the oracle is the only reference implementation this
+path has.
+"""
+import argparse
+import json
+import os
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+M, K, N = 8192, 4096, 4096
+RANK_K, OVERSAMPLE, POWER_ITERS, SEED = 64, 16, 1, 0
+FLOPS = 2.0 * M * N * K
+METRIC = "FP4 split-linear eff. TFLOPS & % of FP4 peak; split+quantize us/layer"
+CONFIG = {"workload": "layer_4096: W bf16 4096x4096 planted spectrum + X bf16 8192x4096, "
+                      "split k=64 p=16 q=1 Gaussian, NVFP4, forward",
+          "M": M, "K": K, "N": N, "k": RANK_K, "p": OVERSAMPLE, "power_iters": POWER_ITERS,
+          "fmt": "nvfp4", "l2": "flushed (512 MB write) before every timed step"}
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    return ap.parse_args()
+
+
+# --------------------------------------------------------------------------
+# distributed plumbing (replicas; barriers and a max-reduction only)
+# --------------------------------------------------------------------------
+
+def dist_init():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def reduce_max(x, world):
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# --------------------------------------------------------------------------
+# clocks during the timed region
+# --------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) >= 9:
+                rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit())
+        loaded = [v for v in sm if v > 0.5 * smax] or sm
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": smax, "reasons": reasons,
+                "samples": len(rows)}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle sample (cpu_baseline and the reference arm)
+# --------------------------------------------------------------------------
+
+def oracle_sample(data, rows=1024):
+    """The oracle's whole step on a bounded sample: the full split of W and its
+    residual quantization, X quantization and the GEMM on `rows` rows of X.
+    Returns (seconds scaled to the full workload, description)."""
+    from oracle import fp4, gemm, split
+    t0 = time.perf_counter()
+    W = data["W"].f64()
+    r = split.split(W, RANK_K, OVERSAMPLE, POWER_ITERS, SEED)
+    Rq = fp4.quantize(r["R"].astype(np.float32), "nv", 0)
+    Uq = fp4.quantize(r["U"].astype(np.float32), "nv", 0)
+    Vq = fp4.quantize(r["V"].astype(np.float32), "nv", 0)
+    t_split = time.perf_counter() - t0
+    t1 = time.perf_counter()
+    x = data["X"].f32()[:rows]
+    xq = fp4.quantize(x, "nv", 1)
+    gemm.gemm(gemm.Operand(xq), gemm.Operand(Rq, RANK_K, Uq, Vq, r["S"]))
+    t_rows = time.perf_counter() - t1
+    full = t_split + t_rows * (M / rows)
+    return full, f"full W split + residual quantize; X quantize + GEMM on {rows} of {M} rows, scaled x{M // rows}"
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max((i.get("num_threads", 1) for i in threadpool_info()), default=1)
+    except Exception:
+        return os.cpu_count() or 1
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return
+    from spectral_domain_quantization_b200 import inputs
+    data = inputs.make("layer_4096")
+    for _ in range(args.warmup):
+        oracle_sample(data, rows=256)
+    times = []
+    desc = ""
+    for _ in range(args.steps):
+        t, desc = oracle_sample(data, rows=256)
+        times.append(t)
+    step_s = float(np.mean(times))
+    value = FLOPS / step_s / 1e12
+    cores = blas_threads()
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": step_s * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "config": CONFIG,
+            "cpu_baseline": {"kind": "oracle", "value": value, "unit": "TFLOPS", "cores": cores,
+                             "sample": desc},
+            "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------------
+# the GPU path
+# --------------------------------------------------------------------------
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        d = json.load(open(path))
+        return d.get("hbm_gbs", 6650.0), d.get("bf16_tflops", 1590.0), "measured"
+    return 6650.0, 1590.0, "fallback"
+
+
+def run_ours(args, rank, world, local):
+    import torch
+    from spectral_domain_quantization_b200 import api, inputs
+
+    assert torch.cuda.is_available(), "bench needs a GPU"
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if not api.lib().metis_device_supported():
+        raise RuntimeError("metis needs an sm_100 (B200) device")
+    data = inputs.make("layer_4096")
+    w_host = torch.from_numpy(data["W"].data.view(np.int16)).view(torch.bfloat16).pin_memory()
+    x_host = torch.from_numpy(data["X"].data.view(np.int16)).view(torch.bfloat16).pin_memory()
+    W = w_host.to(dev)
+    X = x_host.to(dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+
+    def split_w():
+        return api.split(W, RANK_K, OVERSAMPLE, POWER_ITERS, SEED, "nv", rows=False, cols=True, factors=True,
+                         dev_status=status)
+
+    def quant_x():
+        return api.quantize_fp4(X, "nv", 1)
+
+    def step():
+        s = split_w()
+        xq = quant_x()
+        api.linear_fwd(api.Operand(xq), s.operand("right"), M, N, K, Y=Y, dev_status=status)
+
+    def capture(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        torch.cuda.synchronize()
+        return g
+
+    def time_graph(g, steps, warmup):
+        for _ in range(warmup):
+            flush.fill_(1)
+            g.replay()
+        torch.cuda.synchronize()
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        for i in range(steps):
+            flush.fill_(1)
+            starts[i].record()
+            g.replay()
+            ends[i].record()
+        torch.cuda.synchronize()
+        return float(np.mean([s.elapsed_time(e) for s, e in zip(starts, ends)]))
+
+    # --- the step, as one CUDA graph
+    g_step = capture(step)
+    torch.cuda.synchronize()
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())} during warm-up")
+
+    # kernels of this library launched by one step
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        step()
+        torch.cuda.synchronize()
+    launches = sum(1 for e in prof.events() if e.device_type.name == "CUDA" and "metis" in e.name)
+
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    ms = time_graph(g_step, args.steps, args.warmup)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    ms = reduce_max(ms, world)
+
+    # --- phase breakdown (same flush policy)
+    g_split = capture(split_w)
+    ms_split = time_graph(g_split, args.steps, 3)
+    g_quant = capture(quant_x)
+    ms_quant = time_graph(g_quant, args.steps, 3)
+    s = split_w()
+    xq = quant_x()
+    g_gemm = capture(lambda: api.linear_fwd(api.Operand(xq), s.operand("right"), M, N, K, Y=Y, dev_status=status))
+    ms_gemm = time_graph(g_gemm, args.steps, 3)
+    # the FP4 GEMM kernel alone (plain operands: one launch of the kernel)
+    rq = s.R_cols
+    g_plain = capture(lambda: api.linear_fwd(api.Operand(xq), api.Operand(rq), M, N, K, Y=Y, dev_status=status))
+    ms_plain = time_graph(g_plain, args.steps, 3)
+
+    # --- end to end through host buffers
+    e2e = None
+    if not args.no_e2e:
+        y_host = torch.empty((M, N), dtype=torch.bfloat16).pin_memory()
+        stream = torch.cuda.current_stream()
+        for _ in range(2):
+            W.copy_(w_host, non_blocking=True)
+            X.copy_(x_host, non_blocking=True)
+            g_step.replay()
+            y_host.copy_(Y, non_blocking=True)
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(args.steps):
+            W.copy_(w_host, non_blocking=True)
+            X.copy_(x_host, non_blocking=True)
+            g_step.replay()
+            y_host.copy_(Y, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        e2e_ms = reduce_max(e0.elapsed_time(e1) / args.steps, world)
+        e2e = {"value": world * FLOPS / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS",
+               "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(w_host.numel() * 2 + x_host.numel() * 2),
+               "d2h_bytes_per_step": int(y_host.numel() * 2)}
+
+    hbm, bf16_tf, peak_kind = measured_peaks()
+    fp4_peak = 4.0 * bf16_tf   # nominal dense FP4 / bf16 ratio on B200 (9 / 2.25 PFLOP/s)
+    achieved = FLOPS / (ms_plain * 1e-3) / 1e12
+    value = world * FLOPS / (ms * 1e-3) / 1e12
+
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        reps = []
+        desc = ""
+        t_end = time.time() + 20
+        while time.time() < t_end or not reps:
+            t, desc = oracle_sample(data)
+            reps.append(t)
+        cpu = {"value": FLOPS / float(np.mean(reps)) / 1e12, "unit": "TFLOPS", "cores": blas_threads(),
+               "kind": "oracle", "sample": desc + f"; {len(reps)} repetitions"}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp4 (e2m1, nvfp4 scales; fp32 accumulate)", "data": "synthetic",
+            "config": CONFIG,
+            "frac_of_fp4_peak": value / world / fp4_peak,
+            "split_quantize_us_per_layer": (ms_split + ms_quant) * 1e3,
+            "breakdown_us": {"split_W": ms_split * 1e3, "quantize_X": ms_quant * 1e3,
+                             "linear_fwd": ms_gemm * 1e3, "fp4_gemm_kernel": ms_plain * 1e3},
+            "roofline": {"kernel": "gemm_fp4_kernel<256> (8192x4096x4096 NVFP4)", "bound": "tensor",
+                         "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s", "frac": achieved / fp4_peak,
+                         "peak_source": f"{peak_kind} bf16 {bf16_tf} TFLOP/s x 4 (nominal FP4/bf16 ratio)",
+                         "traffic": None},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    # release graphs before the process group goes away
+    del g_step, g_split, g_quant, g_gemm, g_plain
+
+
+def main():
+    args = parse()
+    rank, world, local = dist_init()
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -194,46 +194,45 @@ metis_status skinny(const Source& a, int mode, const __nv_bfloat16* xt, int64_t 
   return run_skinny_gemm(c, s);
 }
 
-// CholeskyQR2 of the split partials of a rows x lp product.  Output: Q (fp32,
-// rows x lp) and Q^T as bf16 hi / lo rows of qt (row stride ldq).
-metis_status cholqr2(const SplitBuffers& b, int splits, int64_t rows, int lp, float* Q, int64_t ldq,
-                     cudaStream_t s) {
+// CholeskyQR of the split partials of a rows x lp product, `passes` times
+// (2 = CholeskyQR2, for the final basis; 1 suffices for the intermediate
+// bases of the power iteration, whose span is all that is used).  Output: Q
+// (fp32, rows x lp) and Q^T as bf16 hi / lo rows of qt (row stride ldq).
+metis_status cholqr(const SplitBuffers& b, int splits, int64_t rows, int lp, float* Q, int64_t ldq, int passes,
+                    cudaStream_t s) {
   launch_gram(b.part, splits, rows, lp, b.Y, b.gpart, b.G, s);
-  METIS_TRY(step_status("cholqr2 gram"));
-  launch_cholesky_inv(b.G, lp, b.Rinv, s);
-  METIS_TRY(step_status("cholqr2 cholesky"));
-  ApplyArgs a{};
-  a.in = b.Y;
-  a.rows = rows;
-  a.kin = lp;
-  a.in_ld = lp;
-  a.M = b.Rinv;
-  a.kout = lp;
-  a.upper = 1;
-  a.out = b.Q1;
-  a.out_ld = lp;
-  a.gpart = b.gpart;
-  launch_apply(a, s);
-  METIS_TRY(step_status("cholqr2 apply"));
-  launch_gram_reduce(b.gpart, static_cast<int>(gram_blocks(rows)), lp, b.G, s);
-  METIS_TRY(step_status("cholqr2 gram reduce"));
-  launch_cholesky_inv(b.G, lp, b.Rinv, s);
-  METIS_TRY(step_status("cholqr2 cholesky 2"));
-  ApplyArgs a2{};
-  a2.in = b.Q1;
-  a2.rows = rows;
-  a2.kin = lp;
-  a2.in_ld = lp;
-  a2.M = b.Rinv;
-  a2.kout = lp;
-  a2.upper = 1;
-  a2.out = Q;
-  a2.out_ld = lp;
-  a2.outT = b.qt;
-  a2.lpT = lp;
-  a2.ldx = ldq;
-  launch_apply(a2, s);
-  return step_status("cholqr2 apply 2");
+  METIS_TRY(step_status("cholqr gram"));
+  const float* in = b.Y;
+  for (int pass = 0; pass < passes; ++pass) {
+    const bool last = pass == passes - 1;
+    launch_cholesky_inv(b.G, lp, b.Rinv, s);
+    METIS_TRY(step_status("cholqr cholesky"));
+    ApplyArgs a{};
+    a.in = in;
+    a.rows = rows;
+    a.kin = lp;
+    a.in_ld = lp;
+    a.M = b.Rinv;
+    a.kout = lp;
+    a.upper = 1;
+    a.out = last ? Q : b.Q1;
+    a.out_ld = lp;
+    if (last) {
+      a.outT = b.qt;
+      a.lpT = lp;
+      a.ldx = ldq;
+    } else {
+      a.gpart = b.gpart;
+    }
+    launch_apply(a, s);
+    METIS_TRY(step_status("cholqr apply"));
+    if (!last) {
+      launch_gram_reduce(b.gpart, static_cast<int>(apply_blocks(rows)), lp, b.G, s);
+      METIS_TRY(step_status("cholqr gram reduce"));
+      in = b.Q1;
+    }
+  }
+  return METIS_OK;
 }
 
 // Range finder + core on `src` (ms x n): returns Z = src^T Q in b.Zn, Q in
@@ -242,12 +241,12 @@ metis_status range_and_core(const SplitPlan& p, const SplitBuffers& b, const Sou
                             int max_sweeps, int32_t* dev_status, cudaStream_t s) {
   const int lp = p.lp;
   METIS_TRY(skinny(src, 0, b.omt, p.ld_n, 1, lp, p.split_m, b.part, dev_status, s));
-  METIS_TRY(cholqr2(b, p.split_m, src.rows, lp, b.Qm, p.ld_m, s));
+  METIS_TRY(cholqr(b, p.split_m, src.rows, lp, b.Qm, p.ld_m, power_iters > 0 ? 1 : 2, s));
   for (int it = 0; it < power_iters; ++it) {
     METIS_TRY(skinny(src, 1, b.qt, p.ld_m, 2, lp, p.split_n, b.part, dev_status, s));
-    METIS_TRY(cholqr2(b, p.split_n, p.n, lp, b.Zn, p.ld_n, s));
+    METIS_TRY(cholqr(b, p.split_n, p.n, lp, b.Zn, p.ld_n, 1, s));
     METIS_TRY(skinny(src, 0, b.qt, p.ld_n, 2, lp, p.split_m, b.part, dev_status, s));
-    METIS_TRY(cholqr2(b, p.split_m, src.rows, lp, b.Qm, p.ld_m, s));
+    METIS_TRY(cholqr(b, p.split_m, src.rows, lp, b.Qm, p.ld_m, it == power_iters - 1 ? 2 : 1, s));
   }
   METIS_TRY(skinny(src, 1, b.qt, p.ld_m, 2, lp, p.split_n, b.part, dev_status, s));
   launch_gram(b.part, p.split_n, p.n, lp, b.Zn, b.gpart, b.G, s);

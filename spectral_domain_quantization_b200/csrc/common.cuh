@@ -262,9 +262,10 @@ MDEV uint32_t e2m1_code(float q) {
   return c | ((__float_as_uint(q) >> 28) & 8u);
 }
 
+// Value of an E2M1 code.  Twice the magnitudes {0,1,2,3,4,6,8,12} are packed
+// as nibbles of one constant, so the lookup stays in registers.
 __host__ __device__ inline float e2m1_value(uint32_t code) {
-  const float mag[8] = {0.f, 0.5f, 1.f, 1.5f, 2.f, 3.f, 4.f, 6.f};
-  float v = mag[code & 7u];
+  const float v = static_cast<float>((0xC8643210u >> (4u * (code & 7u))) & 15u) * 0.5f;
   return (code & 8u) ? -v : v;
 }
 

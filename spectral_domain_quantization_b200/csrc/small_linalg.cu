@@ -63,105 +63,156 @@ __global__ void gram_kernel(const float* partial, int splits, int64_t rows, int 
   gram_block(ys, nr, lp, ld, gpart + static_cast<int64_t>(blockIdx.x) * lp * lp);
 }
 
+// One warp per Gram entry: lanes take blocks lane, lane+32, ... and the warp
+// reduces with a fixed shuffle tree (deterministic).
 __global__ void gram_reduce_kernel(const double* gpart, int nblocks, int n2, double* G) {
-  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  const int lane = threadIdx.x & 31;
   if (e >= n2) return;
   double s = 0.0;
-  for (int b = 0; b < nblocks; ++b) s += gpart[static_cast<int64_t>(b) * n2 + e];
-  G[e] = s;
+  for (int b = lane; b < nblocks; b += 32) s += gpart[static_cast<int64_t>(b) * n2 + e];
+  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
+  if (lane == 0) G[e] = s;
 }
 
 // G = L L^T (with drops), then Rinv = L^-T (upper triangular, float32).
-__global__ void cholesky_inv_kernel(const double* G, int lp, float* Rinv) {
+// 1024 threads as 32 x 32.  One barrier per column: step j updates the
+// trailing matrix with the unscaled column j (times 1/d_j) and scales column
+// j-1; the thread that updates the next diagonal entry also computes the next
+// pivot's 1/sqrt, so the float64 square root overlaps the update.
+__global__ void __launch_bounds__(1024) cholesky_inv_kernel(const double* G, int lp, float* Rinv) {
   extern __shared__ double sm[];
   const int ld = lp + 1;
   double* L = sm;                  // lp x ld
   double* X = L + lp * ld;         // lp x ld, becomes L^-1
   double* diag0 = X + lp * ld;     // lp
-  double* invd = diag0 + lp;       // lp
+  double* invd = diag0 + lp;       // lp: 1/sqrt(pivot) (0 when dropped)
+  double* sqd = invd + lp;         // lp: sqrt(pivot) (0 when dropped)
   const int t = threadIdx.x, nt = blockDim.x;
+  const int tx = t & 31, ty = t >> 5;
   for (int e = t; e < lp * lp; e += nt) {
     const int i = e / lp, j = e - i * lp;
     L[i * ld + j] = G[e];
     X[i * ld + j] = i == j ? 1.0 : 0.0;
   }
+  for (int i = t; i < lp; i += nt) diag0[i] = G[i * lp + i];
   __syncthreads();
-  for (int i = t; i < lp; i += nt) diag0[i] = L[i * ld + i];
+  if (t == 0) {
+    const double d = L[0];
+    const bool drop = !(diag0[0] > 0.0) || !(d > kDropTol * diag0[0]);
+    sqd[0] = drop ? 0.0 : sqrt(d);
+    invd[0] = drop ? 0.0 : 1.0 / sqd[0];
+  }
   __syncthreads();
   for (int j = 0; j < lp; ++j) {
-    if (t == 0) {
-      const double d = L[j * ld + j];
-      const bool drop = !(diag0[j] > 0.0) || !(d > kDropTol * diag0[j]);
-      const double piv = drop ? 0.0 : sqrt(d);
-      invd[j] = drop ? 0.0 : 1.0 / piv;
-      L[j * ld + j] = piv;
-    }
-    __syncthreads();
     const double inv = invd[j];
-    for (int i = j + 1 + t; i < lp; i += nt) L[i * ld + j] *= inv;
-    __syncthreads();
-    const int w = lp - j - 1;
-    for (int e = t; e < w * w; e += nt) {
-      const int i = j + 1 + e / w, c = j + 1 + e % w;
-      if (c <= i) L[i * ld + c] -= L[i * ld + j] * L[c * ld + j];
+    const double inv2 = inv * inv;
+    for (int i = j + 1 + ty; i < lp; i += 32) {
+      const double lij = L[i * ld + j] * inv2;
+      for (int c = j + 1 + tx; c <= i; c += 32) {
+        const double v = L[i * ld + c] - lij * L[c * ld + j];
+        L[i * ld + c] = v;
+        if (i == j + 1 && c == j + 1) {  // next pivot, ready for step j+1
+          const bool drop = !(diag0[c] > 0.0) || !(v > kDropTol * diag0[c]);
+          const double r = drop ? 0.0 : sqrt(v);
+          sqd[c] = r;
+          invd[c] = drop ? 0.0 : 1.0 / r;
+        }
+      }
+    }
+    if (j > 0) {  // deferred scaling of column j-1
+      const double pinv = invd[j - 1];
+      for (int i = j + t; i < lp; i += nt) L[i * ld + j - 1] *= pinv;
+      if (t == 0) L[(j - 1) * ld + j - 1] = sqd[j - 1];
     }
     __syncthreads();
   }
-  // forward substitution for X = L^-1, one row at a time
+  if (t == 0) L[(lp - 1) * ld + lp - 1] = sqd[lp - 1];
+  // X = L^-1 by rows: step k eliminates with the unscaled row k (times
+  // 1/L_kk) and scales row k-1
   for (int k = 0; k < lp; ++k) {
     const double inv = invd[k];
-    for (int c = t; c <= k; c += nt) X[k * ld + c] *= inv;
-    __syncthreads();
-    const int rows = lp - k - 1, cols = k + 1;
-    for (int e = t; e < rows * cols; e += nt) {
-      const int i = k + 1 + e / cols, c = e % cols;
-      X[i * ld + c] -= L[i * ld + k] * X[k * ld + c];
+    for (int i = k + 1 + ty; i < lp; i += 32) {
+      const double lik = L[i * ld + k] * inv;
+      for (int c = tx; c <= k; c += 32) X[i * ld + c] -= lik * X[k * ld + c];
+    }
+    if (k > 0) {
+      const double pinv = invd[k - 1];
+      for (int c = t; c < k; c += nt) X[(k - 1) * ld + c] *= pinv;
     }
     __syncthreads();
   }
+  for (int c = t; c < lp; c += nt) X[(lp - 1) * ld + c] *= invd[lp - 1];
+  __syncthreads();
   for (int e = t; e < lp * lp; e += nt) {
     const int j = e / lp, c = e - j * lp;  // Rinv[j][c] = X[c][j]
     Rinv[e] = c >= j ? static_cast<float>(X[c * ld + j]) : 0.f;
   }
 }
 
-// out = in (rows x kin, row stride in_ld) * Mx (kin x kout, row-major).
-// Optional: fp32 out (row stride out_ld), transposed bf16 hi/lo copy
-// outT[c][row] and outT[lp + c][row] (row stride ldx), Gram partial.
-__global__ void apply_kernel(ApplyArgs a) {
+constexpr int kApplyRows = 64;
+
+// out = in (rows x kin) * M (kin x kout).  64 rows per CTA, 256 threads, each
+// thread a 4-row x ceil(kout/16)-column register block.  Optional fp32 out,
+// transposed bf16 hi/lo copy, Gram partial of the output block.
+__global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) {
   extern __shared__ float smf[];
-  float* Ms = smf;                                     // kin x kout
-  float* In = Ms + a.kin * a.kout;                     // kRowsPerBlock x (kin + 1)
-  float* Out = In + kRowsPerBlock * (a.kin + 1);       // kRowsPerBlock x (kout + 1)
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock;
-  const int nr = static_cast<int>(imin64(kRowsPerBlock, a.rows - r0));
+  float* Ms = smf;                                   // kin x kout
+  float* In = Ms + a.kin * a.kout;                   // kApplyRows x (kin + 1)
+  float* Out = In + kApplyRows * (a.kin + 1);        // kApplyRows x (kout + 1)
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kApplyRows;
+  const int nr = static_cast<int>(imin64(kApplyRows, a.rows - r0));
   for (int e = threadIdx.x; e < a.kin * a.kout; e += blockDim.x) Ms[e] = a.M[e];
-  for (int e = threadIdx.x; e < kRowsPerBlock * a.kin; e += blockDim.x) {
+  for (int e = threadIdx.x; e < kApplyRows * a.kin; e += blockDim.x) {
     const int r = e / a.kin, c = e - r * a.kin;
     In[r * (a.kin + 1) + c] = r < nr ? a.in[(r0 + r) * a.in_ld + c] : 0.f;
   }
   __syncthreads();
-  for (int e = threadIdx.x; e < kRowsPerBlock * a.kout; e += blockDim.x) {
-    const int c = e / kRowsPerBlock, r = e - c * kRowsPerBlock;  // row fastest
-    float acc = 0.f;
-    const int j0 = a.upper ? 0 : 0;
-    const int j1 = a.upper ? c + 1 : a.kin;
-    for (int j = j0; j < j1; ++j) acc = fmaf(In[r * (a.kin + 1) + j], Ms[j * a.kout + c], acc);
-    Out[r * (a.kout + 1) + c] = acc;
-    if (r < nr) {
-      if (a.out) a.out[(r0 + r) * a.out_ld + c] = acc;
-      if (a.outT) {
-        const __nv_bfloat16 hi = __float2bfloat16_rn(acc);
-        const __nv_bfloat16 lo = __float2bfloat16_rn(__fsub_rn(acc, __bfloat162float(hi)));
+  const int tr = threadIdx.x & 15, tc = threadIdx.x >> 4;
+  constexpr int kMaxCols = 7;  // kout <= 112
+  float acc[4][kMaxCols];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int u = 0; u < kMaxCols; ++u) acc[i][u] = 0.f;
+  for (int j = 0; j < a.kin; ++j) {
+    float x[4], m[kMaxCols];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) x[i] = In[(4 * tr + i) * (a.kin + 1) + j];
+#pragma unroll
+    for (int u = 0; u < kMaxCols; ++u) {
+      const int c = tc + 16 * u;
+      m[u] = c < a.kout ? Ms[j * a.kout + c] : 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int u = 0; u < kMaxCols; ++u) acc[i][u] = fmaf(x[i], m[u], acc[i][u]);
+  }
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int u = 0; u < kMaxCols; ++u) {
+      const int c = tc + 16 * u;
+      if (c < a.kout) Out[(4 * tr + i) * (a.kout + 1) + c] = acc[i][u];
+    }
+  __syncthreads();
+  for (int e = threadIdx.x; e < kApplyRows * a.kout; e += blockDim.x) {
+    if (a.out) {
+      const int r = e / a.kout, c = e - r * a.kout;  // column fastest: coalesced rows
+      if (r < nr) a.out[(r0 + r) * a.out_ld + c] = Out[r * (a.kout + 1) + c];
+    }
+    if (a.outT) {
+      const int c = e / kApplyRows, r = e - c * kApplyRows;  // row fastest: coalesced columns of out^T
+      if (r < nr) {
+        const float v = Out[r * (a.kout + 1) + c];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
         a.outT[static_cast<int64_t>(c) * a.ldx + r0 + r] = hi;
-        a.outT[static_cast<int64_t>(a.lpT + c) * a.ldx + r0 + r] = lo;
+        a.outT[static_cast<int64_t>(a.lpT + c) * a.ldx + r0 + r] = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(hi)));
       }
     }
   }
-  if (a.gpart) {
-    __syncthreads();
-    gram_block(Out, nr, a.kout, a.kout + 1, a.gpart + static_cast<int64_t>(blockIdx.x) * a.kout * a.kout);
-  }
+  if (a.gpart) gram_block(Out, nr, a.kout, a.kout + 1, a.gpart + static_cast<int64_t>(blockIdx.x) * a.kout * a.kout);
 }
 
 // Round-robin pairing: in step r of a sweep over n (even) indices, slot i
@@ -171,117 +222,174 @@ MDEV int rr_index(int slot, int step, int n) {
   return ((slot - 1 + step) % (n - 1)) + 1;
 }
 
-// Symmetric Jacobi eigen-decomposition of C (n x n float64, n even), sorted
-// descending.  evec[i * n + j] = component i of eigenvector j.
-__global__ void jacobi_kernel(const double* C, int n, int max_sweeps, double tol, double* eval, float* evec,
-                              int32_t* dev_status) {
-  extern __shared__ double sd[];
+constexpr double kRankTol = 1e-10;   // pivoted Cholesky: relative diagonal cut
+constexpr double kJacobiTol = 1e-6;  // one-sided Jacobi: relative column coupling
+
+// Eigen-decomposition of the l x l core Gram C = Z^T Z (PSD), eigenvalues
+// descending; evec[i * n + j] = component i of eigenvector j.
+//   1. pivoted Cholesky (float64): P C P^T = L L^T (rank-revealing cut);
+//   2. one-sided Jacobi on the columns of L (float32, one warp per column
+//      pair, round-robin order): L J = U diag(sigma), so the normalised
+//      columns are the eigenvectors of P C P^T and sigma^2 its eigenvalues
+//      (this is the one-sided Jacobi SVD of the core, preconditioned by the
+//      pivoted factorization, which needs few sweeps);
+//   3. sort and undo the pivoting.
+__global__ void __launch_bounds__(1024) core_eig_kernel(const double* C, int n, int max_sweeps, double* eval,
+                                                        float* evec, int32_t* dev_status) {
+  extern __shared__ double smd[];
   const int ld = n + 1;
-  double* A = sd;              // n x ld
-  double* V = A + n * ld;      // n x ld
-  double* cs = V + n * ld;     // n/2 cosines
-  double* sn = cs + n / 2;     // n/2 sines
-  double* red = sn + n / 2;    // blockDim reduction scratch
-  __shared__ int pairs_p[64], pairs_q[64];
-  __shared__ int stop;
-  const int t = threadIdx.x, nt = blockDim.x;
-  const int half = n / 2;
-  for (int e = t; e < n * n; e += nt) {
-    const int i = e / n, j = e - i * n;
-    A[i * ld + j] = C[e];
-    V[i * ld + j] = i == j ? 1.0 : 0.0;
-  }
-  if (t == 0) stop = 0;
+  double* G = smd;                                       // n x ld
+  float* X = reinterpret_cast<float*>(G + n * ld);       // column j at X[j * ld + r]
+  int* perm = reinterpret_cast<int*>(X + n * ld);        // n
+  float* norms = reinterpret_cast<float*>(perm + n);     // n
+  __shared__ int piv_sh, rotated_sh;
+  __shared__ double maxd_sh;
+  const int t = threadIdx.x, nt = blockDim.x, warp = t >> 5, lane = t & 31, nwarps = nt >> 5;
+  for (int e = t; e < n * n; e += nt) G[(e / n) * ld + e % n] = C[e];
+  for (int i = t; i < n; i += nt) perm[i] = i;
   __syncthreads();
-  // total squared norm (for the relative stopping rule)
-  double tot = 0.0;
-  for (int e = t; e < n * n; e += nt) {
-    const double v = A[(e / n) * ld + e % n];
-    tot += v * v;
+  if (warp == 0) {
+    double m = 0.0;
+    for (int i = lane; i < n; i += 32) m = fmax(m, G[i * ld + i]);
+    for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
+    if (lane == 0) maxd_sh = m;
   }
-  red[t] = tot;
   __syncthreads();
-  for (int w = nt / 2; w > 0; w >>= 1) {
-    if (t < w) red[t] += red[t + w];
+  const double cut = kRankTol * maxd_sh;
+  int rank = n;
+  for (int j = 0; j < n; ++j) {
+    if (warp == 0) {
+      double best = -1.0;
+      int bi = j;
+      for (int i = j + lane; i < n; i += 32) {
+        const double v = G[i * ld + i];
+        if (v > best) {
+          best = v;
+          bi = i;
+        }
+      }
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ob = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+        const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
+        if (ob > best || (ob == best && oi < bi)) {
+          best = ob;
+          bi = oi;
+        }
+      }
+      if (lane == 0) piv_sh = bi;
+    }
+    __syncthreads();
+    const int p = piv_sh;
+    if (p != j) {
+      for (int c = t; c < n; c += nt) {
+        const double a = G[j * ld + c];
+        G[j * ld + c] = G[p * ld + c];
+        G[p * ld + c] = a;
+      }
+      __syncthreads();
+      for (int r = t; r < n; r += nt) {
+        const double a = G[r * ld + j];
+        G[r * ld + j] = G[r * ld + p];
+        G[r * ld + p] = a;
+      }
+      if (t == 0) {
+        const int a = perm[j];
+        perm[j] = perm[p];
+        perm[p] = a;
+      }
+      __syncthreads();
+    }
+    const double d = G[j * ld + j];
+    if (!(d > cut)) {
+      rank = j;
+      break;
+    }
+    const double inv = 1.0 / sqrt(d);
+    const double invd2 = inv * inv;
+    // the whole (symmetric) Schur complement is kept current, so that the
+    // next pivot swap can exchange complete rows and columns
+    const int w = n - j - 1;
+    for (int e = t; e < w * w; e += nt) {
+      const int i = j + 1 + e / w, c = j + 1 + e % w;
+      G[i * ld + c] -= G[i * ld + j] * G[c * ld + j] * invd2;
+    }
+    __syncthreads();
+    for (int i = j + 1 + t; i < n; i += nt) G[i * ld + j] *= inv;
+    if (t == 0) G[j * ld + j] = d * inv;
     __syncthreads();
   }
-  const double total = red[0];
+  for (int e = t; e < n * n; e += nt) {
+    const int j = e / n, r = e - j * n;
+    X[j * ld + r] = (j < rank && r >= j) ? static_cast<float>(G[r * ld + j]) : 0.f;
+  }
   __syncthreads();
   int sweep = 0;
   for (; sweep < max_sweeps; ++sweep) {
-    // off-diagonal norm
-    double off = 0.0;
-    for (int e = t; e < n * n; e += nt) {
-      const int i = e / n, j = e - i * n;
-      if (i != j) off += A[i * ld + j] * A[i * ld + j];
-    }
-    red[t] = off;
+    if (t == 0) rotated_sh = 0;
     __syncthreads();
-    for (int w = nt / 2; w > 0; w >>= 1) {
-      if (t < w) red[t] += red[t + w];
-      __syncthreads();
-    }
-    if (t == 0) stop = !(red[0] > tol * tol * total);
-    __syncthreads();
-    if (stop) break;
     for (int step = 0; step < n - 1; ++step) {
-      if (t < half) {
-        int p = rr_index(t, step, n), q = rr_index(n - 1 - t, step, n);
+      for (int pair = warp; pair < n / 2; pair += nwarps) {
+        int p = rr_index(pair, step, n), q = rr_index(n - 1 - pair, step, n);
         if (p > q) {
           const int x = p;
           p = q;
           q = x;
         }
-        pairs_p[t] = p;
-        pairs_q[t] = q;
-        const double apq = A[p * ld + q];
-        double c = 1.0, s = 0.0;
-        if (apq != 0.0) {
-          const double theta = (A[q * ld + q] - A[p * ld + p]) / (2.0 * apq);
-          const double tt = (theta >= 0.0 ? 1.0 : -1.0) / (fabs(theta) + sqrt(1.0 + theta * theta));
-          c = 1.0 / sqrt(1.0 + tt * tt);
-          s = tt * c;
+        float a[4], b[4];
+        double al = 0.0, be = 0.0, ga = 0.0;  // float64 sums: the stopping test sees no fp32 noise
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const int r = lane + 32 * k;
+          a[k] = r < n ? X[p * ld + r] : 0.f;
+          b[k] = r < n ? X[q * ld + r] : 0.f;
+          al = fma(static_cast<double>(a[k]), a[k], al);
+          be = fma(static_cast<double>(b[k]), b[k], be);
+          ga = fma(static_cast<double>(a[k]), b[k], ga);
         }
-        cs[t] = c;
-        sn[t] = s;
-      }
-      __syncthreads();
-      // columns p, q of A and V
-      for (int e = t; e < half * n; e += nt) {
-        const int k = e / n, i = e - k * n;
-        const int p = pairs_p[k], q = pairs_q[k];
-        const double c = cs[k], s = sn[k];
-        const double aip = A[i * ld + p], aiq = A[i * ld + q];
-        A[i * ld + p] = c * aip - s * aiq;
-        A[i * ld + q] = s * aip + c * aiq;
-        const double vip = V[i * ld + p], viq = V[i * ld + q];
-        V[i * ld + p] = c * vip - s * viq;
-        V[i * ld + q] = s * vip + c * viq;
-      }
-      __syncthreads();
-      // rows p, q of A
-      for (int e = t; e < half * n; e += nt) {
-        const int k = e / n, j = e - k * n;
-        const int p = pairs_p[k], q = pairs_q[k];
-        const double c = cs[k], s = sn[k];
-        const double apj = A[p * ld + j], aqj = A[q * ld + j];
-        A[p * ld + j] = c * apj - s * aqj;
-        A[q * ld + j] = s * apj + c * aqj;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+          al += __shfl_xor_sync(0xFFFFFFFFu, al, o);
+          be += __shfl_xor_sync(0xFFFFFFFFu, be, o);
+          ga += __shfl_xor_sync(0xFFFFFFFFu, ga, o);
+        }
+        if (ga != 0.0 && fabs(ga) > kJacobiTol * sqrt(al * be)) {
+          const double zeta = (be - al) / (2.0 * ga);
+          const double td = (zeta >= 0.0 ? 1.0 : -1.0) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
+          const float tt = static_cast<float>(td);
+          const float c = rsqrtf(1.f + tt * tt);
+          const float s = c * tt;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int r = lane + 32 * k;
+            if (r < n) {
+              X[p * ld + r] = c * a[k] - s * b[k];
+              X[q * ld + r] = s * a[k] + c * b[k];
+            }
+          }
+          if (lane == 0) rotated_sh = 1;
+        }
       }
       __syncthreads();
     }
+    if (!rotated_sh) break;
   }
   if (t == 0 && sweep >= max_sweeps) report(dev_status, METIS_DEV_NUMERIC);
-  // sort descending (ties: lower index first)
   for (int j = t; j < n; j += nt) {
-    const double lj = A[j * ld + j];
-    int rank = 0;
+    double s2 = 0.0;
+    for (int r = 0; r < n; ++r) s2 += static_cast<double>(X[j * ld + r]) * X[j * ld + r];
+    norms[j] = static_cast<float>(sqrt(s2));
+  }
+  __syncthreads();
+  for (int j = t; j < n; j += nt) {
+    const float sj = norms[j];
+    int rk = 0;
     for (int i = 0; i < n; ++i) {
-      const double li = A[i * ld + i];
-      rank += (li > lj) || (li == lj && i < j);
+      const float si = norms[i];
+      rk += (si > sj) || (si == sj && i < j);
     }
-    eval[rank] = lj;
-    for (int i = 0; i < n; ++i) evec[i * n + rank] = static_cast<float>(V[i * ld + j]);
+    eval[rk] = static_cast<double>(sj) * sj;
+    const float inv = sj > 0.f ? 1.f / sj : 0.f;
+    for (int r = 0; r < n; ++r) evec[perm[r] * n + rk] = X[j * ld + r] * inv;
   }
 }
 
@@ -354,6 +462,8 @@ int blocks(int64_t n, int sms) {
 
 int64_t gram_blocks(int64_t rows) { return (rows + kRowsPerBlock - 1) / kRowsPerBlock; }
 
+int64_t apply_blocks(int64_t rows) { return (rows + kApplyRows - 1) / kApplyRows; }
+
 void launch_gram(const float* partial, int splits, int64_t rows, int lp, float* Y, double* gpart, double* G,
                  cudaStream_t s) {
   const int nb = static_cast<int>(gram_blocks(rows));
@@ -363,28 +473,28 @@ void launch_gram(const float* partial, int splits, int64_t rows, int lp, float* 
 
 void launch_gram_reduce(const double* gpart, int nblocks, int lp, double* G, cudaStream_t s) {
   const int n2 = lp * lp;
-  gram_reduce_kernel<<<(n2 + 255) / 256, 256, 0, s>>>(gpart, nblocks, n2, G);
+  gram_reduce_kernel<<<(n2 + 7) / 8, 256, 0, s>>>(gpart, nblocks, n2, G);
 }
 
 void launch_cholesky_inv(const double* G, int lp, float* Rinv, cudaStream_t s) {
-  const size_t smem = (2 * static_cast<size_t>(lp) * (lp + 1) + 2 * lp) * sizeof(double);
+  const size_t smem = (2 * static_cast<size_t>(lp) * (lp + 1) + 3 * lp) * sizeof(double);
   if (!ensure_smem(reinterpret_cast<const void*>(cholesky_inv_kernel), smem)) return;
-  cholesky_inv_kernel<<<1, 512, smem, s>>>(G, lp, Rinv);
+  cholesky_inv_kernel<<<1, 1024, smem, s>>>(G, lp, Rinv);
 }
 
 void launch_apply(const ApplyArgs& a, cudaStream_t s) {
-  const size_t smem = (static_cast<size_t>(a.kin) * a.kout + kRowsPerBlock * (a.kin + 1) +
-                       kRowsPerBlock * (a.kout + 1)) * sizeof(float);
+  const size_t smem = (static_cast<size_t>(a.kin) * a.kout + kApplyRows * (a.kin + 1) +
+                       kApplyRows * (a.kout + 1)) * sizeof(float);
   if (!ensure_smem(reinterpret_cast<const void*>(apply_kernel), smem)) return;
-  apply_kernel<<<static_cast<unsigned>(gram_blocks(a.rows)), 256, smem, s>>>(a);
+  apply_kernel<<<static_cast<unsigned>(apply_blocks(a.rows)), 256, smem, s>>>(a);
 }
 
 void launch_jacobi(const double* C, int n, int max_sweeps, double* eval, float* evec, int32_t* dev_status,
                    cudaStream_t s) {
-  const int threads = 512;
-  const size_t smem = (2 * static_cast<size_t>(n) * (n + 1) + n + threads) * sizeof(double);
-  if (!ensure_smem(reinterpret_cast<const void*>(jacobi_kernel), smem)) return;
-  jacobi_kernel<<<1, threads, smem, s>>>(C, n, max_sweeps, 1e-13, eval, evec, dev_status);
+  const size_t smem = static_cast<size_t>(n) * (n + 1) * sizeof(double) + static_cast<size_t>(n) * (n + 1) * sizeof(float) +
+                      2 * static_cast<size_t>(n) * sizeof(int);
+  if (!ensure_smem(reinterpret_cast<const void*>(core_eig_kernel), smem)) return;
+  core_eig_kernel<<<1, 1024, smem, s>>>(C, n, max_sweeps, eval, evec, dev_status);
 }
 
 void launch_factor_mats(const double* eval, const float* evec, int lp, int k, float* Mu, float* Mv, float* S,

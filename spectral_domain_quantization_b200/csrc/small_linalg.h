@@ -24,6 +24,8 @@ struct ApplyArgs {
 };
 
 int64_t gram_blocks(int64_t rows);
+// row blocks of launch_apply (its Gram partials come one per block)
+int64_t apply_blocks(int64_t rows);
 // Y (optional) = sum of split partials; G = Y^T Y (float64, lp x lp).
 // gpart: gram_blocks(rows) * lp * lp doubles of scratch.
 void launch_gram(const float* partial, int splits, int64_t rows, int lp, float* Y, double* gpart, double* G,
