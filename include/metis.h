@@ -150,6 +150,38 @@ metis_status metis_quantize_fp4(const void* X, int32_t dtype, int64_t rows, int6
                                 size_t* workspace_bytes, void* stream);
 
 /*
+ * metis_quantize_fp4_noalloc -- metis_quantize_fp4 for callers that cannot
+ * provide scratch memory.  (No counterpart in the source pages: this is a
+ * library convenience, not part of the method.)
+ *
+ * Who needs it: code that may not allocate device memory where it quantizes
+ * (a runtime that owns every device byte through its own arena, a plugin whose
+ * host framework forbids allocation while it runs, a loop that must not block
+ * on the allocator) or a program that simply has no spare device buffer.
+ *
+ * It takes the same arguments as metis_quantize_fp4 minus the workspace and
+ * produces identical bytes.  Its scratch (the NVFP4 tensor-maximum word and,
+ * when out->inner_sum is set, outer * ceil(inner / 64) partial sums) lives in
+ * one fixed array of metis_noalloc_scratch_bytes() (2 MiB) compiled into the
+ * library; every GPU that loads the library keeps that array until the
+ * process exits.  Larger requests return METIS_ERR_WORKSPACE (see
+ * metis_last_error()); use metis_quantize_fp4 for them.
+ *   - The first call on a device looks up the array's device address (this may
+ *     load the library's device code); make that first call before any CUDA
+ *     stream capture.
+ *   - All calls share the one array: calls whose GPU work overlaps (different
+ *     streams, concurrent host threads) race and must be ordered by the caller.
+ *     The call zeroes what must start at zero itself.
+ * The function never calls cudaMalloc, cudaFree or any allocating routine.
+ */
+metis_status metis_quantize_fp4_noalloc(const void* X, int32_t dtype, int64_t rows, int64_t cols,
+                                        int64_t ld, int32_t block_axis, const float* sub_col,
+                                        metis_fp4_tensor* out, void* stream);
+
+/* Host-only: size in bytes of the fixed scratch array of the _noalloc call. */
+size_t metis_noalloc_scratch_bytes(void);
+
+/*
  * Parameters of the randomized split (host struct).
  *   k, p          rank kept and oversampling; l = k + p <= 128, l <= min(m, n)
  *                 (or <= sample_rows), l a multiple of 16 is not required.

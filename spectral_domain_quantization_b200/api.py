@@ -70,6 +70,8 @@ _SIGS = {
     "metis_device_supported": (_I32, []),
     "metis_last_error": (ctypes.c_char_p, []),
     "metis_quantize_fp4": (_I32, [_VP, _I32, _I64, _I64, _I64, _I32, _VP, _FP, _VP, _SZP, _VP]),
+    "metis_quantize_fp4_noalloc": (_I32, [_VP, _I32, _I64, _I64, _I64, _I32, _VP, _FP, _VP]),
+    "metis_noalloc_scratch_bytes": (ctypes.c_size_t, []),
     "metis_split": (_I32, [_VP, _I32, _I64, _I64, _I64, ctypes.POINTER(SplitParams), _VP, _VP, _VP,
                            _FP, _FP, _FP, _FP, _VP, _VP, _VP, _SZP, _VP, _VP]),
     "metis_linear_fwd": (_I32, [_OP, _OP, _I64, _I64, _I64, _VP, _I32, _I64, _VP, _SZP, _VP, _VP]),
@@ -205,6 +207,22 @@ def quantize_fp4(X, fmt, axis=1, sub_col=None, linear=False, inner_sum=False, ou
         L.metis_quantize_fp4,
         (_ptr(X), _dtype_code(X), rows, cols, X.stride(0), axis, _ptr(sub_col), ctypes.byref(s)),
         (_stream(),), X.device, "metis_quantize_fp4")
+    return out
+
+
+def quantize_fp4_noalloc(X, fmt, axis=1, sub_col=None, linear=False, inner_sum=False, out=None):
+    """metis_quantize_fp4_noalloc: the same quantization with the library's
+    fixed scratch instead of a workspace (for callers that cannot allocate)."""
+    if X.dim() != 2 or X.stride(1) != 1:
+        raise ValueError("X must be a row-major 2-D tensor")
+    rows, cols = X.shape
+    outer, inner = (rows, cols) if axis == 1 else (cols, rows)
+    if out is None:
+        out = QTensor(fmt, outer, inner, X.device, linear=linear, inner_sum=inner_sum)
+    s = out.struct()
+    _check(lib().metis_quantize_fp4_noalloc(_ptr(X), _dtype_code(X), rows, cols, X.stride(0), axis,
+                                            _ptr(sub_col), ctypes.byref(s), _stream()),
+           "metis_quantize_fp4_noalloc")
     return out
 
 
