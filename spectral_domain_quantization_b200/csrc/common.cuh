@@ -262,6 +262,23 @@ MDEV uint32_t e2m1_code(float q) {
   return c | ((__float_as_uint(q) >> 28) & 8u);
 }
 
+// E2M1 codes of 8 values packed into 32 bits (element i in bits 4i..4i+3),
+// by the hardware conversion: round to nearest even, saturating at 6, sign
+// kept on zero -- the same rule as e2m1_code.  The instruction converts a
+// pair with its first operand in the upper nibble.
+MDEV uint32_t e2m1_pack8(const float* q) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 b0, b1, b2, b3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b0, %2, %1;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b1, %4, %3;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b2, %6, %5;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 b3, %8, %7;\n\t"
+      "mov.b32 %0, {b0, b1, b2, b3};\n\t}"
+      : "=r"(r)
+      : "f"(q[0]), "f"(q[1]), "f"(q[2]), "f"(q[3]), "f"(q[4]), "f"(q[5]), "f"(q[6]), "f"(q[7]));
+  return r;
+}
+
 // Value of an E2M1 code.  Twice the magnitudes {0,1,2,3,4,6,8,12} are packed
 // as nibbles of one constant, so the lookup stays in registers.
 __host__ __device__ inline float e2m1_value(uint32_t code) {

@@ -12,9 +12,18 @@ MDEV float nv_tensor_scale(float alpha) {
   return alpha == 0.f ? 1.f : __fdiv_rn(alpha, 2688.f);
 }
 
+// Sum of the 8 E2M1 values packed in w, as a multiple of 0.5 (exact).
+MDEV float e2m1_sum8(uint32_t w) {
+  float s = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) s += e2m1_value((w >> (4 * i)) & 15u);
+  return s;
+}
+
 // NVFP4 block of 16.  Returns the E4M3 scale code; writes 16 nibbles to
-// `packed` (element i in bits 4i..4i+3) and the sum of the dequantized
-// values to `dsum`.
+// `packed` (element i in bits 4i..4i+3) and, when SUM, the sum of the
+// dequantized values to `dsum`.
+template <bool SUM = false>
 MDEV uint32_t quant_block_nv(const float* v, float s_t, uint64_t& packed, float& dsum) {
   float a = 0.f;
 #pragma unroll
@@ -26,19 +35,21 @@ MDEV uint32_t quant_block_nv(const float* v, float s_t, uint64_t& packed, float&
   dsum = 0.f;
   if (d == 0.f) return dc;
   const float enc = __fdiv_rn(1.f, __fmul_rn(d, s_t));
-  float csum = 0.f;  // exact: at most 16 values that are multiples of 0.5
+  float q[16];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) {
-    const uint32_t c = e2m1_code(__fmul_rn(v[i], enc));
-    packed |= static_cast<uint64_t>(c) << (4 * i);
-    csum += e2m1_value(c);
+  for (int i = 0; i < 16; ++i) q[i] = __fmul_rn(v[i], enc);
+  const uint32_t w0 = e2m1_pack8(q), w1 = e2m1_pack8(q + 8);
+  packed = static_cast<uint64_t>(w0) | (static_cast<uint64_t>(w1) << 32);
+  if (SUM) {
+    const float csum = e2m1_sum8(w0) + e2m1_sum8(w1);  // exact: 16 multiples of 0.5
+    dsum = __fmul_rn(csum * d, s_t);                     // csum * d is exact in float32
   }
-  dsum = __fmul_rn(csum * d, s_t);  // csum * d is exact in float32
   return dc;
 }
 
 // MXFP4 block of 32.  Returns the E8M0 scale code; writes 32 nibbles to
-// packed[0..1] and the sum of dequantized values to `dsum`.
+// packed[0..1] and, when SUM, the sum of dequantized values to `dsum`.
+template <bool SUM = false>
 MDEV uint32_t quant_block_mx(const float* v, uint64_t* packed, float& dsum) {
   float a = 0.f;
 #pragma unroll
@@ -49,14 +60,18 @@ MDEV uint32_t quant_block_mx(const float* v, uint64_t* packed, float& dsum) {
   int se = floor_log2(a) - 2;
   se = se < -127 ? -127 : (se > 127 ? 127 : se);
   const float inv = pow2f(-se);  // -se in [-125, 127]: a normal float
-  float csum = 0.f;
+  float q[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) {
-    const uint32_t c = e2m1_code(__fmul_rn(v[i], inv));
-    packed[i >> 4] |= static_cast<uint64_t>(c) << (4 * (i & 15));
-    csum += e2m1_value(c);
+  for (int i = 0; i < 32; ++i) q[i] = __fmul_rn(v[i], inv);
+  uint32_t w[4];
+#pragma unroll
+  for (int j = 0; j < 4; ++j) w[j] = e2m1_pack8(q + 8 * j);
+  packed[0] = static_cast<uint64_t>(w[0]) | (static_cast<uint64_t>(w[1]) << 32);
+  packed[1] = static_cast<uint64_t>(w[2]) | (static_cast<uint64_t>(w[3]) << 32);
+  if (SUM) {
+    const float csum = (e2m1_sum8(w[0]) + e2m1_sum8(w[1])) + (e2m1_sum8(w[2]) + e2m1_sum8(w[3]));
+    dsum = ldexpf(csum, se);
   }
-  dsum = ldexpf(csum, se);
   return static_cast<uint32_t>(se + 127);
 }
 

@@ -7,13 +7,12 @@
 //
 // HBM-bound: every element is read once (twice for NVFP4, whose tensor maximum
 // needs a pre-pass) and written as half a byte plus 1/16 or 1/32 byte of
-// scale.  Work unit = one thread per 64 consecutive elements along the block
-// axis (4 NVFP4 blocks or 2 MXFP4 blocks), so each thread writes 32 bytes of
-// codes and a 32- or 16-bit word of the tensor-core scale layout.
+// scale.  Blocks along columns: one thread per 64 consecutive elements (4
+// NVFP4 blocks or 2 MXFP4 blocks), so each thread writes 32 bytes of codes
+// and a 32- or 16-bit word of the tensor-core scale layout.
 //  * blocks along columns (axis 1): a thread reads 64 contiguous elements.
-//  * blocks along rows (axis 0): a thread owns two adjacent columns and reads
-//    64 rows of them; a warp covers 64 columns, i.e. 128 contiguous bytes of
-//    each bf16 row.
+//  * blocks along rows (axis 0): a CTA stages a 64 x 64 tile in shared
+//    memory with coalesced row loads, then quantizes it column by column.
 #include "fp4_block.cuh"
 #include "kernels.h"
 
@@ -43,72 +42,51 @@ MDEV void ld8(const void* X, int dtype, int64_t idx, float* out) {
   }
 }
 
-// two adjacent elements (idx even-aligned)
-MDEV void ld2(const void* X, int dtype, int64_t idx, float& a, float& b) {
-  if (dtype == METIS_BF16) {
-    const uint32_t u = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const __nv_bfloat16*>(X) + idx);
-    a = __uint_as_float(u << 16);
-    b = __uint_as_float(u & 0xFFFF0000u);
-  } else {
-    const float2 f = *reinterpret_cast<const float2*>(reinterpret_cast<const float*>(X) + idx);
-    a = f.x;
-    b = f.y;
-  }
-}
-
 // Quantize `n` (32 or 64) values of one outer index starting at inner offset
-// g*64, write codes / scales / partial sum.
-template <int FMT>
+// g*64, write codes / scales / (SUM) the group's partial sum.
+template <int FMT, bool SUM>
 MDEV void emit_group(const float* v, int n, int64_t o, int64_t g, const QuantParams& p, float s_t) {
   uint8_t* codes = p.codes + o * (p.inner / 2) + g * (kGroup / 2);
   const int64_t c0 = g * (FMT == METIS_NVFP4 ? 4 : 2);
   float dsum_total = 0.f;
   uint32_t sc = 0;
+  uint64_t pk[4] = {0, 0, 0, 0};
+  int nb;
   if (FMT == METIS_NVFP4) {
-    uint64_t pk[4];
-    const int nb = n / 16;
+    nb = n / 16;
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
-      pk[b] = 0;
       if (b < nb) {
         float ds;
-        const uint32_t code = quant_block_nv(v + 16 * b, s_t, pk[b], ds);
+        const uint32_t code = quant_block_nv<SUM>(v + 16 * b, s_t, pk[b], ds);
         sc |= code << (8 * b);
-        dsum_total += ds;
+        if (SUM) dsum_total += ds;
         if (p.scales_linear) p.scales_linear[o * (p.inner / 16) + c0 + b] = static_cast<uint8_t>(code);
       }
     }
-    uint4* dst = reinterpret_cast<uint4*>(codes);
-    dst[0] = make_uint4(static_cast<uint32_t>(pk[0]), static_cast<uint32_t>(pk[0] >> 32),
-                        static_cast<uint32_t>(pk[1]), static_cast<uint32_t>(pk[1] >> 32));
-    if (nb > 2)
-      dst[1] = make_uint4(static_cast<uint32_t>(pk[2]), static_cast<uint32_t>(pk[2] >> 32),
-                          static_cast<uint32_t>(pk[3]), static_cast<uint32_t>(pk[3] >> 32));
     *reinterpret_cast<uint32_t*>(p.scales + tc_scale_offset(o, c0, p.scale_cols)) = sc;
+    nb /= 2;  // 32-element halves written below
   } else {
-    uint64_t pk[4];
-    const int nb = n / 32;
+    nb = n / 32;
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
-      pk[2 * b] = pk[2 * b + 1] = 0;
       if (b < nb) {
         float ds;
-        const uint32_t code = quant_block_mx(v + 32 * b, pk + 2 * b, ds);
+        const uint32_t code = quant_block_mx<SUM>(v + 32 * b, pk + 2 * b, ds);
         sc |= code << (8 * b);
-        dsum_total += ds;
+        if (SUM) dsum_total += ds;
         if (p.scales_linear) p.scales_linear[o * (p.inner / 32) + c0 + b] = static_cast<uint8_t>(code);
       }
     }
-    uint4* dst = reinterpret_cast<uint4*>(codes);
-    dst[0] = make_uint4(static_cast<uint32_t>(pk[0]), static_cast<uint32_t>(pk[0] >> 32),
-                        static_cast<uint32_t>(pk[1]), static_cast<uint32_t>(pk[1] >> 32));
-    if (nb > 1)
-      dst[1] = make_uint4(static_cast<uint32_t>(pk[2]), static_cast<uint32_t>(pk[2] >> 32),
-                          static_cast<uint32_t>(pk[3]), static_cast<uint32_t>(pk[3] >> 32));
-    *reinterpret_cast<uint16_t*>(p.scales + tc_scale_offset(o, c0, p.scale_cols)) =
-        static_cast<uint16_t>(sc);
+    *reinterpret_cast<uint16_t*>(p.scales + tc_scale_offset(o, c0, p.scale_cols)) = static_cast<uint16_t>(sc);
   }
-  if (p.partial_sums) p.partial_sums[o * p.ngroups + g] = dsum_total;
+  uint4* dst = reinterpret_cast<uint4*>(codes);
+  dst[0] = make_uint4(static_cast<uint32_t>(pk[0]), static_cast<uint32_t>(pk[0] >> 32), static_cast<uint32_t>(pk[1]),
+                      static_cast<uint32_t>(pk[1] >> 32));
+  if (nb > 1)
+    dst[1] = make_uint4(static_cast<uint32_t>(pk[2]), static_cast<uint32_t>(pk[2] >> 32),
+                        static_cast<uint32_t>(pk[3]), static_cast<uint32_t>(pk[3] >> 32));
+  if (SUM) p.partial_sums[o * p.ngroups + g] = dsum_total;
 }
 
 MDEV float tensor_scale_of(const QuantParams& p) {
@@ -118,7 +96,7 @@ MDEV float tensor_scale_of(const QuantParams& p) {
 }
 
 // blocks along columns: thread -> (row o, group g)
-template <int FMT>
+template <int FMT, bool SUM>
 __global__ void __launch_bounds__(256) quantize_rows_kernel(QuantParams p) {
   const float s_t = tensor_scale_of(p);
   if (FMT == METIS_NVFP4 && blockIdx.x == 0 && threadIdx.x == 0 && p.tensor_scale) *p.tensor_scale = s_t;
@@ -145,54 +123,83 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QuantParams p) {
       for (int j = 0; j < kGroup; ++j)
         if (j < n) p.r_tap[o * p.tap_ld + i0 + j] = v[j];
     }
-    emit_group<FMT>(v, n, o, g, p, s_t);
+    emit_group<FMT, SUM>(v, n, o, g, p, s_t);
   }
 }
 
-// blocks along rows: thread -> (column pair, group g of 64 rows)
-template <int FMT>
+// blocks along rows: one CTA per 64-row x 64-column tile of X.  The tile is
+// read with 16-byte row-segment loads into shared memory; then each thread
+// quantizes one block of one column (four threads, or two for MXFP4, cover
+// a column's 64 rows, so their codes form one contiguous 32-byte segment).
+constexpr int kColTile = 64;
+
+template <int FMT, bool SUM>
 __global__ void __launch_bounds__(256) quantize_cols_kernel(QuantParams p) {
+  constexpr int kBlk = FMT == METIS_NVFP4 ? 16 : 32;
+  constexpr int kPerCol = kColTile / kBlk;  // threads per column
+  __shared__ float tile[kColTile][kColTile + 1];
+  __shared__ float bsum[kColTile][kPerCol];
   const float s_t = tensor_scale_of(p);
-  if (FMT == METIS_NVFP4 && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 &&
-      threadIdx.y == 0 && p.tensor_scale)
+  if (FMT == METIS_NVFP4 && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && p.tensor_scale)
     *p.tensor_scale = s_t;
   // p.outer = columns of X, p.inner = rows of X
-  const int64_t c = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) * 2;
-  const int64_t g = static_cast<int64_t>(blockIdx.y) * blockDim.y + threadIdx.y;
-  if (c >= p.outer || g >= p.ngroups) return;
-  const int64_t r0 = g * kGroup;
-  const int n = static_cast<int>(imin64(kGroup, p.inner - r0));
-  const bool two = c + 1 < p.outer;
-  float va[kGroup], vb[kGroup];
-  const float sa = p.sub ? p.sub[c] : 0.f;
-  const float sb = (p.sub && two) ? p.sub[c + 1] : 0.f;
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kColTile;
+  const int64_t g = blockIdx.y;
+  const int64_t r0 = g * kColTile;
+  const int nr = static_cast<int>(imin64(kColTile, p.inner - r0));
+  const int nc = static_cast<int>(imin64(kColTile, p.outer - c0));
+  for (int e = threadIdx.x; e < kColTile * (kColTile / 8); e += blockDim.x) {
+    const int r = e >> 3, q = (e & 7) * 8;
+    float v[8];
+    if (r < nr && q + 8 <= nc) {
+      ld8(p.X, p.dtype, (r0 + r) * p.ld + c0 + q, v);
+    } else {
 #pragma unroll
-  for (int j = 0; j < kGroup; ++j) {
-    if (j < n) {
-      const int64_t idx = (r0 + j) * p.ld + c;
-      if (two) {
-        ld2(p.X, p.dtype, idx, va[j], vb[j]);
+      for (int j = 0; j < 8; ++j) v[j] = (r < nr && q + j < nc) ? ld1(p.X, p.dtype, (r0 + r) * p.ld + c0 + q + j) : 0.f;
+    }
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+      if (p.sub && q + j < nc) v[j] = __fsub_rn(v[j], p.sub[c0 + q + j]);
+      tile[r][q + j] = v[j];
+      if (p.r_tap && r < nr && q + j < nc) p.r_tap[(r0 + r) * p.tap_ld + c0 + q + j] = v[j];
+    }
+  }
+  __syncthreads();
+  const int nb = nr / kBlk;
+  if (threadIdx.x < kColTile * kPerCol) {
+    const int b = threadIdx.x % kPerCol, cc = threadIdx.x / kPerCol;
+    if (cc < nc && b < nb) {
+      const int64_t o = c0 + cc;
+      float v[kBlk];
+#pragma unroll
+      for (int i = 0; i < kBlk; ++i) v[i] = tile[b * kBlk + i][cc];
+      float ds = 0.f;
+      uint8_t* dst = p.codes + o * (p.inner / 2) + (r0 + b * kBlk) / 2;
+      const int64_t sc_col = (r0 + b * kBlk) / kBlk;
+      uint32_t code;
+      if (FMT == METIS_NVFP4) {
+        uint64_t pk;
+        code = quant_block_nv<SUM>(v, s_t, pk, ds);
+        *reinterpret_cast<uint2*>(dst) = make_uint2(static_cast<uint32_t>(pk), static_cast<uint32_t>(pk >> 32));
       } else {
-        va[j] = ld1(p.X, p.dtype, idx);
-        vb[j] = 0.f;
+        uint64_t pk[2];
+        code = quant_block_mx<SUM>(v, pk, ds);
+        *reinterpret_cast<uint4*>(dst) = make_uint4(static_cast<uint32_t>(pk[0]), static_cast<uint32_t>(pk[0] >> 32),
+                                                    static_cast<uint32_t>(pk[1]), static_cast<uint32_t>(pk[1] >> 32));
       }
-      if (p.sub) {
-        va[j] = __fsub_rn(va[j], sa);
-        vb[j] = __fsub_rn(vb[j], sb);
-      }
+      p.scales[tc_scale_offset(o, sc_col, p.scale_cols)] = static_cast<uint8_t>(code);
+      if (p.scales_linear) p.scales_linear[o * (p.inner / kBlk) + sc_col] = static_cast<uint8_t>(code);
+      if (SUM) bsum[cc][b] = ds;
     }
   }
-  if (p.r_tap) {
-#pragma unroll
-    for (int j = 0; j < kGroup; ++j) {
-      if (j < n) {
-        p.r_tap[(r0 + j) * p.tap_ld + c] = va[j];
-        if (two) p.r_tap[(r0 + j) * p.tap_ld + c + 1] = vb[j];
-      }
+  if (SUM) {
+    __syncthreads();
+    if (threadIdx.x < nc) {
+      float s = 0.f;
+      for (int b = 0; b < nb; ++b) s += bsum[threadIdx.x][b];
+      p.partial_sums[(c0 + threadIdx.x) * p.ngroups + g] = s;
     }
   }
-  emit_group<FMT>(va, n, c, g, p, s_t);
-  if (two) emit_group<FMT>(vb, n, c + 1, g, p, s_t);
 }
 
 // max |x - sub| over the matrix into *out_bits (float bits, atomicMax).
@@ -253,23 +260,31 @@ void launch_amax(const void* X, int dtype, int64_t rows, int64_t cols, int64_t l
   amax_kernel<<<blocks, 256, 0, s>>>(X, dtype, rows, cols, ld, sub, out_bits);
 }
 
-void launch_quantize(const QuantParams& p, int axis, int num_sms, cudaStream_t s) {
+template <int FMT, bool SUM>
+void launch_quantize_t(const QuantParams& p, int axis, int num_sms, cudaStream_t s) {
   if (axis == 1) {
     const int64_t total = p.outer * p.ngroups;
     int blocks = static_cast<int>(imin64((total + 255) / 256, static_cast<int64_t>(num_sms) * 16));
     if (blocks < 1) blocks = 1;
-    if (p.fmt == METIS_NVFP4)
-      quantize_rows_kernel<METIS_NVFP4><<<blocks, 256, 0, s>>>(p);
-    else
-      quantize_rows_kernel<METIS_MXFP4><<<blocks, 256, 0, s>>>(p);
+    quantize_rows_kernel<FMT, SUM><<<blocks, 256, 0, s>>>(p);
   } else {
-    const dim3 block(64, 4);
-    const dim3 grid(static_cast<unsigned>((p.outer + 127) / 128),
-                    static_cast<unsigned>((p.ngroups + 3) / 4));
-    if (p.fmt == METIS_NVFP4)
-      quantize_cols_kernel<METIS_NVFP4><<<grid, block, 0, s>>>(p);
+    const dim3 grid(static_cast<unsigned>((p.outer + kColTile - 1) / kColTile), static_cast<unsigned>(p.ngroups));
+    quantize_cols_kernel<FMT, SUM><<<grid, 256, 0, s>>>(p);
+  }
+}
+
+void launch_quantize(const QuantParams& p, int axis, int num_sms, cudaStream_t s) {
+  const bool sum = p.partial_sums != nullptr;
+  if (p.fmt == METIS_NVFP4) {
+    if (sum)
+      launch_quantize_t<METIS_NVFP4, true>(p, axis, num_sms, s);
     else
-      quantize_cols_kernel<METIS_MXFP4><<<grid, block, 0, s>>>(p);
+      launch_quantize_t<METIS_NVFP4, false>(p, axis, num_sms, s);
+  } else {
+    if (sum)
+      launch_quantize_t<METIS_MXFP4, true>(p, axis, num_sms, s);
+    else
+      launch_quantize_t<METIS_MXFP4, false>(p, axis, num_sms, s);
   }
   if (p.partial_sums && p.inner_sum) {
     inner_sum_kernel<<<static_cast<unsigned>((p.outer + 255) / 256), 256, 0, s>>>(

@@ -31,16 +31,43 @@ constexpr int kRowsPerBlock = 32;
 constexpr double kDropTol = 1e-12;
 
 // Gram partial of a row block held in shared memory (rows x cols floats with
-// row stride ld): out[i][j] for all i, j (full symmetric matrix).
+// row stride ld, cols a multiple of 4): out[i][j] for all i, j (symmetric).
+// Each thread accumulates a 4 x 4 tile (16 independent float64 chains).
 MDEV void gram_block(const float* ys, int rows, int cols, int ld, double* out) {
-  const int n = cols * cols;
-  for (int e = threadIdx.x; e < n; e += blockDim.x) {
-    const int i = e / cols, j = e - i * cols;
-    if (j < i) continue;
-    double acc = 0.0;
-    for (int r = 0; r < rows; ++r) acc += static_cast<double>(ys[r * ld + i]) * static_cast<double>(ys[r * ld + j]);
-    out[i * cols + j] = acc;
-    out[j * cols + i] = acc;
+  const int nb = cols / 4;
+  const int npairs = nb * (nb + 1) / 2;
+  for (int pidx = threadIdx.x; pidx < npairs; pidx += blockDim.x) {
+    int bi = 0, rem = pidx;
+    while (rem >= nb - bi) {
+      rem -= nb - bi;
+      ++bi;
+    }
+    const int bj = bi + rem;
+    double acc[4][4];
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) acc[x][y] = 0.0;
+    for (int r = 0; r < rows; ++r) {
+      const float* row = ys + r * ld;
+      double a[4], b[4];
+#pragma unroll
+      for (int x = 0; x < 4; ++x) {
+        a[x] = row[4 * bi + x];
+        b[x] = row[4 * bj + x];
+      }
+#pragma unroll
+      for (int x = 0; x < 4; ++x)
+#pragma unroll
+        for (int y = 0; y < 4; ++y) acc[x][y] = fma(a[x], b[y], acc[x][y]);
+    }
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) {
+        out[(4 * bi + x) * cols + 4 * bj + y] = acc[x][y];
+        out[(4 * bj + y) * cols + 4 * bi + x] = acc[x][y];
+      }
   }
 }
 
@@ -75,11 +102,15 @@ __global__ void gram_reduce_kernel(const double* gpart, int nblocks, int n2, dou
   if (lane == 0) G[e] = s;
 }
 
+// Decode e -> (q, e - q*d) for e < 2^22 with a float reciprocal (exact).
+MDEV int fdiv_index(int e, float rcp) { return __float2int_rz((static_cast<float>(e) + 0.5f) * rcp); }
+
 // G = L L^T (with drops), then Rinv = L^-T (upper triangular, float32).
-// 1024 threads as 32 x 32.  One barrier per column: step j updates the
-// trailing matrix with the unscaled column j (times 1/d_j) and scales column
-// j-1; the thread that updates the next diagonal entry also computes the next
-// pivot's 1/sqrt, so the float64 square root overlaps the update.
+// Work is enumerated over flattened index ranges so every thread gets an equal
+// share of the shrinking triangle.  One barrier per column: step j updates the
+// trailing lower triangle with the unscaled column j (times 1/d_j) and scales
+// column j-1; the thread updating the next diagonal entry computes the next
+// pivot's reciprocal square root, overlapping its latency with the update.
 __global__ void __launch_bounds__(1024) cholesky_inv_kernel(const double* G, int lp, float* Rinv) {
   extern __shared__ double sm[];
   const int ld = lp + 1;
@@ -89,7 +120,6 @@ __global__ void __launch_bounds__(1024) cholesky_inv_kernel(const double* G, int
   double* invd = diag0 + lp;       // lp: 1/sqrt(pivot) (0 when dropped)
   double* sqd = invd + lp;         // lp: sqrt(pivot) (0 when dropped)
   const int t = threadIdx.x, nt = blockDim.x;
-  const int tx = t & 31, ty = t >> 5;
   for (int e = t; e < lp * lp; e += nt) {
     const int i = e / lp, j = e - i * lp;
     L[i * ld + j] = G[e];
@@ -105,19 +135,23 @@ __global__ void __launch_bounds__(1024) cholesky_inv_kernel(const double* G, int
   }
   __syncthreads();
   for (int j = 0; j < lp; ++j) {
-    const double inv = invd[j];
-    const double inv2 = inv * inv;
-    for (int i = j + 1 + ty; i < lp; i += 32) {
-      const double lij = L[i * ld + j] * inv2;
-      for (int c = j + 1 + tx; c <= i; c += 32) {
-        const double v = L[i * ld + c] - lij * L[c * ld + j];
-        L[i * ld + c] = v;
-        if (i == j + 1 && c == j + 1) {  // next pivot, ready for step j+1
-          const bool drop = !(diag0[c] > 0.0) || !(v > kDropTol * diag0[c]);
-          const double r = drop ? 0.0 : sqrt(v);
-          sqd[c] = r;
-          invd[c] = drop ? 0.0 : 1.0 / r;
-        }
+    const double inv2 = invd[j] * invd[j];
+    // trailing lower triangle {(i, c): j < c <= i < lp}, row by row:
+    // row i = j + 1 + a holds a + 1 entries; flatten with a triangular decode
+    const int w = lp - j - 1;
+    const int total = w * (w + 1) / 2;
+    for (int e = t; e < total; e += nt) {
+      int a = static_cast<int>((sqrtf(8.f * e + 1.f) - 1.f) * 0.5f);
+      if ((a + 1) * (a + 2) / 2 <= e) ++a;
+      if (a * (a + 1) / 2 > e) --a;
+      const int i = j + 1 + a, c = j + 1 + (e - a * (a + 1) / 2);
+      const double v = L[i * ld + c] - L[i * ld + j] * L[c * ld + j] * inv2;
+      L[i * ld + c] = v;
+      if (e == 0) {  // (j+1, j+1): next pivot
+        const bool drop = !(diag0[c] > 0.0) || !(v > kDropTol * diag0[c]);
+        const double r = drop ? 0.0 : sqrt(v);
+        sqd[c] = r;
+        invd[c] = drop ? 0.0 : 1.0 / r;
       }
     }
     if (j > 0) {  // deferred scaling of column j-1
@@ -128,13 +162,16 @@ __global__ void __launch_bounds__(1024) cholesky_inv_kernel(const double* G, int
     __syncthreads();
   }
   if (t == 0) L[(lp - 1) * ld + lp - 1] = sqd[lp - 1];
-  // X = L^-1 by rows: step k eliminates with the unscaled row k (times
-  // 1/L_kk) and scales row k-1
+  // X = L^-1: step k eliminates with the unscaled row k (times 1/L_kk) over
+  // the rectangle rows k+1.., columns 0..k, and scales row k-1
   for (int k = 0; k < lp; ++k) {
     const double inv = invd[k];
-    for (int i = k + 1 + ty; i < lp; i += 32) {
-      const double lik = L[i * ld + k] * inv;
-      for (int c = tx; c <= k; c += 32) X[i * ld + c] -= lik * X[k * ld + c];
+    const int cols = k + 1, total = (lp - k - 1) * cols;
+    const float rcp = 1.f / static_cast<float>(cols);
+    for (int e = t; e < total; e += nt) {
+      const int q = fdiv_index(e, rcp);
+      const int i = k + 1 + q, c = e - q * cols;
+      X[i * ld + c] -= L[i * ld + k] * inv * X[k * ld + c];
     }
     if (k > 0) {
       const double pinv = invd[k - 1];
@@ -150,10 +187,10 @@ __global__ void __launch_bounds__(1024) cholesky_inv_kernel(const double* G, int
   }
 }
 
-constexpr int kApplyRows = 64;
+constexpr int kApplyRows = 32;
 
-// out = in (rows x kin) * M (kin x kout).  64 rows per CTA, 256 threads, each
-// thread a 4-row x ceil(kout/16)-column register block.  Optional fp32 out,
+// out = in (rows x kin) * M (kin x kout).  32 rows per CTA, 256 threads, each
+// thread a 2-row x ceil(kout/16)-column register tile.  Optional fp32 out,
 // transposed bf16 hi/lo copy, Gram partial of the output block.
 __global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) {
   extern __shared__ float smf[];
@@ -170,31 +207,31 @@ __global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) {
   __syncthreads();
   const int tr = threadIdx.x & 15, tc = threadIdx.x >> 4;
   constexpr int kMaxCols = 7;  // kout <= 112
-  float acc[4][kMaxCols];
+  float acc[2][kMaxCols];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 2; ++i)
 #pragma unroll
     for (int u = 0; u < kMaxCols; ++u) acc[i][u] = 0.f;
+  const float* in0 = In + (2 * tr) * (a.kin + 1);
+  const float* in1 = in0 + (a.kin + 1);
+#pragma unroll 2
   for (int j = 0; j < a.kin; ++j) {
-    float x[4], m[kMaxCols];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) x[i] = In[(4 * tr + i) * (a.kin + 1) + j];
+    const float x0 = in0[j], x1 = in1[j];
+    const float* mrow = Ms + j * a.kout;
 #pragma unroll
     for (int u = 0; u < kMaxCols; ++u) {
       const int c = tc + 16 * u;
-      m[u] = c < a.kout ? Ms[j * a.kout + c] : 0.f;
+      const float m = c < a.kout ? mrow[c] : 0.f;
+      acc[0][u] = fmaf(x0, m, acc[0][u]);
+      acc[1][u] = fmaf(x1, m, acc[1][u]);
     }
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int u = 0; u < kMaxCols; ++u) acc[i][u] = fmaf(x[i], m[u], acc[i][u]);
   }
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 2; ++i)
 #pragma unroll
     for (int u = 0; u < kMaxCols; ++u) {
       const int c = tc + 16 * u;
-      if (c < a.kout) Out[(4 * tr + i) * (a.kout + 1) + c] = acc[i][u];
+      if (c < a.kout) Out[(2 * tr + i) * (a.kout + 1) + c] = acc[i][u];
     }
   __syncthreads();
   for (int e = threadIdx.x; e < kApplyRows * a.kout; e += blockDim.x) {
@@ -223,12 +260,14 @@ MDEV int rr_index(int slot, int step, int n) {
 }
 
 constexpr double kRankTol = 1e-10;   // pivoted Cholesky: relative diagonal cut
-constexpr double kJacobiTol = 1e-6;  // one-sided Jacobi: relative column coupling
+// one-sided Jacobi: rotate while |a.b| > tol |a||b|.  Float32 sums of <= 112
+// products carry ~5e-7 relative noise, so the rule sits well above it.
+constexpr float kJacobiTol = 4e-6f;
 
 // Eigen-decomposition of the l x l core Gram C = Z^T Z (PSD), eigenvalues
 // descending; evec[i * n + j] = component i of eigenvector j.
 //   1. pivoted Cholesky (float64): P C P^T = L L^T (rank-revealing cut);
-//   2. one-sided Jacobi on the columns of L (float32, one warp per column
+//   2. one-sided Jacobi on the columns of L (float32, eight lanes per column
 //      pair, round-robin order): L J = U diag(sigma), so the normalised
 //      columns are the eigenvectors of P C P^T and sigma^2 its eigenvalues
 //      (this is the one-sided Jacobi SVD of the core, preconditioned by the
@@ -309,8 +348,10 @@ __global__ void __launch_bounds__(1024) core_eig_kernel(const double* C, int n, 
     // the whole (symmetric) Schur complement is kept current, so that the
     // next pivot swap can exchange complete rows and columns
     const int w = n - j - 1;
+    const float rcpw = 1.f / static_cast<float>(w > 0 ? w : 1);
     for (int e = t; e < w * w; e += nt) {
-      const int i = j + 1 + e / w, c = j + 1 + e % w;
+      const int q = fdiv_index(e, rcpw);
+      const int i = j + 1 + q, c = j + 1 + (e - q * w);
       G[i * ld + c] -= G[i * ld + j] * G[c * ld + j] * invd2;
     }
     __syncthreads();
@@ -323,50 +364,53 @@ __global__ void __launch_bounds__(1024) core_eig_kernel(const double* C, int n, 
     X[j * ld + r] = (j < rank && r >= j) ? static_cast<float>(G[r * ld + j]) : 0.f;
   }
   __syncthreads();
+  // one-sided Jacobi: 8 lanes per column pair, 4 pairs per warp
+  const int grp = lane >> 3, l8 = lane & 7;
+  const int npairs = n / 2;
   int sweep = 0;
   for (; sweep < max_sweeps; ++sweep) {
     if (t == 0) rotated_sh = 0;
     __syncthreads();
     for (int step = 0; step < n - 1; ++step) {
-      for (int pair = warp; pair < n / 2; pair += nwarps) {
-        int p = rr_index(pair, step, n), q = rr_index(n - 1 - pair, step, n);
-        if (p > q) {
-          const int x = p;
-          p = q;
-          q = x;
+      for (int base = 4 * warp; base < npairs; base += 4 * nwarps) {
+        const int pair = base + grp;
+        const bool act = pair < npairs;
+        int p = 0, q = 1;
+        if (act) {
+          p = rr_index(pair, step, n);
+          q = rr_index(n - 1 - pair, step, n);
+          if (p > q) {
+            const int x = p;
+            p = q;
+            q = x;
+          }
         }
-        float a[4], b[4];
-        double al = 0.0, be = 0.0, ga = 0.0;  // float64 sums: the stopping test sees no fp32 noise
-#pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const int r = lane + 32 * k;
-          a[k] = r < n ? X[p * ld + r] : 0.f;
-          b[k] = r < n ? X[q * ld + r] : 0.f;
-          al = fma(static_cast<double>(a[k]), a[k], al);
-          be = fma(static_cast<double>(b[k]), b[k], be);
-          ga = fma(static_cast<double>(a[k]), b[k], ga);
+        float al = 0.f, be = 0.f, ga = 0.f;
+        if (act) {
+          for (int r = l8; r < n; r += 8) {
+            const float a = X[p * ld + r], b = X[q * ld + r];
+            al = fmaf(a, a, al);
+            be = fmaf(b, b, be);
+            ga = fmaf(a, b, ga);
+          }
         }
 #pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
+        for (int o = 4; o > 0; o >>= 1) {
           al += __shfl_xor_sync(0xFFFFFFFFu, al, o);
           be += __shfl_xor_sync(0xFFFFFFFFu, be, o);
           ga += __shfl_xor_sync(0xFFFFFFFFu, ga, o);
         }
-        if (ga != 0.0 && fabs(ga) > kJacobiTol * sqrt(al * be)) {
-          const double zeta = (be - al) / (2.0 * ga);
-          const double td = (zeta >= 0.0 ? 1.0 : -1.0) / (fabs(zeta) + sqrt(1.0 + zeta * zeta));
-          const float tt = static_cast<float>(td);
-          const float c = rsqrtf(1.f + tt * tt);
+        if (act && ga != 0.f && fabsf(ga) > kJacobiTol * sqrtf(al * be)) {
+          const float zeta = (be - al) / (2.f * ga);
+          const float tt = copysignf(1.f, zeta) / (fabsf(zeta) + sqrtf(fmaf(zeta, zeta, 1.f)));
+          const float c = rsqrtf(fmaf(tt, tt, 1.f));
           const float s = c * tt;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int r = lane + 32 * k;
-            if (r < n) {
-              X[p * ld + r] = c * a[k] - s * b[k];
-              X[q * ld + r] = s * a[k] + c * b[k];
-            }
+          for (int r = l8; r < n; r += 8) {
+            const float a = X[p * ld + r], b = X[q * ld + r];
+            X[p * ld + r] = c * a - s * b;
+            X[q * ld + r] = s * a + c * b;
           }
-          if (lane == 0) rotated_sh = 1;
+          if (l8 == 0) rotated_sh = 1;
         }
       }
       __syncthreads();
