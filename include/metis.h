@@ -183,7 +183,8 @@ size_t metis_noalloc_scratch_bytes(void);
 
 /*
  * Parameters of the randomized split (host struct).
- *   k, p          rank kept and oversampling; l = k + p <= 128, l <= min(m, n)
+ *   k, p          rank kept (a multiple of 4) and oversampling; l = k + p <= 112,
+ *                 l <= min(m, n)
  *                 (or <= sample_rows), l a multiple of 16 is not required.
  *   power_iters   q >= 0 subspace iterations.
  *   seed          Philox4x32-10 key for the sketch and the row sample.
@@ -192,7 +193,9 @@ size_t metis_noalloc_scratch_bytes(void);
  *   sample_rows   0, or the number of rows sampled to find the right singular
  *                 subspace (then power_iters applies to the sample).
  *   fmt           metis_fp4_fmt of every quantized output.
- *   max_jacobi_sweeps  cap on Jacobi sweeps of the core (e.g. 30).
+ *   max_core_iters  cap on the multisection rounds that find each eigenvalue
+ *                 of the core Gram (about 11 are needed; 64 is a safe
+ *                 value); reaching it sets METIS_DEV_NUMERIC in *dev_status.
  */
 typedef struct {
   int32_t k;
@@ -203,7 +206,7 @@ typedef struct {
   int32_t sparse_nnz;
   int64_t sample_rows;
   int32_t fmt;
-  int32_t max_jacobi_sweeps;
+  int32_t max_core_iters;
 } metis_split_params;
 
 /*

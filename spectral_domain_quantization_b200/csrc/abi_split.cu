@@ -62,6 +62,7 @@ struct SplitBuffers {
   __nv_bfloat16* qt = nullptr;       // [2 lp][max(ld_m, ld_n)]
   double* gpart = nullptr;
   double* G = nullptr;
+  double* eig_ws = nullptr;          // core eigensolver scratch
   float* Rinv = nullptr;
   double* eval = nullptr;
   float* evec = nullptr;
@@ -128,6 +129,7 @@ SplitBuffers carve(const SplitPlan& p, int64_t lda, Carver& ws) {
   b.qt = ws.take<__nv_bfloat16>(static_cast<size_t>(2 * wmax) * bigld);
   b.gpart = ws.take<double>(static_cast<size_t>(gram_blocks(big)) * wmax * wmax);
   b.G = ws.take<double>(static_cast<size_t>(wmax) * wmax);
+  b.eig_ws = reinterpret_cast<double*>(ws.take<uint8_t>(core_eig_workspace(wmax)));
   b.Rinv = ws.take<float>(static_cast<size_t>(p.lp) * p.lp);
   b.eval = ws.take<double>(p.lp);
   b.evec = ws.take<float>(static_cast<size_t>(p.lp) * p.lp);
@@ -238,7 +240,7 @@ metis_status cholqr(const SplitBuffers& b, int splits, int64_t rows, int lp, flo
 // Range finder + core on `src` (ms x n): returns Z = src^T Q in b.Zn, Q in
 // b.Qm, and the sorted eigen-decomposition of Z^T Z in b.eval / b.evec.
 metis_status range_and_core(const SplitPlan& p, const SplitBuffers& b, const Source& src, int power_iters,
-                            int max_sweeps, int32_t* dev_status, cudaStream_t s) {
+                            int max_iters, int32_t* dev_status, cudaStream_t s) {
   const int lp = p.lp;
   METIS_TRY(skinny(src, 0, b.omt, p.ld_n, 1, lp, p.split_m, b.part, dev_status, s));
   METIS_TRY(cholqr(b, p.split_m, src.rows, lp, b.Qm, p.ld_m, power_iters > 0 ? 1 : 2, s));
@@ -251,8 +253,8 @@ metis_status range_and_core(const SplitPlan& p, const SplitBuffers& b, const Sou
   METIS_TRY(skinny(src, 1, b.qt, p.ld_m, 2, lp, p.split_n, b.part, dev_status, s));
   launch_gram(b.part, p.split_n, p.n, lp, b.Zn, b.gpart, b.G, s);
   METIS_TRY(step_status("core gram"));
-  launch_jacobi(b.G, lp, max_sweeps, b.eval, b.evec, dev_status, s);
-  return step_status("core jacobi");
+  launch_core_eig(b.G, lp, max_iters, b.eval, b.evec, b.eig_ws, dev_status, s);
+  return step_status("core eigensolver");
 }
 
 metis_status validate_split(const void* A, int dtype, int64_t m, int64_t n, int64_t lda,
@@ -263,7 +265,7 @@ metis_status validate_split(const void* A, int dtype, int64_t m, int64_t n, int6
   METIS_TRY(validate_dense(A, dtype, m, n, lda));
   if (!valid_fmt(prm->fmt)) return METIS_ERR_ARG;
   if (prm->sketch != METIS_SKETCH_GAUSSIAN && prm->sketch != METIS_SKETCH_SPARSE_SIGN) return METIS_ERR_ARG;
-  if (prm->k < 1 || prm->p < 0 || prm->power_iters < 0 || prm->max_jacobi_sweeps < 1) return METIS_ERR_ARG;
+  if (prm->k < 1 || prm->p < 0 || prm->power_iters < 0 || prm->max_core_iters < 1) return METIS_ERR_ARG;
   const int l = prm->k + prm->p;
   if (l > 112) return METIS_ERR_SHAPE;
   if (prm->k % 4) return METIS_ERR_SHAPE;  // U, V rows of k floats start on 16-byte boundaries
@@ -356,7 +358,7 @@ extern "C" metis_status metis_split(const void* A, int32_t dtype, int64_t m, int
   METIS_TRY(step_status("sketch / sampling"));
 
   const int power_iters = prm->power_iters;
-  METIS_TRY(range_and_core(p, b, src, power_iters, prm->max_jacobi_sweeps, dev_status, s));
+  METIS_TRY(range_and_core(p, b, src, power_iters, prm->max_core_iters, dev_status, s));
   launch_factor_mats(b.eval, b.evec, p.lp, p.k, b.Mu, b.Mv, S, s);
   METIS_TRY(step_status("factor matrices"));
 
@@ -402,7 +404,7 @@ extern "C" metis_status metis_split(const void* A, int32_t dtype, int64_t m, int
     const int sp = skinny_splits(m, n, sms);
     METIS_TRY(skinny(full, 0, b.qt, p.ld_n, 2, p.kq, sp, b.part, dev_status, s));
     launch_gram(b.part, sp, m, p.kq, b.P, b.gpart, b.G, s);
-    launch_jacobi(b.G, p.kq, prm->max_jacobi_sweeps, b.eval2, b.evec2, dev_status, s);
+    launch_core_eig(b.G, p.kq, prm->max_core_iters, b.eval2, b.evec2, b.eig_ws, dev_status, s);
     launch_factor_mats(b.eval2, b.evec2, p.kq, p.k, b.Mu, b.Mv, S, s);
     ApplyArgs au{};
     au.in = b.P;

@@ -127,6 +127,91 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QuantParams p) {
   }
 }
 
+// blocks along columns without inner sums (the common case): a grid-stride
+// loop over 32-element units (2 NVFP4 blocks or 1 MXFP4 block); the raw
+// bytes of a thread's next unit are loaded before its current unit is
+// quantized, so every thread keeps a load in flight while it computes.
+template <int FMT, bool BF16>
+__global__ void __launch_bounds__(256) quantize_rows_fast_kernel(QuantParams p) {
+  constexpr int kU = 32;
+  constexpr int kVec = BF16 ? 4 : 8;  // 16-byte words per unit
+  const float s_t = tensor_scale_of(p);
+  if (FMT == METIS_NVFP4 && blockIdx.x == 0 && threadIdx.x == 0 && p.tensor_scale) *p.tensor_scale = s_t;
+  const int64_t upr = p.inner / kU;  // inner is a multiple of 32
+  const int64_t total = p.outer * upr;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const uint8_t* X = reinterpret_cast<const uint8_t*>(p.X);
+  const int64_t esize = BF16 ? 2 : 4;
+  auto src = [&](int64_t unit) {
+    const int64_t o = unit / upr;
+    return reinterpret_cast<const uint4*>(X + (o * p.ld + (unit - o * upr) * kU) * esize);
+  };
+  int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  uint4 cur[kVec], nxt[kVec];
+  if (t < total) {
+    const uint4* a = src(t);
+#pragma unroll
+    for (int k = 0; k < kVec; ++k) cur[k] = a[k];
+  }
+  for (; t < total; t += stride) {
+    const int64_t tn = t + stride;
+    if (tn < total) {
+      const uint4* a = src(tn);
+#pragma unroll
+      for (int k = 0; k < kVec; ++k) nxt[k] = a[k];
+    }
+    const int64_t o = t / upr, u = t - o * upr;
+    float v[kU];
+#pragma unroll
+    for (int k = 0; k < kVec; ++k) {
+      const uint32_t w[4] = {cur[k].x, cur[k].y, cur[k].z, cur[k].w};
+      if (BF16) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          v[8 * k + 2 * i] = __uint_as_float(w[i] << 16);
+          v[8 * k + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+      } else {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) v[4 * k + i] = __uint_as_float(w[i]);
+      }
+    }
+    if (p.sub) {
+#pragma unroll
+      for (int j = 0; j < kU; ++j) v[j] = __fsub_rn(v[j], p.sub[u * kU + j]);
+    }
+    if (p.r_tap) {
+      float* tp = p.r_tap + o * p.tap_ld + u * kU;
+#pragma unroll
+      for (int j = 0; j < kU; ++j) tp[j] = v[j];
+    }
+    uint4* dst = reinterpret_cast<uint4*>(p.codes + o * (p.inner / 2) + u * (kU / 2));
+    float ds;
+    if (FMT == METIS_NVFP4) {
+      uint64_t pk0, pk1;
+      const uint32_t c0 = quant_block_nv<false>(v, s_t, pk0, ds);
+      const uint32_t c1 = quant_block_nv<false>(v + 16, s_t, pk1, ds);
+      *dst = make_uint4(static_cast<uint32_t>(pk0), static_cast<uint32_t>(pk0 >> 32), static_cast<uint32_t>(pk1),
+                        static_cast<uint32_t>(pk1 >> 32));
+      *reinterpret_cast<uint16_t*>(p.scales + tc_scale_offset(o, 2 * u, p.scale_cols)) =
+          static_cast<uint16_t>(c0 | (c1 << 8));
+      if (p.scales_linear) {
+        p.scales_linear[o * (p.inner / 16) + 2 * u] = static_cast<uint8_t>(c0);
+        p.scales_linear[o * (p.inner / 16) + 2 * u + 1] = static_cast<uint8_t>(c1);
+      }
+    } else {
+      uint64_t pk[2];
+      const uint32_t c0 = quant_block_mx<false>(v, pk, ds);
+      *dst = make_uint4(static_cast<uint32_t>(pk[0]), static_cast<uint32_t>(pk[0] >> 32),
+                        static_cast<uint32_t>(pk[1]), static_cast<uint32_t>(pk[1] >> 32));
+      p.scales[tc_scale_offset(o, u, p.scale_cols)] = static_cast<uint8_t>(c0);
+      if (p.scales_linear) p.scales_linear[o * (p.inner / 32) + u] = static_cast<uint8_t>(c0);
+    }
+#pragma unroll
+    for (int k = 0; k < kVec; ++k) cur[k] = nxt[k];
+  }
+}
+
 // blocks along rows: one CTA per 64-row x 64-column tile of X.  The tile is
 // read with 16-byte row-segment loads into shared memory; then each thread
 // quantizes one block of one column (four threads, or two for MXFP4, cover
@@ -262,7 +347,16 @@ void launch_amax(const void* X, int dtype, int64_t rows, int64_t cols, int64_t l
 
 template <int FMT, bool SUM>
 void launch_quantize_t(const QuantParams& p, int axis, int num_sms, cudaStream_t s) {
-  if (axis == 1) {
+  if (axis == 1 && !SUM) {
+    // two or more units per thread, so the prefetch overlaps
+    const int64_t units = p.outer * (p.inner / 32);
+    int blocks = static_cast<int>(imin64((units + 511) / 512, static_cast<int64_t>(num_sms) * 4));
+    if (blocks < 1) blocks = 1;
+    if (p.dtype == METIS_BF16)
+      quantize_rows_fast_kernel<FMT, true><<<blocks, 256, 0, s>>>(p);
+    else
+      quantize_rows_fast_kernel<FMT, false><<<blocks, 256, 0, s>>>(p);
+  } else if (axis == 1) {
     const int64_t total = p.outer * p.ngroups;
     int blocks = static_cast<int>(imin64((total + 255) / 256, static_cast<int64_t>(num_sms) * 16));
     if (blocks < 1) blocks = 1;

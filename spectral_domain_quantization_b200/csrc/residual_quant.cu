@@ -1,24 +1,27 @@
 // Fused residual + FP4 quantization: R = A - U diag(S) V^T, tile by tile,
-// quantized along both block axes in the same pass.
+// quantized along either or both block axes in the same pass.
 //
 // Source: SII release on Metis, section 2.4 item 1 (the long-tail residual is
 // quantized on its own after the dominant part is split off) and section 2.3
 // / Fig. 3 (block-wise scales set by the block maximum); formats from the
 // feature list (MXFP4 / NVFP4).
 //
-// Per 128 x 128 tile of A (one CTA, 128 threads):
-//   1. TMA loads the tile's rows of U (hi, lo) and of W = V diag(S) (hi, lo),
-//      bf16, K = k padded to 64 (zeros).
-//   2. One thread issues U_hi W_hi + U_hi W_lo + U_lo W_hi as kind::f16 MMAs
-//      into a 128 x 128 fp32 TMEM accumulator: L = U S V^T to ~2^-16.
-//   3. Every thread owns one row: for each 64-column chunk it reads L from
-//      TMEM and A from global memory, forms R = fl32(a - l) and
-//        amax pass:  keeps max |R| (NVFP4 needs the tensor maximum first),
-//        quantize:   blocks along n straight from registers (32 bytes of
-//                    codes per thread); blocks along m through a per-warp
-//                    32 x 64 shared-memory transpose (a warp's 32 rows are
-//                    one MXFP4 block or two NVFP4 blocks of every column);
-//                    optional float32 tap of R.
+// Persistent, warp-specialized kernel; one CTA per SM walks a contiguous run
+// of 128 x 64 tiles of A in row-band order:
+//   warp 0      TMA producer: the band's rows of U (hi, lo; reloaded only
+//               when the band changes) and, per tile, the 64 rows of
+//               W = V diag(S) (hi, lo) and the 128 x 64 tile of A, into a ring
+//               of shared-memory stages;
+//   warp 1      TMEM owner and MMA issuer: U_hi W_hi + U_hi W_lo + U_lo W_hi as
+//               kind::f16 MMAs (M 128, N 64) into one of four TMEM
+//               accumulators, so L = U S V^T to ~2^-16 relative;
+//   warps 2-9   epilogue, 32 rows x 32 columns each: L from TMEM, A from the
+//               swizzled stage, R = fl32(a - l); then either the tensor
+//               maximum of |R| (the NVFP4 pre-pass) or the FP4 codes: blocks
+//               along n straight from registers, blocks along m through a
+//               per-warp 32 x 32 shared-memory transpose, plus an optional
+//               float32 tap of R.
+// Loads of the next tiles and MMAs overlap the epilogue of the current one.
 // HBM-bound: A is read once per pass (twice for NVFP4) and FP4 codes plus
 // scales are written once per quantized axis.
 #include "abi_common.h"
@@ -30,44 +33,12 @@ namespace metis {
 
 namespace {
 
-constexpr int kTile = 128;
-
 MDEV bool wait_ns(uint64_t* bar, uint32_t parity, uint64_t ns) {
   const uint64_t t0 = global_timer_ns();
   while (!mbar_try_wait(bar, parity)) {
     if (global_timer_ns() - t0 > ns) return false;
   }
   return true;
-}
-
-MDEV void load64(const void* A, int dtype, int64_t idx, int n, float* v) {
-  if (dtype == METIS_BF16) {
-    const uint4* p = reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(A) + idx);
-#pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      if (8 * q < n) {
-        const uint4 u = p[q];
-        const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          v[8 * q + 2 * i] = __uint_as_float(w[i] << 16);
-          v[8 * q + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
-        }
-      }
-    }
-  } else {
-    const float4* p = reinterpret_cast<const float4*>(reinterpret_cast<const float*>(A) + idx);
-#pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      if (4 * q < n) {
-        const float4 f = p[q];
-        v[4 * q] = f.x;
-        v[4 * q + 1] = f.y;
-        v[4 * q + 2] = f.z;
-        v[4 * q + 3] = f.w;
-      }
-    }
-  }
 }
 
 // Quantize n (32 or 64) values along the block axis: outer index o, first
@@ -120,36 +91,88 @@ MDEV void emit(const float* v, int n, int fmt, float s_t, uint8_t* codes, uint8_
   }
 }
 
-__global__ void __launch_bounds__(128) residual_quant_kernel(const ResidualParams p,
-                                                             const __grid_constant__ CUtensorMap tmUhi,
-                                                             const __grid_constant__ CUtensorMap tmUlo,
-                                                             const __grid_constant__ CUtensorMap tmWhi,
-                                                             const __grid_constant__ CUtensorMap tmWlo) {
+
+constexpr int kBM = 128;         // tile rows (one band)
+constexpr int kBN = 64;          // tile columns
+constexpr int kAccBufs = 4;      // TMEM accumulators of kBN columns
+constexpr int kTmemCols = kAccBufs * kBN;
+constexpr int kEpiWarps = 8;
+constexpr int kThreads = 32 * (2 + kEpiWarps);
+constexpr int kMaxStages = 4;
+constexpr int kSmemLimit = 232448;  // opt-in shared memory per CTA on sm_100
+constexpr int kTransposeBytes = kEpiWarps * 32 * 33 * 4;
+
+struct Layout {
+  int chunks;       // kp / 64
+  int u_bytes;      // U hi + lo
+  int w_bytes;      // per stage: W hi + lo
+  int a_bytes;      // per stage: the A tile
+  int stages;
+  int total;        // dynamic shared memory including 1024 B of alignment slack
+};
+
+__host__ __device__ inline Layout layout(int kp, int dtype) {
+  Layout l{};
+  l.chunks = kp / 64;
+  l.u_bytes = 2 * l.chunks * kBM * 128;
+  l.w_bytes = 2 * l.chunks * kBN * 128;
+  l.a_bytes = kBM * kBN * (dtype == METIS_BF16 ? 2 : 4);
+  const int fixed = 1024 + l.u_bytes + kTransposeBytes + 512;
+  int st = (kSmemLimit - fixed) / (l.w_bytes + l.a_bytes);
+  l.stages = st > kMaxStages ? kMaxStages : st;
+  l.total = fixed + l.stages * (l.w_bytes + l.a_bytes);
+  return l;
+}
+
+__global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const ResidualParams p,
+                                                                     const __grid_constant__ CUtensorMap tmUhi,
+                                                                     const __grid_constant__ CUtensorMap tmUlo,
+                                                                     const __grid_constant__ CUtensorMap tmWhi,
+                                                                     const __grid_constant__ CUtensorMap tmWlo,
+                                                                     const __grid_constant__ CUtensorMap tmA) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const int chunks = p.kp / 64;
-  const int part = chunks * 16384;  // one operand part: 128 rows x kp bf16
+  const Layout lo = layout(p.kp, p.dtype);
+  const int S = lo.stages;
   uint8_t* sUhi = smem;
-  uint8_t* sUlo = sUhi + part;
-  uint8_t* sWhi = sUlo + part;
-  uint8_t* sWlo = sWhi + part;
-  float* stage = reinterpret_cast<float*>(sWlo + part);  // 4 warps x 32 x 65 floats
-  uint64_t* bars = reinterpret_cast<uint64_t*>(stage + 4 * 32 * 65);
-  uint64_t* loaded = bars;
-  uint64_t* done = bars + 1;
-  uint32_t* tmem_sh = reinterpret_cast<uint32_t*>(bars + 2);
+  uint8_t* sUlo = sUhi + lo.u_bytes / 2;
+  uint8_t* sStage = smem + lo.u_bytes;
+  const int stage_bytes = lo.w_bytes + lo.a_bytes;
+  float* tstage = reinterpret_cast<float*>(sStage + S * stage_bytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(tstage) + kTransposeBytes);
+  uint64_t* full = bars;                           // [kMaxStages]
+  uint64_t* empty = full + kMaxStages;             // [kMaxStages]
+  uint64_t* acc_full = empty + kMaxStages;         // [kAccBufs]
+  uint64_t* acc_empty = acc_full + kAccBufs;       // [kAccBufs]
+  uint64_t* u_full = acc_empty + kAccBufs;
+  uint64_t* u_empty = u_full + 1;
+  uint64_t* drain = u_empty + 1;
+  uint32_t* tmem_sh = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_sh + 1);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int tn = blockIdx.x, tm = blockIdx.y;
   if (threadIdx.x == 0) {
-    mbar_init(loaded, 1);
-    mbar_init(done, 1);
+    for (int i = 0; i < kMaxStages; ++i) {
+      mbar_init(&full[i], 1);
+      mbar_init(&empty[i], kEpiWarps);
+    }
+    for (int i = 0; i < kAccBufs; ++i) {
+      mbar_init(&acc_full[i], 1);
+      mbar_init(&acc_empty[i], kEpiWarps);
+    }
+    mbar_init(u_full, 1);
+    mbar_init(u_empty, 1);
+    mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
+    prefetch_tensormap(&tmUhi);
+    prefetch_tensormap(&tmUlo);
+    prefetch_tensormap(&tmWhi);
+    prefetch_tensormap(&tmWlo);
+    prefetch_tensormap(&tmA);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_sh, 128);
+    tmem_alloc(tmem_sh, kTmemCols);
     tmem_relinquish();
   }
   tc_fence_before();
@@ -157,107 +180,220 @@ __global__ void __launch_bounds__(128) residual_quant_kernel(const ResidualParam
   tc_fence_after();
   const uint32_t tmem = *tmem_sh;
 
-  if (threadIdx.x == 0) {
-    mbar_arrive_expect_tx(loaded, 4 * part);
-    for (int c = 0; c < chunks; ++c) {
-      tma_load_2d(sUhi + c * 16384, &tmUhi, loaded, 64 * c, tm * kTile);
-      tma_load_2d(sUlo + c * 16384, &tmUlo, loaded, 64 * c, tm * kTile);
-      tma_load_2d(sWhi + c * 16384, &tmWhi, loaded, 64 * c, tn * kTile);
-      tma_load_2d(sWlo + c * 16384, &tmWlo, loaded, 64 * c, tn * kTile);
-    }
-  } else if (threadIdx.x == 32) {
-    if (mbar_wait(loaded, 0, abort_flag)) {
-      tc_fence_after();
-      const uint32_t idesc = idesc_bf16(128, kTile, false, false);
-      uint32_t acc = 0;
-      for (int c = 0; c < chunks; ++c) {
-        const uint64_t uh = make_sdesc(smem_u32(sUhi + c * 16384), 16, 1024, kSwizzle128B);
-        const uint64_t ul = make_sdesc(smem_u32(sUlo + c * 16384), 16, 1024, kSwizzle128B);
-        const uint64_t wh = make_sdesc(smem_u32(sWhi + c * 16384), 16, 1024, kSwizzle128B);
-        const uint64_t wl = make_sdesc(smem_u32(sWlo + c * 16384), 16, 1024, kSwizzle128B);
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint64_t o = static_cast<uint64_t>(2 * j);
-          mma_bf16(tmem, uh + o, wh + o, idesc, acc);
-          acc = 1;
-          mma_bf16(tmem, uh + o, wl + o, idesc, 1);
-          mma_bf16(tmem, ul + o, wh + o, idesc, 1);
+  // this CTA's contiguous run of tiles, in row-band order
+  const int nt = static_cast<int>((p.n + kBN - 1) / kBN);
+  const int total = static_cast<int>((p.m + kBM - 1) / kBM) * nt;
+  const int per = (total + gridDim.x - 1) / gridDim.x;
+  const int t0 = blockIdx.x * per;
+  const int t1 = min(total, t0 + per);
+  const bool f32 = p.dtype == METIS_F32;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0, issued = 0, u_loads = 0, cur_tm = -1;
+      uint32_t ph = 0, uph = 0;
+      for (int t = t0; t < t1; ++t) {
+        const int tm = t / nt, tn = t - tm * nt;
+        if (tm != cur_tm) {
+          if (cur_tm >= 0) {
+            if (!mbar_wait(u_empty, uph, abort_flag)) break;
+            uph ^= 1u;
+          }
+          mbar_arrive_expect_tx(u_full, lo.u_bytes);
+          for (int c = 0; c < lo.chunks; ++c) {
+            tma_load_2d(sUhi + c * kBM * 128, &tmUhi, u_full, 64 * c, tm * kBM);
+            tma_load_2d(sUlo + c * kBM * 128, &tmUlo, u_full, 64 * c, tm * kBM);
+          }
+          ++u_loads;
+          cur_tm = tm;
+        }
+        if (!mbar_wait(&empty[stage], ph ^ 1u, abort_flag)) break;
+        uint8_t* sW = sStage + stage * stage_bytes;
+        uint8_t* sA = sW + lo.w_bytes;
+        mbar_arrive_expect_tx(&full[stage], stage_bytes);
+        for (int c = 0; c < lo.chunks; ++c) {
+          tma_load_2d(sW + c * kBN * 128, &tmWhi, &full[stage], 64 * c, tn * kBN);
+          tma_load_2d(sW + (lo.chunks + c) * kBN * 128, &tmWlo, &full[stage], 64 * c, tn * kBN);
+        }
+        if (f32) {
+          tma_load_2d(sA, &tmA, &full[stage], tn * kBN, tm * kBM);
+          tma_load_2d(sA + kBM * 128, &tmA, &full[stage], tn * kBN + 32, tm * kBM);
+        } else {
+          tma_load_2d(sA, &tmA, &full[stage], tn * kBN, tm * kBM);
+        }
+        ++issued;
+        if (++stage == S) {
+          stage = 0;
+          ph ^= 1u;
         }
       }
+      if (*abort_flag) {
+        // let copies already in flight land before the CTA exits
+        int st = stage;
+        uint32_t pp = ph;
+        for (int i = 0; i < min(issued, S); ++i) {
+          if (--st < 0) {
+            st = S - 1;
+            pp ^= 1u;
+          }
+          wait_ns(&full[st], pp, 100000000ull);
+        }
+        if (u_loads > 0) wait_ns(u_full, static_cast<uint32_t>(u_loads - 1) & 1u, 100000000ull);
+      }
     }
-    tc_commit(done);
-  }
-  __syncwarp();
-  const bool ok = __all_sync(0xFFFFFFFFu, mbar_wait(done, 0, abort_flag));
-  tc_fence_after();
-
-  float s_t = 1.f;
-  if (p.mode == 1 && p.fmt == METIS_NVFP4) s_t = nv_tensor_scale(__uint_as_float(*p.amax_bits));
-  if (p.mode == 1 && p.fmt == METIS_NVFP4 && tm == 0 && tn == 0 && threadIdx.x == 0) {
-    if (p.ts_rows) *p.ts_rows = s_t;
-    if (p.ts_cols) *p.ts_cols = s_t;
-  }
-  const int64_t row = static_cast<int64_t>(tm) * kTile + 32 * warp + lane;
-  const bool row_ok = row < p.m;
-  float amax = 0.f;
-  float* my_stage = stage + warp * 32 * 65;
-  for (int h = 0; h < 2; ++h) {
-    const int64_t col0 = static_cast<int64_t>(tn) * kTile + 64 * h;
-    const int ncols = static_cast<int>(imax64(0, imin64(64, p.n - col0)));  // 0, 32 or 64
-    float v[64];
-    uint32_t L[64];
-    if (ok) {
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0, acc = 0, bands = 0, cur_tm = -1;
+      uint32_t ph = 0, aph = 0;
+      const uint32_t idesc = idesc_bf16(kBM, kBN, false, false);
+      for (int t = t0; t < t1; ++t) {
+        const int tm = t / nt;
+        if (tm != cur_tm) {
+          if (cur_tm >= 0) tc_commit(u_empty);  // the old U is free once these MMAs retire
+          if (!mbar_wait(u_full, static_cast<uint32_t>(bands) & 1u, abort_flag)) break;
+          ++bands;
+          cur_tm = tm;
+        }
+        if (!mbar_wait(&acc_empty[acc], aph ^ 1u, abort_flag)) break;
+        if (!mbar_wait(&full[stage], ph, abort_flag)) break;
+        tc_fence_after();
+        uint8_t* sW = sStage + stage * stage_bytes;
+        const uint32_t d = tmem + static_cast<uint32_t>(acc * kBN);
+        uint32_t accumulate = 0;
+        for (int c = 0; c < lo.chunks; ++c) {
+          const uint64_t uh = make_sdesc(smem_u32(sUhi + c * kBM * 128), 16, 1024, kSwizzle128B);
+          const uint64_t ul = make_sdesc(smem_u32(sUlo + c * kBM * 128), 16, 1024, kSwizzle128B);
+          const uint64_t wh = make_sdesc(smem_u32(sW + c * kBN * 128), 16, 1024, kSwizzle128B);
+          const uint64_t wl = make_sdesc(smem_u32(sW + (lo.chunks + c) * kBN * 128), 16, 1024, kSwizzle128B);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) tmem_ld16(tmem + (static_cast<uint32_t>(32 * warp) << 16) + 64 * h + 16 * q, L + 16 * q);
+          for (int j = 0; j < 4; ++j) {
+            const uint64_t o = static_cast<uint64_t>(2 * j);  // 32 bytes of K per step
+            mma_bf16(d, uh + o, wh + o, idesc, accumulate);
+            accumulate = 1;
+            mma_bf16(d, uh + o, wl + o, idesc, 1);
+            mma_bf16(d, ul + o, wh + o, idesc, 1);
+          }
+        }
+        tc_commit(&acc_full[acc]);
+        if (++stage == S) {
+          stage = 0;
+          ph ^= 1u;
+        }
+        if (++acc == kAccBufs) {
+          acc = 0;
+          aph ^= 1u;
+        }
+      }
+      if (*abort_flag) {
+        // wait for MMAs already issued before the TMEM is freed
+        tc_commit(drain);
+        wait_ns(drain, 0, 100000000ull);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;             // TMEM lane quadrant: rows 32 q .. 32 q + 31
+    const int h = (warp - 2) >> 2;      // columns 32 h .. 32 h + 31 of the tile
+    float* my_t = tstage + (warp - 2) * 32 * 33;
+    float s_t = 1.f;
+    if (p.mode == 1 && p.fmt == METIS_NVFP4) s_t = nv_tensor_scale(__uint_as_float(*p.amax_bits));
+    if (p.mode == 1 && p.fmt == METIS_NVFP4 && blockIdx.x == 0 && warp == 2 && lane == 0) {
+      if (p.ts_rows) *p.ts_rows = s_t;
+      if (p.ts_cols) *p.ts_cols = s_t;
+    }
+    float amax = 0.f;
+    int stage = 0, acc = 0;
+    uint32_t ph = 0, aph = 0;
+    for (int t = t0; t < t1; ++t) {
+      const int tm = t / nt, tn = t - tm * nt;
+      if (!mbar_wait(&acc_full[acc], aph, abort_flag)) break;
+      tc_fence_after();
+      uint32_t L[32];
+      tmem_ld16(tmem + (static_cast<uint32_t>(32 * q) << 16) + acc * kBN + 32 * h, L);
+      tmem_ld16(tmem + (static_cast<uint32_t>(32 * q) << 16) + acc * kBN + 32 * h + 16, L + 16);
       tmem_ld_wait();
-    }
-    if (ncols == 0) continue;
-    if (row_ok) load64(p.A, p.dtype, row * p.lda + col0, ncols, v);
-#pragma unroll
-    for (int j = 0; j < 64; ++j) {
-      const float l = ok ? __uint_as_float(L[j]) : 0.f;
-      v[j] = (row_ok && j < ncols) ? __fsub_rn(v[j], l) : 0.f;
-    }
-    if (p.mode == 0) {
-#pragma unroll
-      for (int j = 0; j < 64; ++j) amax = fmaxf(amax, fabsf(v[j]));
-      continue;
-    }
-    if (row_ok && p.r_tap) {
-      float* t = p.r_tap + row * p.n + col0;
-      for (int j = 0; j < ncols; j += 4) *reinterpret_cast<float4*>(t + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-    }
-    if (row_ok && p.r_codes) emit(v, ncols, p.fmt, s_t, p.r_codes, p.r_scales, p.r_scale_cols, p.n, row, col0);
-    if (p.c_codes) {
-      // transpose the warp's 32 rows x 64 columns through shared memory
+      tc_fence_before();
       __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      if (!mbar_wait(&full[stage], ph, abort_flag)) break;  // the A tile has landed
+      const int r = 32 * q + lane;                          // row within the tile
+      const uint8_t* arow = sStage + stage * stage_bytes + lo.w_bytes + r * 128;
+      float v[32];
+      if (f32) {
+        const uint8_t* base = arow + h * kBM * 128;  // box h holds columns 32 h ..
 #pragma unroll
-      for (int j = 0; j < 64; ++j) my_stage[lane * 65 + j] = v[j];
-      __syncwarp();
-      const int64_t r0 = static_cast<int64_t>(tm) * kTile + 32 * warp;
-      if (r0 < p.m) {
-        for (int cc = 0; cc < 2; ++cc) {
-          const int c = 2 * lane + cc;
-          if (c < ncols) {
-            float col[32];
+        for (int j = 0; j < 8; ++j) {
+          const float4 f = *reinterpret_cast<const float4*>(base + ((j ^ (r & 7)) << 4));
+          v[4 * j] = f.x;
+          v[4 * j + 1] = f.y;
+          v[4 * j + 2] = f.z;
+          v[4 * j + 3] = f.w;
+        }
+      } else {
 #pragma unroll
-            for (int r = 0; r < 32; ++r) col[r] = my_stage[r * 65 + c];
-            emit(col, 32, p.fmt, s_t, p.c_codes, p.c_scales, p.c_scale_cols, p.m, col0 + c, r0);
+        for (int jj = 0; jj < 4; ++jj) {
+          const int j = 4 * h + jj;
+          const uint4 u = *reinterpret_cast<const uint4*>(arow + ((j ^ (r & 7)) << 4));
+          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            v[8 * jj + 2 * i] = __uint_as_float(w[i] << 16);
+            v[8 * jj + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
           }
         }
       }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[stage]);
+      if (++stage == S) {
+        stage = 0;
+        ph ^= 1u;
+      }
+      if (++acc == kAccBufs) {
+        acc = 0;
+        aph ^= 1u;
+      }
+      const int64_t row0 = static_cast<int64_t>(tm) * kBM + 32 * q;
+      const int64_t col0 = static_cast<int64_t>(tn) * kBN + 32 * h;
+      if (row0 >= p.m || col0 >= p.n) continue;  // m, n are multiples of 32: whole warp
+      const int64_t row = row0 + lane;
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __fsub_rn(v[j], __uint_as_float(L[j]));
+      if (p.mode == 0) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
+        continue;
+      }
+      if (p.r_tap) {
+        float* tp = p.r_tap + row * p.n + col0;
+#pragma unroll
+        for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4*>(tp + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+      }
+      if (p.r_codes) emit(v, 32, p.fmt, s_t, p.r_codes, p.r_scales, p.r_scale_cols, p.n, row, col0);
+      if (p.c_codes) {
+        // the warp's 32 rows x 32 columns, transposed through shared memory
+#pragma unroll
+        for (int j = 0; j < 32; ++j) my_t[lane * 33 + j] = v[j];
+        __syncwarp();
+        float col[32];
+#pragma unroll
+        for (int i = 0; i < 32; ++i) col[i] = my_t[i * 33 + lane];
+        __syncwarp();
+        emit(col, 32, p.fmt, s_t, p.c_codes, p.c_scales, p.c_scale_cols, p.m, col0 + lane, row0);
+      }
+    }
+    if (p.mode == 0) {
+      for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
+      if (lane == 0) atomicMax(p.amax_bits, __float_as_uint(amax));
     }
   }
-  if (p.mode == 0) {
-    for (int o = 16; o > 0; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
-    if (lane == 0) atomicMax(p.amax_bits, __float_as_uint(amax));
-  }
-  if (*abort_flag && threadIdx.x == 32) wait_ns(done, 0, 100000000ull);
   tc_fence_before();
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, 128);
+    tmem_dealloc(tmem, kTmemCols);
   }
   if (threadIdx.x == 0 && *abort_flag) report(p.dev_status, METIS_DEV_TIMEOUT);
 }
@@ -280,12 +416,22 @@ __global__ void hilo_kernel(const float* X, int64_t rows, int k, const float* S,
   }
 }
 
-CUresult map_rows(CUtensorMap* m, const void* base, int64_t rows, int kp) {
+CUresult map_kmajor(CUtensorMap* m, const void* base, int64_t rows, int kp, uint32_t box_rows) {
   const uint64_t dims[2] = {static_cast<uint64_t>(kp), static_cast<uint64_t>(rows)};
   const uint64_t strides[1] = {static_cast<uint64_t>(kp) * 2};
-  const uint32_t box[2] = {64, 128};
+  const uint32_t box[2] = {64, box_rows};
   return encode_tensor_map(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box,
                            CU_TENSOR_MAP_SWIZZLE_128B);
+}
+
+// A (m x n, row stride lda): boxes of 128 bytes of a row x 128 rows.
+CUresult map_a(CUtensorMap* m, const ResidualParams& p) {
+  const bool bf = p.dtype == METIS_BF16;
+  const uint64_t dims[2] = {static_cast<uint64_t>(p.n), static_cast<uint64_t>(p.m)};
+  const uint64_t strides[1] = {static_cast<uint64_t>(p.lda) * (bf ? 2 : 4)};
+  const uint32_t box[2] = {bf ? 64u : 32u, static_cast<uint32_t>(kBM)};
+  return encode_tensor_map(m, bf ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, p.A, dims,
+                           strides, box, CU_TENSOR_MAP_SWIZZLE_128B);
 }
 
 }  // namespace
@@ -298,16 +444,20 @@ void launch_hilo(const float* X, int64_t rows, int k, const float* S, int kp, __
 }
 
 metis_status run_residual_quant(const ResidualParams& p, const ResidualOperands& o, cudaStream_t s) {
-  CUtensorMap uh, ul, wh, wl;
-  if (map_rows(&uh, o.u_hi, p.m, p.kp) != CUDA_SUCCESS || map_rows(&ul, o.u_lo, p.m, p.kp) != CUDA_SUCCESS ||
-      map_rows(&wh, o.w_hi, p.n, p.kp) != CUDA_SUCCESS || map_rows(&wl, o.w_lo, p.n, p.kp) != CUDA_SUCCESS)
+  CUtensorMap uh, ul, wh, wl, ta;
+  if (map_kmajor(&uh, o.u_hi, p.m, p.kp, kBM) != CUDA_SUCCESS || map_kmajor(&ul, o.u_lo, p.m, p.kp, kBM) != CUDA_SUCCESS ||
+      map_kmajor(&wh, o.w_hi, p.n, p.kp, kBN) != CUDA_SUCCESS || map_kmajor(&wl, o.w_lo, p.n, p.kp, kBN) != CUDA_SUCCESS ||
+      map_a(&ta, p) != CUDA_SUCCESS)
     return fail(METIS_ERR_CUDA, "residual tensor map");
-  const int part = (p.kp / 64) * 16384;
-  const int smem = 4 * part + 4 * 32 * 65 * 4 + 64 + 1024;
-  if (!ensure_smem(reinterpret_cast<const void*>(residual_quant_kernel), smem))
+  const Layout lo = layout(p.kp, p.dtype);
+  if (lo.stages < 2) return fail(METIS_ERR_SHAPE, "residual", "factor rank too large for the shared-memory stages");
+  if (!ensure_smem(reinterpret_cast<const void*>(residual_quant_kernel), lo.total))
     return fail(METIS_ERR_CUDA, "residual shared-memory attribute");
-  const dim3 grid(static_cast<unsigned>((p.n + kTile - 1) / kTile), static_cast<unsigned>((p.m + kTile - 1) / kTile));
-  residual_quant_kernel<<<grid, 128, smem, s>>>(p, uh, ul, wh, wl);
+  const int64_t tiles = ((p.m + kBM - 1) / kBM) * ((p.n + kBN - 1) / kBN);
+  const int sms = device_sm_count();
+  const int64_t per = (tiles + sms - 1) / sms;
+  const unsigned grid = static_cast<unsigned>((tiles + per - 1) / per);
+  residual_quant_kernel<<<grid, kThreads, lo.total, s>>>(p, uh, ul, wh, wl, ta);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(METIS_ERR_CUDA, "residual_quant launch", cudaGetErrorString(e));
   return METIS_OK;

@@ -208,7 +208,8 @@ CUresult map_bf16(CUtensorMap* m, const void* base, int64_t rows, int64_t cols, 
 int skinny_splits(int64_t rows_out, int64_t K, int sms) {
   const int64_t tiles = (rows_out + 127) / 128;
   const int64_t ksteps = (K + 63) / 64;
-  int64_t s = (2 * static_cast<int64_t>(sms) + tiles - 1) / tiles;  // about two CTAs per SM
+  // two CTAs fit on an SM: fill that one wave without starting a second
+  int64_t s = 2 * static_cast<int64_t>(sms) / tiles;
   if (s > ksteps) s = ksteps;
   if (s < 1) s = 1;
   return static_cast<int>(s);

@@ -72,125 +72,208 @@ MDEV void gram_block(const float* ys, int rows, int cols, int ld, double* out) {
 }
 
 // Sum split partials into Y (optional) and the Gram partial of each block.
-__global__ void gram_kernel(const float* partial, int splits, int64_t rows, int lp, float* Y, double* gpart) {
+// One thread per 4 consecutive columns of one row (blockDim = 32 lp / 4), so
+// every split partial is one 16-byte load and a thread's loads are
+// independent; the sum keeps the split order.
+__global__ void __launch_bounds__(1024) gram_kernel(const float* __restrict__ partial, int splits, int64_t rows,
+                                                    int lp, float* __restrict__ Y, double* __restrict__ gpart) {
   extern __shared__ float ys[];  // kRowsPerBlock x (lp + 1)
   const int ld = lp + 1;
+  const int q4 = lp / 4;
   const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock;
   const int nr = static_cast<int>(imin64(kRowsPerBlock, rows - r0));
-  for (int e = threadIdx.x; e < kRowsPerBlock * lp; e += blockDim.x) {
-    const int r = e / lp, c = e - r * lp;
-    float v = 0.f;
+  const int64_t stride4 = rows * q4;
+  const float4* src = reinterpret_cast<const float4*>(partial);
+  for (int e = threadIdx.x; e < kRowsPerBlock * q4; e += blockDim.x) {
+    const int r = e / q4, c4 = e - r * q4;
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
     if (r < nr) {
-      for (int s = 0; s < splits; ++s) v += partial[(static_cast<int64_t>(s) * rows + r0 + r) * lp + c];
-      if (Y) Y[(r0 + r) * lp + c] = v;
+      const float4* p = src + (r0 + r) * q4 + c4;
+#pragma unroll 8
+      for (int sp = 0; sp < splits; ++sp) {
+        const float4 x = p[sp * stride4];
+        acc.x += x.x;
+        acc.y += x.y;
+        acc.z += x.z;
+        acc.w += x.w;
+      }
+      if (Y) reinterpret_cast<float4*>(Y)[(r0 + r) * q4 + c4] = acc;
     }
-    ys[r * ld + c] = v;
+    float* d = ys + r * ld + 4 * c4;
+    d[0] = acc.x;
+    d[1] = acc.y;
+    d[2] = acc.z;
+    d[3] = acc.w;
   }
   __syncthreads();
   gram_block(ys, nr, lp, ld, gpart + static_cast<int64_t>(blockIdx.x) * lp * lp);
 }
 
-// One warp per Gram entry: lanes take blocks lane, lane+32, ... and the warp
-// reduces with a fixed shuffle tree (deterministic).
-__global__ void gram_reduce_kernel(const double* gpart, int nblocks, int n2, double* G) {
-  const int e = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-  const int lane = threadIdx.x & 31;
-  if (e >= n2) return;
+// Sum of the block partials: a CTA takes 32 consecutive entries (coalesced
+// 256-byte rows of each partial); its 8 warps take every 8th block, then the
+// 8 partial sums are added in warp order (deterministic).
+constexpr int kReduceGroups = 8;
+__global__ void __launch_bounds__(256) gram_reduce_kernel(const double* __restrict__ gpart, int nblocks, int n2,
+                                                          double* __restrict__ G) {
+  __shared__ double part[kReduceGroups][32];
+  const int lane = threadIdx.x & 31, grp = threadIdx.x >> 5;
+  const int e = blockIdx.x * 32 + lane;
   double s = 0.0;
-  for (int b = lane; b < nblocks; b += 32) s += gpart[static_cast<int64_t>(b) * n2 + e];
-  for (int o = 16; o > 0; o >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, o);
-  if (lane == 0) G[e] = s;
+  if (e < n2) {
+#pragma unroll 8
+    for (int b = grp; b < nblocks; b += kReduceGroups) s += gpart[static_cast<int64_t>(b) * n2 + e];
+  }
+  part[grp][lane] = s;
+  __syncthreads();
+  if (grp == 0 && e < n2) {
+    double t = 0.0;
+#pragma unroll
+    for (int g = 0; g < kReduceGroups; ++g) t += part[g][lane];
+    G[e] = t;
+  }
 }
 
-// Decode e -> (q, e - q*d) for e < 2^22 with a float reciprocal (exact).
-MDEV int fdiv_index(int e, float rcp) { return __float2int_rz((static_cast<float>(e) + 0.5f) * rcp); }
+// Lower-triangle element e (column-major order: column 0 top to bottom, then
+// column 1 ...) of an n x n matrix, packed as (row << 8) | column.
+MDEV int tri_element(int e, int n) {
+  const int ntri = n * (n + 1) / 2;
+  const int er = ntri - 1 - e;  // index counted from the last element
+  // w = length of the column holding er counted from the right: the smallest
+  // w with w (w + 1) / 2 > er
+  int w = static_cast<int>((sqrtf(8.f * er + 1.f) - 1.f) * 0.5f) + 1;
+  while (w * (w + 1) / 2 <= er) ++w;
+  while (w > 1 && (w - 1) * w / 2 > er) --w;
+  const int c = n - w;
+  const int i = n - 1 - (er - (w - 1) * w / 2);
+  return (i << 8) | c;
+}
+
+constexpr int kSmallThreads = 1024;
+constexpr int kMaxOwn = 7;  // ceil(112 * 113 / 2 / 1024): lower-triangle elements per thread
 
 // G = L L^T (with drops), then Rinv = L^-T (upper triangular, float32).
-// Work is enumerated over flattened index ranges so every thread gets an equal
-// share of the shrinking triangle.  One barrier per column: step j updates the
-// trailing lower triangle with the unscaled column j (times 1/d_j) and scales
-// column j-1; the thread updating the next diagonal entry computes the next
-// pivot's reciprocal square root, overlapping its latency with the update.
-__global__ void __launch_bounds__(1024) cholesky_inv_kernel(const double* G, int lp, float* Rinv) {
+//  Cholesky (right-looking, one barrier per column): each thread keeps up to
+//  kMaxOwn lower-triangle elements in registers.  They are dealt out in
+//  reverse column-major order, so the elements still active at step j (those
+//  right of column j) are a prefix of that order and a warp whose share lies
+//  past it skips the slot.  Step j: every active (i, c) takes
+//  v -= v(i, j) v(c, j) / d_j with v(., j) the unscaled column j, published
+//  in shared memory at step j - 1; column j + 1 is then final and is
+//  published for step j + 1, and the owner of (j + 1, j + 1) forms the next
+//  pivot's 1/sqrt.
+//  Inverse: X = L^-1 by 16 x 16 blocks (see below).
+__global__ void __launch_bounds__(kSmallThreads) cholesky_inv_kernel(const double* G, int lp, float* Rinv) {
   extern __shared__ double sm[];
   const int ld = lp + 1;
-  double* L = sm;                  // lp x ld
-  double* X = L + lp * ld;         // lp x ld, becomes L^-1
-  double* diag0 = X + lp * ld;     // lp
-  double* invd = diag0 + lp;       // lp: 1/sqrt(pivot) (0 when dropped)
-  double* sqd = invd + lp;         // lp: sqrt(pivot) (0 when dropped)
-  const int t = threadIdx.x, nt = blockDim.x;
-  for (int e = t; e < lp * lp; e += nt) {
-    const int i = e / lp, j = e - i * lp;
-    L[i * ld + j] = G[e];
-    X[i * ld + j] = i == j ? 1.0 : 0.0;
+  double* buf = sm;               // 2 x lp: the published column
+  double* invd = buf + 2 * lp;    // lp: 1/sqrt(pivot) (0 when dropped)
+  double* sqd = invd + lp;        // lp: sqrt(pivot) (0 when dropped)
+  double* diag0 = sqd + lp;       // lp: the original diagonal (drop rule)
+  double* L = diag0 + lp;         // lp x ld: final L
+  const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+  const int ntri = lp * (lp + 1) / 2;
+  int own[kMaxOwn];
+  double v[kMaxOwn];
+#pragma unroll
+  for (int u = 0; u < kMaxOwn; ++u) {
+    const int er = kSmallThreads * u + t;  // position in reverse column-major order
+    own[u] = er < ntri ? tri_element(ntri - 1 - er, lp) : -1;
+    v[u] = 0.0;
+    if (own[u] >= 0) {
+      const int i = own[u] >> 8, c = own[u] & 255;
+      v[u] = G[i * lp + c];
+      if (i == c) diag0[i] = v[u];
+      if (c == 0) buf[i] = v[u];
+    }
   }
-  for (int i = t; i < lp; i += nt) diag0[i] = G[i * lp + i];
-  __syncthreads();
   if (t == 0) {
-    const double d = L[0];
-    const bool drop = !(diag0[0] > 0.0) || !(d > kDropTol * diag0[0]);
-    sqd[0] = drop ? 0.0 : sqrt(d);
-    invd[0] = drop ? 0.0 : 1.0 / sqd[0];
+    const double d = G[0];
+    const double r = d > 0.0 ? rsqrt(d) : 0.0;
+    invd[0] = r;
+    sqd[0] = d * r;
   }
   __syncthreads();
-  for (int j = 0; j < lp; ++j) {
+  for (int j = 0; j + 1 < lp; ++j) {
+    const double* cur = buf + (j & 1) * lp;
+    double* nxt = buf + ((j + 1) & 1) * lp;
     const double inv2 = invd[j] * invd[j];
-    // trailing lower triangle {(i, c): j < c <= i < lp}, row by row:
-    // row i = j + 1 + a holds a + 1 entries; flatten with a triangular decode
-    const int w = lp - j - 1;
-    const int total = w * (w + 1) / 2;
-    for (int e = t; e < total; e += nt) {
-      int a = static_cast<int>((sqrtf(8.f * e + 1.f) - 1.f) * 0.5f);
-      if ((a + 1) * (a + 2) / 2 <= e) ++a;
-      if (a * (a + 1) / 2 > e) --a;
-      const int i = j + 1 + a, c = j + 1 + (e - a * (a + 1) / 2);
-      const double v = L[i * ld + c] - L[i * ld + j] * L[c * ld + j] * inv2;
-      L[i * ld + c] = v;
-      if (e == 0) {  // (j+1, j+1): next pivot
-        const bool drop = !(diag0[c] > 0.0) || !(v > kDropTol * diag0[c]);
-        const double r = drop ? 0.0 : sqrt(v);
-        sqd[c] = r;
-        invd[c] = drop ? 0.0 : 1.0 / r;
+    const int active = (lp - j - 1) * (lp - j) / 2;  // elements right of column j
+#pragma unroll
+    for (int u = 0; u < kMaxOwn; ++u) {
+      if (kSmallThreads * u + 32 * warp >= active) break;  // warp-uniform
+      if (kSmallThreads * u + t < active) {
+        const int i = own[u] >> 8, c = own[u] & 255;
+        v[u] -= cur[i] * cur[c] * inv2;
+        if (c == j + 1) {
+          nxt[i] = v[u];
+          if (i == c) {
+            const bool drop = !(diag0[c] > 0.0) || !(v[u] > kDropTol * diag0[c]);
+            const double r = drop ? 0.0 : rsqrt(v[u]);
+            invd[c] = r;
+            sqd[c] = v[u] * r;
+          }
+        }
       }
     }
-    if (j > 0) {  // deferred scaling of column j-1
-      const double pinv = invd[j - 1];
-      for (int i = j + t; i < lp; i += nt) L[i * ld + j - 1] *= pinv;
-      if (t == 0) L[(j - 1) * ld + j - 1] = sqd[j - 1];
-    }
     __syncthreads();
   }
-  if (t == 0) L[(lp - 1) * ld + lp - 1] = sqd[lp - 1];
-  // X = L^-1: step k eliminates with the unscaled row k (times 1/L_kk) over
-  // the rectangle rows k+1.., columns 0..k, and scales row k-1
-  for (int k = 0; k < lp; ++k) {
-    const double inv = invd[k];
-    const int cols = k + 1, total = (lp - k - 1) * cols;
-    const float rcp = 1.f / static_cast<float>(cols);
-    for (int e = t; e < total; e += nt) {
-      const int q = fdiv_index(e, rcp);
-      const int i = k + 1 + q, c = e - q * cols;
-      X[i * ld + c] -= L[i * ld + k] * inv * X[k * ld + c];
+#pragma unroll
+  for (int u = 0; u < kMaxOwn; ++u) {
+    if (own[u] >= 0) {
+      const int i = own[u] >> 8, c = own[u] & 255;
+      L[i * ld + c] = i == c ? sqd[c] : v[u] * invd[c];
     }
-    if (k > 0) {
-      const double pinv = invd[k - 1];
-      for (int c = t; c < k; c += nt) X[(k - 1) * ld + c] *= pinv;
-    }
-    __syncthreads();
   }
-  for (int c = t; c < lp; c += nt) X[(lp - 1) * ld + c] *= invd[lp - 1];
   __syncthreads();
-  for (int e = t; e < lp * lp; e += nt) {
-    const int j = e / lp, c = e - j * lp;  // Rinv[j][c] = X[c][j]
-    Rinv[e] = c >= j ? static_cast<float>(X[c * ld + j]) : 0.f;
+  // X = L^-1 by 16 x 16 blocks: the diagonal blocks are inverted by one warp
+  // each (a lane per column, forward substitution), then block row bi is
+  //   T = sum_{k < bi} L(bi, k) X(k, j)   and   X(bi, j) = -X(bi, bi) T
+  // for all j < bi at once (two barriers per block row).
+  double* X = L + lp * ld;        // lp x ld
+  double* T = X + lp * ld;        // 16 x ld
+  const int nb = lp / 16;
+  if (warp < nb && lane < 16) {
+    const int o = 16 * warp, j = lane;
+    double x[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      double sum = 0.0;
+#pragma unroll
+      for (int m = 0; m < i; ++m)
+        if (m >= j) sum += L[(o + i) * ld + o + m] * x[m];
+      x[i] = i < j ? 0.0 : (i == j ? invd[o + i] : -sum * invd[o + i]);
+      X[(o + i) * ld + o + j] = x[i];
+    }
+  }
+  __syncthreads();
+  for (int bi = 1; bi < nb; ++bi) {
+    const int o = 16 * bi;
+    for (int e = t; e < 16 * o; e += kSmallThreads) {
+      const int r = e / o, c = e - r * o;
+      double sum = 0.0;
+      for (int m = c; m < o; ++m) sum += L[(o + r) * ld + m] * X[m * ld + c];
+      T[r * ld + c] = sum;
+    }
+    __syncthreads();
+    for (int e = t; e < 16 * o; e += kSmallThreads) {
+      const int r = e / o, c = e - r * o;
+      double sum = 0.0;
+      for (int q = 0; q <= r; ++q) sum += X[(o + r) * ld + o + q] * T[q * ld + c];
+      X[(o + r) * ld + c] = -sum;
+    }
+    __syncthreads();
+  }
+  // Rinv[c][r] = X[r][c] (upper triangular)
+  for (int e = t; e < lp * lp; e += kSmallThreads) {
+    const int c = e / lp, r = e - c * lp;
+    Rinv[e] = r >= c ? static_cast<float>(X[r * ld + c]) : 0.f;
   }
 }
 
 constexpr int kApplyRows = 32;
 
 // out = in (rows x kin) * M (kin x kout).  32 rows per CTA, 256 threads, each
-// thread a 2-row x ceil(kout/16)-column register tile.  Optional fp32 out,
+// thread a 4-row x 4-column register tile.  Optional fp32 out,
 // transposed bf16 hi/lo copy, Gram partial of the output block.
 __global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) {
   extern __shared__ float smf[];
@@ -199,40 +282,55 @@ __global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) {
   float* Out = In + kApplyRows * (a.kin + 1);        // kApplyRows x (kout + 1)
   const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kApplyRows;
   const int nr = static_cast<int>(imin64(kApplyRows, a.rows - r0));
-  for (int e = threadIdx.x; e < a.kin * a.kout; e += blockDim.x) Ms[e] = a.M[e];
-  for (int e = threadIdx.x; e < kApplyRows * a.kin; e += blockDim.x) {
-    const int r = e / a.kin, c = e - r * a.kin;
-    In[r * (a.kin + 1) + c] = r < nr ? a.in[(r0 + r) * a.in_ld + c] : 0.f;
+  {
+    const float4* M4 = reinterpret_cast<const float4*>(a.M);
+    float4* Ms4 = reinterpret_cast<float4*>(Ms);
+    const int n4 = a.kin * a.kout / 4;
+#pragma unroll 8
+    for (int e = threadIdx.x; e < n4; e += blockDim.x) Ms4[e] = M4[e];
+    const int q4 = a.kin / 4;
+#pragma unroll 4
+    for (int e = threadIdx.x; e < kApplyRows * q4; e += blockDim.x) {
+      const int r = e / q4, c4 = e - r * q4;
+      const float4 x = r < nr ? *reinterpret_cast<const float4*>(a.in + (r0 + r) * a.in_ld + 4 * c4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      float* d = In + r * (a.kin + 1) + 4 * c4;
+      d[0] = x.x;
+      d[1] = x.y;
+      d[2] = x.z;
+      d[3] = x.w;
+    }
   }
   __syncthreads();
-  const int tr = threadIdx.x & 15, tc = threadIdx.x >> 4;
-  constexpr int kMaxCols = 7;  // kout <= 112
-  float acc[2][kMaxCols];
+  // warp w: rows 4 w .. 4 w + 3 (broadcast reads of In); lane: columns
+  // lane, lane + 32, lane + 64, lane + 96 (kout <= 112)
+  const int rg = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  constexpr int kCols = 4;
+  float acc[4][kCols];
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int u = 0; u < kMaxCols; ++u) acc[i][u] = 0.f;
-  const float* in0 = In + (2 * tr) * (a.kin + 1);
-  const float* in1 = in0 + (a.kin + 1);
+    for (int u = 0; u < kCols; ++u) acc[i][u] = 0.f;
+  const float* in0 = In + (4 * rg) * (a.kin + 1);
+  const int ncol = (a.kout - lane + 31) / 32;  // columns this lane owns
 #pragma unroll 2
   for (int j = 0; j < a.kin; ++j) {
-    const float x0 = in0[j], x1 = in1[j];
-    const float* mrow = Ms + j * a.kout;
+    float x[4];
 #pragma unroll
-    for (int u = 0; u < kMaxCols; ++u) {
-      const int c = tc + 16 * u;
-      const float m = c < a.kout ? mrow[c] : 0.f;
-      acc[0][u] = fmaf(x0, m, acc[0][u]);
-      acc[1][u] = fmaf(x1, m, acc[1][u]);
+    for (int i = 0; i < 4; ++i) x[i] = in0[i * (a.kin + 1) + j];
+    const float* mrow = Ms + j * a.kout + lane;
+#pragma unroll
+    for (int u = 0; u < kCols; ++u) {
+      const float m = u < ncol ? mrow[32 * u] : 0.f;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) acc[i][u] = fmaf(x[i], m, acc[i][u]);
     }
   }
 #pragma unroll
-  for (int i = 0; i < 2; ++i)
+  for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int u = 0; u < kMaxCols; ++u) {
-      const int c = tc + 16 * u;
-      if (c < a.kout) Out[(2 * tr + i) * (a.kout + 1) + c] = acc[i][u];
-    }
+    for (int u = 0; u < kCols; ++u)
+      if (u < ncol) Out[(4 * rg + i) * (a.kout + 1) + lane + 32 * u] = acc[i][u];
   __syncthreads();
   for (int e = threadIdx.x; e < kApplyRows * a.kout; e += blockDim.x) {
     if (a.out) {
@@ -254,188 +352,6 @@ __global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) {
 
 // Round-robin pairing: in step r of a sweep over n (even) indices, slot i
 // pairs with slot n-1-i; slot 0 holds index 0, slots 1..n-1 rotate.
-MDEV int rr_index(int slot, int step, int n) {
-  if (slot == 0) return 0;
-  return ((slot - 1 + step) % (n - 1)) + 1;
-}
-
-constexpr double kRankTol = 1e-10;   // pivoted Cholesky: relative diagonal cut
-// one-sided Jacobi: rotate while |a.b| > tol |a||b|.  Float32 sums of <= 112
-// products carry ~5e-7 relative noise, so the rule sits well above it.
-constexpr float kJacobiTol = 4e-6f;
-
-// Eigen-decomposition of the l x l core Gram C = Z^T Z (PSD), eigenvalues
-// descending; evec[i * n + j] = component i of eigenvector j.
-//   1. pivoted Cholesky (float64): P C P^T = L L^T (rank-revealing cut);
-//   2. one-sided Jacobi on the columns of L (float32, eight lanes per column
-//      pair, round-robin order): L J = U diag(sigma), so the normalised
-//      columns are the eigenvectors of P C P^T and sigma^2 its eigenvalues
-//      (this is the one-sided Jacobi SVD of the core, preconditioned by the
-//      pivoted factorization, which needs few sweeps);
-//   3. sort and undo the pivoting.
-__global__ void __launch_bounds__(1024) core_eig_kernel(const double* C, int n, int max_sweeps, double* eval,
-                                                        float* evec, int32_t* dev_status) {
-  extern __shared__ double smd[];
-  const int ld = n + 1;
-  double* G = smd;                                       // n x ld
-  float* X = reinterpret_cast<float*>(G + n * ld);       // column j at X[j * ld + r]
-  int* perm = reinterpret_cast<int*>(X + n * ld);        // n
-  float* norms = reinterpret_cast<float*>(perm + n);     // n
-  __shared__ int piv_sh, rotated_sh;
-  __shared__ double maxd_sh;
-  const int t = threadIdx.x, nt = blockDim.x, warp = t >> 5, lane = t & 31, nwarps = nt >> 5;
-  for (int e = t; e < n * n; e += nt) G[(e / n) * ld + e % n] = C[e];
-  for (int i = t; i < n; i += nt) perm[i] = i;
-  __syncthreads();
-  if (warp == 0) {
-    double m = 0.0;
-    for (int i = lane; i < n; i += 32) m = fmax(m, G[i * ld + i]);
-    for (int o = 16; o > 0; o >>= 1) m = fmax(m, __shfl_xor_sync(0xFFFFFFFFu, m, o));
-    if (lane == 0) maxd_sh = m;
-  }
-  __syncthreads();
-  const double cut = kRankTol * maxd_sh;
-  int rank = n;
-  for (int j = 0; j < n; ++j) {
-    if (warp == 0) {
-      double best = -1.0;
-      int bi = j;
-      for (int i = j + lane; i < n; i += 32) {
-        const double v = G[i * ld + i];
-        if (v > best) {
-          best = v;
-          bi = i;
-        }
-      }
-      for (int o = 16; o > 0; o >>= 1) {
-        const double ob = __shfl_xor_sync(0xFFFFFFFFu, best, o);
-        const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
-        if (ob > best || (ob == best && oi < bi)) {
-          best = ob;
-          bi = oi;
-        }
-      }
-      if (lane == 0) piv_sh = bi;
-    }
-    __syncthreads();
-    const int p = piv_sh;
-    if (p != j) {
-      for (int c = t; c < n; c += nt) {
-        const double a = G[j * ld + c];
-        G[j * ld + c] = G[p * ld + c];
-        G[p * ld + c] = a;
-      }
-      __syncthreads();
-      for (int r = t; r < n; r += nt) {
-        const double a = G[r * ld + j];
-        G[r * ld + j] = G[r * ld + p];
-        G[r * ld + p] = a;
-      }
-      if (t == 0) {
-        const int a = perm[j];
-        perm[j] = perm[p];
-        perm[p] = a;
-      }
-      __syncthreads();
-    }
-    const double d = G[j * ld + j];
-    if (!(d > cut)) {
-      rank = j;
-      break;
-    }
-    const double inv = 1.0 / sqrt(d);
-    const double invd2 = inv * inv;
-    // the whole (symmetric) Schur complement is kept current, so that the
-    // next pivot swap can exchange complete rows and columns
-    const int w = n - j - 1;
-    const float rcpw = 1.f / static_cast<float>(w > 0 ? w : 1);
-    for (int e = t; e < w * w; e += nt) {
-      const int q = fdiv_index(e, rcpw);
-      const int i = j + 1 + q, c = j + 1 + (e - q * w);
-      G[i * ld + c] -= G[i * ld + j] * G[c * ld + j] * invd2;
-    }
-    __syncthreads();
-    for (int i = j + 1 + t; i < n; i += nt) G[i * ld + j] *= inv;
-    if (t == 0) G[j * ld + j] = d * inv;
-    __syncthreads();
-  }
-  for (int e = t; e < n * n; e += nt) {
-    const int j = e / n, r = e - j * n;
-    X[j * ld + r] = (j < rank && r >= j) ? static_cast<float>(G[r * ld + j]) : 0.f;
-  }
-  __syncthreads();
-  // one-sided Jacobi: 8 lanes per column pair, 4 pairs per warp
-  const int grp = lane >> 3, l8 = lane & 7;
-  const int npairs = n / 2;
-  int sweep = 0;
-  for (; sweep < max_sweeps; ++sweep) {
-    if (t == 0) rotated_sh = 0;
-    __syncthreads();
-    for (int step = 0; step < n - 1; ++step) {
-      for (int base = 4 * warp; base < npairs; base += 4 * nwarps) {
-        const int pair = base + grp;
-        const bool act = pair < npairs;
-        int p = 0, q = 1;
-        if (act) {
-          p = rr_index(pair, step, n);
-          q = rr_index(n - 1 - pair, step, n);
-          if (p > q) {
-            const int x = p;
-            p = q;
-            q = x;
-          }
-        }
-        float al = 0.f, be = 0.f, ga = 0.f;
-        if (act) {
-          for (int r = l8; r < n; r += 8) {
-            const float a = X[p * ld + r], b = X[q * ld + r];
-            al = fmaf(a, a, al);
-            be = fmaf(b, b, be);
-            ga = fmaf(a, b, ga);
-          }
-        }
-#pragma unroll
-        for (int o = 4; o > 0; o >>= 1) {
-          al += __shfl_xor_sync(0xFFFFFFFFu, al, o);
-          be += __shfl_xor_sync(0xFFFFFFFFu, be, o);
-          ga += __shfl_xor_sync(0xFFFFFFFFu, ga, o);
-        }
-        if (act && ga != 0.f && fabsf(ga) > kJacobiTol * sqrtf(al * be)) {
-          const float zeta = (be - al) / (2.f * ga);
-          const float tt = copysignf(1.f, zeta) / (fabsf(zeta) + sqrtf(fmaf(zeta, zeta, 1.f)));
-          const float c = rsqrtf(fmaf(tt, tt, 1.f));
-          const float s = c * tt;
-          for (int r = l8; r < n; r += 8) {
-            const float a = X[p * ld + r], b = X[q * ld + r];
-            X[p * ld + r] = c * a - s * b;
-            X[q * ld + r] = s * a + c * b;
-          }
-          if (l8 == 0) rotated_sh = 1;
-        }
-      }
-      __syncthreads();
-    }
-    if (!rotated_sh) break;
-  }
-  if (t == 0 && sweep >= max_sweeps) report(dev_status, METIS_DEV_NUMERIC);
-  for (int j = t; j < n; j += nt) {
-    double s2 = 0.0;
-    for (int r = 0; r < n; ++r) s2 += static_cast<double>(X[j * ld + r]) * X[j * ld + r];
-    norms[j] = static_cast<float>(sqrt(s2));
-  }
-  __syncthreads();
-  for (int j = t; j < n; j += nt) {
-    const float sj = norms[j];
-    int rk = 0;
-    for (int i = 0; i < n; ++i) {
-      const float si = norms[i];
-      rk += (si > sj) || (si == sj && i < j);
-    }
-    eval[rk] = static_cast<double>(sj) * sj;
-    const float inv = sj > 0.f ? 1.f / sj : 0.f;
-    for (int r = 0; r < n; ++r) evec[perm[r] * n + rk] = X[j * ld + r] * inv;
-  }
-}
 
 // Factor matrices from the sorted eigen-decomposition of the core Gram:
 // Mu = W_k (lp x k), Mv = W_k diag(1/sigma) (0 where sigma is negligible),
@@ -511,19 +427,21 @@ int64_t apply_blocks(int64_t rows) { return (rows + kApplyRows - 1) / kApplyRows
 void launch_gram(const float* partial, int splits, int64_t rows, int lp, float* Y, double* gpart, double* G,
                  cudaStream_t s) {
   const int nb = static_cast<int>(gram_blocks(rows));
-  gram_kernel<<<nb, 256, kRowsPerBlock * (lp + 1) * sizeof(float), s>>>(partial, splits, rows, lp, Y, gpart);
+  const int threads = (kRowsPerBlock * (lp / 4) + 31) / 32 * 32;  // lp <= 112: at most 896
+  gram_kernel<<<nb, threads, kRowsPerBlock * (lp + 1) * sizeof(float), s>>>(partial, splits, rows, lp, Y, gpart);
   launch_gram_reduce(gpart, nb, lp, G, s);
 }
 
 void launch_gram_reduce(const double* gpart, int nblocks, int lp, double* G, cudaStream_t s) {
   const int n2 = lp * lp;
-  gram_reduce_kernel<<<(n2 + 7) / 8, 256, 0, s>>>(gpart, nblocks, n2, G);
+  gram_reduce_kernel<<<(n2 + 31) / 32, 32 * kReduceGroups, 0, s>>>(gpart, nblocks, n2, G);
 }
 
 void launch_cholesky_inv(const double* G, int lp, float* Rinv, cudaStream_t s) {
-  const size_t smem = (2 * static_cast<size_t>(lp) * (lp + 1) + 3 * lp) * sizeof(double);
+  // L, buf x2, invd, sqd, diag0, X, T
+  const size_t smem = ((2 * static_cast<size_t>(lp) + 16) * (lp + 1) + 5 * lp) * sizeof(double);
   if (!ensure_smem(reinterpret_cast<const void*>(cholesky_inv_kernel), smem)) return;
-  cholesky_inv_kernel<<<1, 1024, smem, s>>>(G, lp, Rinv);
+  cholesky_inv_kernel<<<1, kSmallThreads, smem, s>>>(G, lp, Rinv);
 }
 
 void launch_apply(const ApplyArgs& a, cudaStream_t s) {
@@ -531,14 +449,6 @@ void launch_apply(const ApplyArgs& a, cudaStream_t s) {
                        kApplyRows * (a.kout + 1)) * sizeof(float);
   if (!ensure_smem(reinterpret_cast<const void*>(apply_kernel), smem)) return;
   apply_kernel<<<static_cast<unsigned>(apply_blocks(a.rows)), 256, smem, s>>>(a);
-}
-
-void launch_jacobi(const double* C, int n, int max_sweeps, double* eval, float* evec, int32_t* dev_status,
-                   cudaStream_t s) {
-  const size_t smem = static_cast<size_t>(n) * (n + 1) * sizeof(double) + static_cast<size_t>(n) * (n + 1) * sizeof(float) +
-                      2 * static_cast<size_t>(n) * sizeof(int);
-  if (!ensure_smem(reinterpret_cast<const void*>(core_eig_kernel), smem)) return;
-  core_eig_kernel<<<1, 1024, smem, s>>>(C, n, max_sweeps, eval, evec, dev_status);
 }
 
 void launch_factor_mats(const double* eval, const float* evec, int lp, int k, float* Mu, float* Mv, float* S,

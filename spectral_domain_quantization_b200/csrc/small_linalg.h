@@ -34,9 +34,14 @@ void launch_gram_reduce(const double* gpart, int nblocks, int lp, double* G, cud
 // Rinv (lp x lp float, upper triangular) with G = R^T R, dropped pivots -> 0.
 void launch_cholesky_inv(const double* G, int lp, float* Rinv, cudaStream_t s);
 void launch_apply(const ApplyArgs& a, cudaStream_t s);
-// Symmetric eigen-decomposition, eigenvalues descending; evec column j.
-void launch_jacobi(const double* C, int n, int max_sweeps, double* eval, float* evec, int32_t* dev_status,
-                   cudaStream_t s);
+// Symmetric eigen-decomposition of C (n x n float64, n <= 112, a multiple of
+// 16), eigenvalues descending in eval, evec[i * n + j] = component i of
+// eigenvector j (core_eig.cu).  ws: core_eig_workspace(n) bytes of scratch;
+// max_iters caps the multisection rounds per eigenvalue (METIS_DEV_NUMERIC
+// when reached).
+size_t core_eig_workspace(int n);
+void launch_core_eig(double* C, int n, int max_iters, double* eval, float* evec, double* ws, int32_t* dev_status,
+                     cudaStream_t s);
 void launch_factor_mats(const double* eval, const float* evec, int lp, int k, float* Mu, float* Mv, float* S,
                         cudaStream_t s);
 int64_t sign_blocks(int64_t rows);
