@@ -51,6 +51,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--profile-steps", type=int, default=0,
+                    help="run this many eager steps (no graphs, no timing) and exit: the command profiled by ncu")
     return ap.parse_args()
 
 
@@ -367,8 +369,31 @@ def run_ours(args, rank, world, local):
     del g_step, g_split, g_quant, g_gemm, g_plain
 
 
+def run_profile(args, local):
+    """The step, eagerly and untimed: a short launch list for profilers."""
+    import torch
+    from spectral_domain_quantization_b200 import api, inputs
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    data = inputs.make("layer_4096")
+    W = torch.from_numpy(data["W"].data.view(np.int16)).view(torch.bfloat16).to(dev)
+    X = torch.from_numpy(data["X"].data.view(np.int16)).view(torch.bfloat16).to(dev)
+    Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    for _ in range(args.profile_steps):
+        s = api.split(W, RANK_K, OVERSAMPLE, POWER_ITERS, SEED, "nv", rows=False, cols=True, factors=True,
+                      dev_status=status)
+        xq = api.quantize_fp4(X, "nv", 1)
+        api.linear_fwd(api.Operand(xq), s.operand("right"), M, N, K, Y=Y, dev_status=status)
+    torch.cuda.synchronize()
+    print(json.dumps({"profile_steps": args.profile_steps, "dev_status": int(status.item())}), flush=True)
+
+
 def main():
     args = parse()
+    if args.profile_steps > 0:
+        run_profile(args, int(os.environ.get("LOCAL_RANK", "0")))
+        return
     rank, world, local = dist_init()
     try:
         if args.impl == "reference":

@@ -148,91 +148,145 @@ MDEV int tri_element(int e, int n) {
   return (i << 8) | c;
 }
 
-constexpr int kSmallThreads = 1024;
-constexpr int kMaxOwn = 7;  // ceil(112 * 113 / 2 / 1024): lower-triangle elements per thread
+constexpr int kSmallThreads = 512;
+constexpr int kTile = 4;  // register tile edge and panel width of the Cholesky
 
 // G = L L^T (with drops), then Rinv = L^-T (upper triangular, float32).
-//  Cholesky (right-looking, one barrier per column): each thread keeps up to
-//  kMaxOwn lower-triangle elements in registers.  They are dealt out in
-//  reverse column-major order, so the elements still active at step j (those
-//  right of column j) are a prefix of that order and a warp whose share lies
-//  past it skips the slot.  Step j: every active (i, c) takes
-//  v -= v(i, j) v(c, j) / d_j with v(., j) the unscaled column j, published
-//  in shared memory at step j - 1; column j + 1 is then final and is
-//  published for step j + 1, and the owner of (j + 1, j + 1) forms the next
-//  pivot's 1/sqrt.
+//  Cholesky, right-looking by panels of 4 columns, two barriers per panel:
+//  thread T owns the 4 x 4 tile (I, J), I >= J, of the lower triangle in
+//  registers.  Panel K (columns 4K .. 4K+3, rows 4K .. lp-1) sits in shared
+//  memory; warp 0 factors it alone (a lane per row, the pivot row broadcast
+//  by shuffles, no block barrier); then every tile right of it takes the
+//  rank-4 update v -= L(I, K) L(J, K)^T and the tiles of column K + 1 write
+//  themselves into the next panel buffer.
 //  Inverse: X = L^-1 by 16 x 16 blocks (see below).
-__global__ void __launch_bounds__(kSmallThreads) cholesky_inv_kernel(const double* G, int lp, float* Rinv) {
+__global__ void __launch_bounds__(kSmallThreads, 1) cholesky_inv_kernel(const double* G, int lp, float* Rinv) {
   extern __shared__ double sm[];
   const int ld = lp + 1;
-  double* buf = sm;               // 2 x lp: the published column
-  double* invd = buf + 2 * lp;    // lp: 1/sqrt(pivot) (0 when dropped)
+  double* pan = sm;               // 2 x lp x 4: panel buffers
+  double* invd = pan + 8 * lp;    // lp: 1/sqrt(pivot) (0 when dropped)
   double* sqd = invd + lp;        // lp: sqrt(pivot) (0 when dropped)
   double* diag0 = sqd + lp;       // lp: the original diagonal (drop rule)
   double* L = diag0 + lp;         // lp x ld: final L
   const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-  const int ntri = lp * (lp + 1) / 2;
-  int own[kMaxOwn];
-  double v[kMaxOwn];
+  const int nb = lp / kTile;
+  const int ntiles = nb * (nb + 1) / 2;
+  int I = 0, J = 0;
+  double v[kTile][kTile];
+  const bool owner = t < ntiles;
+  if (owner) {
+    const int ij = tri_element(t, nb);
+    I = ij >> 8;
+    J = ij & 255;
 #pragma unroll
-  for (int u = 0; u < kMaxOwn; ++u) {
-    const int er = kSmallThreads * u + t;  // position in reverse column-major order
-    own[u] = er < ntri ? tri_element(ntri - 1 - er, lp) : -1;
-    v[u] = 0.0;
-    if (own[u] >= 0) {
-      const int i = own[u] >> 8, c = own[u] & 255;
-      v[u] = G[i * lp + c];
-      if (i == c) diag0[i] = v[u];
-      if (c == 0) buf[i] = v[u];
+    for (int a = 0; a < kTile; ++a)
+#pragma unroll
+      for (int b = 0; b < kTile; ++b) v[a][b] = G[(kTile * I + a) * lp + kTile * J + b];
+    if (I == J) {
+#pragma unroll
+      for (int a = 0; a < kTile; ++a) diag0[kTile * I + a] = v[a][a];
+    }
+    if (J == 0) {
+#pragma unroll
+      for (int a = 0; a < kTile; ++a)
+#pragma unroll
+        for (int b = 0; b < kTile; ++b) pan[(kTile * I + a) * kTile + b] = v[a][b];
     }
   }
-  if (t == 0) {
-    const double d = G[0];
-    const double r = d > 0.0 ? rsqrt(d) : 0.0;
-    invd[0] = r;
-    sqd[0] = d * r;
-  }
   __syncthreads();
-  for (int j = 0; j + 1 < lp; ++j) {
-    const double* cur = buf + (j & 1) * lp;
-    double* nxt = buf + ((j + 1) & 1) * lp;
-    const double inv2 = invd[j] * invd[j];
-    const int active = (lp - j - 1) * (lp - j) / 2;  // elements right of column j
+  for (int K = 0; K < nb; ++K) {
+    double* P = pan + (K & 1) * 4 * lp;
+    double* Pn = pan + ((K + 1) & 1) * 4 * lp;
+    const int r0 = kTile * K;
+    if (warp == 0) {
+      double pr[4][kTile];  // rows r0 + lane + 32 q
 #pragma unroll
-    for (int u = 0; u < kMaxOwn; ++u) {
-      if (kSmallThreads * u + 32 * warp >= active) break;  // warp-uniform
-      if (kSmallThreads * u + t < active) {
-        const int i = own[u] >> 8, c = own[u] & 255;
-        v[u] -= cur[i] * cur[c] * inv2;
-        if (c == j + 1) {
-          nxt[i] = v[u];
-          if (i == c) {
-            const bool drop = !(diag0[c] > 0.0) || !(v[u] > kDropTol * diag0[c]);
-            const double r = drop ? 0.0 : rsqrt(v[u]);
-            invd[c] = r;
-            sqd[c] = v[u] * r;
+      for (int q = 0; q < 4; ++q) {
+        const int row = r0 + lane + 32 * q;
+#pragma unroll
+        for (int c = 0; c < kTile; ++c) pr[q][c] = row < lp ? P[row * kTile + c] : 0.0;
+      }
+      double rinv[kTile], rsq[kTile];
+#pragma unroll
+      for (int c = 0; c < kTile; ++c) {
+        const int gc = r0 + c;
+        const double d = __shfl_sync(0xFFFFFFFFu, pr[0][c], c);  // row gc lives in lane c, q = 0
+        const bool drop = !(diag0[gc] > 0.0) || !(d > kDropTol * diag0[gc]);
+        rinv[c] = drop ? 0.0 : rsqrt(d);
+        rsq[c] = d * rinv[c];
+        const double inv2 = rinv[c] * rinv[c];
+        double prow[kTile];
+#pragma unroll
+        for (int cc = 0; cc < kTile; ++cc) prow[cc] = __shfl_sync(0xFFFFFFFFu, pr[0][cc], c) * inv2;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int row = r0 + lane + 32 * q;
+          if (row > gc) {
+#pragma unroll
+            for (int cc = c + 1; cc < kTile; ++cc) pr[q][cc] = fma(-pr[q][c], prow[cc], pr[q][cc]);
+          }
+        }
+      }
+      if (lane < kTile) {
+        double ri = rinv[0], rs = rsq[0];
+#pragma unroll
+        for (int c = 1; c < kTile; ++c) {
+          ri = lane == c ? rinv[c] : ri;
+          rs = lane == c ? rsq[c] : rs;
+        }
+        invd[r0 + lane] = ri;
+        sqd[r0 + lane] = rs;
+      }
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int row = r0 + lane + 32 * q;
+        if (row < lp) {
+#pragma unroll
+          for (int c = 0; c < kTile; ++c) {
+            const int gc = r0 + c;
+            const double l = row == gc ? rsq[c] : (row > gc ? pr[q][c] * rinv[c] : 0.0);
+            P[row * kTile + c] = l;
+            L[row * ld + gc] = l;
           }
         }
       }
     }
     __syncthreads();
-  }
+    if (owner && J > K) {
+      double li[kTile][kTile], lj[kTile][kTile];
 #pragma unroll
-  for (int u = 0; u < kMaxOwn; ++u) {
-    if (own[u] >= 0) {
-      const int i = own[u] >> 8, c = own[u] & 255;
-      L[i * ld + c] = i == c ? sqd[c] : v[u] * invd[c];
+      for (int a = 0; a < kTile; ++a)
+#pragma unroll
+        for (int c = 0; c < kTile; ++c) {
+          li[a][c] = P[(kTile * I + a) * kTile + c];
+          lj[a][c] = P[(kTile * J + a) * kTile + c];
+        }
+#pragma unroll
+      for (int a = 0; a < kTile; ++a)
+#pragma unroll
+        for (int b = 0; b < kTile; ++b) {
+          double s = v[a][b];
+#pragma unroll
+          for (int c = 0; c < kTile; ++c) s = fma(-li[a][c], lj[b][c], s);
+          v[a][b] = s;
+        }
+      if (J == K + 1) {
+#pragma unroll
+        for (int a = 0; a < kTile; ++a)
+#pragma unroll
+          for (int b = 0; b < kTile; ++b) Pn[(kTile * I + a) * kTile + b] = v[a][b];
+      }
     }
+    __syncthreads();
   }
-  __syncthreads();
   // X = L^-1 by 16 x 16 blocks: the diagonal blocks are inverted by one warp
   // each (a lane per column, forward substitution), then block row bi is
   //   T = sum_{k < bi} L(bi, k) X(k, j)   and   X(bi, j) = -X(bi, bi) T
   // for all j < bi at once (two barriers per block row).
   double* X = L + lp * ld;        // lp x ld
   double* T = X + lp * ld;        // 16 x ld
-  const int nb = lp / 16;
-  if (warp < nb && lane < 16) {
+  const int nb16 = lp / 16;
+  if (warp < nb16 && lane < 16) {
     const int o = 16 * warp, j = lane;
     double x[16];
 #pragma unroll
@@ -246,13 +300,18 @@ __global__ void __launch_bounds__(kSmallThreads) cholesky_inv_kernel(const doubl
     }
   }
   __syncthreads();
-  for (int bi = 1; bi < nb; ++bi) {
+  for (int bi = 1; bi < nb16; ++bi) {
     const int o = 16 * bi;
     for (int e = t; e < 16 * o; e += kSmallThreads) {
       const int r = e / o, c = e - r * o;
-      double sum = 0.0;
-      for (int m = c; m < o; ++m) sum += L[(o + r) * ld + m] * X[m * ld + c];
-      T[r * ld + c] = sum;
+      double s4[4] = {0.0, 0.0, 0.0, 0.0};
+      int m = c;
+      for (; m + 3 < o; m += 4) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) s4[u] = fma(L[(o + r) * ld + m + u], X[(m + u) * ld + c], s4[u]);
+      }
+      for (; m < o; ++m) s4[0] = fma(L[(o + r) * ld + m], X[m * ld + c], s4[0]);
+      T[r * ld + c] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
     }
     __syncthreads();
     for (int e = t; e < 16 * o; e += kSmallThreads) {
@@ -358,58 +417,68 @@ __global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) {
 // S = sigma_k.
 __global__ void factor_mats_kernel(const double* eval, const float* evec, int lp, int k, float* Mu, float* Mv,
                                    float* S) {
-  const double top = eval[0] > 0.0 ? sqrt(eval[0]) : 0.0;
-  for (int e = threadIdx.x; e < lp * k; e += blockDim.x) {
-    const int i = e / k, j = e - i * k;
-    const double ev = eval[j];
-    const double sigma = ev > 0.0 ? sqrt(ev) : 0.0;
-    const float w = evec[i * lp + j];
-    Mu[e] = w;
-    Mv[e] = (sigma > 1e-12 * top && sigma > 0.0) ? static_cast<float>(w / sigma) : 0.f;
-  }
-  for (int j = threadIdx.x; j < k; j += blockDim.x) {
-    const double ev = eval[j];
-    S[j] = static_cast<float>(ev > 0.0 ? sqrt(ev) : 0.0);
-  }
+  // block i, thread j: entry (i, j) of Mu and Mv
+  const int i = blockIdx.x, j = threadIdx.x;
+  if (j >= k) return;
+  const double e0 = eval[0], ev = eval[j];
+  const double top = e0 > 0.0 ? sqrt(e0) : 0.0;
+  const double sigma = ev > 0.0 ? sqrt(ev) : 0.0;
+  const float w = evec[i * lp + j];
+  Mu[i * k + j] = w;
+  Mv[i * k + j] = (sigma > 1e-12 * top && sigma > 0.0) ? static_cast<float>(w / sigma) : 0.f;
+  if (i == 0) S[j] = static_cast<float>(sigma);
 }
 
-// Per row block: for each column, the largest |U| and its lowest row index.
-__global__ void colmax_kernel(const float* U, int64_t rows, int k, float* bmax, int64_t* bidx) {
+// Per block of kSignRows rows: for each column, the largest |U| and its lowest
+// row index.
+constexpr int kSignRows = 32;
+__global__ void colmax_kernel(const float* __restrict__ U, int64_t rows, int k, float* bmax, int64_t* bidx) {
   const int j = threadIdx.x;
   if (j >= k) return;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * 256;
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kSignRows;
+  float v[kSignRows];
+#pragma unroll
+  for (int r = 0; r < kSignRows; ++r) v[r] = r0 + r < rows ? fabsf(U[(r0 + r) * k + j]) : -1.f;
   float best = -1.f;
-  int64_t bi = 0;
-  for (int64_t r = r0; r < imin64(r0 + 256, rows); ++r) {
-    const float v = fabsf(U[r * k + j]);
-    if (v > best) {
-      best = v;
-      bi = r;
+  int64_t bi = r0;
+#pragma unroll
+  for (int r = 0; r < kSignRows; ++r) {
+    if (v[r] > best) {
+      best = v[r];
+      bi = r0 + r;
     }
   }
   bmax[static_cast<int64_t>(blockIdx.x) * k + j] = best;
   bidx[static_cast<int64_t>(blockIdx.x) * k + j] = bi;
 }
 
-__global__ void sign_kernel(const float* U, const float* bmax, const int64_t* bidx, int nblocks, int k, float* sign) {
+__global__ void sign_kernel(const float* __restrict__ U, const float* __restrict__ bmax,
+                            const int64_t* __restrict__ bidx, int nblocks, int k, float* sign) {
   const int j = threadIdx.x;
   if (j >= k) return;
   float best = -1.f;
-  int64_t bi = 0;
+  int bb = 0;
+#pragma unroll 8
   for (int b = 0; b < nblocks; ++b) {
     const float v = bmax[static_cast<int64_t>(b) * k + j];
     if (v > best) {
       best = v;
-      bi = bidx[static_cast<int64_t>(b) * k + j];
+      bb = b;
     }
   }
+  const int64_t bi = bidx[static_cast<int64_t>(bb) * k + j];
   sign[j] = U[bi * k + j] < 0.f ? -1.f : 1.f;
 }
 
-__global__ void flip_kernel(float* X, int64_t rows, int k, const float* sign) {
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < rows * k;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    X[e] *= sign[e % k];
+// U (m x k) and V (n x k) columns times sign, one launch.
+__global__ void flip_kernel(float* U, int64_t mk, float* V, int64_t nk, int k, const float* sign) {
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < mk + nk;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    if (e < mk)
+      U[e] *= sign[e % k];
+    else
+      V[e - mk] *= sign[(e - mk) % k];
+  }
 }
 
 int blocks(int64_t n, int sms) {
@@ -438,8 +507,8 @@ void launch_gram_reduce(const double* gpart, int nblocks, int lp, double* G, cud
 }
 
 void launch_cholesky_inv(const double* G, int lp, float* Rinv, cudaStream_t s) {
-  // L, buf x2, invd, sqd, diag0, X, T
-  const size_t smem = ((2 * static_cast<size_t>(lp) + 16) * (lp + 1) + 5 * lp) * sizeof(double);
+  // panels x2, invd, sqd, diag0, L, X, T
+  const size_t smem = ((2 * static_cast<size_t>(lp) + 16) * (lp + 1) + 11 * lp) * sizeof(double);
   if (!ensure_smem(reinterpret_cast<const void*>(cholesky_inv_kernel), smem)) return;
   cholesky_inv_kernel<<<1, kSmallThreads, smem, s>>>(G, lp, Rinv);
 }
@@ -453,18 +522,17 @@ void launch_apply(const ApplyArgs& a, cudaStream_t s) {
 
 void launch_factor_mats(const double* eval, const float* evec, int lp, int k, float* Mu, float* Mv, float* S,
                         cudaStream_t s) {
-  factor_mats_kernel<<<1, 256, 0, s>>>(eval, evec, lp, k, Mu, Mv, S);
+  factor_mats_kernel<<<lp, (k + 31) / 32 * 32, 0, s>>>(eval, evec, lp, k, Mu, Mv, S);
 }
 
-int64_t sign_blocks(int64_t rows) { return (rows + 255) / 256; }
+int64_t sign_blocks(int64_t rows) { return (rows + kSignRows - 1) / kSignRows; }
 
 void launch_signs(float* U, int64_t m, float* V, int64_t n, int k, float* bmax, int64_t* bidx, float* sign, int sms,
                   cudaStream_t s) {
   const int nb = static_cast<int>(sign_blocks(m));
   colmax_kernel<<<nb, 128, 0, s>>>(U, m, k, bmax, bidx);
   sign_kernel<<<1, 128, 0, s>>>(U, bmax, bidx, nb, k, sign);
-  flip_kernel<<<blocks(m * k, sms), 256, 0, s>>>(U, m, k, sign);
-  flip_kernel<<<blocks(n * k, sms), 256, 0, s>>>(V, n, k, sign);
+  flip_kernel<<<blocks(m * k + n * k, sms), 256, 0, s>>>(U, m * k, V, n * k, k, sign);
 }
 
 }  // namespace metis
