@@ -134,13 +134,15 @@ def _dtype_code(t):
 
 
 class _Workspace:
-    """Grow-only workspace per device (allocated by torch, the caller side)."""
+    """Grow-only workspace per device and stream (allocated by torch, the
+    caller side), so that calls enqueued on different streams never share
+    scratch memory."""
 
     def __init__(self):
         self.buf = {}
 
     def get(self, nbytes, device):
-        key = torch.device(device).index
+        key = (torch.device(device).index, torch.cuda.current_stream(device).cuda_stream)
         cur = self.buf.get(key)
         if cur is None or cur.numel() < nbytes:
             cur = torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)

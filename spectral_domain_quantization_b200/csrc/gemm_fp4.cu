@@ -35,18 +35,17 @@ namespace metis {
 
 namespace {
 
-constexpr int kStages = 4;
 constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
 
-template <int BN>
+template <int BN, int STAGES>
 struct Smem {
   static constexpr int kA = 128 * 128;
   static constexpr int kB = BN * 128;
   static constexpr int kSFA = 2048;
-  static constexpr int kSFB = 4096;
+  static constexpr int kSFB = BN > 128 ? 4096 : 2048;
   static constexpr int kStage = kA + kB + kSFA + kSFB;
-  static constexpr int kBytes = kStages * kStage + 1024 /*align*/ + 256 /*barriers*/;
+  static constexpr int kBytes = STAGES * kStage + 1024 /*align*/ + 256 /*barriers*/;
 };
 
 MDEV bool wait_ns(uint64_t* bar, uint32_t parity, uint64_t ns) {
@@ -57,12 +56,15 @@ MDEV bool wait_ns(uint64_t* bar, uint32_t parity, uint64_t ns) {
   return true;
 }
 
-template <int BN>
-__global__ void __launch_bounds__(kThreads, 1)
+// BN: MMA N; STAGES: shared-memory ring depth; CTAS: CTAs per SM (2 halves
+// the TMEM allocation and lets one CTA's epilogue overlap the other's MMAs).
+template <int BN, int STAGES, int CTAS>
+__global__ void __launch_bounds__(kThreads, CTAS)
     gemm_fp4_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmLA,
                     const __grid_constant__ CUtensorMap tmLB) {
-  using S = Smem<BN>;
+  using S = Smem<BN, STAGES>;
+  constexpr int kStages = STAGES;
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * S::kStage);
@@ -80,7 +82,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr int kBHalves = BN > 128 ? 2 : 1;      // 128-row scale chunk groups of B
   const int sfb_cols = 4 * atoms_per_kt * kBHalves;
   const int sf_stage_cols = sfa_cols + sfb_cols;
-  constexpr uint32_t kTmemCols = 512;
+  constexpr uint32_t kTmemCols = CTAS == 2 ? 256 : 512;
+  constexpr uint32_t kSfBase = CTAS == 2 ? BN : 256;  // TMEM columns of the accumulator
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
@@ -200,7 +203,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (it < kt1) {
             uint8_t* sSFA = sB + S::kB;
             uint8_t* sSFB = sSFA + S::kSFA;
-            const uint32_t sfa_t = tmem + 256 + stage * sf_stage_cols;
+            const uint32_t sfa_t = tmem + kSfBase + stage * sf_stage_cols;
             const uint32_t sfb_t = sfa_t + sfa_cols + sfb_off;
             for (int a = 0; a < atoms_per_kt; ++a) {
               tc_cp_32x128b_warpx4(sfa_t + 4 * a, make_sdesc(smem_u32(sSFA + 512 * a), 0, 128, kSwizzleNone));
@@ -350,12 +353,15 @@ __global__ void splitk_reduce_kernel(const float* partial, int splits, int64_t M
   }
 }
 
-template <int BN>
+template <int BN, int STAGES, int CTAS>
 cudaError_t launch_bn(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& la,
-                      const CUtensorMap& lb, int grid, cudaStream_t s) {
-  const int bytes = Smem<BN>::kBytes;
-  if (!ensure_smem(reinterpret_cast<const void*>(gemm_fp4_kernel<BN>), bytes)) return cudaErrorInvalidValue;
-  gemm_fp4_kernel<BN><<<grid, kThreads, bytes, s>>>(p, a, b, la, lb);
+                      const CUtensorMap& lb, int tiles, cudaStream_t s) {
+  const int bytes = Smem<BN, STAGES>::kBytes;
+  if (!ensure_smem(reinterpret_cast<const void*>(gemm_fp4_kernel<BN, STAGES, CTAS>), bytes))
+    return cudaErrorInvalidValue;
+  const int slots = device_sm_count() * CTAS;
+  const int grid = tiles < slots ? tiles : slots;
+  gemm_fp4_kernel<BN, STAGES, CTAS><<<grid, kThreads, bytes, s>>>(p, a, b, la, lb);
   return cudaGetLastError();
 }
 
@@ -398,6 +404,13 @@ metis_status run_gemm_fp4(const GemmCall& g, cudaStream_t s) {
   p.vec_ok = (g.ldc % 4 == 0) && ((reinterpret_cast<uintptr_t>(g.C) & 15u) == 0);
   p.dev_status = g.dev_status;
   p.splits = g.splits < 1 ? 1 : g.splits;
+  if (p.splits > p.num_kt) p.splits = p.num_kt;
+  {
+    // every split must own at least one K tile (an empty split would leave
+    // its accumulator unwritten): use the fewest splits of the same length
+    const int per = (p.num_kt + p.splits - 1) / p.splits;
+    p.splits = (p.num_kt + per - 1) / per;
+  }
   p.partial = g.partial;
   if (p.splits > 1 && !p.partial) return METIS_ERR_ARG;
   if (p.splits > 1 && p.lr_chunks) return METIS_ERR_ARG;
@@ -413,14 +426,13 @@ metis_status run_gemm_fp4(const GemmCall& g, cudaStream_t s) {
     mlb = mb;
   }
   const int tiles = static_cast<int>(((g.M + 127) / 128) * ((g.N + bn - 1) / bn)) * p.splits;
-  const int grid = tiles < device_sm_count() ? tiles : device_sm_count();
   cudaError_t e;
   if (bn == 256)
-    e = launch_bn<256>(p, ma, mb, mla, mlb, grid, s);
+    e = launch_bn<256, 4, 1>(p, ma, mb, mla, mlb, tiles, s);
   else if (bn == 128)
-    e = launch_bn<128>(p, ma, mb, mla, mlb, grid, s);
+    e = launch_bn<128, 4, 1>(p, ma, mb, mla, mlb, tiles, s);
   else if (bn == 64)
-    e = launch_bn<64>(p, ma, mb, mla, mlb, grid, s);
+    e = launch_bn<64, 4, 1>(p, ma, mb, mla, mlb, tiles, s);
   else
     return METIS_ERR_ARG;
   if (e != cudaSuccess) return fail(METIS_ERR_CUDA, "gemm_fp4 launch", cudaGetErrorString(e));

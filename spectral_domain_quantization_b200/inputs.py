@@ -126,36 +126,41 @@ def averis_activation(m, n, seed, stream, dtype="bf16"):
 # workloads
 # --------------------------------------------------------------------------
 
-def make(name, scale=None):
+def make(name, scale=None, keys=None):
     """Generate a workload's inputs.  ``scale`` optionally overrides sizes
-    (dict of M/K/N) to get a smaller case with the same recipe."""
+    (dict of M/K/N) to get a smaller case with the same recipe; ``keys``
+    optionally limits the matrices generated (each matrix has its own seeded
+    stream, so the selection does not change their values)."""
     cfg = dict(WORKLOADS[name])
     if scale:
         cfg.update(scale)
     s = cfg["seed"]
     M, K, N = cfg["M"], cfg["K"], cfg["N"]
-    out = dict(cfg=cfg)
     if name == "tiny_256":
-        out["W"] = planted(K, N, [4.0 / i for i in range(1, 17)], 0.02, s, 1, "f32")
-        out["X"] = gaussian((M, K), 1.0, s, 2, "f32")
+        gen = {"W": lambda: planted(K, N, [4.0 / i for i in range(1, 17)], 0.02, s, 1, "f32"),
+               "X": lambda: gaussian((M, K), 1.0, s, 2, "f32")}
     elif name == "layer_4096":
-        out["W"] = planted(K, N, [8.0 / i for i in range(1, 257)], 0.02, s, 1)
-        out["X"] = gaussian((M, K), 1.0, s, 2)
+        gen = {"W": lambda: planted(K, N, [8.0 / i for i in range(1, 257)], 0.02, s, 1),
+               "X": lambda: gaussian((M, K), 1.0, s, 2)}
     elif name == "averis_32768":
-        out["X"] = averis_activation(M, K, s, 1)
-        out["W"] = gaussian((K, N), 0.02, s, 2)
-        out["dY"] = gaussian((M, N), 0.01, s, 3)
+        gen = {"X": lambda: averis_activation(M, K, s, 1),
+               "W": lambda: gaussian((K, N), 0.02, s, 2),
+               "dY": lambda: gaussian((M, N), 0.01, s, 3)}
     elif name == "llama3_8b_mlp":
         sig = [8.0 / i for i in range(1, 257)]
-        out["W"] = planted(K, N, sig, 0.02, s, 1)          # gate / up projection
-        out["W_down"] = planted(N, K, sig, 0.02, s, 2)     # down projection
-        out["X"] = gaussian((M, K), 1.0, s, 3)
-        out["H"] = gaussian((M, N), 1.0, s, 4)
-        out["dY"] = gaussian((M, N), 0.01, s, 5)           # gradient of gate / up output
-        out["dY_down"] = gaussian((M, K), 0.01, s, 6)      # gradient of down output
+        gen = {"W": lambda: planted(K, N, sig, 0.02, s, 1),          # gate / up projection
+               "W_down": lambda: planted(N, K, sig, 0.02, s, 2),     # down projection
+               "X": lambda: gaussian((M, K), 1.0, s, 3),
+               "H": lambda: gaussian((M, N), 1.0, s, 4),
+               "dY": lambda: gaussian((M, N), 0.01, s, 5),           # gradient of gate / up output
+               "dY_down": lambda: gaussian((M, K), 0.01, s, 6)}      # gradient of down output
     elif name == "sampled_65536":
-        out["A"] = planted(M, K, [50.0 * i ** -1.5 for i in range(1, 33)], 1.0, s, 1)
-        out["W"] = gaussian((K, N), 0.02, s, 2)
+        gen = {"A": lambda: planted(M, K, [50.0 * i ** -1.5 for i in range(1, 33)], 1.0, s, 1),
+               "W": lambda: gaussian((K, N), 0.02, s, 2)}
     else:
         raise KeyError(name)
+    out = dict(cfg=cfg)
+    for key, fn in gen.items():
+        if keys is None or key in keys:
+            out[key] = fn()
     return out

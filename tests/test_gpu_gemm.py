@@ -98,6 +98,22 @@ def test_both_split_product(fmt):
     assert rel_fro(y.cpu().numpy(), want) < TOL
 
 
+def test_both_split_long_contraction():
+    # K = 14336 (56 K tiles) with few output tiles: the low-rank products run
+    # split-K with a split count that does not divide the K tiles evenly
+    fmt = "nv"
+    M, N, K, ka, kb = 128, 4096, 14336, 64, 64
+    qra, rra = _q(_rand((M, K), 51, 0.2), fmt, 1)
+    qPa, rPa, qFa, rFa, Sa = _factors(M, K, ka, fmt, 52)
+    qrb, rrb = _q(_rand((K, N), 53, 0.02), fmt, 0)
+    qPb, rPb, qFb, rFb, Sb = _factors(N, K, kb, fmt, 54)
+    y = api.linear_fwd(api.Operand(qra, ka, qPa, qFa, torch.from_numpy(Sa).cuda()),
+                       api.Operand(qrb, kb, qPb, qFb, torch.from_numpy(Sb).cuda()), M, N, K)
+    torch.cuda.synchronize()
+    want = gemm.gemm(gemm.Operand(rra, ka, rPa, rFa, Sa), gemm.Operand(rrb, kb, rPb, rFb, Sb))
+    assert rel_fro(y.cpu().numpy(), want) < TOL
+
+
 def test_averis_ones_factors():
     # left operand X = 1 mu^T + R (F = ones), right operand plain; and the dW
     # form X^T dY with both means (P = ones on both sides)
