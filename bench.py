@@ -36,6 +36,10 @@ sys.path.insert(0, ROOT)
 M, K, N = 8192, 4096, 4096
 RANK_K, OVERSAMPLE, POWER_ITERS, SEED = 64, 16, 1, 0
 FLOPS = 2.0 * M * N * K
+# DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
+# the plain-operand FP4 GEMM, from one ncu capture of the current kernel; to
+# be set to None whenever the kernel changes after that capture.
+GEMM_NCU_DRAM_BYTES = 34.902272e6 + 21.137920e6
 METRIC = "FP4 split-linear eff. TFLOPS & % of FP4 peak; split+quantize us/layer"
 CONFIG = {"workload": "layer_4096: W bf16 4096x4096 planted spectrum + X bf16 8192x4096, "
                       "split k=64 p=16 q=1 Gaussian, NVFP4, forward",
@@ -363,10 +367,10 @@ def run_ours(args, rank, world, local):
             "split_quantize_us_per_layer": (ms_split + ms_quant) * 1e3,
             "breakdown_us": {"split_W": ms_split * 1e3, "quantize_X": ms_quant * 1e3,
                              "linear_fwd": ms_gemm * 1e3, "fp4_gemm_kernel": ms_plain * 1e3},
-            "roofline": {"kernel": "gemm_fp4_kernel<256> (8192x4096x4096 NVFP4)", "bound": "tensor",
+            "roofline": {"kernel": "gemm_fp4_kernel<256,4,1> (8192x4096x4096 NVFP4)", "bound": "tensor",
                          "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s", "frac": achieved / fp4_peak,
                          "peak_source": f"{peak_kind} bf16 {bf16_tf} TFLOP/s x 4 (nominal FP4/bf16 ratio)",
-                         "traffic": None},
+                         "traffic": GEMM_NCU_DRAM_BYTES},
             "cpu_baseline": cpu,
             "e2e": e2e,
             "gpu_launches": launches,
