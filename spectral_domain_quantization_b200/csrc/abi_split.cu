@@ -148,7 +148,7 @@ SplitBuffers carve(const SplitPlan& p, int64_t lda, Carver& ws) {
   b.u_lo = ws.take<__nv_bfloat16>(static_cast<size_t>(p.m) * p.kp);
   b.w_hi = ws.take<__nv_bfloat16>(static_cast<size_t>(p.n) * p.kp);
   b.w_lo = ws.take<__nv_bfloat16>(static_cast<size_t>(p.n) * p.kp);
-  b.amax = ws.take<unsigned>(1);
+  b.amax = ws.take<unsigned>(3);
   return b;
 }
 
@@ -243,7 +243,15 @@ metis_status range_and_core(const SplitPlan& p, const SplitBuffers& b, const Sou
                             int max_iters, int32_t* dev_status, cudaStream_t s) {
   const int lp = p.lp;
   METIS_TRY(skinny(src, 0, b.omt, p.ld_n, 1, lp, p.split_m, b.part, dev_status, s));
-  METIS_TRY(cholqr(b, p.split_m, src.rows, lp, b.Qm, p.ld_m, power_iters > 0 ? 1 : 2, s));
+  if (power_iters > 0) {
+    // A^T Y0 spans the same space as A^T orth(Y0): Y0 = A Omega goes to the
+    // next product as it is (its hi / lo transpose), and the next basis is
+    // orthonormalised
+    launch_sum_hilo(b.part, p.split_m, src.rows, lp, b.qt, p.ld_m, s);
+    METIS_TRY(step_status("sketch hi/lo"));
+  } else {
+    METIS_TRY(cholqr(b, p.split_m, src.rows, lp, b.Qm, p.ld_m, 2, s));
+  }
   for (int it = 0; it < power_iters; ++it) {
     METIS_TRY(skinny(src, 1, b.qt, p.ld_m, 2, lp, p.split_n, b.part, dev_status, s));
     METIS_TRY(cholqr(b, p.split_n, p.n, lp, b.Zn, p.ld_n, 1, s));
@@ -430,13 +438,15 @@ extern "C" metis_status metis_split(const void* A, int32_t dtype, int64_t m, int
   METIS_TRY(step_status("factors"));
   launch_signs(U, m, V, n, p.k, b.bmax, b.bidx, b.sign, sms, s);
   METIS_TRY(step_status("signs"));
-  if (U_q) METIS_TRY(enqueue_quantize(U, METIS_F32, m, p.k, p.k, 0, nullptr, U_q, nullptr, nullptr, ws, s));
-  if (V_q) METIS_TRY(enqueue_quantize(V, METIS_F32, n, p.k, p.k, 0, nullptr, V_q, nullptr, nullptr, ws, s));
+  const bool residual = R_rows || R_cols || R_f32;
+  cudaMemsetAsync(b.amax, 0, 3 * sizeof(unsigned), s);  // [0] |U|, [1] |V|, [2] |R|
+  launch_factor_finish(U, m, V, n, p.k, b.sign, S, p.kp, residual ? b.u_hi : nullptr, b.u_lo, b.w_hi, b.w_lo,
+                       b.amax, sms, s);
+  METIS_TRY(step_status("factor signs and operands"));
+  if (U_q) METIS_TRY(enqueue_quantize(U, METIS_F32, m, p.k, p.k, 0, nullptr, U_q, b.amax, nullptr, ws, s));
+  if (V_q) METIS_TRY(enqueue_quantize(V, METIS_F32, n, p.k, p.k, 0, nullptr, V_q, b.amax + 1, nullptr, ws, s));
 
-  if (R_rows || R_cols || R_f32) {
-    launch_hilo(U, m, p.k, nullptr, p.kp, b.u_hi, b.u_lo, sms, s);
-    launch_hilo(V, n, p.k, S, p.kp, b.w_hi, b.w_lo, sms, s);
-    METIS_TRY(step_status("residual operands"));
+  if (residual) {
     ResidualOperands ro{b.u_hi, b.u_lo, b.w_hi, b.w_lo};
     ResidualParams rp{};
     rp.A = A;
@@ -446,10 +456,9 @@ extern "C" metis_status metis_split(const void* A, int32_t dtype, int64_t m, int
     rp.lda = lda;
     rp.kp = p.kp;
     rp.fmt = prm->fmt;
-    rp.amax_bits = b.amax;
+    rp.amax_bits = b.amax + 2;
     rp.dev_status = dev_status;
     if (prm->fmt == METIS_NVFP4) {
-      cudaMemsetAsync(b.amax, 0, sizeof(unsigned), s);
       rp.mode = 0;
       METIS_TRY(run_residual_quant(rp, ro, s));
     }

@@ -398,21 +398,54 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
   if (threadIdx.x == 0 && *abort_flag) report(p.dev_status, METIS_DEV_TIMEOUT);
 }
 
-// U (rows x k) times diag(S) (optional) -> hi / lo bf16 [rows][kp], zero padded.
-__global__ void hilo_kernel(const float* X, int64_t rows, int k, const float* S, int kp, __nv_bfloat16* hi,
-                            __nv_bfloat16* lo) {
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < rows * kp;
+// The split's factors after the sign choice, in one pass over U (m x k) and
+// V (n x k): both are multiplied by sign (in place); U and V diag(S) are
+// written as bf16 hi / lo pairs [rows][kp] (zero padded, when hi pointers are
+// given), and the tensor maxima of |U| and |V| are atomically maxed into
+// amax[0], amax[1] (when given; the NVFP4 quantizer of U and V reads them).
+__global__ void __launch_bounds__(256) factor_finish_kernel(float* U, int64_t m, float* V, int64_t n, int k,
+                                                            const float* sign, const float* S, int kp,
+                                                            __nv_bfloat16* u_hi, __nv_bfloat16* u_lo,
+                                                            __nv_bfloat16* w_hi, __nv_bfloat16* w_lo,
+                                                            unsigned* amax) {
+  float mu = 0.f, mv = 0.f;
+  const int64_t eu = m * kp, total = eu + n * kp;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
        e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = e / kp;
-    const int c = static_cast<int>(e - r * kp);
-    float x = 0.f;
+    const bool isu = e < eu;
+    const int64_t el = isu ? e : e - eu;
+    const int64_t r = el / kp;
+    const int c = static_cast<int>(el - r * kp);
+    float w = 0.f;
     if (c < k) {
-      x = X[r * k + c];
-      if (S) x = __fmul_rn(x, S[c]);
+      float* x = (isu ? U : V) + r * k + c;
+      const float v = *x * sign[c];
+      *x = v;
+      if (isu) {
+        mu = fmaxf(mu, fabsf(v));
+        w = v;
+      } else {
+        mv = fmaxf(mv, fabsf(v));
+        w = __fmul_rn(v, S[c]);
+      }
     }
-    const __nv_bfloat16 h = __float2bfloat16_rn(x);
-    hi[e] = h;
-    lo[e] = __float2bfloat16_rn(__fsub_rn(x, __bfloat162float(h)));
+    __nv_bfloat16* hi = isu ? u_hi : w_hi;
+    __nv_bfloat16* lo = isu ? u_lo : w_lo;
+    if (hi) {
+      const __nv_bfloat16 h = __float2bfloat16_rn(w);
+      hi[el] = h;
+      lo[el] = __float2bfloat16_rn(__fsub_rn(w, __bfloat162float(h)));
+    }
+  }
+  if (amax) {
+    for (int o = 16; o > 0; o >>= 1) {
+      mu = fmaxf(mu, __shfl_xor_sync(0xFFFFFFFFu, mu, o));
+      mv = fmaxf(mv, __shfl_xor_sync(0xFFFFFFFFu, mv, o));
+    }
+    if ((threadIdx.x & 31) == 0) {
+      if (mu > 0.f) atomicMax(amax, __float_as_uint(mu));
+      if (mv > 0.f) atomicMax(amax + 1, __float_as_uint(mv));
+    }
   }
 }
 
@@ -436,11 +469,13 @@ CUresult map_a(CUtensorMap* m, const ResidualParams& p) {
 
 }  // namespace
 
-void launch_hilo(const float* X, int64_t rows, int k, const float* S, int kp, __nv_bfloat16* hi, __nv_bfloat16* lo,
-                 int sms, cudaStream_t s) {
-  int64_t b = (rows * kp + 255) / 256;
+void launch_factor_finish(float* U, int64_t m, float* V, int64_t n, int k, const float* sign, const float* S, int kp,
+                          __nv_bfloat16* u_hi, __nv_bfloat16* u_lo, __nv_bfloat16* w_hi, __nv_bfloat16* w_lo,
+                          unsigned* amax, int sms, cudaStream_t s) {
+  int64_t b = ((m + n) * kp + 255) / 256;
   if (b > sms * 8) b = sms * 8;
-  hilo_kernel<<<static_cast<unsigned>(b < 1 ? 1 : b), 256, 0, s>>>(X, rows, k, S, kp, hi, lo);
+  factor_finish_kernel<<<static_cast<unsigned>(b < 1 ? 1 : b), 256, 0, s>>>(U, m, V, n, k, sign, S, kp, u_hi, u_lo,
+                                                                           w_hi, w_lo, amax);
 }
 
 metis_status run_residual_quant(const ResidualParams& p, const ResidualOperands& o, cudaStream_t s) {

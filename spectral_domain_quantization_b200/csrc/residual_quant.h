@@ -34,9 +34,13 @@ struct ResidualOperands {
   const __nv_bfloat16 *w_hi, *w_lo;  // n x kp, W = V diag(S)
 };
 
-// hi / lo bf16 split of X (rows x k, optionally times diag(S)), padded to kp.
-void launch_hilo(const float* X, int64_t rows, int k, const float* S, int kp, __nv_bfloat16* hi, __nv_bfloat16* lo,
-                 int sms, cudaStream_t s);
+// Sign flip of the factors U (m x k) and V (n x k) in place, bf16 hi / lo
+// copies of U and V diag(S) padded to kp columns (skipped when u_hi is
+// NULL), and the maxima of |U|, |V| into amax[0..1] (skipped when NULL; the
+// caller zeroes them first).
+void launch_factor_finish(float* U, int64_t m, float* V, int64_t n, int k, const float* sign, const float* S, int kp,
+                          __nv_bfloat16* u_hi, __nv_bfloat16* u_lo, __nv_bfloat16* w_hi, __nv_bfloat16* w_lo,
+                          unsigned* amax, int sms, cudaStream_t s);
 metis_status run_residual_quant(const ResidualParams& p, const ResidualOperands& o, cudaStream_t s);
 
 }  // namespace metis

@@ -76,7 +76,8 @@ MDEV void gram_block(const float* ys, int rows, int cols, int ld, double* out) {
 // every split partial is one 16-byte load and a thread's loads are
 // independent; the sum keeps the split order.
 __global__ void __launch_bounds__(1024) gram_kernel(const float* __restrict__ partial, int splits, int64_t rows,
-                                                    int lp, float* __restrict__ Y, double* __restrict__ gpart) {
+                                                    int lp, float* __restrict__ Y, double* __restrict__ gpart,
+                                                    __nv_bfloat16* __restrict__ outT, int64_t ldx) {
   extern __shared__ float ys[];  // kRowsPerBlock x (lp + 1)
   const int ld = lp + 1;
   const int q4 = lp / 4;
@@ -106,7 +107,18 @@ __global__ void __launch_bounds__(1024) gram_kernel(const float* __restrict__ pa
     d[3] = acc.w;
   }
   __syncthreads();
-  gram_block(ys, nr, lp, ld, gpart + static_cast<int64_t>(blockIdx.x) * lp * lp);
+  if (outT) {  // transposed bf16 hi / lo copy (rows lp apart), coalesced along the rows
+    for (int e = threadIdx.x; e < kRowsPerBlock * lp; e += blockDim.x) {
+      const int c = e / kRowsPerBlock, r = e - c * kRowsPerBlock;
+      if (r < nr) {
+        const float v = ys[r * ld + c];
+        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
+        outT[static_cast<int64_t>(c) * ldx + r0 + r] = hi;
+        outT[static_cast<int64_t>(lp + c) * ldx + r0 + r] = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(hi)));
+      }
+    }
+  }
+  if (gpart) gram_block(ys, nr, lp, ld, gpart + static_cast<int64_t>(blockIdx.x) * lp * lp);
 }
 
 // Sum of the block partials: a CTA takes 32 consecutive entries (coalesced
@@ -470,17 +482,6 @@ __global__ void sign_kernel(const float* __restrict__ U, const float* __restrict
   sign[j] = U[bi * k + j] < 0.f ? -1.f : 1.f;
 }
 
-// U (m x k) and V (n x k) columns times sign, one launch.
-__global__ void flip_kernel(float* U, int64_t mk, float* V, int64_t nk, int k, const float* sign) {
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < mk + nk;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    if (e < mk)
-      U[e] *= sign[e % k];
-    else
-      V[e - mk] *= sign[(e - mk) % k];
-  }
-}
-
 int blocks(int64_t n, int sms) {
   int64_t b = (n + 255) / 256;
   if (b > sms * 8) b = sms * 8;
@@ -497,8 +498,17 @@ void launch_gram(const float* partial, int splits, int64_t rows, int lp, float* 
                  cudaStream_t s) {
   const int nb = static_cast<int>(gram_blocks(rows));
   const int threads = (kRowsPerBlock * (lp / 4) + 31) / 32 * 32;  // lp <= 112: at most 896
-  gram_kernel<<<nb, threads, kRowsPerBlock * (lp + 1) * sizeof(float), s>>>(partial, splits, rows, lp, Y, gpart);
+  gram_kernel<<<nb, threads, kRowsPerBlock * (lp + 1) * sizeof(float), s>>>(partial, splits, rows, lp, Y, gpart,
+                                                                            nullptr, 0);
   launch_gram_reduce(gpart, nb, lp, G, s);
+}
+
+void launch_sum_hilo(const float* partial, int splits, int64_t rows, int lp, __nv_bfloat16* outT, int64_t ldx,
+                     cudaStream_t s) {
+  const int nb = static_cast<int>(gram_blocks(rows));
+  const int threads = (kRowsPerBlock * (lp / 4) + 31) / 32 * 32;
+  gram_kernel<<<nb, threads, kRowsPerBlock * (lp + 1) * sizeof(float), s>>>(partial, splits, rows, lp, nullptr,
+                                                                            nullptr, outT, ldx);
 }
 
 void launch_gram_reduce(const double* gpart, int nblocks, int lp, double* G, cudaStream_t s) {
@@ -532,7 +542,6 @@ void launch_signs(float* U, int64_t m, float* V, int64_t n, int k, float* bmax, 
   const int nb = static_cast<int>(sign_blocks(m));
   colmax_kernel<<<nb, 128, 0, s>>>(U, m, k, bmax, bidx);
   sign_kernel<<<1, 128, 0, s>>>(U, bmax, bidx, nb, k, sign);
-  flip_kernel<<<blocks(m * k + n * k, sms), 256, 0, s>>>(U, m * k, V, n * k, k, sign);
 }
 
 }  // namespace metis

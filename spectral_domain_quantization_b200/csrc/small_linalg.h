@@ -30,6 +30,11 @@ int64_t apply_blocks(int64_t rows);
 // gpart: gram_blocks(rows) * lp * lp doubles of scratch.
 void launch_gram(const float* partial, int splits, int64_t rows, int lp, float* Y, double* gpart, double* G,
                  cudaStream_t s);
+// Sum of split partials written only as a transposed bf16 hi / lo copy
+// ([2 lp][ldx]: hi rows 0..lp-1, lo rows lp..2lp-1): the operand of the next
+// skinny product when this basis needs no orthonormalisation.
+void launch_sum_hilo(const float* partial, int splits, int64_t rows, int lp, __nv_bfloat16* outT, int64_t ldx,
+                     cudaStream_t s);
 void launch_gram_reduce(const double* gpart, int nblocks, int lp, double* G, cudaStream_t s);
 // Rinv (lp x lp float, upper triangular) with G = R^T R, dropped pivots -> 0.
 void launch_cholesky_inv(const double* G, int lp, float* Rinv, cudaStream_t s);
@@ -45,8 +50,8 @@ void launch_core_eig(double* C, int n, int max_iters, double* eval, float* evec,
 void launch_factor_mats(const double* eval, const float* evec, int lp, int k, float* Mu, float* Mv, float* S,
                         cudaStream_t s);
 int64_t sign_blocks(int64_t rows);
-// Make the largest-|.| entry (lowest row on ties) of each U column positive,
-// flipping the matching V column.
+// sign[j] = the sign that makes the largest-|.| entry (lowest row on ties)
+// of column j of U positive (applied by launch_factor_finish).
 void launch_signs(float* U, int64_t m, float* V, int64_t n, int k, float* bmax, int64_t* bidx, float* sign, int sms,
                   cudaStream_t s);
 
