@@ -256,7 +256,9 @@ metis_status range_and_core(const SplitPlan& p, const SplitBuffers& b, const Sou
     METIS_TRY(skinny(src, 1, b.qt, p.ld_m, 2, lp, p.split_n, b.part, dev_status, s));
     METIS_TRY(cholqr(b, p.split_n, p.n, lp, b.Zn, p.ld_n, 1, s));
     METIS_TRY(skinny(src, 0, b.qt, p.ld_n, 2, lp, p.split_m, b.part, dev_status, s));
-    METIS_TRY(cholqr(b, p.split_m, src.rows, lp, b.Qm, p.ld_m, it == power_iters - 1 ? 2 : 1, s));
+    // one pass also for the final basis: the Gram is formed in float64 from
+    // float32 data, so a pass leaves |Q^T Q - I| near kappa(Y) 2^-23
+    METIS_TRY(cholqr(b, p.split_m, src.rows, lp, b.Qm, p.ld_m, 1, s));
   }
   METIS_TRY(skinny(src, 1, b.qt, p.ld_m, 2, lp, p.split_n, b.part, dev_status, s));
   launch_gram(b.part, p.split_n, p.n, lp, b.Zn, b.gpart, b.G, s);

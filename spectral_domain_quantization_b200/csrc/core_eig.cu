@@ -489,7 +489,7 @@ MDEV double warp_norm(const double* v, int n) {
   return sqrt(s);
 }
 
-__global__ void __launch_bounds__(256) core_finish_kernel(int n, double* ws, double* eval, float* evec) {
+__global__ void __launch_bounds__(1024) core_finish_kernel(int n, double* ws, double* eval, float* evec) {
   __shared__ double lam[kMaxN];
   const EigScratch S = scratch(ws, n);
   double* X = S.X;
@@ -543,6 +543,7 @@ __global__ void __launch_bounds__(256) core_finish_kernel(int n, double* ws, dou
   }
   __syncthreads();
   // descending order: rank = n - 1 - idx
+#pragma unroll 4
   for (int e = threadIdx.x; e < n * n; e += blockDim.x) {
     const int r = e / n, rk = e - r * n;
     evec[e] = static_cast<float>(X[r * n + (n - 1 - rk)]);
@@ -563,7 +564,7 @@ void launch_core_eig(double* C, int n, int max_iters, double* eval, float* evec,
   const size_t vsmem = static_cast<size_t>(n) * n * sizeof(double);
   if (!ensure_smem(reinterpret_cast<const void*>(core_vector_kernel), vsmem)) return;
   core_vector_kernel<<<n, 32, vsmem, s>>>(n, ws, max_iters, dev_status);
-  core_finish_kernel<<<1, 256, 0, s>>>(n, ws, eval, evec);
+  core_finish_kernel<<<1, 1024, 0, s>>>(n, ws, eval, evec);
 }
 
 }  // namespace metis

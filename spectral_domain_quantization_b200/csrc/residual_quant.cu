@@ -408,33 +408,33 @@ __global__ void __launch_bounds__(256) factor_finish_kernel(float* U, int64_t m,
                                                             __nv_bfloat16* u_hi, __nv_bfloat16* u_lo,
                                                             __nv_bfloat16* w_hi, __nv_bfloat16* w_lo,
                                                             unsigned* amax) {
+  // thread (c, ry): column c of rows blockIdx.x * blockDim.y + ry (U's rows
+  // first, then V's)
+  const int c = threadIdx.x;
+  const int64_t row = static_cast<int64_t>(blockIdx.x) * blockDim.y + threadIdx.y;
   float mu = 0.f, mv = 0.f;
-  const int64_t eu = m * kp, total = eu + n * kp;
-  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
-       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const bool isu = e < eu;
-    const int64_t el = isu ? e : e - eu;
-    const int64_t r = el / kp;
-    const int c = static_cast<int>(el - r * kp);
+  if (row < m + n) {
+    const bool isu = row < m;
+    const int64_t r = isu ? row : row - m;
     float w = 0.f;
     if (c < k) {
       float* x = (isu ? U : V) + r * k + c;
       const float v = *x * sign[c];
       *x = v;
       if (isu) {
-        mu = fmaxf(mu, fabsf(v));
+        mu = fabsf(v);
         w = v;
       } else {
-        mv = fmaxf(mv, fabsf(v));
+        mv = fabsf(v);
         w = __fmul_rn(v, S[c]);
       }
     }
     __nv_bfloat16* hi = isu ? u_hi : w_hi;
     __nv_bfloat16* lo = isu ? u_lo : w_lo;
-    if (hi) {
+    if (hi && c < kp) {
       const __nv_bfloat16 h = __float2bfloat16_rn(w);
-      hi[el] = h;
-      lo[el] = __float2bfloat16_rn(__fsub_rn(w, __bfloat162float(h)));
+      hi[r * kp + c] = h;
+      lo[r * kp + c] = __float2bfloat16_rn(__fsub_rn(w, __bfloat162float(h)));
     }
   }
   if (amax) {
@@ -471,11 +471,11 @@ CUresult map_a(CUtensorMap* m, const ResidualParams& p) {
 
 void launch_factor_finish(float* U, int64_t m, float* V, int64_t n, int k, const float* sign, const float* S, int kp,
                           __nv_bfloat16* u_hi, __nv_bfloat16* u_lo, __nv_bfloat16* w_hi, __nv_bfloat16* w_lo,
-                          unsigned* amax, int sms, cudaStream_t s) {
-  int64_t b = ((m + n) * kp + 255) / 256;
-  if (b > sms * 8) b = sms * 8;
-  factor_finish_kernel<<<static_cast<unsigned>(b < 1 ? 1 : b), 256, 0, s>>>(U, m, V, n, k, sign, S, kp, u_hi, u_lo,
-                                                                           w_hi, w_lo, amax);
+                          unsigned* amax, int, cudaStream_t s) {
+  const int cols = ((kp > k ? kp : k) + 31) / 32 * 32;  // <= 128
+  const dim3 block(cols, 256 / cols);
+  const unsigned grid = static_cast<unsigned>((m + n + block.y - 1) / block.y);
+  factor_finish_kernel<<<grid, block, 0, s>>>(U, m, V, n, k, sign, S, kp, u_hi, u_lo, w_hi, w_lo, amax);
 }
 
 metis_status run_residual_quant(const ResidualParams& p, const ResidualOperands& o, cudaStream_t s) {

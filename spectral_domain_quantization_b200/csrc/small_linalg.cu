@@ -464,22 +464,33 @@ __global__ void colmax_kernel(const float* __restrict__ U, int64_t rows, int k, 
   bidx[static_cast<int64_t>(blockIdx.x) * k + j] = bi;
 }
 
+// One warp per column: lanes take every 32nd block, then a shuffle reduction
+// keeps the largest |U| (the lowest block, hence the lowest row, on ties).
 __global__ void sign_kernel(const float* __restrict__ U, const float* __restrict__ bmax,
                             const int64_t* __restrict__ bidx, int nblocks, int k, float* sign) {
-  const int j = threadIdx.x;
-  if (j >= k) return;
+  const int j = blockIdx.x, lane = threadIdx.x;
   float best = -1.f;
-  int bb = 0;
-#pragma unroll 8
-  for (int b = 0; b < nblocks; ++b) {
+  int bb = nblocks;
+#pragma unroll 4
+  for (int b = lane; b < nblocks; b += 32) {
     const float v = bmax[static_cast<int64_t>(b) * k + j];
     if (v > best) {
       best = v;
       bb = b;
     }
   }
-  const int64_t bi = bidx[static_cast<int64_t>(bb) * k + j];
-  sign[j] = U[bi * k + j] < 0.f ? -1.f : 1.f;
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+    const int ob = __shfl_xor_sync(0xFFFFFFFFu, bb, o);
+    if (ov > best || (ov == best && ob < bb)) {
+      best = ov;
+      bb = ob;
+    }
+  }
+  if (lane == 0) {
+    const int64_t bi = bidx[static_cast<int64_t>(bb) * k + j];
+    sign[j] = U[bi * k + j] < 0.f ? -1.f : 1.f;
+  }
 }
 
 int blocks(int64_t n, int sms) {
@@ -541,7 +552,7 @@ void launch_signs(float* U, int64_t m, float* V, int64_t n, int k, float* bmax, 
                   cudaStream_t s) {
   const int nb = static_cast<int>(sign_blocks(m));
   colmax_kernel<<<nb, 128, 0, s>>>(U, m, k, bmax, bidx);
-  sign_kernel<<<1, 128, 0, s>>>(U, bmax, bidx, nb, k, sign);
+  sign_kernel<<<k, 32, 0, s>>>(U, bmax, bidx, nb, k, sign);
 }
 
 }  // namespace metis
