@@ -279,10 +279,25 @@ MDEV int sturm_count(const double* d, const double* e2, int n, double x) {
 }
 
 __global__ void __launch_bounds__(32) core_vector_kernel(int n, double* ws, int max_rounds, int32_t* dev_status) {
-  __shared__ double d[kMaxN], e[kMaxN], e2[kMaxN], dp[kMaxN], dm[kMaxN], lp[kMaxN], um[kMaxN], z[kMaxN], bs[kMaxN];
-  extern __shared__ double Vs[];  // n x n reflectors
+  __shared__ double d[kMaxN], e[kMaxN], e2[kMaxN], dp[kMaxN], dm[kMaxN], lp[kMaxN], um[kMaxN], z[kMaxN];
+  __shared__ __align__(16) double bs[kMaxN];
+  extern __shared__ __align__(16) double Vs[];  // n x n reflectors
+  __shared__ uint64_t vbar;
+  __shared__ int vabort;
   const EigScratch S = scratch(ws, n);
   const int lane = threadIdx.x, idx = blockIdx.x;  // eigenvalue idx in ascending order
+  // the reflectors and their betas come in by one bulk copy each, started
+  // now so that they land while the eigenvalue is found
+  const uint32_t vbytes = static_cast<uint32_t>(n) * n * sizeof(double);
+  if (lane == 0) {
+    vabort = 0;
+    mbar_init(&vbar, 1);
+    fence_barrier_init();
+    mbar_arrive_expect_tx(&vbar, vbytes + static_cast<uint32_t>(n) * sizeof(double));
+    bulk_load(Vs, S.V, vbytes, &vbar);
+    bulk_load(bs, S.beta, static_cast<uint32_t>(n) * sizeof(double), &vbar);
+  }
+  __syncwarp();
   // scale T by a power of two so that |d|, |e| <= 1
   double mx = 0.0;
   for (int i = lane; i < n; i += 32) {
@@ -420,9 +435,18 @@ __global__ void __launch_bounds__(32) core_vector_kernel(int n, double* ws, int 
   __syncwarp();
   // x = H_0 H_1 ... H_{n-3} z, the reflectors staged in shared memory;
   // lane l holds entries l, l + 32, l + 64, l + 96
-  for (int e = lane; e < n * n; e += 32) Vs[e] = S.V[e];
-  for (int i = lane; i < n; i += 32) bs[i] = S.beta[i];
-  __syncwarp();
+  const bool landed = mbar_wait(&vbar, 0, &vabort);  // bounded wait
+  if (!__all_sync(0xFFFFFFFFu, landed)) {
+    if (lane == 0) {
+      report(dev_status, METIS_DEV_TIMEOUT);
+      // the copies were issued by this warp: give them a bounded time to land
+      const uint64_t t0 = global_timer_ns();
+      while (!mbar_try_wait(&vbar, 0) && global_timer_ns() - t0 < 100000000ull) {
+      }
+    }
+    __syncwarp();
+    return;
+  }
   double xv[4];
 #pragma unroll
   for (int q = 0; q < 4; ++q) xv[q] = lane + 32 * q < n ? z[lane + 32 * q] : 0.0;
@@ -495,7 +519,18 @@ __global__ void __launch_bounds__(1024) core_finish_kernel(int n, double* ws, do
   double* X = S.X;
   for (int i = threadIdx.x; i < n; i += blockDim.x) lam[i] = S.lam[i];
   __syncthreads();
+  // is there any cluster at all?  (one warp vote; usually not)
+  bool any = false;
   if (threadIdx.x < 32) {
+    double top = 0.0;
+    for (int i = threadIdx.x; i < n; i += 32) top = fmax(top, fabs(lam[i]));
+    for (int o = 16; o > 0; o >>= 1) top = fmax(top, __shfl_xor_sync(0xFFFFFFFFu, top, o));
+    const double tol = kClusterTol * top;
+    bool gap_small = false;
+    for (int i = threadIdx.x; i + 1 < n; i += 32) gap_small |= lam[i + 1] - lam[i] <= tol;
+    any = __any_sync(0xFFFFFFFFu, gap_small);
+  }
+  if (threadIdx.x < 32 && any) {
     double top = 0.0;
     for (int i = 0; i < n; ++i) top = fmax(top, fabs(lam[i]));
     const double tol = kClusterTol * top;

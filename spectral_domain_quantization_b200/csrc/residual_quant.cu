@@ -408,12 +408,14 @@ __global__ void __launch_bounds__(256) factor_finish_kernel(float* U, int64_t m,
                                                             __nv_bfloat16* u_hi, __nv_bfloat16* u_lo,
                                                             __nv_bfloat16* w_hi, __nv_bfloat16* w_lo,
                                                             unsigned* amax) {
-  // thread (c, ry): column c of rows blockIdx.x * blockDim.y + ry (U's rows
-  // first, then V's)
+  // thread (c, ry): column c of rows ry, ry + blockDim.y, ... of this CTA's
+  // share (U's rows first, then V's); one atomic per CTA and matrix
+  __shared__ float red[2][32];
   const int c = threadIdx.x;
-  const int64_t row = static_cast<int64_t>(blockIdx.x) * blockDim.y + threadIdx.y;
+  const int nthr = blockDim.x * blockDim.y, tid = threadIdx.y * blockDim.x + threadIdx.x;
   float mu = 0.f, mv = 0.f;
-  if (row < m + n) {
+  for (int64_t row = static_cast<int64_t>(blockIdx.x) * blockDim.y + threadIdx.y; row < m + n;
+       row += static_cast<int64_t>(gridDim.x) * blockDim.y) {
     const bool isu = row < m;
     const int64_t r = isu ? row : row - m;
     float w = 0.f;
@@ -422,10 +424,10 @@ __global__ void __launch_bounds__(256) factor_finish_kernel(float* U, int64_t m,
       const float v = *x * sign[c];
       *x = v;
       if (isu) {
-        mu = fabsf(v);
+        mu = fmaxf(mu, fabsf(v));
         w = v;
       } else {
-        mv = fabsf(v);
+        mv = fmaxf(mv, fabsf(v));
         w = __fmul_rn(v, S[c]);
       }
     }
@@ -442,7 +444,16 @@ __global__ void __launch_bounds__(256) factor_finish_kernel(float* U, int64_t m,
       mu = fmaxf(mu, __shfl_xor_sync(0xFFFFFFFFu, mu, o));
       mv = fmaxf(mv, __shfl_xor_sync(0xFFFFFFFFu, mv, o));
     }
-    if ((threadIdx.x & 31) == 0) {
+    if ((tid & 31) == 0) {
+      red[0][tid >> 5] = mu;
+      red[1][tid >> 5] = mv;
+    }
+    __syncthreads();
+    if (tid == 0) {
+      for (int w = 1; w < nthr / 32; ++w) {
+        mu = fmaxf(mu, red[0][w]);
+        mv = fmaxf(mv, red[1][w]);
+      }
       if (mu > 0.f) atomicMax(amax, __float_as_uint(mu));
       if (mv > 0.f) atomicMax(amax + 1, __float_as_uint(mv));
     }
@@ -471,11 +482,13 @@ CUresult map_a(CUtensorMap* m, const ResidualParams& p) {
 
 void launch_factor_finish(float* U, int64_t m, float* V, int64_t n, int k, const float* sign, const float* S, int kp,
                           __nv_bfloat16* u_hi, __nv_bfloat16* u_lo, __nv_bfloat16* w_hi, __nv_bfloat16* w_lo,
-                          unsigned* amax, int, cudaStream_t s) {
+                          unsigned* amax, int sms, cudaStream_t s) {
   const int cols = ((kp > k ? kp : k) + 31) / 32 * 32;  // <= 128
   const dim3 block(cols, 256 / cols);
-  const unsigned grid = static_cast<unsigned>((m + n + block.y - 1) / block.y);
-  factor_finish_kernel<<<grid, block, 0, s>>>(U, m, V, n, k, sign, S, kp, u_hi, u_lo, w_hi, w_lo, amax);
+  int64_t grid = (m + n + block.y - 1) / block.y;
+  if (grid > 2 * sms) grid = 2 * sms;  // a few atomics per matrix, not one per warp
+  factor_finish_kernel<<<static_cast<unsigned>(grid), block, 0, s>>>(U, m, V, n, k, sign, S, kp, u_hi, u_lo, w_hi,
+                                                                     w_lo, amax);
 }
 
 metis_status run_residual_quant(const ResidualParams& p, const ResidualOperands& o, cudaStream_t s) {

@@ -344,7 +344,7 @@ __global__ void __launch_bounds__(kSmallThreads, 1) cholesky_inv_kernel(const do
 constexpr int kApplyRows = 32;
 
 // out = in (rows x kin) * M (kin x kout).  32 rows per CTA, 256 threads, each
-// thread a 4-row x 4-column register tile.  Optional fp32 out,
+// thread a 4-row x 4-column register tile (4 consecutive columns).  Optional fp32 out,
 // transposed bf16 hi/lo copy, Gram partial of the output block.
 __global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) {
   extern __shared__ float smf[];
@@ -373,35 +373,34 @@ __global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) {
     }
   }
   __syncthreads();
-  // warp w: rows 4 w .. 4 w + 3 (broadcast reads of In); lane: columns
-  // lane, lane + 32, lane + 64, lane + 96 (kout <= 112)
+  // warp w: rows 4 w .. 4 w + 3 (broadcast reads of In); lane l < kout / 4:
+  // columns 4 l .. 4 l + 3 (one 16-byte read of M per step; kout <= 112)
   const int rg = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  constexpr int kCols = 4;
-  float acc[4][kCols];
+  const bool has = 4 * lane < a.kout;
+  float acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int u = 0; u < kCols; ++u) acc[i][u] = 0.f;
+    for (int u = 0; u < 4; ++u) acc[i][u] = 0.f;
   const float* in0 = In + (4 * rg) * (a.kin + 1);
-  const int ncol = (a.kout - lane + 31) / 32;  // columns this lane owns
+  if (has) {
 #pragma unroll 2
-  for (int j = 0; j < a.kin; ++j) {
-    float x[4];
+    for (int j = 0; j < a.kin; ++j) {
+      float x[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) x[i] = in0[i * (a.kin + 1) + j];
-    const float* mrow = Ms + j * a.kout + lane;
+      for (int i = 0; i < 4; ++i) x[i] = in0[i * (a.kin + 1) + j];
+      const float4 m = *reinterpret_cast<const float4*>(Ms + j * a.kout + 4 * lane);
+      const float mv[4] = {m.x, m.y, m.z, m.w};
 #pragma unroll
-    for (int u = 0; u < kCols; ++u) {
-      const float m = u < ncol ? mrow[32 * u] : 0.f;
+      for (int u = 0; u < 4; ++u)
 #pragma unroll
-      for (int i = 0; i < 4; ++i) acc[i][u] = fmaf(x[i], m, acc[i][u]);
+        for (int i = 0; i < 4; ++i) acc[i][u] = fmaf(x[i], mv[u], acc[i][u]);
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int u = 0; u < 4; ++u) Out[(4 * rg + i) * (a.kout + 1) + 4 * lane + u] = acc[i][u];
   }
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int u = 0; u < kCols; ++u)
-      if (u < ncol) Out[(4 * rg + i) * (a.kout + 1) + lane + 32 * u] = acc[i][u];
   __syncthreads();
   for (int e = threadIdx.x; e < kApplyRows * a.kout; e += blockDim.x) {
     if (a.out) {
@@ -493,11 +492,6 @@ __global__ void sign_kernel(const float* __restrict__ U, const float* __restrict
   }
 }
 
-int blocks(int64_t n, int sms) {
-  int64_t b = (n + 255) / 256;
-  if (b > sms * 8) b = sms * 8;
-  return static_cast<int>(b < 1 ? 1 : b);
-}
 
 }  // namespace
 
