@@ -62,7 +62,7 @@ typedef enum {
 } metis_status;
 
 /* bits OR-ed into *dev_status by kernels */
-#define METIS_DEV_NUMERIC 1  /* Jacobi did not converge within max sweeps       */
+#define METIS_DEV_NUMERIC 1  /* the core eigensolver hit max_core_iters          */
 #define METIS_DEV_TIMEOUT 2  /* a bounded device wait expired; outputs invalid   */
 #define METIS_DEV_SAMPLING 4 /* a sparse-sign row could not draw its columns     */
 
@@ -117,6 +117,18 @@ int32_t metis_device_supported(void);
  * (which step failed and the CUDA error string); "" if none.  The string is
  * owned by the library and overwritten by the next failure on the thread. */
 const char* metis_last_error(void);
+
+/*
+ * metis_selftest_wait_timeout -- check of the failure detection every kernel
+ * relies on.  One thread runs the library's bounded barrier wait on a phase
+ * that nothing completes, with a limit of limit_ns (1 .. 1e9 ns), and must
+ * OR METIS_DEV_TIMEOUT into *dev_status (device int32, caller-owned) and
+ * return.  The pages have no counterpart: this is the library's own check
+ * that a stalled wait ends with a status instead of hanging.
+ * Errors: METIS_ERR_NULL (dev_status), METIS_ERR_ARG (limit out of range),
+ * METIS_ERR_UNSUPPORTED (no sm_100 device), METIS_ERR_CUDA (launch).
+ */
+metis_status metis_selftest_wait_timeout(uint64_t limit_ns, int32_t* dev_status, void* stream);
 
 /*
  * metis_quantize_fp4 -- block-quantize a dense matrix to FP4.

@@ -72,6 +72,7 @@ _SIGS = {
     "metis_quantize_fp4": (_I32, [_VP, _I32, _I64, _I64, _I64, _I32, _VP, _FP, _VP, _SZP, _VP]),
     "metis_quantize_fp4_noalloc": (_I32, [_VP, _I32, _I64, _I64, _I64, _I32, _VP, _FP, _VP]),
     "metis_noalloc_scratch_bytes": (ctypes.c_size_t, []),
+    "metis_selftest_wait_timeout": (_I32, [ctypes.c_uint64, ctypes.c_void_p, ctypes.c_void_p]),
     "metis_split": (_I32, [_VP, _I32, _I64, _I64, _I64, ctypes.POINTER(SplitParams), _VP, _VP, _VP,
                            _FP, _FP, _FP, _FP, _VP, _VP, _VP, _SZP, _VP, _VP]),
     "metis_linear_fwd": (_I32, [_OP, _OP, _I64, _I64, _I64, _VP, _I32, _I64, _VP, _SZP, _VP, _VP]),
@@ -401,3 +402,13 @@ def averis_split(X, fmt="nv", rows=True, cols=True, tap=False, dev_status=None):
         (_ptr(dev_status), _stream()), dev, "averis_split")
     return AverisSplit(mean=mean, mean_q=mean_q, R_rows=R_rows, R_cols=R_cols, R_f32=R_f32,
                        dev_status=dev_status, fmt=f)
+
+
+def selftest_wait_timeout(limit_ns=1_000_000, device="cuda"):
+    """Run the library's bounded device wait on a barrier that never
+    completes (metis_selftest_wait_timeout); returns the device status word
+    after the launch finished (DEV_TIMEOUT set when the wait ended itself)."""
+    st = torch.zeros(1, dtype=torch.int32, device=device)
+    _check(lib().metis_selftest_wait_timeout(int(limit_ns), _ptr(st), _stream()), "metis_selftest_wait_timeout")
+    torch.cuda.synchronize()
+    return int(st.item())

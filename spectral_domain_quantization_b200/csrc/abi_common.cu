@@ -156,3 +156,26 @@ int32_t metis_device_supported(void) { return metis::device_is_sm100() ? 1 : 0; 
 const char* metis_last_error(void) { return metis::g_last_error; }
 
 }  // extern "C"
+
+namespace {
+
+// One thread waits, with the kernels' own bounded wait, on a barrier phase
+// that nothing completes; the timeout must end the wait and be reported.
+__global__ void wait_selftest_kernel(uint64_t limit_ns, int32_t* dev_status) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  abort_flag = 0;
+  metis::mbar_init(&bar, 1);
+  metis::fence_barrier_init();
+  if (!metis::mbar_wait_for(&bar, 0, &abort_flag, limit_ns)) metis::report(dev_status, METIS_DEV_TIMEOUT);
+}
+
+}  // namespace
+
+extern "C" metis_status metis_selftest_wait_timeout(uint64_t limit_ns, int32_t* dev_status, void* stream) {
+  if (!dev_status) return METIS_ERR_NULL;
+  if (limit_ns == 0 || limit_ns > 1000000000ull) return METIS_ERR_ARG;
+  if (!metis::device_is_sm100()) return METIS_ERR_UNSUPPORTED;
+  wait_selftest_kernel<<<1, 1, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns, dev_status);
+  return metis::launch_status();
+}

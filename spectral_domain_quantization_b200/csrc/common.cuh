@@ -85,20 +85,25 @@ MDEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for phase `parity` of `bar`.  Returns false once *abort is set (by this
-// or another thread) or after kWaitTimeoutNs; a timeout sets *abort.
-MDEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+// or another thread) or after limit_ns; a timeout sets *abort.
+MDEV bool mbar_wait_for(uint64_t* bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = global_timer_ns();
   for (uint32_t it = 1;; ++it) {
     if (mbar_try_wait(bar, parity)) return true;
     if ((it & 63u) == 0) {
       if (*abort) return false;
-      if (global_timer_ns() - t0 > kWaitTimeoutNs) {
+      if (global_timer_ns() - t0 > limit_ns) {
         *abort = 1;
         return false;
       }
     }
   }
+}
+
+// The wait every kernel uses: limit kWaitTimeoutNs.
+MDEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
+  return mbar_wait_for(bar, parity, abort, kWaitTimeoutNs);
 }
 
 // ---------------------------------------------------------------------------

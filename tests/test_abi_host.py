@@ -85,3 +85,14 @@ def test_unbuilt_entry_points_report_instead_of_crashing():
     size = ctypes.c_size_t(0)
     st = L.metis_linear_fwd(None, None, 1, 1, 32, None, api.F32, 1, None, ctypes.byref(size), None, None)
     assert st != api.OK
+
+
+ERR_NULL, ERR_ARG = 1, 7  # metis_status codes of include/metis.h
+
+
+def test_selftest_wait_argument_checks():
+    L = api.lib()
+    assert L.metis_selftest_wait_timeout(1000, None, None) == ERR_NULL
+    fake = ctypes.c_int32(0)
+    assert L.metis_selftest_wait_timeout(0, ctypes.addressof(fake), None) == ERR_ARG
+    assert L.metis_selftest_wait_timeout(2_000_000_000, ctypes.addressof(fake), None) == ERR_ARG
