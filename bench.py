@@ -100,26 +100,81 @@ def reduce_max(x, world):
 # --------------------------------------------------------------------------
 
 class ClockSampler:
+    """SM clock, its maximum and the clock-event (throttle) reasons, sampled
+    during the timed region.  NVML is read from a thread every 2 ms (a timed
+    region of a few tens of milliseconds still gets samples); where NVML is
+    not importable, `nvidia-smi -lms 50` runs instead, started before the
+    region.  Nothing here changes a setting of the GPU."""
+
+    REASONS = (("hw_slowdown", 8), ("hw_thermal_slowdown", 64), ("sw_thermal_slowdown", 32),
+               ("sw_power_cap", 4), ("hw_power_brake_slowdown", 128))
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index):
         self.index = index
+        self.rows = []
+        self.thread = None
         self.proc = None
         self.path = None
+        self.source = None
+
+    def _nvml_handle(self):
+        import pynvml
+        import torch
+        pynvml.nvmlInit()
+        uuid = str(torch.cuda.get_device_properties(self.index).uuid)
+        if not uuid.startswith("GPU-"):
+            uuid = "GPU-" + uuid
+        return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid)
 
     def start(self):
+        import threading
+        try:
+            nv, h = self._nvml_handle()
+            self.smax = float(nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM))
+            self.stop_evt = threading.Event()
+
+            def run():
+                while not self.stop_evt.is_set():
+                    try:
+                        self.rows.append((float(nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM)),
+                                          int(nv.nvmlDeviceGetCurrentClocksEventReasons(h))))
+                    except Exception:
+                        pass
+                    self.stop_evt.wait(0.002)
+
+            self.thread = threading.Thread(target=run, daemon=True)
+            self.thread.start()
+            self.source = "nvml (2 ms)"
+            return
+        except Exception:
+            self.thread = None
         try:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
-                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+                 "-lms", "50"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+            t0 = time.time()
+            while os.path.getsize(self.path) == 0 and time.time() - t0 < 5.0:
+                time.sleep(0.01)   # the first sample lands before the timed region starts
+            self.source = "nvidia-smi (50 ms)"
         except Exception:
             self.proc = None
 
     def stop(self):
+        if self.thread is not None:
+            self.stop_evt.set()
+            self.thread.join(timeout=5)
+            if not self.rows:
+                return None
+            sm = [r[0] for r in self.rows]
+            loaded = [v for v in sm if v > 0.5 * self.smax] or sm
+            reasons = sorted({name for _, bits in self.rows for name, bit in self.REASONS if bits & bit})
+            return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": self.smax, "reasons": reasons,
+                    "samples": len(self.rows), "source": self.source}
         if self.proc is None:
             return None
         self.proc.terminate()
@@ -141,7 +196,7 @@ class ClockSampler:
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
         return {"sm_mhz": float(np.median(loaded)), "sm_max_mhz": smax, "reasons": reasons,
-                "samples": len(rows)}
+                "samples": len(rows), "source": self.source}
 
 
 # --------------------------------------------------------------------------

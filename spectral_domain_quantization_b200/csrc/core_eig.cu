@@ -10,9 +10,9 @@
 // The problem is tiny and latency-bound, so the work is cut into three
 // launches that each keep their sequential chains short:
 //   1. core_tridiag_kernel (one CTA): Householder reduction C = Q T Q^T to a
-//      symmetric tridiagonal T (diagonal d, off-diagonal e), accumulating Q,
-//      with A and Q held in per-thread register tiles; three barriers per
-//      column.
+//      symmetric tridiagonal T (diagonal d, off-diagonal e), keeping the
+//      reflectors; A's rows held in registers by thread pairs, two barriers
+//      per column.
 //   2. core_vector_kernel (one CTA of one warp per eigenvalue): the
 //      eigenvalue by multisection on Sturm counts (32 points per round, the
 //      counts from the division-free determinant recurrence with power-of-two
@@ -32,7 +32,6 @@ namespace metis {
 
 namespace {
 
-constexpr int kTriThreads = 512;  // >= the 406 tiles of n = 112
 constexpr int kMaxN = 112;
 constexpr double kClusterTol = 1e-9; // relative gap below which vectors are re-orthogonalised
 
@@ -55,81 +54,77 @@ __host__ __device__ inline EigScratch scratch(double* ws, int n) {
 }
 
 // ---------------------------------------------------------------------------
-// Tile (I, J), I >= J, of an nb x nb lower block triangle: its index in
-// row-major order of the triangle, and the inverse map (packed (I << 8) | J).
-MDEV int tri_pos(int I, int J, int) { return I * (I + 1) / 2 + J; }
-MDEV int tri_index(int t, int) {
-  int I = static_cast<int>((sqrtf(8.f * t + 1.f) - 1.f) * 0.5f);
-  while ((I + 1) * (I + 2) / 2 <= t) ++I;
-  while (I * (I + 1) / 2 > t) --I;
-  return (I << 8) | (t - I * (I + 1) / 2);
-}
-
-// Column c (a runtime index) of a 4 x 4 register tile into dst[0..3],
-// selected without dynamic register indexing.
-MDEV void publish_col(const double (&a)[4][4], int c, double* dst) {
-#pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    double v = a[r][0];
-#pragma unroll
-    for (int q = 1; q < 4; ++q) v = q == c ? a[r][q] : v;
-    dst[r] = v;
-  }
-}
-
-// ---------------------------------------------------------------------------
 // 1. Householder tridiagonalisation
 // ---------------------------------------------------------------------------
 // Column j: x = A[j+1.., j], alpha = -sign(x0) |x|, v = x - alpha e_1,
-// beta = 2 / v^T v, p = beta A' v, w = p - (beta/2)(p^T v) v,
-// A' -= v w^T + w v^T; (v, beta) are kept so that the eigenvectors can be
-// taken back through H_0 ... H_{n-3} later.
-// Register tiles: thread T < nA owns the 4 x 4 tile (I, J), I >= J, of the
-// symmetric A (a diagonal tile holds its whole block).  A step publishes
-// nothing but vectors:
-//   (a) every tile multiplies by the v it needs (its rows and, off the
-//       diagonal, its columns) into per-tile partial sums;
-//   (b) one thread per row adds the partials in a fixed order (p);
-//   (c) every tile applies its rank-2 update and the tiles holding column
-//       j + 1 publish it for the next step.
+// beta = 2 / v^T v, p = beta A' v, K = (beta/2) p^T v, w = p - K v and
+// A' -= v w^T + w v^T, which is A' -= q v^T + v p^T with q = p - 2 K v.
+// (v, beta) are kept so that the eigenvectors can be taken back through
+// H_0 ... H_{n-3} later.
+//
+// Layout: a thread pair per row.  Thread (i, h) holds the row's columns
+// base + 2 r + h (r < NH) in registers, base = j rounded down to even, so
+// the two halves shrink together and after every second column the row
+// moves one register to the left.  Row warps skip 16-column chunks that lie
+// past n and the work of warps whose rows are all finished.  The full
+// square is kept (no symmetric packing): the product then needs no
+// transposed partial sums.
+//
+// Two barriers per column:
+//   (a) row warps: u = A' x with x0 (not v0) at column j + 1, the sums
+//       S1 = sum_{i>j+1} u_i x_i and S2 = sum_{i>j+1} A[i][j+1] x_i, and
+//       the values of row j + 1; meanwhile one extra warp finds alpha,
+//       beta and v0 from |x|^2 (reduced in the column before) and x0;
+//   (b) all: p_i = beta (u_i + A[i][j+1] (v0 - x0)) and
+//       p^T v = p_{j+1} v0 + beta (S1 + (v0 - x0) S2) give K and q; the
+//       holders of column j + 1 update it first and reduce the next
+//       column's |x|^2;
+//   (c) row warps: the rest of the rank-2 update.
 
-__global__ void __launch_bounds__(kTriThreads, 1) core_tridiag_kernel(const double* C, int n, double* ws) {
-  extern __shared__ double sm[];
-  const int nb = n / 4;
-  const int nA = nb * (nb + 1) / 2;
-  double* xb = sm;                 // 2 x n: column j of A below the diagonal (double-buffered)
-  double* pb = xb + 2 * n;         // n: beta A' v
-  double* partA = pb + n;          // nA x 4: row sums of each A tile
-  double* partT = partA + 4 * nA;  // nA x 4: column sums of each off-diagonal A tile
-  const EigScratch S = scratch(ws, n);
-  const int t = threadIdx.x, lane = t & 31;
-  // ---- tile ownership
-  const bool isA = t < nA;
-  int I = 0, J = 0;
-  double a[4][4];
-  if (isA) {
-    const int ij = tri_index(t, nb);
-    I = ij >> 8;
-    J = ij & 255;
-#pragma unroll
-    for (int r = 0; r < 4; ++r)
-#pragma unroll
-      for (int c = 0; c < 4; ++c) a[r][c] = C[(4 * I + r) * n + 4 * J + c];
-    if (J == 0) {
-#pragma unroll
-      for (int r = 0; r < 4; ++r) xb[4 * I + r] = a[r][0];
-    }
+template <int NH>
+struct TriShared {
+  static constexpr int kBuf = 4 * NH + 8;   // row windows reach base + 2 NH - 1 <= n + 2 NH - 4
+  static constexpr int kWarps = (4 * NH + 31) / 32;
+  double xb[2][kBuf];   // x entries of the column by row (0 outside the active rows)
+  double pb[2][kBuf];   // p_i by row (0 outside the active rows)
+  double red1a[kWarps], red1b[kWarps], red2[kWarps];
+  double row1[2];       // row j + 1: u_{j+1} and A[j+1][j+1]
+  double refl[2];       // beta, v0 of the current column
+};
+
+// Sum of v[0 .. cnt) in a fixed order, two interleaved accumulators.
+MDEV double sum_fixed(const double* v, int cnt) {
+  double s0 = 0.0, s1 = 0.0;
+  int w = 0;
+  for (; w + 1 < cnt; w += 2) {
+    s0 += v[w];
+    s1 += v[w + 1];
   }
-  __syncthreads();
-  for (int j = 0; j + 2 < n; ++j) {
-    const double* x = xb + (j & 1) * n;        // x[i] = A[i][j], i > j
-    double* xn = xb + ((j + 1) & 1) * n;
-    // every warp: alpha, beta, v0 (the same arithmetic in every warp)
-    double sg = 0.0;
-    for (int i = j + 2 + lane; i < n; i += 32) sg = fma(x[i], x[i], sg);
+  if (w < cnt) s0 += v[w];
+  return s0 + s1;
+}
+
+MDEV double warp_sum(double v) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) sg += __shfl_xor_sync(0xFFFFFFFFu, sg, o);
-    const double x0 = x[j + 1];
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xFFFFFFFFu, v, o);
+  return v;
+}
+
+// One column step; ODD = j & 1 (registers hold columns base + 2 r + h,
+// base = j - ODD).  Warps 0 .. nwr - 1 hold rows; warp nwr the scalars.
+template <int NH, int ODD>
+MDEV void tri_step(double (&a)[NH], TriShared<NH>& sh, const EigScratch& S, int j, int n, int i, int h,
+                   int lane, int warp, int nwr) {
+  constexpr int kHoldR = ODD ? 1 : 0;   // register of column j + 1, in thread h = 1 - ODD
+  const int hold_h = 1 - ODD;
+  const int base = j - ODD;
+  const double* xcur = sh.xb[j & 1];
+  double* xnext = sh.xb[(j + 1) & 1];
+  double* pcur = sh.pb[j & 1];
+  const bool scalar_warp = warp == nwr;
+  if (scalar_warp) {
+    const double sg = sum_fixed(sh.red2, nwr);
+    const double x0 = xcur[j + 1];
     double alpha = x0, beta = 0.0, v0 = 0.0;
     if (sg > 0.0) {
       const double nrm = sqrt(fma(x0, x0, sg));
@@ -137,107 +132,163 @@ __global__ void __launch_bounds__(kTriThreads, 1) core_tridiag_kernel(const doub
       v0 = x0 - alpha;
       beta = 2.0 / fma(v0, v0, sg);
     }
-    if (t == 0) {
+    if (lane == 0) {
+      sh.refl[0] = beta;
+      sh.refl[1] = v0;
       S.e[j] = alpha;
       S.beta[j] = beta;
     }
-    if (isA && I == j / 4 && J == I) {
-      const int jm = j % 4;
-      double dj = a[0][0];
+  }
+  const bool row_ok = !scalar_warp && i < n;
+  const bool act = row_ok && i > j;                            // rows of the trailing block
+  const bool warp_live = !scalar_warp && 16 * warp + 15 > j;   // some row of the warp is active
+  // (a) u_i = sum_c A[i][c] x_c over the row's window
+  double u = 0.0;
+  if (warp_live) {
+    double s[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
+    const double* xw = xcur + base + h;
 #pragma unroll
-      for (int r = 1; r < 4; ++r) dj = r == jm ? a[r][r] : dj;
-      S.d[j] = dj;
-    }
-    if (beta == 0.0) {  // nothing to eliminate (uniform): column j + 1 is already final
-      for (int i = t; i < n; i += kTriThreads) S.V[j * n + i] = 0.0;
-      if (isA && J == (j + 1) / 4) publish_col(a, (j + 1) % 4, xn + 4 * I);
-      __syncthreads();
-      continue;
-    }
-    auto vel = [&](int i) { return i <= j ? 0.0 : (i == j + 1 ? v0 : x[i]); };
-    for (int i = t; i < n; i += kTriThreads) S.V[j * n + i] = vel(i);
-    // (a) partial products
-    const bool actA = isA && 4 * J + 3 > j;
-    if (actA) {
-      double vr[4], vc[4];
+    for (int c = 0; c < NH / 8; ++c) {
+      if (base + 16 * c < n) {
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        vr[r] = vel(4 * I + r);
-        vc[r] = vel(4 * J + r);
+        for (int r = 8 * c; r < 8 * c + 8; ++r) s[r & 7] = fma(a[r], xw[2 * r], s[r & 7]);
       }
+    }
+    u = ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
+  }
+  u += __shfl_xor_sync(0xFFFFFFFFu, u, 1);
+  const double ah = __shfl_sync(0xFFFFFFFFu, a[kHoldR], (lane & ~1) | hold_h);   // A[i][j+1]
+  const double xi = act ? xcur[i] : 0.0;
+  if (row_ok && i == j && h == ODD) S.d[j] = a[0];
+  double s1 = 0.0, s2 = 0.0;
+  if (h == 0 && act && i >= j + 2) {
+    s1 = u * xi;
+    s2 = ah * xi;
+  }
+  if (h == 0 && row_ok && i == j + 1) {
+    sh.row1[0] = u;
+    sh.row1[1] = ah;
+  }
 #pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        double s = 0.0;
+  for (int o = 16; o > 0; o >>= 1) {
+    s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, o);
+    s2 += __shfl_xor_sync(0xFFFFFFFFu, s2, o);
+  }
+  if (lane == 0 && !scalar_warp) {
+    sh.red1a[warp] = s1;
+    sh.red1b[warp] = s2;
+  }
+  __syncthreads();
+  // (b) p, K, q; column j + 1 and the next |x|^2
+  const double beta = sh.refl[0], v0 = sh.refl[1];
+  const double dv = v0 - xcur[j + 1];
+  const double S1 = sum_fixed(sh.red1a, nwr), S2 = sum_fixed(sh.red1b, nwr);
+  const double pj1 = beta * fma(sh.row1[1], dv, sh.row1[0]);
+  const double K = 0.5 * beta * fma(pj1, v0, beta * fma(dv, S2, S1));
+  const double pi = act ? beta * fma(ah, dv, u) : 0.0;
+  const double vi = !act ? 0.0 : (i == j + 1 ? v0 : xi);
+  const double qi = fma(-2.0 * K, vi, pi);
+  if (h == 0 && row_ok) {
+    pcur[i] = pi;
+    S.V[j * n + i] = beta == 0.0 ? 0.0 : vi;
+    if (i <= j + 1) xnext[i] = 0.0;
+  }
+  double sq = 0.0;
+  if (h == hold_h && row_ok) {
+    a[kHoldR] = fma(-qi, v0, fma(-vi, pj1, a[kHoldR]));
+    if (i >= j + 2) xnext[i] = a[kHoldR];
+    if (i >= j + 3) sq = a[kHoldR] * a[kHoldR];
+  }
+  sq = warp_sum(sq);
+  if (lane == 0 && !scalar_warp) sh.red2[warp] = sq;
+  __syncthreads();
+  // (c) the rest of the update: a_ic -= q_i v_c + v_i p_c (v_c = x_c past
+  // column j + 1, whose register was updated above)
+  if (warp_live) {
+    const double* xw = xcur + base + h;
+    const double* pw = pcur + base + h;
 #pragma unroll
-        for (int c = 0; c < 4; ++c) s = fma(a[r][c], vc[c], s);
-        partA[4 * t + r] = s;
-      }
-      if (I != J) {
+    for (int c = 0; c < NH / 8; ++c) {
+      if (base + 16 * c < n) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          double s = 0.0;
-#pragma unroll
-          for (int r = 0; r < 4; ++r) s = fma(a[r][c], vr[r], s);
-          partT[4 * t + c] = s;
+        for (int r = 8 * c; r < 8 * c + 8; ++r) {
+          if (h == hold_h && r == kHoldR) continue;
+          a[r] = fma(-qi, xw[2 * r], fma(-vi, pw[2 * r], a[r]));
         }
       }
     }
+  }
+}
+
+// One CTA of round32(2 n) + 32 threads, n <= 2 NH.
+template <int NH>
+__global__ void __launch_bounds__(4 * NH + 32, 1) core_tridiag_kernel(const double* C, int n, double* ws) {
+  __shared__ TriShared<NH> sh;
+  const EigScratch S = scratch(ws, n);
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int nwr = (blockDim.x >> 5) - 1;
+  const int i = t >> 1, h = t & 1;
+  const bool row_ok = warp < nwr && i < n;
+  double a[NH];
+#pragma unroll
+  for (int r = 0; r < NH; ++r) {
+    const int c = 2 * r + h;
+    a[r] = (row_ok && c < n) ? C[i * n + c] : 0.0;
+  }
+  for (int e = t; e < 2 * TriShared<NH>::kBuf; e += blockDim.x) {
+    (&sh.xb[0][0])[e] = 0.0;
+    (&sh.pb[0][0])[e] = 0.0;
+  }
+  __syncthreads();
+  {
+    // column 0: x_i = A[i][0] (i >= 1) and |x|^2 without x0
+    if (h == 0 && row_ok && i >= 1) sh.xb[0][i] = a[0];
+    const double s = warp_sum((h == 0 && row_ok && i >= 2) ? a[0] * a[0] : 0.0);
+    if (lane == 0 && warp < nwr) sh.red2[warp] = s;
     __syncthreads();
-    // (b) p_i (rows i > j): fixed-order sums of the tile partials
-    if (t < n) {
-      const int i = t;
-      if (i > j) {
-        const int Ii = i / 4, ri = i % 4;
-        // four interleaved partial sums in a fixed order (short dependent chains)
-        const int J0 = (j + 1) / 4;
-        const int na = Ii - J0 + 1, total = na + (nb - Ii - 1);
-        auto term = [&](int k) {
-          return k < na ? partA[4 * tri_pos(Ii, J0 + k, nb) + ri] : partT[4 * tri_pos(Ii + 1 + (k - na), Ii, nb) + ri];
-        };
-        double s0 = 0.0, s1 = 0.0, s2 = 0.0, s3 = 0.0;
-        int k = 0;
-        for (; k + 3 < total; k += 4) {
-          s0 += term(k);
-          s1 += term(k + 1);
-          s2 += term(k + 2);
-          s3 += term(k + 3);
+  }
+  int j = 0;
+  bool even_next = true;   // registers hold base = j
+  while (j + 2 < n) {
+    tri_step<NH, 0>(a, sh, S, j, n, i, h, lane, warp, nwr);
+    ++j;
+    even_next = false;
+    if (j + 2 >= n) break;
+    tri_step<NH, 1>(a, sh, S, j, n, i, h, lane, warp, nwr);
+    if (warp < nwr && 16 * warp + 15 > j) {
+      // move the row one register left (chunks past n hold zeros already)
+#pragma unroll
+      for (int c = 0; c < NH / 8; ++c) {
+        if (j - 1 + 16 * c < n) {
+#pragma unroll
+          for (int r = 8 * c; r < 8 * c + 8; ++r) a[r] = r + 1 < NH ? a[r + 1] : 0.0;
         }
-        if (k < total) s0 += term(k);
-        if (k + 1 < total) s1 += term(k + 1);
-        if (k + 2 < total) s2 += term(k + 2);
-        pb[i] = beta * ((s0 + s1) + (s2 + s3));
       }
     }
-    __syncthreads();
-    // (c) updates; K = (beta / 2) p^T v in every warp
-    double kk = 0.0;
-    for (int i = j + 1 + lane; i < n; i += 32) kk = fma(pb[i], vel(i), kk);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) kk += __shfl_xor_sync(0xFFFFFFFFu, kk, o);
-    const double K = 0.5 * beta * kk;
-    if (actA) {
-      double vr[4], wr[4], vc[4], wc[4];
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int i = 4 * I + r, c = 4 * J + r;
-        vr[r] = vel(i);
-        wr[r] = i > j ? fma(-K, vr[r], pb[i]) : 0.0;
-        vc[r] = vel(c);
-        wc[r] = c > j ? fma(-K, vc[r], pb[c]) : 0.0;
-      }
-#pragma unroll
-      for (int r = 0; r < 4; ++r)
-#pragma unroll
-        for (int c = 0; c < 4; ++c) a[r][c] -= fma(vr[r], wc[c], wr[r] * vc[c]);
-      if (J == (j + 1) / 4) publish_col(a, (j + 1) % 4, xn + 4 * I);
-    }
-    __syncthreads();
+    ++j;
+    even_next = true;
   }
-  if (isA && I == nb - 1 && J == nb - 1) {
-    S.d[n - 2] = a[2][2];
-    S.d[n - 1] = a[3][3];
-    S.e[n - 2] = a[3][2];
+  if (!row_ok) return;
+  if (n == 1) {
+    S.d[0] = a[0];
+    return;
   }
+  // the last 2 x 2 block, columns n - 2 and n - 1
+  if (even_next) {   // base = n - 2: column n - 2 in (h 0, r 0), n - 1 in (h 1, r 0)
+    if (i == n - 2 && h == 0) S.d[n - 2] = a[0];
+    if (i == n - 1 && h == 0) S.e[n - 2] = a[0];
+    if (i == n - 1 && h == 1) S.d[n - 1] = a[0];
+  } else {           // base = n - 3: column n - 2 in (h 1, r 0), n - 1 in (h 0, r 1)
+    if (i == n - 2 && h == 1) S.d[n - 2] = a[0];
+    if (i == n - 1 && h == 1) S.e[n - 2] = a[0];
+    if (i == n - 1 && h == 0) S.d[n - 1] = a[1];
+  }
+}
+
+template <int NH>
+void launch_tridiag(const double* C, int n, double* ws, cudaStream_t s) {
+  const int threads = (2 * n + 31) / 32 * 32 + 32;
+  core_tridiag_kernel<NH><<<1, threads, 0, s>>>(C, n, ws);
 }
 
 // ---------------------------------------------------------------------------
@@ -592,10 +643,10 @@ size_t core_eig_workspace(int n) { return (2 * static_cast<size_t>(n) * n + 4 * 
 
 void launch_core_eig(double* C, int n, int max_iters, double* eval, float* evec, double* ws, int32_t* dev_status,
                      cudaStream_t s) {
-  const int nb = n / 4, nA = nb * (nb + 1) / 2;
-  const size_t smem = (3 * static_cast<size_t>(n) + 8 * nA) * sizeof(double);
-  if (!ensure_smem(reinterpret_cast<const void*>(core_tridiag_kernel), smem)) return;
-  core_tridiag_kernel<<<1, kTriThreads, smem, s>>>(C, n, ws);
+  if (n <= 32) launch_tridiag<16>(C, n, ws, s);
+  else if (n <= 48) launch_tridiag<24>(C, n, ws, s);
+  else if (n <= 80) launch_tridiag<40>(C, n, ws, s);
+  else launch_tridiag<56>(C, n, ws, s);
   const size_t vsmem = static_cast<size_t>(n) * n * sizeof(double);
   if (!ensure_smem(reinterpret_cast<const void*>(core_vector_kernel), vsmem)) return;
   core_vector_kernel<<<n, 32, vsmem, s>>>(n, ws, max_iters, dev_status);
