@@ -166,14 +166,24 @@ metis_status enqueue_product(const metis_operand* A, const metis_operand* B, int
       if (B->P) {
         GemmCall g = base_call(A->R, B->P, M, p.kb, K, dev_status);
         g.bn = p.kb <= 64 ? 64 : 128;
-        g.C = b.t1;
         g.c_dtype = METIS_F32;
         g.ldc = p.kb;
         g.splits = p.s1;
         g.partial = b.t1p;
+        const int splits = gemm_effective_splits(K, p.s1);
+        if (splits > 1) {
+          // keep the partial sums: build_la adds them (no separate reduction)
+          g.C = nullptr;
+          la.t1part = b.t1p;
+          la.t1_splits = splits;
+          la.t1_ts_a = A->R->fmt == METIS_NVFP4 ? A->R->tensor_scale : nullptr;
+          la.t1_ts_b = B->P->fmt == METIS_NVFP4 ? B->P->tensor_scale : nullptr;
+        } else {
+          g.C = b.t1;
+          la.t1raw = b.t1;
+          la.t1_ld = p.kb;
+        }
         METIS_TRY(run_gemm_fp4(g, s));
-        la.t1raw = b.t1;
-        la.t1_ld = p.kb;
       } else {
         la.t1raw = A->R->inner_sum;  // R_A 1
         la.t1_ld = 1;

@@ -408,26 +408,25 @@ __global__ void __launch_bounds__(32) core_vector_kernel(int n, double* ws, int 
     if (!done && lane == 0) report(dev_status, METIS_DEV_NUMERIC);
     lam = 0.5 * (lo + hi);
     // twisted factorisation of T - lam I: lane 0 runs the top-down LDL^T
-    // recurrence, lane 1 the bottom-up UDU^T one at the same time
+    // recurrence, lane 1 the bottom-up UDU^T one, in lockstep (one
+    // instruction stream, per-lane indices)
     const double pivmin = 0x1p-100;
-    if (lane == 0) {
-      double Dp = d[0] - lam;
-      for (int i = 0; i + 1 < n; ++i) {
-        if (fabs(Dp) < pivmin) Dp = Dp < 0.0 ? -pivmin : pivmin;
-        dp[i] = Dp;
-        lp[i] = e[i] / Dp;
-        Dp = (d[i + 1] - lam) - lp[i] * e[i];
+    if (lane < 2) {
+      const bool up = lane == 1;
+      double* Dst = up ? dm : dp;
+      double* Lst = up ? um : lp;
+      double D = (up ? d[n - 1] : d[0]) - lam;
+      for (int st = 0; st + 1 < n; ++st) {
+        const int ie = up ? n - 2 - st : st;      // e index of this step
+        const int inext = up ? n - 2 - st : st + 1;
+        const double ee = e[ie], dn = d[inext];
+        if (fabs(D) < pivmin) D = D < 0.0 ? -pivmin : pivmin;
+        Dst[up ? n - 1 - st : st] = D;
+        const double l = ee / D;
+        Lst[ie] = l;
+        D = (dn - lam) - l * ee;
       }
-      dp[n - 1] = Dp;
-    } else if (lane == 1) {
-      double Dm = d[n - 1] - lam;
-      for (int i = n - 1; i > 0; --i) {
-        if (fabs(Dm) < pivmin) Dm = Dm < 0.0 ? -pivmin : pivmin;
-        dm[i] = Dm;
-        um[i - 1] = e[i - 1] / Dm;
-        Dm = (d[i - 1] - lam) - um[i - 1] * e[i - 1];
-      }
-      dm[0] = Dm;
+      Dst[up ? 0 : n - 1] = D;
     }
     __syncwarp();
     // twist index r: the smallest |gamma_r| = |D+_r + D-_r - (d_r - lam)|
@@ -450,23 +449,28 @@ __global__ void __launch_bounds__(32) core_vector_kernel(int n, double* ws, int 
         r = orr;
       }
     }
-    // z_r = 1; lane 0 walks up, lane 1 walks down (each rescales its own side
-    // by 1e-150 if it grows past 1e150; the sides are reconciled after)
+    // z_r = 1; lane 0 walks up, lane 1 walks down, in lockstep (each
+    // rescales its own side by 1e-150 if it grows past 1e150; the sides are
+    // reconciled after)
     int sc = 0;
-    if (lane == 0) {
-      for (int i = r - 1; i >= 0; --i) {
-        z[i] = -lp[i] * (i + 1 == r ? 1.0 : z[i + 1]);
-        if (fabs(z[i]) > 1e150) {
-          for (int q = i; q < r; ++q) z[q] *= 1e-150;
-          ++sc;
-        }
-      }
-    } else if (lane == 1) {
-      for (int i = r; i + 1 < n; ++i) {
-        z[i + 1] = -um[i] * (i == r ? 1.0 : z[i]);
-        if (fabs(z[i + 1]) > 1e150) {
-          for (int q = r + 1; q <= i + 1; ++q) z[q] *= 1e-150;
-          ++sc;
+    if (lane < 2) {
+      const bool up = lane == 0;
+      const double* mul = up ? lp : um;
+      const int steps = up ? r : n - 1 - r;
+      const int smax = r > n - 1 - r ? r : n - 1 - r;
+      double zc = 1.0;
+      for (int st = 0; st < smax; ++st) {
+        if (st < steps) {
+          const int i = up ? r - 1 - st : r + st;      // multiplier index
+          const int dst = up ? r - 1 - st : r + 1 + st;
+          zc = -mul[i] * zc;
+          z[dst] = zc;
+          if (fabs(zc) > 1e150) {
+            const int q0 = up ? dst : r + 1, q1 = up ? r - 1 : dst;
+            for (int q = q0; q <= q1; ++q) z[q] *= 1e-150;
+            zc *= 1e-150;
+            ++sc;
+          }
         }
       }
     }

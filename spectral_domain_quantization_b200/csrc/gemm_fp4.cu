@@ -353,6 +353,20 @@ __global__ void splitk_reduce_kernel(const float* partial, int splits, int64_t M
   }
 }
 
+}  // namespace
+
+int gemm_effective_splits(int64_t K, int splits) {
+  const int num_kt = static_cast<int>((K + 255) / 256);
+  int s = splits < 1 ? 1 : splits;
+  if (s > num_kt) s = num_kt;
+  // every split must own at least one K tile (an empty split would leave
+  // its accumulator unwritten): the fewest splits of the same length
+  const int per = (num_kt + s - 1) / s;
+  return (num_kt + per - 1) / per;
+}
+
+namespace {
+
 template <int BN, int STAGES, int CTAS>
 cudaError_t launch_bn(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& la,
                       const CUtensorMap& lb, int tiles, cudaStream_t s) {
@@ -403,14 +417,7 @@ metis_status run_gemm_fp4(const GemmCall& g, cudaStream_t s) {
   p.ldc = g.ldc;
   p.vec_ok = (g.ldc % 4 == 0) && ((reinterpret_cast<uintptr_t>(g.C) & 15u) == 0);
   p.dev_status = g.dev_status;
-  p.splits = g.splits < 1 ? 1 : g.splits;
-  if (p.splits > p.num_kt) p.splits = p.num_kt;
-  {
-    // every split must own at least one K tile (an empty split would leave
-    // its accumulator unwritten): use the fewest splits of the same length
-    const int per = (p.num_kt + p.splits - 1) / p.splits;
-    p.splits = (p.num_kt + per - 1) / per;
-  }
+  p.splits = gemm_effective_splits(g.K, g.splits);
   p.partial = g.partial;
   if (p.splits > 1 && !p.partial) return METIS_ERR_ARG;
   if (p.splits > 1 && p.lr_chunks) return METIS_ERR_ARG;

@@ -54,4 +54,10 @@ struct GemmCall {
 
 metis_status run_gemm_fp4(const GemmCall& g, cudaStream_t s);
 
+// The split count run_gemm_fp4 uses for a requested one: at most one split
+// per 256-element K tile, and the fewest splits of the same length (so
+// every split owns at least one K tile).  Partial sums are laid out
+// [split][M][N].
+int gemm_effective_splits(int64_t K, int splits);
+
 }  // namespace metis

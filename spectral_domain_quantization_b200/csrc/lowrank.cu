@@ -65,63 +65,74 @@ MDEV float alpha_main(const LowRankArgs& a) {
   return v;
 }
 
-// LA rows: one thread per (m, column of LA).
+// T1 element (m, j) before S_B: from T1 itself or from its split-K
+// partials, summed in split order and scaled as the GEMM's own split-K
+// reduction does (the same float operations, so the same value).
+MDEV float t1_value(const LowRankArgs& a, int64_t m, int j) {
+  if (a.t1part) {
+    float s = 0.f;
+    for (int k = 0; k < a.t1_splits; ++k) s += a.t1part[(k * a.M + m) * a.kb + j];
+    float alpha = 1.f;
+    if (a.t1_ts_a) alpha = __fmul_rn(alpha, *a.t1_ts_a);
+    if (a.t1_ts_b) alpha = __fmul_rn(alpha, *a.t1_ts_b);
+    return __fmul_rn(alpha, s);
+  }
+  return a.t1raw ? a.t1raw[m * a.t1_ld + j] : 0.f;
+}
+
+// LA: a row per block iteration, a column per thread.
 __global__ void build_la_kernel(LowRankArgs a) {
-  const int64_t total = a.M * a.lr_k;
   const float inv_alpha = 1.f / alpha_main(a);
   const float s_fb = tscale(a.fb);
   const float s_fa = tscale(a.fa);
-  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
-       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t m = t / a.lr_k;
-    const int c = static_cast<int>(t - m * a.lr_k);
-    __nv_bfloat16 out = __float2bfloat16_rn(0.f);
-    if (c < 2 * a.kb) {
-      const int j = c % a.kb;
-      float v = a.t1raw ? a.t1raw[m * a.t1_ld + j] : 0.f;
-      if (a.ka > 0 && a.cab) {
-        float acc = 0.f;
-        for (int i = 0; i < a.ka; ++i) {
-          const float sa = a.s_a ? a.s_a[i] : 1.f;
-          acc += factor_value(a.fa, i, m) * s_fa * sa * a.cab[i * a.kb + j];
+  for (int64_t m = blockIdx.x; m < a.M; m += gridDim.x) {
+    for (int c = threadIdx.x; c < a.lr_k; c += blockDim.x) {
+      __nv_bfloat16 out = __float2bfloat16_rn(0.f);
+      if (c < 2 * a.kb) {
+        const int j = c < a.kb ? c : c - a.kb;
+        float v = t1_value(a, m, j);
+        if (a.ka > 0 && a.cab) {
+          float acc = 0.f;
+          for (int i = 0; i < a.ka; ++i) {
+            const float sa = a.s_a ? a.s_a[i] : 1.f;
+            acc += factor_value(a.fa, i, m) * s_fa * sa * a.cab[i * a.kb + j];
+          }
+          v += acc;
         }
-        v += acc;
+        const float sb = a.s_b ? a.s_b[j] : 1.f;
+        v = v * sb * s_fb * inv_alpha;
+        __nv_bfloat16 hi, lo;
+        split_hi_lo(v, hi, lo);
+        out = c < a.kb ? hi : lo;
+      } else if (c < 2 * a.kb + 2 * a.ka) {
+        const int i = (c - 2 * a.kb) % a.ka;
+        out = __float2bfloat16_rn(factor_value(a.fa, i, m));
       }
-      const float sb = a.s_b ? a.s_b[j] : 1.f;
-      v = v * sb * s_fb * inv_alpha;
-      __nv_bfloat16 hi, lo;
-      split_hi_lo(v, hi, lo);
-      out = c < a.kb ? hi : lo;
-    } else if (c < 2 * a.kb + 2 * a.ka) {
-      const int i = (c - 2 * a.kb) % a.ka;
-      out = __float2bfloat16_rn(factor_value(a.fa, i, m));
+      a.la[m * a.lr_k + c] = out;
     }
-    a.la[m * a.lr_k + c] = out;
   }
 }
 
-// LB rows: one thread per (n, column of LB).
+// LB: a row per block iteration, a column per thread.
 __global__ void build_lb_kernel(LowRankArgs a) {
-  const int64_t total = a.N * a.lr_k;
   const float inv_alpha = 1.f / alpha_main(a);
   const float s_fa = tscale(a.fa);
-  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
-       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t n = t / a.lr_k;
-    const int c = static_cast<int>(t - n * a.lr_k);
-    __nv_bfloat16 out = __float2bfloat16_rn(0.f);
-    if (c < 2 * a.kb) {
-      out = __float2bfloat16_rn(factor_value(a.fb, c % a.kb, n));
-    } else if (c < 2 * a.kb + 2 * a.ka) {
-      const int cc = c - 2 * a.kb;
-      const int i = cc % a.ka;
-      const float sa = a.s_a ? a.s_a[i] : 1.f;
-      const float v = a.t2raw[i * a.t2_ld + n] * sa * s_fa * inv_alpha;
-      __nv_bfloat16 hi, lo;
-      split_hi_lo(v, hi, lo);
-      out = cc < a.ka ? hi : lo;
+  for (int64_t n = blockIdx.x; n < a.N; n += gridDim.x) {
+    for (int c = threadIdx.x; c < a.lr_k; c += blockDim.x) {
+      __nv_bfloat16 out = __float2bfloat16_rn(0.f);
+      if (c < 2 * a.kb) {
+        out = __float2bfloat16_rn(factor_value(a.fb, c < a.kb ? c : c - a.kb, n));
+      } else if (c < 2 * a.kb + 2 * a.ka) {
+        const int cc = c - 2 * a.kb;
+        const int i = cc % a.ka;
+        const float sa = a.s_a ? a.s_a[i] : 1.f;
+        const float v = a.t2raw[i * a.t2_ld + n] * sa * s_fa * inv_alpha;
+        __nv_bfloat16 hi, lo;
+        split_hi_lo(v, hi, lo);
+        out = cc < a.ka ? hi : lo;
+      }
+      a.lb[n * a.lr_k + c] = out;
     }
-    a.lb[n * a.lr_k + c] = out;
   }
 }
 
@@ -144,9 +155,15 @@ void launch_cab(const FactorView& pa, const FactorView& pb, int64_t K, int ka, i
   cab_kernel<<<dim3(kb, ka), 256, 0, s>>>(pa, pb, K, kb, cab);
 }
 
+int row_blocks(int64_t rows, int sms) {
+  const int64_t b = rows < sms * 16 ? rows : sms * 16;
+  return static_cast<int>(b < 1 ? 1 : b);
+}
+
 void launch_build_lowrank(const LowRankArgs& a, int sms, cudaStream_t s) {
-  build_la_kernel<<<blocks_for(a.M * a.lr_k, sms), 256, 0, s>>>(a);
-  build_lb_kernel<<<blocks_for(a.N * a.lr_k, sms), 256, 0, s>>>(a);
+  const int threads = a.lr_k >= 128 ? 128 : 64;
+  build_la_kernel<<<row_blocks(a.M, sms), threads, 0, s>>>(a);
+  build_lb_kernel<<<row_blocks(a.N, sms), threads, 0, s>>>(a);
 }
 
 void launch_copy(const float* src, float* dst, int64_t n, int sms, cudaStream_t s) {

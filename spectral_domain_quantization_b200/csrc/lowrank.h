@@ -31,6 +31,10 @@ struct LowRankArgs {
   const float* s_b;         // S_B (kb) or NULL
   const float* t1raw;       // R_A P_B, M x kb (row stride t1_ld), or NULL
   int64_t t1_ld;
+  const float* t1part;      // or its split-K partial sums (t1_splits x M x kb), summed here
+  int t1_splits;
+  const float* t1_ts_a;     // tensor scales of that product's operands (NVFP4) or NULL
+  const float* t1_ts_b;
   const float* t2raw;       // P_A^T R_B, ka x N (row stride t2_ld)
   int64_t t2_ld;
   const float* cab;         // P_A^T P_B, ka x kb, or NULL

@@ -1,24 +1,19 @@
-// Small dense linear algebra of the randomized split (l = k + p <= 128):
-// Gram matrices, Cholesky with rank drop, triangular inverse (CholeskyQR),
-// row-block products, the Jacobi eigensolver of the core, factor assembly and
-// the sign convention.
+// Small dense linear algebra of the randomized split (l = k + p <= 112):
+// Gram matrices, Cholesky with rank drop and triangular inverse (CholeskyQR),
+// row-block products, factor assembly and the sign convention.  The core's
+// eigen-decomposition lives in core_eig.cu.
 //
 // Source: SII release on Metis, section 2.4 item 1 (spectral decomposition in
 // a low-dimensional space after randomized reduction); older Metis abstract
 // item (i) (random embedding separates dominant from long-tail parts).
 //
 // Numerics: Gram matrices are accumulated in float64 from float32 rows;
-// Cholesky, the triangular inverse and Jacobi run in float64 in one CTA's
-// shared memory; tall row blocks are multiplied in float32.
+// Cholesky and the triangular inverse run in float64 in one CTA; tall row
+// blocks are multiplied in float32.
 //   * CholeskyQR: G = Y^T Y = L L^T, Q = Y L^-T.  A pivot that falls below
 //     1e-12 of its original diagonal (a numerically dependent sketch column,
 //     e.g. for an exactly low-rank input) is dropped: that column of Q
 //     becomes zero instead of amplified rounding noise.
-//   * Core SVD via one-sided Jacobi of B^T, carried out on its l x l Gram
-//     C = B B^T (rotations chosen from the Gram entries, as one-sided Jacobi
-//     does): C = W diag(sigma^2) W^T, then U = Q W_k, V = B^T W_k / sigma.
-//     Rotations use the parallel (round-robin) ordering: l/2 disjoint pairs
-//     per step, l-1 steps per sweep.
 #include "common.cuh"
 #include "abi_common.h"
 #include "small_linalg.h"
@@ -163,14 +158,147 @@ MDEV int tri_element(int e, int n) {
 constexpr int kSmallThreads = 512;
 constexpr int kTile = 4;  // register tile edge and panel width of the Cholesky
 
+// Block row BI of X = L^-1 (16 x 16 blocks, o = 16 BI), after blocks
+// 0 .. BI-1 of X and the diagonal block X(BI, BI) are known:
+//   T = L(BI, 0:BI) X(0:BI, 0:BI)   and   X(BI, 0:BI) = -X(BI, BI) T.
+// Thread t < 256 owns row r = t / 16 of the block row and the columns
+// c0 + 16 u (c0 = t % 16, u < BI): 16 lanes read 16 consecutive entries of
+// an X row (no bank conflicts).  Only the lower block triangle of X is
+// read: row block mb of the sum meets column blocks u <= mb (the diagonal
+// blocks hold zeros above their diagonal).  Two accumulators per column
+// (even and odd m) halve the dependent chains.
+template <int BI>
+MDEV void inverse_block_row(const double* L, double* X, double* T, int ld, int t) {
+  constexpr int o = 16 * BI;
+  const int r = t >> 4, c0 = t & 15;
+  if (t < 256) {
+    double e[BI], f[BI];
+#pragma unroll
+    for (int u = 0; u < BI; ++u) e[u] = f[u] = 0.0;
+    const double* Lr = L + (o + r) * ld;
+#pragma unroll
+    for (int mb = 0; mb < BI; ++mb) {
+#pragma unroll 4
+      for (int mm = 0; mm < 16; mm += 2) {
+        const int m = 16 * mb + mm;
+        const double l0 = Lr[m], l1 = Lr[m + 1];
+        const double* X0 = X + m * ld + c0;
+        const double* X1 = X0 + ld;
+#pragma unroll
+        for (int u = 0; u <= mb; ++u) {
+          e[u] = fma(l0, X0[16 * u], e[u]);
+          f[u] = fma(l1, X1[16 * u], f[u]);
+        }
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < BI; ++u) T[r * ld + c0 + 16 * u] = e[u] + f[u];
+  }
+  __syncthreads();
+  if (t < 256) {
+    double acc[BI];
+#pragma unroll
+    for (int u = 0; u < BI; ++u) acc[u] = 0.0;
+    const double* Xr = X + (o + r) * ld + o;
+    for (int q = 0; q <= r; ++q) {
+      const double x = Xr[q];
+#pragma unroll
+      for (int u = 0; u < BI; ++u) acc[u] = fma(x, T[q * ld + c0 + 16 * u], acc[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < BI; ++u) X[(o + r) * ld + c0 + 16 * u] = -acc[u];
+  }
+  __syncthreads();
+}
+
+// Warp 0: factor panel K (columns 4K .. 4K+3, rows 4K .. lp-1, held in P
+// as lp x 4) in place: a lane per row (rows r0 + lane + 32 q), the pivot row
+// broadcast by shuffles.  Writes L's columns, 1/sqrt(pivot) and sqrt(pivot).
+MDEV void factor_panel(int K, double* P, double* L, double* invd, double* sqd, const double* diag0, int lp,
+                       int ld, int lane) {
+  const int r0 = kTile * K;
+  double pr[4][kTile];  // rows r0 + lane + 32 q
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int row = r0 + lane + 32 * q;
+#pragma unroll
+    for (int c = 0; c < kTile; ++c) pr[q][c] = row < lp ? P[row * kTile + c] : 0.0;
+  }
+  double rinv[kTile], rsq[kTile];
+#pragma unroll
+  for (int c = 0; c < kTile; ++c) {
+    const int gc = r0 + c;
+    const double d = __shfl_sync(0xFFFFFFFFu, pr[0][c], c);  // row gc lives in lane c, q = 0
+    double prow[kTile];
+#pragma unroll
+    for (int cc = 0; cc < kTile; ++cc) prow[cc] = __shfl_sync(0xFFFFFFFFu, pr[0][cc], c);
+    const bool drop = !(diag0[gc] > 0.0) || !(d > kDropTol * diag0[gc]);
+    rinv[c] = drop ? 0.0 : rsqrt(d);
+    rsq[c] = d * rinv[c];
+    const double inv2 = rinv[c] * rinv[c];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int row = r0 + lane + 32 * q;
+      if (row > gc) {
+#pragma unroll
+        for (int cc = c + 1; cc < kTile; ++cc) pr[q][cc] = fma(-pr[q][c], prow[cc] * inv2, pr[q][cc]);
+      }
+    }
+  }
+  if (lane < kTile) {
+    double ri = rinv[0], rs = rsq[0];
+#pragma unroll
+    for (int c = 1; c < kTile; ++c) {
+      ri = lane == c ? rinv[c] : ri;
+      rs = lane == c ? rsq[c] : rs;
+    }
+    invd[r0 + lane] = ri;
+    sqd[r0 + lane] = rs;
+  }
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int row = r0 + lane + 32 * q;
+    if (row < lp) {
+#pragma unroll
+      for (int c = 0; c < kTile; ++c) {
+        const int gc = r0 + c;
+        const double l = row == gc ? rsq[c] : (row > gc ? pr[q][c] * rinv[c] : 0.0);
+        P[row * kTile + c] = l;
+        L[row * ld + gc] = l;
+      }
+    }
+  }
+}
+
+// Rank-4 update of the register tile (I, J) with panel P: v -= L(I, K) L(J, K)^T.
+MDEV void panel_update(double (&v)[kTile][kTile], const double* P, int I, int J) {
+  double li[kTile][kTile], lj[kTile][kTile];
+#pragma unroll
+  for (int a = 0; a < kTile; ++a)
+#pragma unroll
+    for (int c = 0; c < kTile; ++c) {
+      li[a][c] = P[(kTile * I + a) * kTile + c];
+      lj[a][c] = P[(kTile * J + a) * kTile + c];
+    }
+#pragma unroll
+  for (int a = 0; a < kTile; ++a)
+#pragma unroll
+    for (int b = 0; b < kTile; ++b) {
+      double s = v[a][b];
+#pragma unroll
+      for (int c = 0; c < kTile; ++c) s = fma(-li[a][c], lj[b][c], s);
+      v[a][b] = s;
+    }
+}
+
 // G = L L^T (with drops), then Rinv = L^-T (upper triangular, float32).
-//  Cholesky, right-looking by panels of 4 columns, two barriers per panel:
-//  thread T owns the 4 x 4 tile (I, J), I >= J, of the lower triangle in
-//  registers.  Panel K (columns 4K .. 4K+3, rows 4K .. lp-1) sits in shared
-//  memory; warp 0 factors it alone (a lane per row, the pivot row broadcast
-//  by shuffles, no block barrier); then every tile right of it takes the
-//  rank-4 update v -= L(I, K) L(J, K)^T and the tiles of column K + 1 write
-//  themselves into the next panel buffer.
+//  Cholesky, right-looking by panels of 4 columns with look-ahead: thread
+//  32 + T owns the 4 x 4 tile (I, J), I >= J, of the lower triangle in
+//  registers; panel K sits in shared memory.  Per panel, two barriers:
+//    (1) the tiles of column K + 1 take the rank-4 update of panel K and
+//        write themselves into the next panel buffer;
+//    (2) warp 0 factors panel K + 1 while every other tile right of it
+//        takes the update of panel K.
 //  Inverse: X = L^-1 by 16 x 16 blocks (see below).
 __global__ void __launch_bounds__(kSmallThreads, 1) cholesky_inv_kernel(const double* G, int lp, float* Rinv) {
   extern __shared__ double sm[];
@@ -185,9 +313,9 @@ __global__ void __launch_bounds__(kSmallThreads, 1) cholesky_inv_kernel(const do
   const int ntiles = nb * (nb + 1) / 2;
   int I = 0, J = 0;
   double v[kTile][kTile];
-  const bool owner = t < ntiles;
+  const bool owner = t >= 32 && t - 32 < ntiles;
   if (owner) {
-    const int ij = tri_element(t, nb);
+    const int ij = tri_element(t - 32, nb);
     I = ij >> 8;
     J = ij & 255;
 #pragma unroll
@@ -206,89 +334,23 @@ __global__ void __launch_bounds__(kSmallThreads, 1) cholesky_inv_kernel(const do
     }
   }
   __syncthreads();
-  for (int K = 0; K < nb; ++K) {
-    double* P = pan + (K & 1) * 4 * lp;
+  if (warp == 0) factor_panel(0, pan, L, invd, sqd, diag0, lp, ld, lane);
+  __syncthreads();
+  for (int K = 0; K + 1 < nb; ++K) {
+    const double* P = pan + (K & 1) * 4 * lp;
     double* Pn = pan + ((K + 1) & 1) * 4 * lp;
-    const int r0 = kTile * K;
-    if (warp == 0) {
-      double pr[4][kTile];  // rows r0 + lane + 32 q
+    if (owner && J == K + 1) {
+      panel_update(v, P, I, J);
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int row = r0 + lane + 32 * q;
+      for (int a = 0; a < kTile; ++a)
 #pragma unroll
-        for (int c = 0; c < kTile; ++c) pr[q][c] = row < lp ? P[row * kTile + c] : 0.0;
-      }
-      double rinv[kTile], rsq[kTile];
-#pragma unroll
-      for (int c = 0; c < kTile; ++c) {
-        const int gc = r0 + c;
-        const double d = __shfl_sync(0xFFFFFFFFu, pr[0][c], c);  // row gc lives in lane c, q = 0
-        const bool drop = !(diag0[gc] > 0.0) || !(d > kDropTol * diag0[gc]);
-        rinv[c] = drop ? 0.0 : rsqrt(d);
-        rsq[c] = d * rinv[c];
-        const double inv2 = rinv[c] * rinv[c];
-        double prow[kTile];
-#pragma unroll
-        for (int cc = 0; cc < kTile; ++cc) prow[cc] = __shfl_sync(0xFFFFFFFFu, pr[0][cc], c) * inv2;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int row = r0 + lane + 32 * q;
-          if (row > gc) {
-#pragma unroll
-            for (int cc = c + 1; cc < kTile; ++cc) pr[q][cc] = fma(-pr[q][c], prow[cc], pr[q][cc]);
-          }
-        }
-      }
-      if (lane < kTile) {
-        double ri = rinv[0], rs = rsq[0];
-#pragma unroll
-        for (int c = 1; c < kTile; ++c) {
-          ri = lane == c ? rinv[c] : ri;
-          rs = lane == c ? rsq[c] : rs;
-        }
-        invd[r0 + lane] = ri;
-        sqd[r0 + lane] = rs;
-      }
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int row = r0 + lane + 32 * q;
-        if (row < lp) {
-#pragma unroll
-          for (int c = 0; c < kTile; ++c) {
-            const int gc = r0 + c;
-            const double l = row == gc ? rsq[c] : (row > gc ? pr[q][c] * rinv[c] : 0.0);
-            P[row * kTile + c] = l;
-            L[row * ld + gc] = l;
-          }
-        }
-      }
+        for (int b = 0; b < kTile; ++b) Pn[(kTile * I + a) * kTile + b] = v[a][b];
     }
     __syncthreads();
-    if (owner && J > K) {
-      double li[kTile][kTile], lj[kTile][kTile];
-#pragma unroll
-      for (int a = 0; a < kTile; ++a)
-#pragma unroll
-        for (int c = 0; c < kTile; ++c) {
-          li[a][c] = P[(kTile * I + a) * kTile + c];
-          lj[a][c] = P[(kTile * J + a) * kTile + c];
-        }
-#pragma unroll
-      for (int a = 0; a < kTile; ++a)
-#pragma unroll
-        for (int b = 0; b < kTile; ++b) {
-          double s = v[a][b];
-#pragma unroll
-          for (int c = 0; c < kTile; ++c) s = fma(-li[a][c], lj[b][c], s);
-          v[a][b] = s;
-        }
-      if (J == K + 1) {
-#pragma unroll
-        for (int a = 0; a < kTile; ++a)
-#pragma unroll
-          for (int b = 0; b < kTile; ++b) Pn[(kTile * I + a) * kTile + b] = v[a][b];
-      }
-    }
+    if (warp == 0)
+      factor_panel(K + 1, Pn, L, invd, sqd, diag0, lp, ld, lane);
+    else if (owner && J > K + 1)
+      panel_update(v, P, I, J);
     __syncthreads();
   }
   // X = L^-1 by 16 x 16 blocks: the diagonal blocks are inverted by one warp
@@ -313,32 +375,19 @@ __global__ void __launch_bounds__(kSmallThreads, 1) cholesky_inv_kernel(const do
   }
   __syncthreads();
   for (int bi = 1; bi < nb16; ++bi) {
-    const int o = 16 * bi;
-    for (int e = t; e < 16 * o; e += kSmallThreads) {
-      const int r = e / o, c = e - r * o;
-      double s4[4] = {0.0, 0.0, 0.0, 0.0};
-      int m = c;
-      for (; m + 3 < o; m += 4) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) s4[u] = fma(L[(o + r) * ld + m + u], X[(m + u) * ld + c], s4[u]);
-      }
-      for (; m < o; ++m) s4[0] = fma(L[(o + r) * ld + m], X[m * ld + c], s4[0]);
-      T[r * ld + c] = (s4[0] + s4[1]) + (s4[2] + s4[3]);
+    switch (bi) {
+      case 1: inverse_block_row<1>(L, X, T, ld, t); break;
+      case 2: inverse_block_row<2>(L, X, T, ld, t); break;
+      case 3: inverse_block_row<3>(L, X, T, ld, t); break;
+      case 4: inverse_block_row<4>(L, X, T, ld, t); break;
+      case 5: inverse_block_row<5>(L, X, T, ld, t); break;
+      default: inverse_block_row<6>(L, X, T, ld, t); break;
     }
-    __syncthreads();
-    for (int e = t; e < 16 * o; e += kSmallThreads) {
-      const int r = e / o, c = e - r * o;
-      double sum = 0.0;
-      for (int q = 0; q <= r; ++q) sum += X[(o + r) * ld + o + q] * T[q * ld + c];
-      X[(o + r) * ld + c] = -sum;
-    }
-    __syncthreads();
   }
-  // Rinv[c][r] = X[r][c] (upper triangular)
-  for (int e = t; e < lp * lp; e += kSmallThreads) {
-    const int c = e / lp, r = e - c * lp;
-    Rinv[e] = r >= c ? static_cast<float>(X[r * ld + c]) : 0.f;
-  }
+  // Rinv[c][r] = X[r][c] (upper triangular): a warp per column c, lanes
+  // along r (coalesced stores)
+  for (int c = warp; c < lp; c += kSmallThreads / 32)
+    for (int r = lane; r < lp; r += 32) Rinv[c * lp + r] = r >= c ? static_cast<float>(X[r * ld + c]) : 0.f;
 }
 
 constexpr int kApplyRows = 32;
