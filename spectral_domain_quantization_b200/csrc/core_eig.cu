@@ -85,8 +85,9 @@ template <int NH>
 struct TriShared {
   static constexpr int kBuf = 4 * NH + 8;   // row windows reach base + 2 NH - 1 <= n + 2 NH - 4
   static constexpr int kWarps = (4 * NH + 31) / 32;
-  double xb[2][kBuf];   // x entries of the column by row (0 outside the active rows)
-  double pb[2][kBuf];   // p_i by row (0 outside the active rows)
+  // per column parity, by row: .x = x entry of the column, .y = p_i (both 0
+  // outside the active rows); the update reads both with one 16-byte load
+  double2 xp[2][kBuf];
   double red1a[kWarps], red1b[kWarps], red2[kWarps];
   double row1[2];       // row j + 1: u_{j+1} and A[j+1][j+1]
   double refl[2];       // beta, v0 of the current column
@@ -118,13 +119,12 @@ MDEV void tri_step(double (&a)[NH], TriShared<NH>& sh, const EigScratch& S, int 
   constexpr int kHoldR = ODD ? 1 : 0;   // register of column j + 1, in thread h = 1 - ODD
   const int hold_h = 1 - ODD;
   const int base = j - ODD;
-  const double* xcur = sh.xb[j & 1];
-  double* xnext = sh.xb[(j + 1) & 1];
-  double* pcur = sh.pb[j & 1];
+  double2* cur = sh.xp[j & 1];
+  double2* nxt = sh.xp[(j + 1) & 1];
   const bool scalar_warp = warp == nwr;
   if (scalar_warp) {
     const double sg = sum_fixed(sh.red2, nwr);
-    const double x0 = xcur[j + 1];
+    const double x0 = cur[j + 1].x;
     double alpha = x0, beta = 0.0, v0 = 0.0;
     if (sg > 0.0) {
       const double nrm = sqrt(fma(x0, x0, sg));
@@ -146,19 +146,19 @@ MDEV void tri_step(double (&a)[NH], TriShared<NH>& sh, const EigScratch& S, int 
   double u = 0.0;
   if (warp_live) {
     double s[8] = {0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0, 0.0};
-    const double* xw = xcur + base + h;
+    const double2* xw = cur + base + h;
 #pragma unroll
     for (int c = 0; c < NH / 8; ++c) {
       if (base + 16 * c < n) {
 #pragma unroll
-        for (int r = 8 * c; r < 8 * c + 8; ++r) s[r & 7] = fma(a[r], xw[2 * r], s[r & 7]);
+        for (int r = 8 * c; r < 8 * c + 8; ++r) s[r & 7] = fma(a[r], xw[2 * r].x, s[r & 7]);
       }
     }
     u = ((s[0] + s[1]) + (s[2] + s[3])) + ((s[4] + s[5]) + (s[6] + s[7]));
   }
   u += __shfl_xor_sync(0xFFFFFFFFu, u, 1);
   const double ah = __shfl_sync(0xFFFFFFFFu, a[kHoldR], (lane & ~1) | hold_h);   // A[i][j+1]
-  const double xi = act ? xcur[i] : 0.0;
+  const double xi = act ? cur[i].x : 0.0;
   if (row_ok && i == j && h == ODD) S.d[j] = a[0];
   double s1 = 0.0, s2 = 0.0;
   if (h == 0 && act && i >= j + 2) {
@@ -181,7 +181,7 @@ MDEV void tri_step(double (&a)[NH], TriShared<NH>& sh, const EigScratch& S, int 
   __syncthreads();
   // (b) p, K, q; column j + 1 and the next |x|^2
   const double beta = sh.refl[0], v0 = sh.refl[1];
-  const double dv = v0 - xcur[j + 1];
+  const double dv = v0 - cur[j + 1].x;
   const double S1 = sum_fixed(sh.red1a, nwr), S2 = sum_fixed(sh.red1b, nwr);
   const double pj1 = beta * fma(sh.row1[1], dv, sh.row1[0]);
   const double K = 0.5 * beta * fma(pj1, v0, beta * fma(dv, S2, S1));
@@ -189,14 +189,14 @@ MDEV void tri_step(double (&a)[NH], TriShared<NH>& sh, const EigScratch& S, int 
   const double vi = !act ? 0.0 : (i == j + 1 ? v0 : xi);
   const double qi = fma(-2.0 * K, vi, pi);
   if (h == 0 && row_ok) {
-    pcur[i] = pi;
+    cur[i].y = pi;
     S.V[j * n + i] = beta == 0.0 ? 0.0 : vi;
-    if (i <= j + 1) xnext[i] = 0.0;
+    if (i <= j + 1) nxt[i].x = 0.0;
   }
   double sq = 0.0;
   if (h == hold_h && row_ok) {
     a[kHoldR] = fma(-qi, v0, fma(-vi, pj1, a[kHoldR]));
-    if (i >= j + 2) xnext[i] = a[kHoldR];
+    if (i >= j + 2) nxt[i].x = a[kHoldR];
     if (i >= j + 3) sq = a[kHoldR] * a[kHoldR];
   }
   sq = warp_sum(sq);
@@ -205,15 +205,15 @@ MDEV void tri_step(double (&a)[NH], TriShared<NH>& sh, const EigScratch& S, int 
   // (c) the rest of the update: a_ic -= q_i v_c + v_i p_c (v_c = x_c past
   // column j + 1, whose register was updated above)
   if (warp_live) {
-    const double* xw = xcur + base + h;
-    const double* pw = pcur + base + h;
+    const double2* xw = cur + base + h;
 #pragma unroll
     for (int c = 0; c < NH / 8; ++c) {
       if (base + 16 * c < n) {
 #pragma unroll
         for (int r = 8 * c; r < 8 * c + 8; ++r) {
           if (h == hold_h && r == kHoldR) continue;
-          a[r] = fma(-qi, xw[2 * r], fma(-vi, pw[2 * r], a[r]));
+          const double2 xpc = xw[2 * r];
+          a[r] = fma(-qi, xpc.x, fma(-vi, xpc.y, a[r]));
         }
       }
     }
@@ -235,14 +235,11 @@ __global__ void __launch_bounds__(4 * NH + 32, 1) core_tridiag_kernel(const doub
     const int c = 2 * r + h;
     a[r] = (row_ok && c < n) ? C[i * n + c] : 0.0;
   }
-  for (int e = t; e < 2 * TriShared<NH>::kBuf; e += blockDim.x) {
-    (&sh.xb[0][0])[e] = 0.0;
-    (&sh.pb[0][0])[e] = 0.0;
-  }
+  for (int e = t; e < 2 * TriShared<NH>::kBuf; e += blockDim.x) (&sh.xp[0][0])[e] = make_double2(0.0, 0.0);
   __syncthreads();
   {
     // column 0: x_i = A[i][0] (i >= 1) and |x|^2 without x0
-    if (h == 0 && row_ok && i >= 1) sh.xb[0][i] = a[0];
+    if (h == 0 && row_ok && i >= 1) sh.xp[0][i].x = a[0];
     const double s = warp_sum((h == 0 && row_ok && i >= 2) ? a[0] * a[0] : 0.0);
     if (lane == 0 && warp < nwr) sh.red2[warp] = s;
     __syncthreads();

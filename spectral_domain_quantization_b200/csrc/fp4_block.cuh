@@ -47,6 +47,35 @@ MDEV uint32_t quant_block_nv(const float* v, float s_t, uint64_t& packed, float&
   return dc;
 }
 
+// The NVFP4 encode factors of one tensor: entry dc = 1 / (d(dc) s_t) for
+// every E4M3 scale code dc (0 where d = 0), by the same float operations as
+// quant_block_nv, so a block quantized through the table has the same codes.
+// The calling CTA fills the 128 entries and synchronises before use.
+MDEV void nv_enc_table(float s_t, float* tab) {
+  for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+    const float d = e4m3_value(static_cast<uint32_t>(c));
+    tab[c] = d == 0.f ? 0.f : __fdiv_rn(1.f, __fmul_rn(d, s_t));
+  }
+}
+
+// quant_block_nv without the per-block reciprocal (taken from nv_enc_table).
+MDEV uint32_t quant_block_nv_tab(const float* v, float s_t, const float* enc_tab, uint64_t& packed) {
+  float a = 0.f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[i]));
+  const float t = __fdiv_rn(__fdiv_rn(a, s_t), 6.f);
+  const uint32_t dc = e4m3_code(t);
+  packed = 0;
+  if (dc == 0u) return dc;  // d(0) = 0 and every other code has d > 0
+  const float enc = enc_tab[dc];
+  float q[16];
+#pragma unroll
+  for (int i = 0; i < 16; ++i) q[i] = __fmul_rn(v[i], enc);
+  const uint32_t w0 = e2m1_pack8(q), w1 = e2m1_pack8(q + 8);
+  packed = static_cast<uint64_t>(w0) | (static_cast<uint64_t>(w1) << 32);
+  return dc;
+}
+
 // MXFP4 block of 32.  Returns the E8M0 scale code; writes 32 nibbles to
 // packed[0..1] and, when SUM, the sum of dequantized values to `dsum`.
 template <bool SUM = false>

@@ -135,15 +135,25 @@ template <int FMT, bool BF16>
 __global__ void __launch_bounds__(256) quantize_rows_fast_kernel(QuantParams p) {
   constexpr int kU = 32;
   constexpr int kVec = BF16 ? 4 : 8;  // 16-byte words per unit
+  __shared__ float enc_tab[128];
   const float s_t = tensor_scale_of(p);
   if (FMT == METIS_NVFP4 && blockIdx.x == 0 && threadIdx.x == 0 && p.tensor_scale) *p.tensor_scale = s_t;
+  if (FMT == METIS_NVFP4) {
+    nv_enc_table(s_t, enc_tab);
+    __syncthreads();
+  }
   const int64_t upr = p.inner / kU;  // inner is a multiple of 32
   const int64_t total = p.outer * upr;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const uint8_t* X = reinterpret_cast<const uint8_t*>(p.X);
   const int64_t esize = BF16 ? 2 : 4;
+  // unit -> row: a 32-bit division while the unit count allows it
+  const bool narrow = total < (int64_t{1} << 31);
+  auto row_of = [&](int64_t unit) {
+    return narrow ? static_cast<int64_t>(static_cast<uint32_t>(unit) / static_cast<uint32_t>(upr)) : unit / upr;
+  };
   auto src = [&](int64_t unit) {
-    const int64_t o = unit / upr;
+    const int64_t o = row_of(unit);
     return reinterpret_cast<const uint4*>(X + (o * p.ld + (unit - o * upr) * kU) * esize);
   };
   int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
@@ -160,7 +170,7 @@ __global__ void __launch_bounds__(256) quantize_rows_fast_kernel(QuantParams p) 
 #pragma unroll
       for (int k = 0; k < kVec; ++k) nxt[k] = a[k];
     }
-    const int64_t o = t / upr, u = t - o * upr;
+    const int64_t o = row_of(t), u = t - o * upr;
     float v[kU];
 #pragma unroll
     for (int k = 0; k < kVec; ++k) {
@@ -189,8 +199,8 @@ __global__ void __launch_bounds__(256) quantize_rows_fast_kernel(QuantParams p) 
     float ds;
     if (FMT == METIS_NVFP4) {
       uint64_t pk0, pk1;
-      const uint32_t c0 = quant_block_nv<false>(v, s_t, pk0, ds);
-      const uint32_t c1 = quant_block_nv<false>(v + 16, s_t, pk1, ds);
+      const uint32_t c0 = quant_block_nv_tab(v, s_t, enc_tab, pk0);
+      const uint32_t c1 = quant_block_nv_tab(v + 16, s_t, enc_tab, pk1);
       *dst = make_uint4(static_cast<uint32_t>(pk0), static_cast<uint32_t>(pk0 >> 32), static_cast<uint32_t>(pk1),
                         static_cast<uint32_t>(pk1 >> 32));
       *reinterpret_cast<uint16_t*>(p.scales + tc_scale_offset(o, 2 * u, p.scale_cols)) =
@@ -292,6 +302,24 @@ __global__ void __launch_bounds__(256) amax_kernel(const void* X, int dtype, int
                                                    int64_t ld, const float* sub, unsigned* out_bits) {
   float m = 0.f;
   const int64_t total = rows * cols;
+  if (!sub && ld == cols && cols % 8 == 0) {
+    // a dense matrix: one flat stream, two adjacent 8-element units per
+    // thread and step (32 or 64 contiguous bytes), no index arithmetic
+    const int64_t units = total / 8;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+    for (int64_t t = 2 * (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x); t < units; t += 2 * stride) {
+      float v0[8], v1[8];
+      ld8(X, dtype, 8 * t, v0);
+      if (t + 1 < units) {
+        ld8(X, dtype, 8 * (t + 1), v1);
+      } else {
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v1[j] = 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) m = fmaxf(m, fmaxf(fabsf(v0[j]), fabsf(v1[j])));
+    }
+  } else
   for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t * 8 < total;
        t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
     const int64_t e = t * 8;
@@ -339,8 +367,13 @@ int64_t quant_groups(int64_t inner) { return (inner + kGroup - 1) / kGroup; }
 
 void launch_amax(const void* X, int dtype, int64_t rows, int64_t cols, int64_t ld, const float* sub,
                  unsigned* out_bits, int num_sms, cudaStream_t s) {
+  // no more CTAs than are resident at once: the grid-stride loop is
+  // latency-bound, so a second wave would add its full length
+  int per_sm = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, amax_kernel, 256, 0) != cudaSuccess || per_sm < 1)
+    per_sm = 1;
   const int64_t work = (rows * cols + 7) / 8;
-  int blocks = static_cast<int>(imin64((work + 255) / 256, static_cast<int64_t>(num_sms) * 8));
+  int blocks = static_cast<int>(imin64((work + 255) / 256, static_cast<int64_t>(num_sms) * per_sm));
   if (blocks < 1) blocks = 1;
   amax_kernel<<<blocks, 256, 0, s>>>(X, dtype, rows, cols, ld, sub, out_bits);
 }
@@ -348,9 +381,15 @@ void launch_amax(const void* X, int dtype, int64_t rows, int64_t cols, int64_t l
 template <int FMT, bool SUM>
 void launch_quantize_t(const QuantParams& p, int axis, int num_sms, cudaStream_t s) {
   if (axis == 1 && !SUM) {
-    // two or more units per thread, so the prefetch overlaps
+    // two or more units per thread, so the prefetch overlaps; no more CTAs
+    // than are resident at once (the grid-stride loop is latency-bound, so a
+    // second wave would add its full length)
     const int64_t units = p.outer * (p.inner / 32);
-    int blocks = static_cast<int>(imin64((units + 511) / 512, static_cast<int64_t>(num_sms) * 4));
+    const void* k = p.dtype == METIS_BF16 ? reinterpret_cast<const void*>(quantize_rows_fast_kernel<FMT, true>)
+                                          : reinterpret_cast<const void*>(quantize_rows_fast_kernel<FMT, false>);
+    int per_sm = 0;
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, 256, 0) != cudaSuccess || per_sm < 1) per_sm = 1;
+    int blocks = static_cast<int>(imin64((units + 511) / 512, static_cast<int64_t>(num_sms) * per_sm));
     if (blocks < 1) blocks = 1;
     if (p.dtype == METIS_BF16)
       quantize_rows_fast_kernel<FMT, true><<<blocks, 256, 0, s>>>(p);
