@@ -43,8 +43,8 @@ MDEV bool wait_ns(uint64_t* bar, uint32_t parity, uint64_t ns) {
 
 // Quantize n (32 or 64) values along the block axis: outer index o, first
 // element at inner offset i0 (a multiple of 32).
-MDEV void emit(const float* v, int n, int fmt, float s_t, uint8_t* codes, uint8_t* scales, int64_t scale_cols,
-               int64_t inner, int64_t o, int64_t i0) {
+MDEV void emit(const float* v, int n, int fmt, float s_t, const float* enc_tab, uint8_t* codes, uint8_t* scales,
+               int64_t scale_cols, int64_t inner, int64_t o, int64_t i0) {
   uint8_t* dst = codes + o * (inner / 2) + i0 / 2;
   if (fmt == METIS_NVFP4) {
     uint64_t pk[4] = {0, 0, 0, 0};
@@ -53,8 +53,7 @@ MDEV void emit(const float* v, int n, int fmt, float s_t, uint8_t* codes, uint8_
 #pragma unroll
     for (int b = 0; b < 4; ++b) {
       if (b < nb) {
-        float ds;
-        sc |= quant_block_nv(v + 16 * b, s_t, pk[b], ds) << (8 * b);
+        sc |= quant_block_nv_tab(v + 16 * b, s_t, enc_tab, pk[b]) << (8 * b);
       }
     }
     reinterpret_cast<uint4*>(dst)[0] = make_uint4(static_cast<uint32_t>(pk[0]), static_cast<uint32_t>(pk[0] >> 32),
@@ -117,7 +116,7 @@ __host__ __device__ inline Layout layout(int kp, int dtype) {
   l.u_bytes = 2 * l.chunks * kBM * 128;
   l.w_bytes = 2 * l.chunks * kBN * 128;
   l.a_bytes = kBM * kBN * (dtype == METIS_BF16 ? 2 : 4);
-  const int fixed = 1024 + l.u_bytes + kTransposeBytes + 512;
+  const int fixed = 1024 + l.u_bytes + kTransposeBytes + 1024;  // barriers 256 B, encode table 512 B
   int st = (kSmemLimit - fixed) / (l.w_bytes + l.a_bytes);
   l.stages = st > kMaxStages ? kMaxStages : st;
   l.total = fixed + l.stages * (l.w_bytes + l.a_bytes);
@@ -149,6 +148,7 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
   uint64_t* drain = u_empty + 1;
   uint32_t* tmem_sh = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_sh + 1);
+  float* enc_tab = reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(bars) + 256);  // NVFP4 encode factors
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -175,6 +175,7 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
     tmem_alloc(tmem_sh, kTmemCols);
     tmem_relinquish();
   }
+  if (p.mode == 1 && p.fmt == METIS_NVFP4) nv_enc_table(nv_tensor_scale(__uint_as_float(*p.amax_bits)), enc_tab);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -371,7 +372,7 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
 #pragma unroll
         for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4*>(tp + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
       }
-      if (p.r_codes) emit(v, 32, p.fmt, s_t, p.r_codes, p.r_scales, p.r_scale_cols, p.n, row, col0);
+      if (p.r_codes) emit(v, 32, p.fmt, s_t, enc_tab, p.r_codes, p.r_scales, p.r_scale_cols, p.n, row, col0);
       if (p.c_codes) {
         // the warp's 32 rows x 32 columns, transposed through shared memory
 #pragma unroll
@@ -381,7 +382,7 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
 #pragma unroll
         for (int i = 0; i < 32; ++i) col[i] = my_t[i * 33 + lane];
         __syncwarp();
-        emit(col, 32, p.fmt, s_t, p.c_codes, p.c_scales, p.c_scale_cols, p.m, col0 + lane, row0);
+        emit(col, 32, p.fmt, s_t, enc_tab, p.c_codes, p.c_scales, p.c_scale_cols, p.m, col0 + lane, row0);
       }
     }
     if (p.mode == 0) {

@@ -148,3 +148,22 @@ def test_quantize_full_size_activation(axis):
     torch.cuda.synchronize()
     ref = fp4.quantize(d["X"].f32(), "nv", axis)
     assert_fp4_equal(q, ref)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+@pytest.mark.parametrize("axis", [0, 1])
+def test_quantize_strided_view(dtype, axis):
+    # a column view of a wider matrix (leading dimension 320 > 256 columns):
+    # the NVFP4 tensor maximum and the codes must ignore the columns outside
+    # the view, which hold the largest values of the buffer
+    rows, cols, ld = 224, 256, 320
+    x = _data(rows, ld, 21)
+    x[:, cols:] *= 1e3
+    if dtype == "bf16":
+        Xp, xval = bf16_tensor(x)
+    else:
+        Xp, xval = torch.from_numpy(x).cuda(), x
+    q = api.quantize_fp4(Xp[:, :cols], "nv", axis, linear=True)
+    torch.cuda.synchronize()
+    ref = fp4.quantize(np.ascontiguousarray(xval[:, :cols]), "nv", axis)
+    assert_fp4_equal(q, ref)
