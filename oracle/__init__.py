@@ -37,8 +37,8 @@ Sources followed (page title, section)
   separately, the same split on the output gradient in the backward pass.
 
 Everything the pages leave open (sketch distribution, QR/SVD form, FP4 scale
-rules, op order, sampling law) follows the readings listed in the design doc's
-"Readings" table; the functions below name the reading they implement.
+rules, op order, sampling law) follows one stated reading, numbered R1, R2,
+...; each function below names the reading it implements and states it.
 
 Parity status: every function here is pinned by ``tests/test_oracle_*.py``
 against closed forms, brute force, published test vectors or independent

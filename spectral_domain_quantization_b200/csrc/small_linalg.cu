@@ -422,10 +422,13 @@ __global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) {
     }
   }
   __syncthreads();
-  // warp w: rows 4 w .. 4 w + 3 (broadcast reads of In); lane l < kout / 4:
-  // columns 4 l .. 4 l + 3 (one 16-byte read of M per step; kout <= 112)
-  const int rg = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const bool has = 4 * lane < a.kout;
+  // thread t < 8 kout / 4: rows 4 rg .. 4 rg + 3 (broadcast reads of In) and
+  // columns 4 cg .. 4 cg + 3 (one 16-byte read of M per step), rg = t / (kout
+  // / 4), cg = t % (kout / 4): every lane of the first warps works (kout <= 112)
+  const int ncg = a.kout / 4;
+  const int t = threadIdx.x;
+  const bool has = t < 8 * ncg;
+  const int rg = has ? t / ncg : 0, cg = has ? t - rg * ncg : 0;
   float acc[4][4];
 #pragma unroll
   for (int i = 0; i < 4; ++i)
@@ -438,7 +441,7 @@ __global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) {
       float x[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i) x[i] = in0[i * (a.kin + 1) + j];
-      const float4 m = *reinterpret_cast<const float4*>(Ms + j * a.kout + 4 * lane);
+      const float4 m = *reinterpret_cast<const float4*>(Ms + j * a.kout + 4 * cg);
       const float mv[4] = {m.x, m.y, m.z, m.w};
 #pragma unroll
       for (int u = 0; u < 4; ++u)
@@ -448,7 +451,7 @@ __global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int u = 0; u < 4; ++u) Out[(4 * rg + i) * (a.kout + 1) + 4 * lane + u] = acc[i][u];
+      for (int u = 0; u < 4; ++u) Out[(4 * rg + i) * (a.kout + 1) + 4 * cg + u] = acc[i][u];
   }
   __syncthreads();
   for (int e = threadIdx.x; e < kApplyRows * a.kout; e += blockDim.x) {
