@@ -73,12 +73,12 @@ __host__ __device__ inline EigScratch scratch(double* ws, int n) {
 // Two barriers per column:
 //   (a) row warps: u = A' x with x0 (not v0) at column j + 1, the sums
 //       S1 = sum_{i>j+1} u_i x_i and S2 = sum_{i>j+1} A[i][j+1] x_i, and
-//       the values of row j + 1; meanwhile one extra warp finds alpha,
-//       beta and v0 from |x|^2 (reduced in the column before) and x0;
+//       the values of row j + 1; meanwhile one extra warp sums |x|^2
+//       from the per-row squares and finds alpha, beta and v0;
 //   (b) all: p_i = beta (u_i + A[i][j+1] (v0 - x0)) and
 //       p^T v = p_{j+1} v0 + beta (S1 + (v0 - x0) S2) give K and q; the
-//       holders of column j + 1 update it first and reduce the next
-//       column's |x|^2;
+//       holders of column j + 1 update it first and write the squares of
+//       its entries below the next x0 (the extra warp reduces them);
 //   (c) row warps: the rest of the rank-2 update.
 
 template <int NH>
@@ -88,7 +88,8 @@ struct TriShared {
   // per column parity, by row: .x = x entry of the column, .y = p_i (both 0
   // outside the active rows); the update reads both with one 16-byte load
   double2 xp[2][kBuf];
-  double red1a[kWarps], red1b[kWarps], red2[kWarps];
+  double red1a[kWarps], red1b[kWarps];
+  double sq[2 * NH];    // by row: x_i^2 of the next column's entries below x0 (0 elsewhere)
   double row1[2];       // row j + 1: u_{j+1} and A[j+1][j+1]
   double refl[2];       // beta, v0 of the current column
 };
@@ -123,7 +124,11 @@ MDEV void tri_step(double (&a)[NH], TriShared<NH>& sh, const EigScratch& S, int 
   double2* nxt = sh.xp[(j + 1) & 1];
   const bool scalar_warp = warp == nwr;
   if (scalar_warp) {
-    const double sg = sum_fixed(sh.red2, nwr);
+    // |x|^2 without x0, summed by this warp in a fixed order (the row
+    // warps only wrote their rows' squares)
+    double sg = 0.0;
+    for (int r = lane; r < n; r += 32) sg += sh.sq[r];
+    sg = warp_sum(sg);
     const double x0 = cur[j + 1].x;
     double alpha = x0, beta = 0.0, v0 = 0.0;
     if (sg > 0.0) {
@@ -193,14 +198,11 @@ MDEV void tri_step(double (&a)[NH], TriShared<NH>& sh, const EigScratch& S, int 
     S.V[j * n + i] = beta == 0.0 ? 0.0 : vi;
     if (i <= j + 1) nxt[i].x = 0.0;
   }
-  double sq = 0.0;
   if (h == hold_h && row_ok) {
     a[kHoldR] = fma(-qi, v0, fma(-vi, pj1, a[kHoldR]));
     if (i >= j + 2) nxt[i].x = a[kHoldR];
-    if (i >= j + 3) sq = a[kHoldR] * a[kHoldR];
+    sh.sq[i] = i >= j + 3 ? a[kHoldR] * a[kHoldR] : 0.0;
   }
-  sq = warp_sum(sq);
-  if (lane == 0 && !scalar_warp) sh.red2[warp] = sq;
   __syncthreads();
   // (c) the rest of the update: a_ic -= q_i v_c + v_i p_c (v_c = x_c past
   // column j + 1, whose register was updated above)
@@ -240,8 +242,7 @@ __global__ void __launch_bounds__(4 * NH + 32, 1) core_tridiag_kernel(const doub
   {
     // column 0: x_i = A[i][0] (i >= 1) and |x|^2 without x0
     if (h == 0 && row_ok && i >= 1) sh.xp[0][i].x = a[0];
-    const double s = warp_sum((h == 0 && row_ok && i >= 2) ? a[0] * a[0] : 0.0);
-    if (lane == 0 && warp < nwr) sh.red2[warp] = s;
+    if (h == 0 && row_ok) sh.sq[i] = i >= 2 ? a[0] * a[0] : 0.0;
     __syncthreads();
   }
   int j = 0;
