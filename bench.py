@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--composite", action="store_true",
+                    help="measure the mean + spectral composite split of the Averis-shaped activation instead")
     ap.add_argument("--profile-steps", type=int, default=0,
                     help="run this many eager steps (no graphs, no timing) and exit: the command profiled by ncu")
     return ap.parse_args()
@@ -489,10 +491,73 @@ def run_profile(args, local):
     print(json.dumps({"profile_steps": args.profile_steps, "dev_status": int(status.item())}), flush=True)
 
 
+def run_composite(args, local):
+    """The mean + spectral composite: averis_split of an activation with a
+    column mean (X bf16 32768 x 4096 = 1 mu^T + Z), the spectral split of its
+    float32 mean-free residual (k = 64, p = 16, q = 1), the rank-65 FP4
+    factors, then Y = X W with the composite X and a plain NVFP4 W.  Eager
+    calls timed with CUDA events on the current stream, L2 flushed before
+    every step; one JSON line."""
+    import torch
+    from spectral_domain_quantization_b200 import api, inputs
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    data = inputs.make("averis_32768", keys=("X", "W"))
+    c = data["cfg"]
+    Mx, Kx, Nx = c["M"], c["K"], c["N"]
+    X = torch.from_numpy(data["X"].data.view(np.int16)).view(torch.bfloat16).to(dev)
+    W = torch.from_numpy(data["W"].data.view(np.int16)).view(torch.bfloat16).to(dev)
+    qw = api.quantize_fp4(W, "nv", 0)                       # outer N, blocks along K
+    Y = torch.empty((Mx, Nx), dtype=torch.bfloat16, device=dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    flush = torch.empty(256 * 1024 * 1024, dtype=torch.int16, device=dev)
+    t_split, t_fwd = [], []
+    for i in range(args.warmup + args.steps):
+        flush.fill_(1)
+        e0, e1, e2 = (torch.cuda.Event(enable_timing=True) for _ in range(3))
+        e0.record()
+        comp = api.composite_split(X, RANK_K, OVERSAMPLE, POWER_ITERS, SEED, "nv", rows=True, cols=False,
+                                   dev_status=status)
+        e1.record()
+        api.linear_fwd(comp.operand("left"), api.Operand(qw), Mx, Nx, Kx, Y=Y, dev_status=status)
+        e2.record()
+        torch.cuda.synchronize()
+        if i >= args.warmup:
+            t_split.append(e0.elapsed_time(e1))
+            t_fwd.append(e1.elapsed_time(e2))
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item())}")
+    split_ms, fwd_ms = float(np.mean(t_split)), float(np.mean(t_fwd))
+    flops = 2.0 * Mx * Nx * Kx
+    line = {"metric": "mean + spectral composite split us/layer; composite forward eff. TFLOPS",
+            "value": split_ms * 1e3, "unit": "us", "higher_is_better": False, "n_gpus": 1,
+            "steps": args.steps, "warmup": args.warmup, "dtype": "fp4 (e2m1, nvfp4 scales; fp32 accumulate)",
+            "data": "synthetic",
+            "config": {"workload": f"averis_32768 activation X bf16 {Mx}x{Kx} = 1 mu^T + Z; composite split "
+                                   f"k={RANK_K} p={OVERSAMPLE} q={POWER_ITERS} (rank {RANK_K + 1} with the mean), "
+                                   f"NVFP4; Y = X W with W bf16 {Kx}x{Nx} plain NVFP4",
+                       "timing": "eager calls, CUDA events, L2 flushed (512 MB write) before every step"},
+            "breakdown_us": {"composite_split": split_ms * 1e3, "forward_product": fwd_ms * 1e3},
+            "forward_tflops": flops / (fwd_ms * 1e-3) / 1e12}
+    if not args.no_cpu_baseline:
+        from oracle import composite
+        rows = 2048
+        x32 = data["X"].f32()[:rows]
+        t0 = time.perf_counter()
+        composite.split(x32, RANK_K, OVERSAMPLE, POWER_ITERS, SEED)
+        dt = (time.perf_counter() - t0) * (Mx / rows)
+        line["cpu_baseline"] = {"value": dt * 1e6, "unit": "us", "cores": blas_threads(), "kind": "oracle",
+                                "sample": f"composite split of the first {rows} of {Mx} rows, scaled x{Mx // rows}"}
+    print(json.dumps(line), flush=True)
+
+
 def main():
     args = parse()
     if args.profile_steps > 0:
         run_profile(args, int(os.environ.get("LOCAL_RANK", "0")))
+        return
+    if args.composite:
+        run_composite(args, int(os.environ.get("LOCAL_RANK", "0")))
         return
     rank, world, local = dist_init()
     try:

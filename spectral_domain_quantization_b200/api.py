@@ -404,6 +404,60 @@ def averis_split(X, fmt="nv", rows=True, cols=True, tap=False, dev_status=None):
                        dev_status=dev_status, fmt=f)
 
 
+# --------------------------------------------------------------------------
+# mean + spectral composite
+# --------------------------------------------------------------------------
+
+class CompositeSplit:
+    """A = 1 mu^T + U diag(S) V^T + R2 from averis_split then metis_split of
+    the float32 mean-free residual.  The mean and the spectral part form one
+    rank-(k + 1) low-rank part F diag(S1) P^T with F = [1 | U], P = [mu | V],
+    S1 = [1, S]; F_q (outer k + 1, inner m) and P_q (outer k + 1, inner n) are
+    their FP4 quantizations along the long axis.  F32 and P32 are float32
+    column views of the factors as quantized (leading dimension padded)."""
+
+    def __init__(self, **kw):
+        self.__dict__.update(kw)
+
+    def operand(self, side, axis_rows=True):
+        """As Split.operand: "right" for W in X W, "left" for X in X W."""
+        if side == "right":
+            return Operand(self.R_cols if axis_rows else self.R_rows, self.k1, self.F_q, self.P_q, self.S1)
+        return Operand(self.R_rows, self.k1, self.P_q, self.F_q, self.S1)
+
+
+def composite_split(A, k, p, q=1, seed=0, fmt="nv", sketch="gaussian", nnz=4, max_iters=64,
+                    rows=True, cols=True, tap=False, dev_status=None):
+    """Mean removal (averis_split, float32 residual tap) followed by the
+    spectral split of the residual (metis_split), then the FP4 factors of the
+    rank-(k + 1) low-rank part (metis_quantize_fp4).  Every step runs in the
+    library's kernels; this function only arranges buffers."""
+    if A.dim() != 2 or A.stride(1) != 1:
+        raise ValueError("A must be a row-major 2-D tensor")
+    m, n = A.shape
+    dev = A.device
+    if dev_status is None:
+        dev_status = torch.zeros(1, dtype=torch.int32, device=dev)
+    av = averis_split(A, fmt, rows=False, cols=False, tap=True, dev_status=dev_status)
+    sp = split(av.R_f32, k, p, q, seed, fmt, sketch=sketch, nnz=nnz, max_iters=max_iters, rows=rows,
+               cols=cols, factors=False, tap=tap, dev_status=dev_status)
+    k1 = k + 1
+    ldk = (k1 + 3) // 4 * 4                     # rows start on 16-byte boundaries
+    Fbuf = torch.zeros((m, ldk), dtype=torch.float32, device=dev)
+    Pbuf = torch.zeros((n, ldk), dtype=torch.float32, device=dev)
+    Fbuf[:, 0] = 1.0
+    Fbuf[:, 1:k1] = sp.U
+    Pbuf[:, 0] = av.mean
+    Pbuf[:, 1:k1] = sp.V
+    F32, P32 = Fbuf[:, :k1], Pbuf[:, :k1]
+    F_q = quantize_fp4(F32, fmt, 0)
+    P_q = quantize_fp4(P32, fmt, 0)
+    S1 = torch.cat([torch.ones(1, dtype=torch.float32, device=dev), sp.S])
+    return CompositeSplit(mean=av.mean, R1=av.R_f32, U=sp.U, S=sp.S, V=sp.V, F32=F32, P32=P32, F_q=F_q,
+                          P_q=P_q, S1=S1, R_rows=sp.R_rows, R_cols=sp.R_cols, R2_f32=sp.R_f32, k=k, k1=k1,
+                          fmt=sp.fmt, dev_status=dev_status)
+
+
 def selftest_wait_timeout(limit_ns=1_000_000, device="cuda"):
     """Run the library's bounded device wait on a barrier that never
     completes (metis_selftest_wait_timeout); returns the device status word

@@ -73,8 +73,11 @@ extern "C" metis_status averis_split(const void* X, int32_t dtype, int64_t m, in
                                s));
     tapped = R_f32 != nullptr;
   }
-  if (R_cols)
+  if (R_cols) {
     METIS_TRY(enqueue_quantize(X, dtype, m, n, ld, 0, mean, R_cols, fmt == METIS_NVFP4 ? b.amax : nullptr,
                                tapped ? nullptr : R_f32, ws, s));
+    tapped = R_f32 != nullptr;
+  }
+  if (R_f32 && !tapped) launch_residual_tap(X, dtype, m, n, ld, mean, R_f32, device_sm_count(), s);
   return launch_status();
 }

@@ -133,4 +133,28 @@ void launch_colstats(const void* X, int dtype, int64_t m, int64_t n, int64_t ld,
       psum, pmin, pmax, static_cast<int>(nchunks), m, n, mean, amax_bits);
 }
 
+// The float32 mean-free matrix alone: R[i][j] = fl32(x_ij - mu_j), the same
+// float operation as the quantizers' tap (for callers that want the residual
+// without its FP4 codes).  A grid-stride loop over elements, row-major.
+__global__ void residual_tap_kernel(const void* X, int dtype, int64_t m, int64_t n, int64_t ld, const float* mu,
+                                    float* R) {
+  const int64_t total = m * n;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < total;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t i = e / n, j = e - i * n;
+    const float x = dtype == METIS_BF16 ? __bfloat162float(reinterpret_cast<const __nv_bfloat16*>(X)[i * ld + j])
+                                        : reinterpret_cast<const float*>(X)[i * ld + j];
+    R[e] = __fsub_rn(x, mu[j]);
+  }
+}
+
+void launch_residual_tap(const void* X, int dtype, int64_t m, int64_t n, int64_t ld, const float* mu, float* R,
+                         int num_sms, cudaStream_t s) {
+  const int64_t total = m * n;
+  int64_t blocks = (total + 255) / 256;
+  if (blocks > static_cast<int64_t>(num_sms) * 8) blocks = static_cast<int64_t>(num_sms) * 8;
+  if (blocks < 1) blocks = 1;
+  residual_tap_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(X, dtype, m, n, ld, mu, R);
+}
+
 }  // namespace metis

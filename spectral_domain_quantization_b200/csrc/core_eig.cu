@@ -447,6 +447,7 @@ __global__ void __launch_bounds__(32) core_vector_kernel(int n, double* ws, int 
         r = orr;
       }
     }
+    if (r >= n) r = 0;  // no finite gamma (a non-finite input): any in-range twist
     // z_r = 1; lane 0 walks up, lane 1 walks down, in lockstep (each
     // rescales its own side by 1e-150 if it grows past 1e150; the sides are
     // reconciled after)

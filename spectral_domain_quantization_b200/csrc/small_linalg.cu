@@ -520,7 +520,10 @@ __global__ void colmax_kernel(const float* __restrict__ U, int64_t rows, int k, 
 __global__ void sign_kernel(const float* __restrict__ U, const float* __restrict__ bmax,
                             const int64_t* __restrict__ bidx, int nblocks, int k, float* sign) {
   const int j = blockIdx.x, lane = threadIdx.x;
-  float best = -1.f;
+  // below every block maximum (colmax reports -1 for a block with no value
+  // above -1, e.g. NaN entries), so each lane with a block picks one and the
+  // chosen block index is always in range
+  float best = -2.f;
   int bb = nblocks;
 #pragma unroll 4
   for (int b = lane; b < nblocks; b += 32) {
@@ -539,6 +542,7 @@ __global__ void sign_kernel(const float* __restrict__ U, const float* __restrict
     }
   }
   if (lane == 0) {
+    if (bb >= nblocks) bb = 0;   // only when nblocks == 0, which the shape checks exclude
     const int64_t bi = bidx[static_cast<int64_t>(bb) * k + j];
     sign[j] = U[bi * k + j] < 0.f ? -1.f : 1.f;
   }
