@@ -55,6 +55,8 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--compensate", action="store_true",
+                    help="the split forms the error-compensated residual A - deq(U_q) S deq(V_q)^T")
     ap.add_argument("--composite", action="store_true",
                     help="measure the mean + spectral composite split of the Averis-shaped activation instead")
     ap.add_argument("--profile-steps", type=int, default=0,
@@ -291,7 +293,7 @@ def run_ours(args, rank, world, local):
     def make_step(Wb, Xb, Yb):
         def split_w():
             return api.split(Wb, RANK_K, OVERSAMPLE, POWER_ITERS, SEED, "nv", rows=False, cols=True, factors=True,
-                             dev_status=status)
+                             compensate=args.compensate, dev_status=status)
 
         def quant_x():
             return api.quantize_fp4(Xb, "nv", 1)
@@ -452,7 +454,8 @@ def run_ours(args, rank, world, local):
             "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "fp4 (e2m1, nvfp4 scales; fp32 accumulate)", "data": "synthetic",
-            "config": CONFIG,
+            "config": dict(CONFIG, residual="error-compensated: A - deq(U_q) S deq(V_q)^T") if args.compensate
+            else CONFIG,
             "frac_of_fp4_peak": value / world / fp4_peak,
             "split_quantize_us_per_layer": (ms_split + ms_quant) * 1e3,
             "breakdown_us": {"split_W": ms_split * 1e3, "quantize_X": ms_quant * 1e3,

@@ -208,6 +208,13 @@ size_t metis_noalloc_scratch_bytes(void);
  *   max_core_iters  cap on the multisection rounds that find each eigenvalue
  *                 of the core Gram (about 11 are needed; 64 is a safe
  *                 value); reaching it sets METIS_DEV_NUMERIC in *dev_status.
+ *   compensate    0: R = A - U diag(S) V^T with the float32 factors (the
+ *                 pages' split).  1: the error-compensated residual
+ *                 R = A - deq(U_q) diag(S) deq(V_q)^T, formed from the FP4
+ *                 factors as quantized, so that the quantized residual also
+ *                 absorbs the factors' quantization error; needs U_q and V_q
+ *                 (METIS_ERR_NULL otherwise).  Zero-initialise the struct
+ *                 to get 0.
  */
 typedef struct {
   int32_t k;
@@ -219,6 +226,7 @@ typedef struct {
   int64_t sample_rows;
   int32_t fmt;
   int32_t max_core_iters;
+  int32_t compensate;
 } metis_split_params;
 
 /*
@@ -229,10 +237,13 @@ typedef struct {
  * Quantization" abstract (random projection and sparse random sampling);
  * older Metis abstract item (i) (random embedding).
  * Steps: [sample rows] -> Omega (Philox Gaussian / sparse sign, bf16) ->
- * Y = A Omega -> CholeskyQR2 -> q x (A^T Q, QR, A Q, QR) -> B^T = A^T Q ->
- * one-sided Jacobi on the l-wide core (via its l x l Gram, float64) -> top k,
- * U = Q U~, V = B^T U~ S^-1, signs (largest-|.| entry of each U column made
- * positive) -> R = A - U S V^T fused with FP4 quantization.
+ * Y = A Omega -> q x (A^T Y, CholeskyQR, A Q, CholeskyQR) (with q = 0 a
+ * two-pass CholeskyQR of Y) -> Z = A^T Q -> eigen-decomposition of the l x l
+ * core Gram C = Z^T Z in float64 (Householder tridiagonalisation, multisection
+ * on Sturm counts, eigenvectors from the twisted factorisation) -> top k,
+ * U = Q W, V = Z W S^-1, signs (largest-|.| entry of each U column made
+ * positive) -> R = A - U S V^T (or, with compensate, A minus the product of
+ * the dequantized FP4 factors) fused with FP4 quantization.
  * With sample_rows > 0: V_s from the sampled rows, P = A V_s, CholeskyQR2 of
  * P, SVD of its triangular factor; U = Q_P W1, V = V_s W2.
  *

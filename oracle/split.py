@@ -94,6 +94,16 @@ def residual(A, U, S, V):
     return np.asarray(A, dtype=np.float64) - (U * S) @ V.T
 
 
+def compensated_residual(A, Uq, S, Vq):
+    """R = A - deq(U_q) diag(S) deq(V_q)^T (float64): the residual against
+    the FP4 factors as quantized (the variant of R10 that the option
+    `compensate` selects; reading R29).  Uq, Vq: FP4Tensor with outer = k
+    (inner m and n)."""
+    Ud = Uq.dequantize().T          # m x k
+    Vd = Vq.dequantize().T          # n x k
+    return np.asarray(A, dtype=np.float64) - (Ud * np.asarray(S, dtype=np.float64)) @ Vd.T
+
+
 def make_sketch(n, l, seed, kind="gaussian", nnz=4):
     if kind == "gaussian":
         return sketch.gaussian_omega(n, l, seed)

@@ -48,7 +48,8 @@ class SplitParams(ctypes.Structure):
     _fields_ = [("k", ctypes.c_int32), ("p", ctypes.c_int32), ("power_iters", ctypes.c_int32),
                 ("seed", ctypes.c_uint64), ("sketch", ctypes.c_int32),
                 ("sparse_nnz", ctypes.c_int32), ("sample_rows", ctypes.c_int64),
-                ("fmt", ctypes.c_int32), ("max_core_iters", ctypes.c_int32)]
+                ("fmt", ctypes.c_int32), ("max_core_iters", ctypes.c_int32),
+                ("compensate", ctypes.c_int32)]
 
 
 class OperandStruct(ctypes.Structure):
@@ -325,8 +326,9 @@ class Split:
 
 
 def split(A, k, p, q=1, seed=0, fmt="nv", sketch="gaussian", nnz=4, sample_rows=0, max_iters=64,
-          rows=True, cols=True, factors=True, tap=False, dev_status=None):
-    """Spectral split A = U diag(S) V^T + R with FP4 outputs (metis_split)."""
+          rows=True, cols=True, factors=True, tap=False, compensate=False, dev_status=None):
+    """Spectral split A = U diag(S) V^T + R with FP4 outputs (metis_split).
+    compensate: R = A - deq(U_q) diag(S) deq(V_q)^T (needs factors=True)."""
     if A.dim() != 2 or A.stride(1) != 1:
         raise ValueError("A must be a row-major 2-D tensor")
     m, n = A.shape
@@ -344,7 +346,7 @@ def split(A, k, p, q=1, seed=0, fmt="nv", sketch="gaussian", nnz=4, sample_rows=
     if dev_status is None:
         dev_status = torch.zeros(1, dtype=torch.int32, device=dev)
     prm = SplitParams(k=k, p=p, power_iters=q, seed=seed, sketch=SKETCH[sketch], sparse_nnz=nnz,
-                      sample_rows=sample_rows, fmt=f, max_core_iters=max_iters)
+                      sample_rows=sample_rows, fmt=f, max_core_iters=max_iters, compensate=int(bool(compensate)))
     st = [t.struct() if t is not None else None for t in (U_q, V_q, R_rows, R_cols)]
     refs = [ctypes.byref(s) if s is not None else None for s in st]
     _call_with_workspace(

@@ -23,6 +23,7 @@
 #include "abi_internal.h"
 #include "common.cuh"
 #include "kernels.h"
+#include "lowrank.h"
 #include "residual_quant.h"
 #include "sketch.h"
 #include "skinny_gemm.h"
@@ -31,6 +32,8 @@
 namespace metis {
 
 namespace {
+
+static_assert(sizeof(metis_split_params) == 56, "metis_split_params layout (the Python binding mirrors it)");
 
 int round_up(int x, int m) { return (x + m - 1) / m * m; }
 int64_t round_up64(int64_t x, int64_t m) { return (x + m - 1) / m * m; }
@@ -276,6 +279,8 @@ metis_status validate_split(const void* A, int dtype, int64_t m, int64_t n, int6
   if (!valid_fmt(prm->fmt)) return METIS_ERR_ARG;
   if (prm->sketch != METIS_SKETCH_GAUSSIAN && prm->sketch != METIS_SKETCH_SPARSE_SIGN) return METIS_ERR_ARG;
   if (prm->k < 1 || prm->p < 0 || prm->power_iters < 0 || prm->max_core_iters < 1) return METIS_ERR_ARG;
+  if (prm->compensate != 0 && prm->compensate != 1) return METIS_ERR_ARG;
+  if (prm->compensate && (!U_q || !V_q)) return METIS_ERR_NULL;
   const int l = prm->k + prm->p;
   if (l > 112) return METIS_ERR_SHAPE;
   if (prm->k % 4) return METIS_ERR_SHAPE;  // U, V rows of k floats start on 16-byte boundaries
@@ -447,6 +452,23 @@ extern "C" metis_status metis_split(const void* A, int32_t dtype, int64_t m, int
   METIS_TRY(step_status("factor signs and operands"));
   if (U_q) METIS_TRY(enqueue_quantize(U, METIS_F32, m, p.k, p.k, 0, nullptr, U_q, b.amax, nullptr, ws, s));
   if (V_q) METIS_TRY(enqueue_quantize(V, METIS_F32, n, p.k, p.k, 0, nullptr, V_q, b.amax + 1, nullptr, ws, s));
+  if (residual && prm->compensate) {
+    // the residual against the factors as quantized: its operands become
+    // hi / lo of deq(U_q) and deq(V_q) diag(S)
+    auto view = [](const metis_fp4_tensor* t) {
+      FactorView f{};
+      f.ones = 0;
+      f.fmt = t->fmt;
+      f.inner = t->inner;
+      f.scale_cols = tc_scale_cols(t->fmt, t->inner);
+      f.codes = t->codes;
+      f.scales = t->scales;
+      f.tensor_scale = t->fmt == METIS_NVFP4 ? t->tensor_scale : nullptr;
+      return f;
+    };
+    launch_compensated_operands(view(U_q), view(V_q), m, n, p.k, S, p.kp, b.u_hi, b.u_lo, b.w_hi, b.w_lo, sms, s);
+    METIS_TRY(step_status("compensated residual operands"));
+  }
 
   if (residual) {
     ResidualOperands ro{b.u_hi, b.u_lo, b.w_hi, b.w_lo};

@@ -142,6 +142,32 @@ __global__ void copy_rows_kernel(const float* src, float* dst, int64_t n) {
     dst[i] = src[i];
 }
 
+// Operands of the error-compensated residual: thread per (row, column c <
+// kp) of [U rows | V rows]; column c < k holds hi / lo of deq(U_q)[row][c]
+// (U's rows) or of fl32(deq(V_q)[row][c] S[c]) (V's rows), padding columns 0.
+// deq includes the NVFP4 tensor scale.  The same [rows][kp] layout as the
+// float32 factors' operands, which these replace.
+__global__ void compensated_operands_kernel(FactorView fu, FactorView fv, int64_t m, int64_t n, int k,
+                                            const float* S, int kp, __nv_bfloat16* u_hi, __nv_bfloat16* u_lo,
+                                            __nv_bfloat16* w_hi, __nv_bfloat16* w_lo) {
+  const float tu = tscale(fu), tv = tscale(fv);
+  const int64_t total = (m + n) * kp;
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < total;
+       t += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t row = t / kp;
+    const int c = static_cast<int>(t - row * kp);
+    const bool isu = row < m;
+    const int64_t r = isu ? row : row - m;
+    float w = 0.f;
+    if (c < k) w = isu ? __fmul_rn(factor_value(fu, c, r), tu) : __fmul_rn(__fmul_rn(factor_value(fv, c, r), tv), S[c]);
+    const __nv_bfloat16 h = __float2bfloat16_rn(w);
+    __nv_bfloat16* hi = isu ? u_hi : w_hi;
+    __nv_bfloat16* lo = isu ? u_lo : w_lo;
+    hi[r * kp + c] = h;
+    lo[r * kp + c] = __float2bfloat16_rn(__fsub_rn(w, __bfloat162float(h)));
+  }
+}
+
 int blocks_for(int64_t n, int sms) {
   int64_t b = (n + 255) / 256;
   if (b > sms * 8) b = sms * 8;
@@ -164,6 +190,13 @@ void launch_build_lowrank(const LowRankArgs& a, int sms, cudaStream_t s) {
   const int threads = a.lr_k >= 128 ? 128 : 64;
   build_la_kernel<<<row_blocks(a.M, sms), threads, 0, s>>>(a);
   build_lb_kernel<<<row_blocks(a.N, sms), threads, 0, s>>>(a);
+}
+
+void launch_compensated_operands(const FactorView& fu, const FactorView& fv, int64_t m, int64_t n, int k,
+                                 const float* S, int kp, __nv_bfloat16* u_hi, __nv_bfloat16* u_lo,
+                                 __nv_bfloat16* w_hi, __nv_bfloat16* w_lo, int sms, cudaStream_t s) {
+  compensated_operands_kernel<<<blocks_for((m + n) * kp, sms), 256, 0, s>>>(fu, fv, m, n, k, S, kp, u_hi, u_lo, w_hi,
+                                                                           w_lo);
 }
 
 void launch_copy(const float* src, float* dst, int64_t n, int sms, cudaStream_t s) {

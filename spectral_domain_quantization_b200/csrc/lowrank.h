@@ -48,5 +48,11 @@ void launch_cab(const FactorView& pa, const FactorView& pb, int64_t K, int ka, i
                 cudaStream_t s);
 void launch_build_lowrank(const LowRankArgs& a, int sms, cudaStream_t s);
 void launch_copy(const float* src, float* dst, int64_t n, int sms, cudaStream_t s);
+// hi / lo bf16 operands [rows][kp] of deq(U_q) (m rows) and deq(V_q) diag(S)
+// (n rows) for the error-compensated residual (fu: U_q, fv: V_q, k factors).
+void launch_compensated_operands(const FactorView& fu, const FactorView& fv, int64_t m, int64_t n, int k,
+                                 const float* S, int kp, __nv_bfloat16* u_hi, __nv_bfloat16* u_lo,
+                                 __nv_bfloat16* w_hi, __nv_bfloat16* w_lo, int sms, cudaStream_t s);
+
 
 }  // namespace metis

@@ -96,3 +96,14 @@ def test_selftest_wait_argument_checks():
     fake = ctypes.c_int32(0)
     assert L.metis_selftest_wait_timeout(0, ctypes.addressof(fake), None) == ERR_ARG
     assert L.metis_selftest_wait_timeout(2_000_000_000, ctypes.addressof(fake), None) == ERR_ARG
+
+
+def test_split_params_layout_matches_the_header():
+    # the library asserts sizeof(metis_split_params) == 56 at compile time;
+    # the ctypes mirror must have the same size and field offsets
+    import ctypes
+    P = api.SplitParams
+    assert ctypes.sizeof(P) == 56
+    assert [P.k.offset, P.p.offset, P.power_iters.offset, P.seed.offset, P.sketch.offset, P.sparse_nnz.offset,
+            P.sample_rows.offset, P.fmt.offset, P.max_core_iters.offset, P.compensate.offset] == \
+        [0, 4, 8, 16, 24, 28, 32, 40, 44, 48]

@@ -11,7 +11,7 @@ import torch
 from oracle import fp4, sketch, split
 from spectral_domain_quantization_b200 import api, inputs
 
-from gpu_helpers import assert_fp4_equal, rel_fro, to_device
+from gpu_helpers import assert_fp4_equal, read_fp4, rel_fro, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -131,3 +131,32 @@ def test_split_largest_cores(k, p):
     torch.cuda.synchronize()
     A64 = A.astype(np.float64)
     _check(A64, res, split.split(A64, k, p, 1, 3), "nv", tap_scale=np.linalg.norm(A64))
+
+
+@pytest.mark.parametrize("fmt", ["nv", "mx"])
+def test_split_compensated_residual(fmt):
+    # R = A - deq(U_q) S deq(V_q)^T against the oracle fed the GPU's own FP4
+    # factors; U, S, V and their codes are those of the plain split; the
+    # quantized operand R_q + deq(U_q) S deq(V_q)^T is closer to A than with
+    # the plain residual
+    d = inputs.make("layer_4096", scale=dict(K=512, N=768, M=128))
+    A = to_device(d["W"])
+    plain = api.split(A, 64, 16, 1, 0, fmt, tap=True)
+    comp = api.split(A, 64, 16, 1, 0, fmt, tap=True, compensate=True)
+    torch.cuda.synchronize()
+    assert int(comp.dev_status.cpu()[0]) == 0
+    for name in ("U", "S", "V"):
+        assert torch.equal(getattr(plain, name), getattr(comp, name))
+    assert torch.equal(plain.U_q.codes, comp.U_q.codes) and torch.equal(plain.V_q.codes, comp.V_q.codes)
+    A64 = d["W"].f64()
+    Uq, Vq = read_fp4(comp.U_q), read_fp4(comp.V_q)
+    S = comp.S.cpu().numpy().astype(np.float64)
+    Rc = split.compensated_residual(A64, Uq, S, Vq)
+    R = comp.R_f32.cpu().numpy()
+    assert rel_fro(R, Rc) < TOL
+    assert_fp4_equal(comp.R_rows, fp4.quantize(R, fmt, 1), check_linear=False)
+    assert_fp4_equal(comp.R_cols, fp4.quantize(R, fmt, 0), check_linear=False)
+    low = (Uq.dequantize().T * S) @ Vq.dequantize()
+    err_c = rel_fro(low + read_fp4(comp.R_rows).dequantize(), A64)
+    err_p = rel_fro(low + read_fp4(plain.R_rows).dequantize(), A64)
+    assert err_c < err_p

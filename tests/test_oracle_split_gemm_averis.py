@@ -221,3 +221,47 @@ def test_averis_residual_amax_from_columns():
     mu = X.astype(np.float64).mean(axis=0).astype(np.float32)
     r = averis.residual_f32(X, mu)
     assert averis.residual_amax_from_columns(X, mu) == np.abs(r).max()
+
+
+# --------------------------------------------------------------------------
+# error-compensated residual (R29)
+# --------------------------------------------------------------------------
+
+def test_compensated_residual_equals_plain_for_representable_factors():
+    # factors whose entries are FP4 values times a power-of-two block scale
+    # are exact in MXFP4: the compensated residual is the plain one
+    rng = _rng(41)
+    grid = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+    U = rng.choice(grid, (64, 4)) * rng.choice([-1.0, 1.0], (64, 4)) / 8.0
+    V = rng.choice(grid, (96, 4)) * rng.choice([-1.0, 1.0], (96, 4)) / 16.0
+    U[0] = 6.0 / 8.0          # every 32-row block keeps its maximum at 6 x scale
+    U[32] = 6.0 / 8.0
+    V[0] = V[32] = V[64] = 6.0 / 16.0
+    S = np.array([3.0, 2.0, 1.5, 1.0])
+    A = rng.standard_normal((64, 96))
+    Uq = fp4.quantize(U.astype(np.float32), "mx", 0)
+    Vq = fp4.quantize(V.astype(np.float32), "mx", 0)
+    assert np.array_equal(Uq.dequantize().T, U) and np.array_equal(Vq.dequantize().T, V)
+    assert np.array_equal(split.compensated_residual(A, Uq, S, Vq), split.residual(A, U, S, V))
+
+
+@pytest.mark.parametrize("fmt", ["nv", "mx"])
+def test_compensated_residual_absorbs_the_factor_error(fmt):
+    # with an exact (unquantized) residual the compensated operand is A
+    # itself, while the plain residual leaves the factors' FP4 error; after
+    # quantizing the residual too, the compensated operand is the closer one
+    rng = _rng(42)
+    m, n, k = 256, 192, 16
+    A = (rng.standard_normal((m, k)) * (8.0 / (1 + np.arange(k)))) @ rng.standard_normal((k, n)) / np.sqrt(n)
+    A += 0.02 * rng.standard_normal((m, n))
+    r = split.split(A, k, 8, 1, 3)
+    Uq = fp4.quantize(r["U"].astype(np.float32), fmt, 0)
+    Vq = fp4.quantize(r["V"].astype(np.float32), fmt, 0)
+    low = (Uq.dequantize().T * r["S"]) @ Vq.dequantize()
+    Rc = split.compensated_residual(A, Uq, r["S"], Vq)
+    assert np.allclose(low + Rc, A, rtol=0, atol=1e-12)
+    plain_err = np.linalg.norm(low + r["R"] - A)
+    assert plain_err > 1e-3 * np.linalg.norm(A)
+    e_plain = np.linalg.norm(low + fp4.quantize(r["R"].astype(np.float32), fmt, 1).dequantize() - A)
+    e_comp = np.linalg.norm(low + fp4.quantize(Rc.astype(np.float32), fmt, 1).dequantize() - A)
+    assert e_comp < e_plain
