@@ -136,12 +136,6 @@ __global__ void build_lb_kernel(LowRankArgs a) {
   }
 }
 
-__global__ void copy_rows_kernel(const float* src, float* dst, int64_t n) {
-  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < n;
-       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
-    dst[i] = src[i];
-}
-
 // Operands of the error-compensated residual: thread per (row, column c <
 // kp) of [U rows | V rows]; column c < k holds hi / lo of deq(U_q)[row][c]
 // (U's rows) or of fl32(deq(V_q)[row][c] S[c]) (V's rows), padding columns 0.
@@ -197,10 +191,6 @@ void launch_compensated_operands(const FactorView& fu, const FactorView& fv, int
                                  __nv_bfloat16* w_hi, __nv_bfloat16* w_lo, int sms, cudaStream_t s) {
   compensated_operands_kernel<<<blocks_for((m + n) * kp, sms), 256, 0, s>>>(fu, fv, m, n, k, S, kp, u_hi, u_lo, w_hi,
                                                                            w_lo);
-}
-
-void launch_copy(const float* src, float* dst, int64_t n, int sms, cudaStream_t s) {
-  copy_rows_kernel<<<blocks_for(n, sms), 256, 0, s>>>(src, dst, n);
 }
 
 }  // namespace metis

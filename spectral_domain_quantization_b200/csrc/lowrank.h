@@ -47,7 +47,6 @@ struct LowRankArgs {
 void launch_cab(const FactorView& pa, const FactorView& pb, int64_t K, int ka, int kb, float* cab,
                 cudaStream_t s);
 void launch_build_lowrank(const LowRankArgs& a, int sms, cudaStream_t s);
-void launch_copy(const float* src, float* dst, int64_t n, int sms, cudaStream_t s);
 // hi / lo bf16 operands [rows][kp] of deq(U_q) (m rows) and deq(V_q) diag(S)
 // (n rows) for the error-compensated residual (fu: U_q, fv: V_q, k factors).
 void launch_compensated_operands(const FactorView& fu, const FactorView& fv, int64_t m, int64_t n, int k,
