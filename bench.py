@@ -560,7 +560,9 @@ def main():
         run_profile(args, int(os.environ.get("LOCAL_RANK", "0")))
         return
     if args.composite:
-        run_composite(args, int(os.environ.get("LOCAL_RANK", "0")))
+        # a single-GPU measurement: under a multi-process launch only rank 0 runs it
+        if int(os.environ.get("RANK", "0")) == 0:
+            run_composite(args, int(os.environ.get("LOCAL_RANK", "0")))
         return
     rank, world, local = dist_init()
     try:
