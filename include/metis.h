@@ -244,8 +244,10 @@ typedef struct {
  * U = Q W, V = Z W S^-1, signs (largest-|.| entry of each U column made
  * positive) -> R = A - U S V^T (or, with compensate, A minus the product of
  * the dequantized FP4 factors) fused with FP4 quantization.
- * With sample_rows > 0: V_s from the sampled rows, P = A V_s, CholeskyQR2 of
- * P, SVD of its triangular factor; U = Q_P W1, V = V_s W2.
+ * With sample_rows > 0: V_s from the sampled rows, P = A V_s, the
+ * eigen-decomposition P^T P = W diag(sigma^2) W^T with the same solver (the SVD
+ * of P's triangular QR factor in exact arithmetic); U = P W / sigma,
+ * V = V_s W.
  *
  *   A, dtype, m, n, lda   device input (bf16 or f32), row-major, 16-byte rows.
  *   U       device m x k float (row-major), S device k floats (descending),

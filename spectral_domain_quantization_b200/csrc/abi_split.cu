@@ -9,10 +9,13 @@
 //   [sample rows -> gather A_s]                      sketch.cu
 //   Omega^T (Philox Gaussian / sparse sign, bf16)    sketch.cu
 //   Y = A Omega                                      skinny_gemm.cu (tcgen05)
-//   Q = orth(Y)  CholeskyQR2                         small_linalg.cu
-//   q x { Q = orth(A^T Q); Q = orth(A Q) }
+//   q = 0: Q = orth(Y), two CholeskyQR passes        small_linalg.cu
+//   q >= 1: Y as is, then q x { Q1 = orth(A^T Y); Y = A Q1; Q = orth(Y) },
+//           one CholeskyQR pass each
 //   Z = B^T = A^T Q, C = Z^T Z                       skinny GEMM + Gram
-//   C = W diag(sigma^2) W^T (Jacobi), top k          small_linalg.cu
+//   C = W diag(sigma^2) W^T, top k                   core_eig.cu (tridiagonal
+//                                                    reduction, multisection,
+//                                                    twisted factorisation)
 //   U = Q W_k, V = Z W_k / sigma, S = sigma          row-block products
 //   signs; U_q, V_q                                  quantize.cu
 //   R = A - U S V^T, FP4 along n and/or m            residual_quant.cu
@@ -200,8 +203,8 @@ metis_status skinny(const Source& a, int mode, const __nv_bfloat16* xt, int64_t 
 }
 
 // CholeskyQR of the split partials of a rows x lp product, `passes` times
-// (2 = CholeskyQR2, for the final basis; 1 suffices for the intermediate
-// bases of the power iteration, whose span is all that is used).  Output: Q
+// (2 for the only basis when there is no power iteration; otherwise 1 for
+// every basis: the Gram is float64 from float32 data).  Output: Q
 // (fp32, rows x lp) and Q^T as bf16 hi / lo rows of qt (row stride ldq).
 metis_status cholqr(const SplitBuffers& b, int splits, int64_t rows, int lp, float* Q, int64_t ldq, int passes,
                     cudaStream_t s) {

@@ -472,9 +472,6 @@ __global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) {
   if (a.gpart) gram_block(Out, nr, a.kout, a.kout + 1, a.gpart + static_cast<int64_t>(blockIdx.x) * a.kout * a.kout);
 }
 
-// Round-robin pairing: in step r of a sweep over n (even) indices, slot i
-// pairs with slot n-1-i; slot 0 holds index 0, slots 1..n-1 rotate.
-
 // Factor matrices from the sorted eigen-decomposition of the core Gram:
 // Mu = W_k (lp x k), Mv = W_k diag(1/sigma) (0 where sigma is negligible),
 // S = sigma_k.
