@@ -333,6 +333,328 @@ __global__ void __launch_bounds__(kThreads, CTAS)
   if (threadIdx.x == 0 && *abort_flag) report(p.dev_status, METIS_DEV_TIMEOUT);
 }
 
+// ---------------------------------------------------------------------------
+// Wide tile: two 128-row M halves share one 192-row B tile (256 x 192 per
+// CTA).  Per flop it moves 22 % fewer operand bytes from L2 than a 128 x 256
+// tile and issues fewer scale copies.  TMEM: the two halves' accumulators in
+// columns 0-383 and the scale factors in two 64-column slots; a slot is
+// refilled only after the commit of the stage that last read it.  B's scale
+// chunks come from the 128-row chunk at or below the tile's first row: a tile
+// that starts 64 rows into a chunk (odd tn) reads them two TMEM columns
+// further.  Rows past M and columns past N are computed on zero-filled (TMA)
+// operands and never stored.  No split-K.
+constexpr int kWideBN = 192;
+constexpr int kWideStages = 3;
+struct WideSmem {
+  static constexpr int kA = 128 * 128;         // one M half, K = 256 FP4
+  static constexpr int kB = kWideBN * 128;
+  static constexpr int kSFA = 2048;            // per half
+  static constexpr int kSFB = 4096;            // two 128-row chunks
+  static constexpr int kStage = 2 * kA + kB + 2 * kSFA + kSFB;
+  static constexpr int kBytes = kWideStages * kStage + 1024 /*align*/ + 256 /*barriers*/;
+};
+
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_fp4_wide_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmA,
+                         const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmLA,
+                         const __grid_constant__ CUtensorMap tmLB) {
+  using S = WideSmem;
+  constexpr int kStages = kWideStages;
+  constexpr int BN = kWideBN;
+  constexpr uint32_t kSfBase = 2 * BN;   // first TMEM column after the accumulators
+  constexpr uint32_t kSlotCols = 64;     // per slot: A scales 2 x 16, B scales 32
+  extern __shared__ __align__(1024) uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + kStages * S::kStage);
+  uint64_t* empty = full + kStages;
+  uint64_t* acc_full = empty + kStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* sf_free = acc_empty + 1;     // [2]
+  uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(sf_free + 2);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_sh + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const bool nv = p.fmt == METIS_NVFP4;
+  const int atoms_per_kt = nv ? 4 : 2;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kEpiWarps);
+    mbar_init(&sf_free[0], 1);
+    mbar_init(&sf_free[1], 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+    if (p.lr_chunks) {
+      prefetch_tensormap(&tmLA);
+      prefetch_tensormap(&tmLB);
+    }
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_base_sh, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_base_sh;
+
+  const int tiles_m = (p.M + 255) / 256;
+  const int tiles_n = (p.N + BN - 1) / BN;
+  const int num_tiles = tiles_m * tiles_n;
+  const int nk = p.num_kt + p.lr_chunks;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      int stage = 0, issued = 0;
+      uint32_t phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int tm = t % tiles_m, tn = t / tiles_m;
+        const bool half1 = 256 * tm + 128 < p.M;               // A scales of the second half exist
+        const int nb0 = tn * BN / 128;                         // B scale chunk at or below the tile
+        const bool second = (nb0 + 1) * 128 < p.sfb_rows;
+        for (int it = 0; it < nk; ++it) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag)) { ok = false; break; }
+          uint8_t* sA0 = smem + stage * S::kStage;
+          uint8_t* sA1 = sA0 + S::kA;
+          uint8_t* sB = sA1 + S::kA;
+          uint8_t* sSFA0 = sB + S::kB;
+          uint8_t* sSFA1 = sSFA0 + S::kSFA;
+          uint8_t* sSFB = sSFA1 + S::kSFA;
+          if (it < p.num_kt) {
+            const int kt = it;
+            const uint32_t sf_bytes = 512u * atoms_per_kt;
+            const uint32_t bytes = 2 * S::kA + S::kB + sf_bytes * ((half1 ? 2 : 1) + (second ? 2 : 1));
+            mbar_arrive_expect_tx(&full[stage], bytes);
+            tma_load_2d(sA0, &tmA, &full[stage], kt * 128, 256 * tm);
+            tma_load_2d(sA1, &tmA, &full[stage], kt * 128, 256 * tm + 128);
+            tma_load_2d(sB, &tmB, &full[stage], kt * 128, tn * BN);
+            bulk_load(sSFA0, p.sfa + (static_cast<int64_t>(2 * tm) * p.sfa_chunks + kt * atoms_per_kt) * 512, sf_bytes,
+                      &full[stage]);
+            if (half1)
+              bulk_load(sSFA1, p.sfa + (static_cast<int64_t>(2 * tm + 1) * p.sfa_chunks + kt * atoms_per_kt) * 512,
+                        sf_bytes, &full[stage]);
+            bulk_load(sSFB, p.sfb + (static_cast<int64_t>(nb0) * p.sfb_chunks + kt * atoms_per_kt) * 512, sf_bytes,
+                      &full[stage]);
+            if (second)
+              bulk_load(sSFB + 2048, p.sfb + (static_cast<int64_t>(nb0 + 1) * p.sfb_chunks + kt * atoms_per_kt) * 512,
+                        sf_bytes, &full[stage]);
+          } else {
+            const int c = it - p.num_kt;
+            mbar_arrive_expect_tx(&full[stage], 2 * S::kA + S::kB);
+            tma_load_2d(sA0, &tmLA, &full[stage], c * 64, 256 * tm);
+            tma_load_2d(sA1, &tmLA, &full[stage], c * 64, 256 * tm + 128);
+            tma_load_2d(sB, &tmLB, &full[stage], c * 64, tn * BN);
+          }
+          ++issued;
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      if (*abort_flag) {
+        // let copies already in flight land before the CTA exits
+        int s = stage;
+        uint32_t ph = phase;
+        for (int i = 0; i < min(issued, kStages); ++i) {
+          if (--s < 0) { s = kStages - 1; ph ^= 1u; }
+          wait_ns(&full[s], ph, 100000000ull);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0, g = 0;
+      uint32_t phase = 0, acc_phase = 0;
+      bool ok = true;
+      const uint32_t acc0 = tmem, acc1 = tmem + BN;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int tn = t / tiles_m;
+        const uint32_t shift = (tn & 1) ? 2u : 0u;   // the tile starts 64 rows into its first B scale chunk
+        if (!mbar_wait(acc_empty, acc_phase ^ 1u, abort_flag)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t accumulate = 0;
+        for (int it = 0; it < nk; ++it) {
+          if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          tc_fence_after();
+          uint8_t* sA0 = smem + stage * S::kStage;
+          uint8_t* sA1 = sA0 + S::kA;
+          uint8_t* sB = sA1 + S::kA;
+          const uint64_t a0 = make_sdesc(smem_u32(sA0), 16, 1024, kSwizzle128B);
+          const uint64_t a1 = make_sdesc(smem_u32(sA1), 16, 1024, kSwizzle128B);
+          const uint64_t bd = make_sdesc(smem_u32(sB), 16, 1024, kSwizzle128B);
+          if (it < p.num_kt) {
+            const int slot = g & 1;
+            if (g >= 2) {
+              // the MMAs that last read this slot (stage g - 2) have retired
+              if (!mbar_wait(&sf_free[slot], static_cast<uint32_t>((g >> 1) - 1) & 1u, abort_flag)) { ok = false; break; }
+              tc_fence_after();
+            }
+            uint8_t* sSFA0 = sB + S::kB;
+            uint8_t* sSFA1 = sSFA0 + S::kSFA;
+            uint8_t* sSFB = sSFA1 + S::kSFA;
+            const uint32_t sf = tmem + kSfBase + slot * kSlotCols;
+            const uint32_t sfa0 = sf, sfa1 = sf + 16, sfb = sf + 32;
+            for (int a = 0; a < atoms_per_kt; ++a) {
+              tc_cp_32x128b_warpx4(sfa0 + 4 * a, make_sdesc(smem_u32(sSFA0 + 512 * a), 0, 128, kSwizzleNone));
+              tc_cp_32x128b_warpx4(sfa1 + 4 * a, make_sdesc(smem_u32(sSFA1 + 512 * a), 0, 128, kSwizzleNone));
+              for (int h = 0; h < 2; ++h)
+                tc_cp_32x128b_warpx4(sfb + 8 * a + 4 * h,
+                                     make_sdesc(smem_u32(sSFB + 2048 * h + 512 * a), 0, 128, kSwizzleNone));
+            }
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint64_t koff = static_cast<uint64_t>((j * 32) >> 4);
+              if (nv) {
+                const uint32_t id = idesc_fp4(128, BN, false, 0, 0);
+                mma_nvf4(acc0, a0 + koff, bd + koff, id, sfa0 + 4 * j, sfb + 8 * j + shift, accumulate);
+                mma_nvf4(acc1, a1 + koff, bd + koff, id, sfa1 + 4 * j, sfb + 8 * j + shift, accumulate);
+              } else {
+                const uint32_t sid = 2u * (j & 1);
+                const uint32_t id = idesc_fp4(128, BN, true, sid, sid);
+                const uint32_t sb = (sfb + 8 * (j >> 1) + shift) | (sid << 30);
+                mma_mxf4(acc0, a0 + koff, bd + koff, id, (sfa0 + 4 * (j >> 1)) | (sid << 30), sb, accumulate);
+                mma_mxf4(acc1, a1 + koff, bd + koff, id, (sfa1 + 4 * (j >> 1)) | (sid << 30), sb, accumulate);
+              }
+              accumulate = 1;
+            }
+            tc_commit(&sf_free[slot]);
+            ++g;
+          } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              const uint64_t koff = static_cast<uint64_t>((j * 32) >> 4);
+              const uint32_t id = idesc_bf16(128, BN, false, false);
+              mma_bf16(acc0, a0 + koff, bd + koff, id, accumulate);
+              mma_bf16(acc1, a1 + koff, bd + koff, id, accumulate);
+              accumulate = 1;
+            }
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+        acc_phase ^= 1u;
+      }
+      if (*abort_flag) {
+        // wait for MMAs already issued before the TMEM is freed
+        tc_commit(acc_full);
+        wait_ns(acc_full, acc_phase, 100000000ull);
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;               // TMEM lane quadrant of this warp
+    const int h = (warp - 2) >> 2;        // M half (accumulator)
+    float alpha = 1.f;
+    if (p.ts_a) alpha = __fmul_rn(alpha, *p.ts_a);
+    if (p.ts_b) alpha = __fmul_rn(alpha, *p.ts_b);
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x) {
+      const int tm = t % tiles_m, tn = t / tiles_m;
+      if (!mbar_wait(acc_full, acc_phase, abort_flag)) break;
+      tc_fence_after();
+      acc_phase ^= 1u;
+      const int64_t row = static_cast<int64_t>(tm) * 256 + 128 * h + 32 * q + lane;
+      const bool row_ok = row < p.M;
+      const uint32_t tbase = tmem + (static_cast<uint32_t>(32 * q) << 16) + h * BN;
+      const int64_t col0 = static_cast<int64_t>(tn) * BN;
+      if (p.c_dtype != METIS_F32 && col0 + BN <= p.N && p.vec16_ok) {
+        // bf16, full-width tile: the whole row fits in registers as packed
+        // pairs, so the accumulator is released before any store
+        uint32_t pk[BN / 2];
+#pragma unroll
+        for (int cc = 0; cc < BN / 16; ++cc) {
+          uint32_t v[16];
+          tmem_ld16(tbase + 16 * cc, v);
+          tmem_ld_wait();
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const __nv_bfloat16 lo = __float2bfloat16_rn(__fmul_rn(alpha, __uint_as_float(v[2 * e])));
+            const __nv_bfloat16 hi = __float2bfloat16_rn(__fmul_rn(alpha, __uint_as_float(v[2 * e + 1])));
+            pk[8 * cc + e] = static_cast<uint32_t>(__bfloat16_as_ushort(lo)) |
+                             (static_cast<uint32_t>(__bfloat16_as_ushort(hi)) << 16);
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(acc_empty);
+        if (!row_ok) continue;
+        uint4* dst = reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.C) + row * p.ldc + col0);
+#pragma unroll
+        for (int c = 0; c < BN / 8; ++c) dst[c] = make_uint4(pk[4 * c], pk[4 * c + 1], pk[4 * c + 2], pk[4 * c + 3]);
+        continue;
+      }
+      // otherwise drained 32 columns at a time and released after the last load
+      for (int cc = 0; cc < BN / 32; ++cc) {
+        uint32_t v[32];
+        tmem_ld16(tbase + 32 * cc, v);
+        tmem_ld16(tbase + 32 * cc + 16, v + 16);
+        tmem_ld_wait();
+        if (cc == BN / 32 - 1) {
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(acc_empty);
+        }
+        if (!row_ok) continue;
+        const int64_t cb = col0 + 32 * cc;
+        if (p.c_dtype == METIS_F32) {
+          float* dst = reinterpret_cast<float*>(p.C) + row * p.ldc;
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            const int64_t col = cb + c;
+            const float4 f = make_float4(__fmul_rn(alpha, __uint_as_float(v[c])), __fmul_rn(alpha, __uint_as_float(v[c + 1])),
+                                         __fmul_rn(alpha, __uint_as_float(v[c + 2])), __fmul_rn(alpha, __uint_as_float(v[c + 3])));
+            if (col + 3 < p.N && p.vec_ok) {
+              *reinterpret_cast<float4*>(dst + col) = f;
+            } else {
+              const float fe[4] = {f.x, f.y, f.z, f.w};
+              for (int e = 0; e < 4; ++e)
+                if (col + e < p.N) dst[col + e] = fe[e];
+            }
+          }
+        } else {
+          __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(p.C) + row * p.ldc;
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            const int64_t col = cb + c;
+            __nv_bfloat16 b[4];
+            for (int e = 0; e < 4; ++e) b[e] = __float2bfloat16_rn(__fmul_rn(alpha, __uint_as_float(v[c + e])));
+            if (col + 3 < p.N && p.vec_ok) {
+              uint2 u;
+              u.x = static_cast<uint32_t>(__bfloat16_as_ushort(b[0])) | (static_cast<uint32_t>(__bfloat16_as_ushort(b[1])) << 16);
+              u.y = static_cast<uint32_t>(__bfloat16_as_ushort(b[2])) | (static_cast<uint32_t>(__bfloat16_as_ushort(b[3])) << 16);
+              *reinterpret_cast<uint2*>(dst + col) = u;
+            } else {
+              for (int e = 0; e < 4; ++e)
+                if (col + e < p.N) dst[col + e] = b[e];
+            }
+          }
+        }
+      }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, 512);
+  }
+  if (threadIdx.x == 0 && *abort_flag) report(p.dev_status, METIS_DEV_TIMEOUT);
+}
+
 // Deterministic split-K reduction: C = alpha * sum_s partial[s] (+ nothing).
 __global__ void splitk_reduce_kernel(const float* partial, int splits, int64_t M, int64_t N, const float* ts_a,
                                      const float* ts_b, void* C, int c_dtype, int64_t ldc) {
@@ -379,6 +701,16 @@ cudaError_t launch_bn(const GemmParams& p, const CUtensorMap& a, const CUtensorM
   return cudaGetLastError();
 }
 
+cudaError_t launch_wide(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b, const CUtensorMap& la,
+                        const CUtensorMap& lb, int tiles, cudaStream_t s) {
+  const int bytes = WideSmem::kBytes;
+  if (!ensure_smem(reinterpret_cast<const void*>(gemm_fp4_wide_kernel), bytes)) return cudaErrorInvalidValue;
+  const int slots = device_sm_count();
+  const int grid = tiles < slots ? tiles : slots;
+  gemm_fp4_wide_kernel<<<grid, kThreads, bytes, s>>>(p, a, b, la, lb);
+  return cudaGetLastError();
+}
+
 CUresult fp4_map(CUtensorMap* m, const uint8_t* codes, int64_t rows, int64_t inner, uint32_t box_rows) {
   const uint64_t dims[2] = {static_cast<uint64_t>(inner / 2), static_cast<uint64_t>(rows)};
   const uint64_t strides[1] = {static_cast<uint64_t>(inner / 2)};
@@ -416,12 +748,25 @@ metis_status run_gemm_fp4(const GemmCall& g, cudaStream_t s) {
   p.c_dtype = g.c_dtype;
   p.ldc = g.ldc;
   p.vec_ok = (g.ldc % 4 == 0) && ((reinterpret_cast<uintptr_t>(g.C) & 15u) == 0);
+  p.vec16_ok = (g.ldc % 8 == 0) && ((reinterpret_cast<uintptr_t>(g.C) & 15u) == 0);
   p.dev_status = g.dev_status;
   p.splits = gemm_effective_splits(g.K, g.splits);
   p.partial = g.partial;
   if (p.splits > 1 && !p.partial) return METIS_ERR_ARG;
   if (p.splits > 1 && p.lr_chunks) return METIS_ERR_ARG;
-  const int bn = g.bn;
+  // The wide tile (two 128-row halves sharing a 192-row B tile) covers 1.5
+  // times the work of a 128 x 256 tile and, measured on an NVFP4
+  // 8192 x 4096 x 4096 product, runs a unit of work 4.5 % faster
+  // (17.4 against 18.2 us per 128 x 256 x 4096 unit).  It is taken for
+  // unsplit products when its rounds of tiles over the SMs cost less.
+  bool wide = false;
+  if (g.bn == 256 && p.splits == 1 && g.M >= 256 && g.N >= 384) {
+    const int64_t sms = device_sm_count();
+    const int64_t rounds_n = (((g.M + 127) / 128) * ((g.N + 255) / 256) + sms - 1) / sms;
+    const int64_t rounds_w = (((g.M + 255) / 256) * ((g.N + kWideBN - 1) / kWideBN) + sms - 1) / sms;
+    wide = rounds_w * 1433 < rounds_n * 1000;   // 1.5 x 0.955
+  }
+  const int bn = wide ? kWideBN : g.bn;
   CUtensorMap ma, mb, mla, mlb;
   if (fp4_map(&ma, g.a_codes, g.M, g.K, 128) != CUDA_SUCCESS) return fail(METIS_ERR_CUDA, "gemm_fp4 tensor map");
   if (fp4_map(&mb, g.b_codes, g.N, g.K, static_cast<uint32_t>(bn)) != CUDA_SUCCESS) return fail(METIS_ERR_CUDA, "gemm_fp4 tensor map");
@@ -434,7 +779,9 @@ metis_status run_gemm_fp4(const GemmCall& g, cudaStream_t s) {
   }
   const int tiles = static_cast<int>(((g.M + 127) / 128) * ((g.N + bn - 1) / bn)) * p.splits;
   cudaError_t e;
-  if (bn == 256)
+  if (wide)
+    e = launch_wide(p, ma, mb, mla, mlb, static_cast<int>(((g.M + 255) / 256) * ((g.N + bn - 1) / bn)), s);
+  else if (bn == 256)
     e = launch_bn<256, 4, 1>(p, ma, mb, mla, mlb, tiles, s);
   else if (bn == 128)
     e = launch_bn<128, 4, 1>(p, ma, mb, mla, mlb, tiles, s);

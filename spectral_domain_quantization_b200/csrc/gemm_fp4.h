@@ -24,7 +24,8 @@ struct GemmParams {
   void* C;
   int c_dtype;
   int64_t ldc;
-  int vec_ok;
+  int vec_ok;               // 16-byte aligned rows of 4 columns (f32) or 4 bf16
+  int vec16_ok;             // 16-byte aligned rows of 8 bf16 columns
   int32_t* dev_status;
   int splits;               // split-K factor (1 = none)
   float* partial;           // split-K partial sums [splits][M][N] (raw, no alpha)

@@ -61,6 +61,41 @@ def test_plain_product_bf16_output():
     assert rel_fro(y.float().cpu().numpy(), want) < 5e-3
 
 
+# Shapes whose rounds of tiles over 148 SMs favour the 256 x 192 tile (two
+# 128-row halves sharing one B tile): full-width and ragged tiles, rows of C
+# with and without 16-byte alignment.
+WIDE_SHAPES = [(2048, 2560, 512), (2000, 2500, 512)]
+
+
+@pytest.mark.parametrize("fmt", ["mx", "nv"])
+@pytest.mark.parametrize("M,N,K", WIDE_SHAPES)
+def test_wide_tile_product(fmt, M, N, K):
+    a = _rand((M, K), M + 3)
+    b = _rand((K, N), N + 5)
+    qa, ra = _q(a, fmt, 1)
+    qb, rb = _q(b, fmt, 0)
+    y = api.linear_fwd(api.Operand(qa), api.Operand(qb), M, N, K)
+    y16 = api.linear_fwd(api.Operand(qa), api.Operand(qb), M, N, K, out_dtype=torch.bfloat16)
+    torch.cuda.synchronize()
+    want = gemm.gemm(gemm.Operand(ra), gemm.Operand(rb))
+    assert rel_fro(y.cpu().numpy(), want) < 1e-5
+    # the bf16 output is the float32 one rounded once (same accumulation)
+    assert torch.equal(y16.cpu(), y.cpu().to(torch.bfloat16))
+
+
+@pytest.mark.parametrize("fmt", ["mx", "nv"])
+def test_wide_tile_right_split_product(fmt):
+    # the low-rank chunks appended to the K loop of the wide tile
+    M, N, K, kb = 2000, 2560, 512, 64
+    qa, ra = _q(_rand((M, K), 17), fmt, 1)
+    qr, rr = _q(_rand((K, N), 18, 0.1), fmt, 0)
+    qP, rP, qF, rF, S = _factors(N, K, kb, fmt, 19)
+    y = api.linear_fwd(api.Operand(qa), api.Operand(qr, kb, qP, qF, torch.from_numpy(S).cuda()), M, N, K)
+    torch.cuda.synchronize()
+    want = gemm.gemm(gemm.Operand(ra), gemm.Operand(rr, kb, rP, rF, S))
+    assert rel_fro(y.cpu().numpy(), want) < TOL
+
+
 def _factors(n_free, K, k, fmt, seed):
     P = (_rand((K, k), seed) / np.sqrt(K)).astype(np.float32)
     F = (_rand((n_free, k), seed + 1) / np.sqrt(n_free)).astype(np.float32)
