@@ -27,6 +27,11 @@
 //               store raw partial sums for split-K.
 // Every wait is bounded (METIS_DEV_TIMEOUT) and the kernel always frees its
 // TMEM.  Shared memory per stage: A 16 KB + B BN*128 B + scales 6 KB.
+//
+// A second kernel, gemm_fp4_wide_kernel, runs the same pipeline on a
+// 256 x 192 tile (two 128-row M halves sharing one B tile, three stages);
+// run_gemm_fp4 picks it for unsplit products when its rounds of tiles over
+// the SMs cost less than the 128 x 256 tile's.
 #include "abi_common.h"
 #include "common.cuh"
 #include "gemm_fp4.h"

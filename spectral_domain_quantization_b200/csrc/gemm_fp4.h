@@ -47,7 +47,7 @@ struct GemmCall {
   void* C;                  // output (NULL allowed with splits > 1 to keep partials only)
   int c_dtype;
   int64_t ldc;
-  int bn;                   // MMA N tile: 64, 128 or 256
+  int bn;                   // MMA N tile: 64, 128 or 256 (an unsplit 256 may run as the 256 x 192 wide tile)
   int splits;
   float* partial;
   int32_t* dev_status;
