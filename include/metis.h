@@ -46,6 +46,14 @@
 #include <stddef.h>
 #include <stdint.h>
 
+/* Entry points are the library's only exported symbols (it is built with
+ * hidden visibility). */
+#if defined(__GNUC__)
+#define METIS_API __attribute__((visibility("default")))
+#else
+#define METIS_API
+#endif
+
 #ifdef __cplusplus
 extern "C" {
 #endif
@@ -104,19 +112,19 @@ typedef struct {
 } metis_fp4_tensor;
 
 /* Host-only helpers (no device work): buffer sizes for a metis_fp4_tensor. */
-size_t metis_fp4_codes_bytes(int64_t outer, int64_t inner);
-size_t metis_fp4_scales_bytes(int32_t fmt, int64_t outer, int64_t inner);
+METIS_API size_t metis_fp4_codes_bytes(int64_t outer, int64_t inner);
+METIS_API size_t metis_fp4_scales_bytes(int32_t fmt, int64_t outer, int64_t inner);
 
 /* Host-only: short description of a status code (static string). */
-const char* metis_status_string(int32_t status);
+METIS_API const char* metis_status_string(int32_t status);
 
 /* Host-only: 1 if a device of compute capability 10.x is current, else 0. */
-int32_t metis_device_supported(void);
+METIS_API int32_t metis_device_supported(void);
 
 /* Host-only: description of the last METIS_ERR_CUDA reported on this thread
  * (which step failed and the CUDA error string); "" if none.  The string is
  * owned by the library and overwritten by the next failure on the thread. */
-const char* metis_last_error(void);
+METIS_API const char* metis_last_error(void);
 
 /*
  * metis_selftest_wait_timeout -- check of the failure detection every kernel
@@ -128,7 +136,7 @@ const char* metis_last_error(void);
  * Errors: METIS_ERR_NULL (dev_status), METIS_ERR_ARG (limit out of range),
  * METIS_ERR_UNSUPPORTED (no sm_100 device), METIS_ERR_CUDA (launch).
  */
-metis_status metis_selftest_wait_timeout(uint64_t limit_ns, int32_t* dev_status, void* stream);
+METIS_API metis_status metis_selftest_wait_timeout(uint64_t limit_ns, int32_t* dev_status, void* stream);
 
 /*
  * metis_quantize_fp4 -- block-quantize a dense matrix to FP4.
@@ -156,7 +164,7 @@ metis_status metis_selftest_wait_timeout(uint64_t limit_ns, int32_t* dev_status,
  *                multiple of 32 (METIS_ERR_SHAPE).
  * Workspace: NVFP4 needs a few bytes for the tensor maximum.
  */
-metis_status metis_quantize_fp4(const void* X, int32_t dtype, int64_t rows, int64_t cols,
+METIS_API metis_status metis_quantize_fp4(const void* X, int32_t dtype, int64_t rows, int64_t cols,
                                 int64_t ld, int32_t block_axis, const float* sub_col,
                                 metis_fp4_tensor* out, void* workspace,
                                 size_t* workspace_bytes, void* stream);
@@ -186,12 +194,12 @@ metis_status metis_quantize_fp4(const void* X, int32_t dtype, int64_t rows, int6
  *     The call zeroes what must start at zero itself.
  * The function never calls cudaMalloc, cudaFree or any allocating routine.
  */
-metis_status metis_quantize_fp4_noalloc(const void* X, int32_t dtype, int64_t rows, int64_t cols,
+METIS_API metis_status metis_quantize_fp4_noalloc(const void* X, int32_t dtype, int64_t rows, int64_t cols,
                                         int64_t ld, int32_t block_axis, const float* sub_col,
                                         metis_fp4_tensor* out, void* stream);
 
 /* Host-only: size in bytes of the fixed scratch array of the _noalloc call. */
-size_t metis_noalloc_scratch_bytes(void);
+METIS_API size_t metis_noalloc_scratch_bytes(void);
 
 /*
  * Parameters of the randomized split (host struct).
@@ -261,7 +269,7 @@ typedef struct {
  *   dev_status  device int32 (required).
  * Quantized outputs need m and n multiples of 32 along their blocked axis.
  */
-metis_status metis_split(const void* A, int32_t dtype, int64_t m, int64_t n, int64_t lda,
+METIS_API metis_status metis_split(const void* A, int32_t dtype, int64_t m, int64_t n, int64_t lda,
                          const metis_split_params* prm, float* U, float* S, float* V,
                          metis_fp4_tensor* U_q, metis_fp4_tensor* V_q,
                          metis_fp4_tensor* R_rows, metis_fp4_tensor* R_cols, float* R_f32,
@@ -303,7 +311,7 @@ typedef struct {
  *   Y  device M x N, y_dtype METIS_F32 or METIS_BF16, leading dimension ldy.
  * K must be a multiple of 32.
  */
-metis_status metis_linear_fwd(const metis_operand* X, const metis_operand* W, int64_t M,
+METIS_API metis_status metis_linear_fwd(const metis_operand* X, const metis_operand* W, int64_t M,
                               int64_t N, int64_t K, void* Y, int32_t y_dtype, int64_t ldy,
                               void* workspace, size_t* workspace_bytes, int32_t* dev_status,
                               void* stream);
@@ -320,7 +328,7 @@ metis_status metis_linear_fwd(const metis_operand* X, const metis_operand* W, in
  *   out_dtype METIS_F32 or METIS_BF16; ld_dx, ld_dw leading dimensions.
  * N must be a multiple of 32 for dX and M a multiple of 32 for dW.
  */
-metis_status metis_linear_bwd(const metis_operand* dY_n, const metis_operand* Wt,
+METIS_API metis_status metis_linear_bwd(const metis_operand* dY_n, const metis_operand* Wt,
                               const metis_operand* Xt, const metis_operand* dY_m, int64_t M,
                               int64_t N, int64_t K, void* dX, int64_t ld_dx, void* dW,
                               int64_t ld_dw, int32_t out_dtype, void* workspace,
@@ -341,7 +349,7 @@ metis_status metis_linear_bwd(const metis_operand* dY_n, const metis_operand* Wt
  * NVFP4 takes the residual's tensor maximum from the column minima and maxima
  * (exact: rounding is monotonic), so X is read twice in total.
  */
-metis_status averis_split(const void* X, int32_t dtype, int64_t m, int64_t n, int64_t ld,
+METIS_API metis_status averis_split(const void* X, int32_t dtype, int64_t m, int64_t n, int64_t ld,
                           int32_t fmt, float* mean, metis_fp4_tensor* mean_q,
                           metis_fp4_tensor* R_rows, metis_fp4_tensor* R_cols, float* R_f32,
                           void* workspace, size_t* workspace_bytes, int32_t* dev_status,

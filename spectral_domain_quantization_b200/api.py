@@ -104,7 +104,8 @@ def header_functions():
     """Names of the functions declared in include/metis.h."""
     src = open(HEADER).read()
     src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\**\s+\**(\w+)\s*\(", src, flags=re.M)))
+    return sorted(set(re.findall(r"^\s*(?:METIS_API\s+)?(?:const\s+)?[a-z_0-9]+\s*\**\s+\**(\w+)\s*\(", src,
+                                 flags=re.M)))
 
 
 def status_string(status):

@@ -20,7 +20,7 @@ BUILD = os.path.join(ROOT, "_build")
 LIB = os.path.join(HERE, "libmetis_b200.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2",
+FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-Xcompiler", "-O2", "-Xcompiler", "-fvisibility=hidden",
          "--expt-relaxed-constexpr", "-I", INCLUDE]
 
 
@@ -49,7 +49,8 @@ def _stale(target, deps):
 
 def _compile(src, extra, verbose):
     obj = os.path.join(BUILD, os.path.basename(src) + ".o")
-    if not _stale(obj, [src] + _headers()):
+    # the compile flags live in this file: a change to it rebuilds everything
+    if not _stale(obj, [src, os.path.abspath(__file__)] + _headers()):
         return obj
     cmd = [nvcc(), *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
     if verbose:
