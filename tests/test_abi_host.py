@@ -6,6 +6,7 @@ import subprocess
 
 import numpy as np
 import pytest
+import torch
 
 from oracle import fp4
 from spectral_domain_quantization_b200 import api
@@ -108,3 +109,156 @@ def test_split_params_layout_matches_the_header():
     assert [P.k.offset, P.p.offset, P.power_iters.offset, P.seed.offset, P.sketch.offset, P.sparse_nnz.offset,
             P.sample_rows.offset, P.fmt.offset, P.max_core_iters.offset, P.compensate.offset] == \
         [0, 4, 8, 16, 24, 28, 32, 40, 44, 48]
+
+
+# ---------------------------------------------------------------------------
+# argument checks of the split, product and Averis entry points: every case
+# returns before any device work (workspace query or a rejected argument), so
+# the pointers below are never dereferenced.  The one call that passes every
+# check with a workspace runs only without a GPU (where it must report
+# METIS_ERR_UNSUPPORTED); on a GPU it would launch on these fake pointers.
+# ---------------------------------------------------------------------------
+
+ERR_SHAPE, ERR_ALIGN, ERR_UNSUPPORTED, ERR_WORKSPACE = 2, 3, 4, 5
+_A, _U, _S, _V, _ST, _WS = 0x40000, 0x50000, 0x58000, 0x60000, 0x68000, 0x70000
+
+
+def _params(k=8, p=8, q=1, sketch=0, nnz=4, sample_rows=0, fmt=api.NVFP4, iters=64, compensate=0):
+    prm = api.SplitParams()
+    prm.k, prm.p, prm.power_iters, prm.seed = k, p, q, 0
+    prm.sketch, prm.sparse_nnz, prm.sample_rows = sketch, nnz, sample_rows
+    prm.fmt, prm.max_core_iters, prm.compensate = fmt, iters, compensate
+    return prm
+
+
+def _split(m=256, n=128, lda=None, prm=None, A=_A, U_q=None, V_q=None, R_rows=None, R_cols=None, ws=None,
+           wsb=None, dtype=None):
+    L = api.lib()
+    size = ctypes.c_size_t(0 if wsb is None else wsb)
+    prm = _params() if prm is None else prm
+    ref = lambda t: ctypes.byref(t) if t is not None else None
+    st = L.metis_split(A, api.BF16 if dtype is None else dtype, m, n, n if lda is None else lda,
+                       ctypes.byref(prm) if prm is not False else None, _U, _S, _V,
+                       ref(U_q), ref(V_q), ref(R_rows), ref(R_cols), None, None, ws, ctypes.byref(size),
+                       _ST, None)
+    return st, size.value
+
+
+def test_split_argument_checks_and_workspace_query():
+    st, need = _split()
+    assert st == api.OK and need > 0
+    assert _split(R_rows=_fake_fp4(api.NVFP4, 256, 128), R_cols=_fake_fp4(api.NVFP4, 128, 256))[0] == api.OK
+    assert _split(prm=False)[0] == ERR_NULL
+    assert _split(A=None)[0] == ERR_NULL
+    assert _split(m=0)[0] == ERR_SHAPE
+    assert _split(lda=100)[0] == ERR_SHAPE                        # lda < n
+    assert _split(A=0x40002)[0] == ERR_ALIGN
+    assert _split(lda=132)[0] == ERR_ALIGN                        # rows not on 16-byte boundaries
+    assert _split(dtype=9)[0] == ERR_ARG
+    assert _split(prm=_params(fmt=5))[0] == ERR_ARG
+    assert _split(prm=_params(sketch=3))[0] == ERR_ARG
+    assert _split(prm=_params(k=0))[0] == ERR_ARG
+    assert _split(prm=_params(q=-1))[0] == ERR_ARG
+    assert _split(prm=_params(iters=0))[0] == ERR_ARG
+    assert _split(prm=_params(sketch=1, nnz=0))[0] == ERR_ARG
+    assert _split(prm=_params(sketch=1, nnz=17))[0] == ERR_ARG
+    assert _split(prm=_params(compensate=2))[0] == ERR_ARG
+    assert _split(prm=_params(compensate=1))[0] == ERR_NULL       # compensation needs U_q and V_q
+    assert _split(prm=_params(k=64, p=64))[0] == ERR_SHAPE       # l = k + p above the core's limit
+    assert _split(prm=_params(k=6))[0] == ERR_SHAPE              # k not a multiple of 4
+    assert _split(n=64, prm=_params(k=40, p=40))[0] == ERR_SHAPE  # l > n
+    assert _split(prm=_params(sample_rows=512))[0] == ERR_SHAPE   # more sampled rows than rows
+    assert _split(prm=_params(k=40, p=40, sample_rows=64))[0] == ERR_SHAPE  # l > sampled rows
+    assert _split(m=96 + 8, n=128)[0] == ERR_SHAPE               # m not a multiple of 32
+    assert _split(R_rows=_fake_fp4(api.NVFP4, 128, 256))[0] == ERR_SHAPE   # rows tensor must be m x n
+    assert _split(R_rows=_fake_fp4(api.MXFP4, 256, 128))[0] == ERR_ARG     # format differs from the params
+    assert _split(U_q=_fake_fp4(api.NVFP4, 8, 256))[0] == api.OK          # U_q: outer k, inner m
+    assert _split(U_q=_fake_fp4(api.NVFP4, 256, 8))[0] == ERR_SHAPE
+    assert _split(ws=ctypes.c_void_p(_WS), wsb=need - 1)[0] == ERR_WORKSPACE
+    assert _split(ws=ctypes.c_void_p(_WS + 8), wsb=need)[0] == ERR_WORKSPACE  # not 256-byte aligned
+    if not torch.cuda.is_available():
+        assert _split(ws=ctypes.c_void_p(_WS), wsb=need)[0] == ERR_UNSUPPORTED
+
+
+def _operand(fmt, outer, inner, k=0, P=None, F=None, inner_sum=False):
+    R = _fake_fp4(fmt, outer, inner)
+    if inner_sum:
+        R.inner_sum = 0x78000
+    op = api.OperandStruct()
+    op.R = ctypes.pointer(R)
+    op.k = k
+    op.P = ctypes.pointer(P) if P is not None else None
+    op.F = ctypes.pointer(F) if F is not None else None
+    op.S = 0x7C000 if k else None
+    op._keep = (R, P, F)
+    return op
+
+
+def _fwd(X, W, M, N, K, Y=0x80000, ydt=None, ldy=None, ws=None, wsb=None):
+    L = api.lib()
+    size = ctypes.c_size_t(0 if wsb is None else wsb)
+    st = L.metis_linear_fwd(ctypes.byref(X) if X is not None else None, ctypes.byref(W) if W is not None else None,
+                            M, N, K, Y, api.F32 if ydt is None else ydt, N if ldy is None else ldy, ws,
+                            ctypes.byref(size), _ST, None)
+    return st, size.value
+
+
+def test_linear_argument_checks_and_workspace_query():
+    nv, mx = api.NVFP4, api.MXFP4
+    M, N, K = 256, 128, 512
+    X, W = _operand(nv, M, K), _operand(nv, N, K)
+    assert _fwd(X, W, M, N, K)[0] == api.OK
+    assert _fwd(None, W, M, N, K)[0] == ERR_NULL
+    assert _fwd(X, W, M, N, K, Y=None)[0] == ERR_NULL
+    assert _fwd(X, W, 0, N, K)[0] == ERR_SHAPE
+    assert _fwd(X, W, M, N, K + 16)[0] == ERR_SHAPE                 # K not a multiple of 32
+    assert _fwd(X, W, M + 1, N, K)[0] == ERR_SHAPE                  # X is not M x K
+    assert _fwd(X, _operand(mx, N, K), M, N, K)[0] == ERR_ARG       # formats differ
+    assert _fwd(X, W, M, N, K, ydt=9)[0] == ERR_ARG
+    assert _fwd(X, W, M, N, K, ldy=N - 1)[0] == ERR_SHAPE
+    # split right operand: P (k x K) and F (k x N) quantized along K and N
+    P, F = _fake_fp4(nv, 8, K), _fake_fp4(nv, 8, N)
+    st, need = _fwd(X, _operand(nv, N, K, 8, P, F), M, N, K)
+    assert st == api.OK and need > 0
+    assert _fwd(X, _operand(nv, N, K, 8, _fake_fp4(nv, 8, N), F), M, N, K)[0] == ERR_SHAPE   # P must be k x K
+    assert _fwd(X, _operand(nv, N, K, 200, P, F), M, N, K)[0] == ERR_ARG                     # k above 128
+    assert _fwd(X, _operand(nv, N, K, 2), M, N, K)[0] == ERR_ARG        # only k = 1 may omit P and F (ones)
+    # an all-ones P (the Averis rank-1 form) needs the other operand's inner sums
+    ones = _operand(nv, N, K, 1, None, _fake_fp4(nv, 1, N))
+    assert _fwd(X, ones, M, N, K)[0] == ERR_NULL
+    assert _fwd(_operand(nv, M, K, inner_sum=True), ones, M, N, K)[0] == api.OK
+    st, need = _fwd(X, _operand(nv, N, K, 8, P, F), M, N, K)
+    assert _fwd(X, _operand(nv, N, K, 8, P, F), M, N, K, ws=ctypes.c_void_p(_WS), wsb=need - 1)[0] == ERR_WORKSPACE
+    # backward: at least one output
+    L = api.lib()
+    size = ctypes.c_size_t(0)
+    assert L.metis_linear_bwd(ctypes.byref(X), ctypes.byref(W), ctypes.byref(X), ctypes.byref(W), M, N, K,
+                              None, K, None, N, api.F32, None, ctypes.byref(size), _ST, None) == ERR_NULL
+
+
+def _averis(m=256, n=128, ld=None, fmt=api.NVFP4, mean=0x90000, mean_q=None, R_rows=None, R_cols=None, X=_A,
+            ws=None, wsb=None):
+    L = api.lib()
+    size = ctypes.c_size_t(0 if wsb is None else wsb)
+    ref = lambda t: ctypes.byref(t) if t is not None else None
+    st = L.averis_split(X, api.BF16, m, n, n if ld is None else ld, fmt, mean, ref(mean_q), ref(R_rows),
+                        ref(R_cols), None, ws, ctypes.byref(size), _ST, None)
+    return st, size.value
+
+
+def test_averis_argument_checks_and_workspace_query():
+    st, need = _averis(mean_q=_fake_fp4(api.NVFP4, 1, 128), R_rows=_fake_fp4(api.NVFP4, 256, 128),
+                       R_cols=_fake_fp4(api.NVFP4, 128, 256))
+    assert st == api.OK and need > 0
+    assert _averis(mean=None)[0] == ERR_NULL
+    assert _averis(X=None)[0] == ERR_NULL
+    assert _averis(mean=0x90004)[0] == ERR_ALIGN
+    assert _averis(fmt=5)[0] == ERR_ARG
+    assert _averis(m=0)[0] == ERR_SHAPE
+    assert _averis(mean_q=_fake_fp4(api.NVFP4, 2, 128))[0] == ERR_SHAPE      # the mean is one row
+    assert _averis(R_rows=_fake_fp4(api.MXFP4, 256, 128))[0] == ERR_ARG
+    assert _averis(R_cols=_fake_fp4(api.NVFP4, 256, 128))[0] == ERR_SHAPE    # blocks along m: outer n
+    st, need1 = _averis(mean_q=_fake_fp4(api.NVFP4, 1, 128))
+    assert st == api.OK and 0 < need1 < need
+    assert _averis(ws=ctypes.c_void_p(_WS), wsb=need1 - 1,
+                   mean_q=_fake_fp4(api.NVFP4, 1, 128))[0] == ERR_WORKSPACE
