@@ -309,7 +309,7 @@ typedef struct {
  * accumulator (T1 = (R_X P_W + F_X S_X P_X^T P_W) S_W, T2 = S_X P_X^T R_W).
  *   X  left operand (M x K), W right operand (K x N).
  *   Y  device M x N, y_dtype METIS_F32 or METIS_BF16, leading dimension ldy.
- * K must be a multiple of 32.
+ * K must be a multiple of 32, and M, N, K at most INT32_MAX (METIS_ERR_SHAPE).
  */
 METIS_API metis_status metis_linear_fwd(const metis_operand* X, const metis_operand* W, int64_t M,
                               int64_t N, int64_t K, void* Y, int32_t y_dtype, int64_t ldy,
@@ -326,7 +326,8 @@ METIS_API metis_status metis_linear_fwd(const metis_operand* X, const metis_oper
  * gradients, G4); Averis paragraphs (the output gradient is split too).
  *   dX  device M x K (or NULL to skip), dW device K x N (or NULL to skip),
  *   out_dtype METIS_F32 or METIS_BF16; ld_dx, ld_dw leading dimensions.
- * N must be a multiple of 32 for dX and M a multiple of 32 for dW.
+ * N must be a multiple of 32 for dX and M a multiple of 32 for dW; M, N and
+ * K are at most INT32_MAX (METIS_ERR_SHAPE).
  */
 METIS_API metis_status metis_linear_bwd(const metis_operand* dY_n, const metis_operand* Wt,
                               const metis_operand* Xt, const metis_operand* dY_m, int64_t M,

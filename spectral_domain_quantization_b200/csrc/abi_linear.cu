@@ -131,6 +131,8 @@ ProductBuffers carve(const ProductPlan& p, const metis_operand* A, const metis_o
 metis_status check_product(const metis_operand* A, const metis_operand* B, int64_t M, int64_t N, int64_t K) {
   if (!A || !B || !A->R || !B->R) return METIS_ERR_NULL;
   if (M <= 0 || N <= 0 || K <= 0 || K % 32) return METIS_ERR_SHAPE;
+  // the GEMM indexes rows, columns and K tiles of one product in 32 bits
+  if (M > INT32_MAX || N > INT32_MAX || K > INT32_MAX) return METIS_ERR_SHAPE;
   const int fmt = A->R->fmt;
   if (!valid_fmt(fmt)) return METIS_ERR_ARG;
   METIS_TRY(check_operand(A, M, K, fmt));

@@ -212,6 +212,8 @@ def test_linear_argument_checks_and_workspace_query():
     assert _fwd(X, W, M, N, K, Y=None)[0] == ERR_NULL
     assert _fwd(X, W, 0, N, K)[0] == ERR_SHAPE
     assert _fwd(X, W, M, N, K + 16)[0] == ERR_SHAPE                 # K not a multiple of 32
+    big = 1 << 31                                                   # rows past 32-bit indexing
+    assert _fwd(_operand(nv, big, K), W, big, N, K)[0] == ERR_SHAPE
     assert _fwd(X, W, M + 1, N, K)[0] == ERR_SHAPE                  # X is not M x K
     assert _fwd(X, _operand(mx, N, K), M, N, K)[0] == ERR_ARG       # formats differ
     assert _fwd(X, W, M, N, K, ydt=9)[0] == ERR_ARG
