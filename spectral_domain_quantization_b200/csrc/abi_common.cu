@@ -1,4 +1,5 @@
 // Host-side helpers of the C ABI and the entry points that need no kernels.
+#include <atomic>
 #include <cstdio>
 #include <mutex>
 
@@ -9,8 +10,11 @@ namespace metis {
 
 namespace {
 constexpr int kMaxDevices = 64;
-int g_sm_count[kMaxDevices] = {0};
-int g_major[kMaxDevices] = {0};
+// Per-device properties, filled on first use.  g_major is written before
+// g_sm_count is published (release), and readers check g_sm_count first
+// (acquire), so a thread that sees the count also sees the major version.
+std::atomic<int> g_sm_count[kMaxDevices];
+std::atomic<int> g_major[kMaxDevices];
 std::once_flag g_driver_once;
 // signature of cuTensorMapEncodeTiled (driver API, CUDA 12.0+)
 typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
@@ -26,12 +30,12 @@ int current_device() {
 }
 
 void fill_props(int dev) {
-  if (dev < 0 || dev >= kMaxDevices || g_sm_count[dev] != 0) return;
+  if (dev < 0 || dev >= kMaxDevices || g_sm_count[dev].load(std::memory_order_acquire) != 0) return;
   int sms = 0, major = 0;
   cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
-  g_major[dev] = major;
-  g_sm_count[dev] = sms;
+  g_major[dev].store(major, std::memory_order_relaxed);
+  g_sm_count[dev].store(sms, std::memory_order_release);
 }
 }  // namespace
 
@@ -39,14 +43,16 @@ int device_sm_count() {
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices) return 148;
   fill_props(dev);
-  return g_sm_count[dev] > 0 ? g_sm_count[dev] : 148;
+  const int sms = g_sm_count[dev].load(std::memory_order_acquire);
+  return sms > 0 ? sms : 148;
 }
 
 bool device_is_sm100() {
   const int dev = current_device();
   if (dev < 0 || dev >= kMaxDevices) return false;
   fill_props(dev);
-  return g_major[dev] == 10;
+  if (g_sm_count[dev].load(std::memory_order_acquire) == 0) return false;
+  return g_major[dev].load(std::memory_order_relaxed) == 10;
 }
 
 CUresult encode_tensor_map(CUtensorMap* map, CUtensorMapDataType dtype, int rank,
@@ -89,22 +95,27 @@ metis_status fail(metis_status st, const char* where, const char* detail) {
   return st;
 }
 
+// The dynamic shared-memory limit is a per-device attribute of a kernel:
+// the cache of limits already set is keyed by (kernel, device).
 bool ensure_smem(const void* kernel, size_t bytes) {
   static std::mutex mu;
-  static const void* keys[64];
-  static size_t vals[64];
+  static const void* keys[128];
+  static int devs[128];
+  static size_t vals[128];
   static int count = 0;
+  const int dev = current_device();
   std::lock_guard<std::mutex> lock(mu);
   int slot = -1;
   for (int i = 0; i < count; ++i)
-    if (keys[i] == kernel) slot = i;
+    if (keys[i] == kernel && devs[i] == dev) slot = i;
   if (slot >= 0 && vals[slot] >= bytes) return true;
   if (cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(bytes)) !=
       cudaSuccess)
     return false;
-  if (slot < 0 && count < 64) {
+  if (slot < 0 && count < 128) {
     slot = count++;
     keys[slot] = kernel;
+    devs[slot] = dev;
   }
   if (slot >= 0) vals[slot] = bytes;
   return true;
