@@ -26,6 +26,8 @@ of the two dequantized dense operands.
 
 import numpy as np
 
+from . import fp4
+
 
 class Operand:
     """Oracle-side operand: R (FP4Tensor), optional k, P, F (FP4Tensor or the
@@ -73,3 +75,72 @@ def gemm(opA, opB, rows=None):
     if rows is not None:
         A = A[rows]
     return A @ dense_right(opB)
+
+
+# ---------------------------------------------------------------------------
+# Re-quantized low-rank intermediates (reading R30)
+# ---------------------------------------------------------------------------
+
+def intermediates(opA, opB):
+    """The low-rank intermediates of C = A B in float64 (reading R16):
+
+        C = R_A R_B + T1 F_B^T + F_A T2,
+        T1 = (R_A P_B + F_A diag(S_A) P_A^T P_B) diag(S_B)   (M x k_B),
+        T2 = diag(S_A) P_A^T R_B                             (k_A x N).
+
+    Returns (R_A, R_B, T1, F_B, F_A, T2); the absent terms are None."""
+    RA = opA.R.dequantize()                     # M x K
+    RB = opB.R.dequantize().T                   # K x N
+    M, K = RA.shape
+    N = RB.shape[1]
+    FA = PA = FB = PB = T1 = T2 = None
+    if opA.k:
+        FA = _factor(opA.F, M, opA.k)           # M x k_A
+        PA = _factor(opA.P, K, opA.k)           # K x k_A
+        T2 = (PA * opA.S).T @ RB
+    if opB.k:
+        PB = _factor(opB.P, K, opB.k)           # K x k_B
+        FB = _factor(opB.F, N, opB.k)           # N x k_B
+        T1 = RA @ PB
+        if opA.k:
+            T1 = T1 + (FA * opA.S) @ (PA.T @ PB)
+        T1 = T1 * opB.S
+    return RA, RB, T1, FB, FA, T2
+
+
+def requantize(X32, fmt, axis):
+    """deq(Q(X)) for a float32 matrix, blocks along ``axis`` (1: along the
+    columns, 0: along the rows).  A blocked length that is not a multiple of
+    the block size is zero-padded to one; the zeros change no block maximum
+    and are dropped again (reading R30)."""
+    X32 = np.asarray(X32, dtype=np.float32)
+    bs = 32 if fmt == "mx" else 16
+    n = X32.shape[axis]
+    pad = (-n) % bs
+    if pad:
+        widths = [(0, 0), (0, 0)]
+        widths[axis] = (0, pad)
+        X32 = np.pad(X32, widths)
+    d = fp4.quantize(X32, fmt, axis).dequantize()      # outer x inner
+    if axis == 0:
+        d = d.T
+    return d[:, :n] if axis == 1 else d[:n, :]
+
+
+def gemm_requant(opA, opB, fmt, t1_32=None, t2_32=None):
+    """C = A B with the low-rank intermediates re-quantized to FP4 along the
+    axis they are contracted over (reading R30): T1 (M x k_B) in blocks along
+    k_B, T2 (k_A x N) in blocks along k_A, each with its own NVFP4 tensor
+    scale.  The values quantized are float32: by default fl32 of the exact
+    T1 / T2; ``t1_32`` / ``t2_32`` supply other float32 values (the ones a
+    device computed), so that both sides take the same FP4 decisions.  The
+    factors F_A, F_B enter as they are (already FP4)."""
+    RA, RB, T1, FB, FA, T2 = intermediates(opA, opB)
+    C = RA @ RB
+    if T1 is not None:
+        v = np.float32(T1) if t1_32 is None else np.asarray(t1_32, dtype=np.float32)
+        C = C + requantize(v, fmt, 1) @ FB.T
+    if T2 is not None:
+        v = np.float32(T2) if t2_32 is None else np.asarray(t2_32, dtype=np.float32)
+        C = C + FA @ requantize(v, fmt, 0)
+    return C
