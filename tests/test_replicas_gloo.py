@@ -40,7 +40,7 @@ def _worker(rank, world, port, out):
 
 def test_two_ranks_reduce_to_the_slowest():
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_worker, args=(2, port, out), nprocs=2, join=True)
         res = dict(out)
@@ -73,7 +73,7 @@ def _ref_worker(rank, world, port, out):
 
 def test_reference_arm_runs_on_rank_zero_only():
     port = _free_port()
-    with mp.Manager() as mgr:
+    with mp.get_context("spawn").Manager() as mgr:
         out = mgr.dict()
         mp.spawn(_ref_worker, args=(2, port, out), nprocs=2, join=True)
         assert dict(out) == {0: "skipped", 1: "returned"}
