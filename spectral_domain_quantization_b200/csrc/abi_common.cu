@@ -1,10 +1,20 @@
 // Host-side helpers of the C ABI and the entry points that need no kernels.
 #include <atomic>
+#include <cstddef>
 #include <cstdio>
 #include <mutex>
 
 #include "abi_common.h"
 #include "common.cuh"
+
+// The Python binding mirrors these structs field by field (ctypes); a layout
+// change must change both sides.
+static_assert(sizeof(metis_fp4_tensor) == 64 && offsetof(metis_fp4_tensor, outer) == 8 &&
+                  offsetof(metis_fp4_tensor, codes) == 24 && offsetof(metis_fp4_tensor, inner_sum) == 56,
+              "metis_fp4_tensor layout");
+static_assert(sizeof(metis_operand) == 40 && offsetof(metis_operand, k) == 8 && offsetof(metis_operand, P) == 16 &&
+                  offsetof(metis_operand, S) == 32,
+              "metis_operand layout");
 
 namespace metis {
 

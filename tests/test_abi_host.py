@@ -100,6 +100,16 @@ def test_selftest_wait_argument_checks():
     assert L.metis_selftest_wait_timeout(2_000_000_000, ctypes.addressof(fake), None) == ERR_ARG
 
 
+def test_fp4_tensor_and_operand_layouts_match_the_header():
+    # the library asserts the same sizes and offsets at compile time
+    T, O = api.FP4Struct, api.OperandStruct
+    assert ctypes.sizeof(T) == 64
+    assert [T.fmt.offset, T.outer.offset, T.inner.offset, T.codes.offset, T.scales.offset,
+            T.scales_linear.offset, T.tensor_scale.offset, T.inner_sum.offset] == [0, 8, 16, 24, 32, 40, 48, 56]
+    assert ctypes.sizeof(O) == 40
+    assert [O.R.offset, O.k.offset, O.P.offset, O.F.offset, O.S.offset] == [0, 8, 16, 24, 32]
+
+
 def test_split_params_layout_matches_the_header():
     # the library asserts sizeof(metis_split_params) == 56 at compile time;
     # the ctypes mirror must have the same size and field offsets
