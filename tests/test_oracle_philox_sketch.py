@@ -124,6 +124,30 @@ def test_gaussian_sketch_box_muller_pairs():
             assert abs(got - r2) <= 2 * 2 ** -7 * r2 + 1e-30
 
 
+def test_gaussian_sketch_box_muller_angle():
+    # the angle of the pair (even entry, odd entry) is 2 pi u2 with u2 from
+    # the raw word x1: the even entry is r cos(theta) and the odd r sin(theta).
+    # bf16 rounding moves each entry by at most 2**-9 of r, so the angle by at
+    # most 2**-8; swapped cos / sin, u2 from another word, theta = pi u2 or a
+    # flipped sign would all miss by far more on most pairs.
+    n, l, seed = 96, 32, 4
+    om = sketch.gaussian_omega(n, l, seed)
+    k0, k1 = philox.seed_key(seed)
+    checked = 0
+    for i in range(n):
+        for c in range(l // 2):
+            x0, x1, _, _ = philox.philox4x32_10(c, i, philox.STREAM_OMEGA, 0, k0, k1)
+            r = math.sqrt(-2 * math.log((int(x0) + 1) / 2 ** 32))
+            if r < 1e-3:
+                continue
+            theta = 2 * math.pi * (int(x1) / 2 ** 32)
+            got = math.atan2(om[i, 2 * c + 1], om[i, 2 * c])
+            diff = (got - theta + math.pi) % (2 * math.pi) - math.pi
+            assert abs(diff) <= 2 ** -8 + 1e-12, (i, c, got, theta)
+            checked += 1
+    assert checked > 0.99 * n * (l // 2)
+
+
 def test_sparse_sign_structure():
     n, l, nnz = 4096, 48, 4
     om = sketch.sparse_sign_omega(n, l, nnz, 0)
