@@ -5,13 +5,16 @@ import json
 import os
 import subprocess
 import sys
+import time
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 
 def test_reference_arm_prints_one_contract_line():
+    t0 = time.time()
     r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--steps", "1",
                         "--warmup", "0"], capture_output=True, text=True, cwd=ROOT, timeout=600)
+    wall = time.time() - t0
     assert r.returncode == 0, r.stderr[-2000:]
     lines = [ln for ln in r.stdout.splitlines() if ln.strip()]
     assert len(lines) == 1, r.stdout
@@ -23,6 +26,11 @@ def test_reference_arm_prints_one_contract_line():
     assert line["metric"] == bench.METRIC and line["config"] == bench.CONFIG
     assert line["unit"] == "TFLOPS" and line["higher_is_better"] is True
     assert line["value"] > 0 and line["ms_per_step"] > 0
+    # ms_per_step is the sampled step as it ran (it fits in the run's wall
+    # time); the metric uses the step extrapolated to all M rows
+    assert line["steps"] * line["ms_per_step"] <= wall * 1e3
+    assert line["full_step_ms_extrapolated"] >= line["ms_per_step"]
+    assert abs(line["value"] - bench.FLOPS / (line["full_step_ms_extrapolated"] * 1e-3) / 1e12) < 1e-9 * line["value"]
     assert (line["n_gpus"], line["steps"], line["warmup"]) == (1, 1, 0)
     assert line["scaling"] == "weak" and line["vs_baseline"] is None
     assert line["data"] == "synthetic" and isinstance(line["dtype"], str)

@@ -3,7 +3,8 @@
 The layer has no cross-GPU exchange, so N GPUs run N independent replicas; the
 only collectives are a barrier and a max-reduction of the per-rank timings
 (the job's time is the slowest rank's).  These tests run that plumbing with
-world size 2 on the host.
+world size 2 on the host; METIS_DIST_BACKEND=gloo keeps them on the gloo
+backend and host tensors even where a GPU is present.
 """
 import os
 import socket
@@ -23,12 +24,13 @@ def _free_port():
 
 def _worker(rank, world, port, out):
     os.environ.update({"RANK": str(rank), "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank),
-                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port), "METIS_DIST_BACKEND": "gloo"})
     sys.path.insert(0, ROOT)
     import bench
     import torch.distributed as dist
     r, w, local = bench.dist_init()
     try:
+        assert dist.get_backend() == "gloo"
         bench.barrier(w)
         # rank 1 is the slow one: the job time is its time
         t = bench.reduce_max(1.5 if r == 1 else 1.0, w)
@@ -52,7 +54,7 @@ def test_two_ranks_reduce_to_the_slowest():
 
 def _ref_worker(rank, world, port, out):
     os.environ.update({"RANK": str(rank), "WORLD_SIZE": str(world), "LOCAL_RANK": str(rank),
-                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port)})
+                       "MASTER_ADDR": "127.0.0.1", "MASTER_PORT": str(port), "METIS_DIST_BACKEND": "gloo"})
     sys.path.insert(0, ROOT)
     import bench
     import torch.distributed as dist
