@@ -268,6 +268,11 @@ typedef struct {
  *   sample_idx  optional device int32[sample_rows]: the sampled rows.
  *   dev_status  device int32 (required).
  * Quantized outputs need m and n multiples of 32 along their blocked axis.
+ * Sketch tap: after the call, in stream order, the first lp * round_up(n, 8)
+ * bf16 values of the workspace hold Omega^T (lp = round_up(k + p, 16) rows of
+ * round_up(n, 8) entries, row j = column j of Omega; rows past k + p and
+ * entries past n are zero).  It is read-only output for tests; the rest of
+ * the workspace is scratch.
  */
 METIS_API metis_status metis_split(const void* A, int32_t dtype, int64_t m, int64_t n, int64_t lda,
                          const metis_split_params* prm, float* U, float* S, float* V,

@@ -156,11 +156,17 @@ class _Workspace:
 _ws = _Workspace()
 
 
-def _call_with_workspace(fn, args_before_ws, args_after_ws, device, what):
-    """Query the workspace size, provide it, then run the call."""
+def _call_with_workspace(fn, args_before_ws, args_after_ws, device, what, workspace=None):
+    """Query the workspace size, provide it (the caller's uint8 tensor when
+    given, else the shared per-stream one), then run the call."""
     size = ctypes.c_size_t(0)
     _check(fn(*args_before_ws, None, ctypes.byref(size), *args_after_ws), what + " (workspace query)")
-    ws = _ws.get(size.value, device)
+    if workspace is not None:
+        if workspace.dtype != torch.uint8 or workspace.numel() < size.value:
+            raise ValueError(f"{what}: the workspace needs {size.value} bytes (uint8)")
+        ws = workspace
+    else:
+        ws = _ws.get(size.value, device)
     size2 = ctypes.c_size_t(ws.numel())
     _check(fn(*args_before_ws, _ptr(ws), ctypes.byref(size2), *args_after_ws), what)
 
@@ -327,9 +333,10 @@ class Split:
 
 
 def split(A, k, p, q=1, seed=0, fmt="nv", sketch="gaussian", nnz=4, sample_rows=0, max_iters=64,
-          rows=True, cols=True, factors=True, tap=False, compensate=False, dev_status=None):
+          rows=True, cols=True, factors=True, tap=False, compensate=False, dev_status=None, workspace=None):
     """Spectral split A = U diag(S) V^T + R with FP4 outputs (metis_split).
-    compensate: R = A - deq(U_q) diag(S) deq(V_q)^T (needs factors=True)."""
+    compensate: R = A - deq(U_q) diag(S) deq(V_q)^T (needs factors=True).
+    workspace: optional caller-owned uint8 CUDA tensor (see sketch_tap)."""
     if A.dim() != 2 or A.stride(1) != 1:
         raise ValueError("A must be a row-major 2-D tensor")
     m, n = A.shape
@@ -354,9 +361,20 @@ def split(A, k, p, q=1, seed=0, fmt="nv", sketch="gaussian", nnz=4, sample_rows=
         lib().metis_split,
         (_ptr(A), _dtype_code(A), m, n, A.stride(0), ctypes.byref(prm), _ptr(U), _ptr(S), _ptr(V), *refs,
          _ptr(R_f32), _ptr(idx)),
-        (_ptr(dev_status), _stream()), dev, "metis_split")
+        (_ptr(dev_status), _stream()), dev, "metis_split", workspace=workspace)
     return Split(U=U, S=S, V=V, U_q=U_q, V_q=V_q, R_rows=R_rows, R_cols=R_cols, R_f32=R_f32, idx=idx,
                  dev_status=dev_status, k=k, fmt=f)
+
+
+def sketch_tap(workspace, n, k, p):
+    """The sketch Omega (n x l, float32 from bf16) that the last metis_split
+    on `workspace` used: the first round_up(l, 16) x round_up(n, 8) bf16
+    values of the workspace hold Omega^T (the tap metis.h documents)."""
+    l = k + p
+    lp = (l + 15) // 16 * 16
+    ldn = (n + 7) // 8 * 8
+    omt = workspace[: lp * ldn * 2].view(torch.bfloat16).view(lp, ldn)
+    return omt, omt[:l, :n].float().t()
 
 
 # --------------------------------------------------------------------------
