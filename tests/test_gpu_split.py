@@ -34,12 +34,15 @@ def _check(A64, res, ref, fmt, check_vectors=True, r_tol=TOL, tap_scale=None):
     den = np.linalg.norm(R) if tap_scale is None else tap_scale
     assert np.linalg.norm(R.astype(np.float64) - (A64 - L)) / den < 1e-5
     if check_vectors:
+        # a singular vector is unique (up to the sign both sides fix the same
+        # way) only where its value is separated from its neighbours; there
+        # the columns are held to the factor tolerance
         s = ref["S"]
         gap = np.minimum(np.abs(np.diff(np.r_[np.inf, s])), np.abs(np.diff(np.r_[s, -np.inf])))
         sep = gap / s > 0.05
         for j in np.flatnonzero(sep):
-            assert rel_fro(U[:, j], ref["U"][:, j]) < 1e-2, j
-            assert rel_fro(V[:, j], ref["V"][:, j]) < 1e-2, j
+            assert rel_fro(U[:, j], ref["U"][:, j]) < TOL, j
+            assert rel_fro(V[:, j], ref["V"][:, j]) < TOL, j
     # FP4 outputs: bit-exact on the GPU's own float32 values
     k = U.shape[1]
     assert_fp4_equal(res.U_q, fp4.quantize(res.U.cpu().numpy(), fmt, 0), check_linear=False)
@@ -114,7 +117,7 @@ def test_split_full_size_layer_weight():
     torch.cuda.synchronize()
     A64 = d["W"].f64()
     ref = split.split(A64, c["k"], c["p"], c["q"], c["sketch_seed"])
-    _check(A64, res, ref, "nv", check_vectors=False)
+    _check(A64, res, ref, "nv")
 
 
 @pytest.mark.parametrize("k,p", [(96, 16), (92, 3)])
