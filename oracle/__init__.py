@@ -45,4 +45,4 @@ against closed forms, brute force, published test vectors or independent
 formulations.
 """
 
-from . import philox, sketch, fp4, split, gemm, averis, composite, mlp  # noqa: F401
+from . import philox, sketch, fp4, split, gemm, averis, composite, mlp, spectral_lr  # noqa: F401
