@@ -188,7 +188,9 @@ METIS_API metis_status metis_quantize_fp4(const void* X, int32_t dtype, int64_t 
  * metis_last_error()); use metis_quantize_fp4 for them.
  *   - The first call on a device looks up the array's device address (this may
  *     load the library's device code); make that first call before any CUDA
- *     stream capture.
+ *     stream capture.  The address is kept per device and context: after the
+ *     context is destroyed and re-created (cudaDeviceReset), the next call
+ *     looks it up again, so make that call before any capture too.
  *   - All calls share the one array: calls whose GPU work overlaps (different
  *     streams, concurrent host threads) race and must be ordered by the caller.
  *     The call zeroes what must start at zero itself.
@@ -303,7 +305,14 @@ typedef struct {
   const metis_fp4_tensor* P;
   const metis_fp4_tensor* F;
   const float* S;
+  /* bit 0 (METIS_REQUANT_LOWRANK): re-quantize to FP4 the low-rank
+   * intermediate formed from this operand's factors (T1 for a right operand,
+   * T2 for a left operand), in blocks along its k, before it enters the
+   * product.  0 keeps it in float32 (bf16 hi/lo).  Other bits: 0. */
+  int32_t flags;
 } metis_operand;
+
+#define METIS_REQUANT_LOWRANK 1
 
 /*
  * metis_linear_fwd -- Y = X W on FP4 operands (W4A4 forward).

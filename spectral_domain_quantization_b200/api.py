@@ -55,7 +55,10 @@ class SplitParams(ctypes.Structure):
 class OperandStruct(ctypes.Structure):
     _fields_ = [("R", ctypes.POINTER(FP4Struct)), ("k", ctypes.c_int32),
                 ("P", ctypes.POINTER(FP4Struct)), ("F", ctypes.POINTER(FP4Struct)),
-                ("S", ctypes.c_void_p)]
+                ("S", ctypes.c_void_p), ("flags", ctypes.c_int32)]
+
+
+REQUANT_LOWRANK = 1
 
 
 _lib = None
@@ -248,10 +251,13 @@ class Operand:
     right operand B (K x N) = R + P diag(S) F^T
     R: QTensor quantized along K; P: QTensor (outer k, inner K) or None for
     the all-ones vector; F: QTensor (outer k, inner M or N) or None for ones;
-    S: CUDA float tensor of k values or None (ones)."""
+    S: CUDA float tensor of k values or None (ones).
+    requant: re-quantize the low-rank intermediate formed from this
+    operand's factors to FP4 along its k (METIS_REQUANT_LOWRANK)."""
 
-    def __init__(self, R, k=0, P=None, F=None, S=None):
+    def __init__(self, R, k=0, P=None, F=None, S=None, requant=False):
         self.R, self.k, self.P, self.F, self.S = R, int(k), P, F, S
+        self.requant = bool(requant)
 
     def struct(self):
         o = OperandStruct()
@@ -263,6 +269,7 @@ class Operand:
         o.P = ctypes.pointer(self._p) if self._p is not None else None
         o.F = ctypes.pointer(self._f) if self._f is not None else None
         o.S = self.S.data_ptr() if self.S is not None else None
+        o.flags = REQUANT_LOWRANK if self.requant else 0
         self._o = o
         return o
 

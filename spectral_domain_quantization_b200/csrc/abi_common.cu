@@ -12,8 +12,8 @@
 static_assert(sizeof(metis_fp4_tensor) == 64 && offsetof(metis_fp4_tensor, outer) == 8 &&
                   offsetof(metis_fp4_tensor, codes) == 24 && offsetof(metis_fp4_tensor, inner_sum) == 56,
               "metis_fp4_tensor layout");
-static_assert(sizeof(metis_operand) == 40 && offsetof(metis_operand, k) == 8 && offsetof(metis_operand, P) == 16 &&
-                  offsetof(metis_operand, S) == 32,
+static_assert(sizeof(metis_operand) == 48 && offsetof(metis_operand, k) == 8 && offsetof(metis_operand, P) == 16 &&
+                  offsetof(metis_operand, S) == 32 && offsetof(metis_operand, flags) == 40,
               "metis_operand layout");
 
 namespace metis {

@@ -27,6 +27,7 @@ metis_status check_operand(const metis_operand* op, int64_t free_dim, int64_t K,
   if (!op || !op->R) return METIS_ERR_NULL;
   METIS_TRY(check_fp4(op->R, free_dim, K, fmt));
   if (op->k < 0 || op->k > 128) return METIS_ERR_ARG;
+  if (op->flags & ~METIS_REQUANT_LOWRANK) return METIS_ERR_ARG;
   if (op->k == 0) return METIS_OK;
   if (op->P) {
     METIS_TRY(check_fp4(op->P, op->k, K, fmt));
@@ -108,6 +109,8 @@ ProductPlan plan(const metis_operand* A, const metis_operand* B, int64_t M, int6
 struct ProductBuffers {
   __nv_bfloat16 *la = nullptr, *lb = nullptr;
   float *t1 = nullptr, *t1p = nullptr, *t2 = nullptr, *t2p = nullptr, *cab = nullptr;
+  float* t1full = nullptr;      // re-quantized T1: its float32 values
+  unsigned* amax = nullptr;     // [2]: max |T1|, max |T2| (NVFP4)
 };
 
 ProductBuffers carve(const ProductPlan& p, const metis_operand* A, const metis_operand* B, int64_t M,
@@ -125,6 +128,9 @@ ProductBuffers carve(const ProductPlan& p, const metis_operand* A, const metis_o
     if (p.s2 > 1) b.t2p = ws.take<float>(static_cast<size_t>(p.s2) * p.ka * N);
   }
   if (p.ka && p.kb) b.cab = ws.take<float>(static_cast<size_t>(p.ka) * p.kb);
+  if (p.kb && (B->flags & METIS_REQUANT_LOWRANK)) b.t1full = ws.take<float>(static_cast<size_t>(M) * p.kb);
+  if ((p.kb && (B->flags & METIS_REQUANT_LOWRANK)) || (p.ka && (A->flags & METIS_REQUANT_LOWRANK)))
+    b.amax = ws.take<unsigned>(2);
   return b;
 }
 
@@ -164,6 +170,12 @@ metis_status enqueue_product(const metis_operand* A, const metis_operand* B, int
     la.ts_rb = B->R->fmt == METIS_NVFP4 ? B->R->tensor_scale : nullptr;
     la.la = b.la;
     la.lb = b.lb;
+    la.fmt = A->R->fmt;
+    la.requant_t1 = p.kb && (B->flags & METIS_REQUANT_LOWRANK);
+    la.requant_t2 = p.ka && (A->flags & METIS_REQUANT_LOWRANK);
+    la.t1full = b.t1full;
+    la.amax1 = b.amax;
+    la.amax2 = b.amax ? b.amax + 1 : nullptr;
     if (p.kb) {
       if (B->P) {
         GemmCall g = base_call(A->R, B->P, M, p.kb, K, dev_status);

@@ -12,6 +12,8 @@
 //
 // The arithmetic is exactly that of metis_quantize_fp4 (the same kernels are
 // enqueued); only where the scratch lives differs.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "abi_common.h"
@@ -26,24 +28,63 @@ __device__ __align__(256) unsigned char g_fixed_scratch[kFixedScratchBytes];
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-void* g_scratch_addr[kMaxDevices] = {};
+
+// The address is cached per device together with the unique ID of the CUDA
+// context it was looked up in: after a context is destroyed and re-created
+// (cudaDeviceReset), the library's device code may load at another address,
+// so a new context ID means a new lookup.
+struct CachedAddr {
+  unsigned long long ctx_id;
+  void* addr;
+};
+CachedAddr g_scratch_addr[kMaxDevices] = {};
+
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+using CtxGetIdFn = CUresult (*)(CUcontext, unsigned long long*);
+std::once_flag g_ctx_fns_once;
+CtxGetCurrentFn g_ctx_get_current = nullptr;
+CtxGetIdFn g_ctx_get_id = nullptr;
+
+// Unique ID of the current context (0 if it cannot be read).
+unsigned long long current_ctx_id() {
+  std::call_once(g_ctx_fns_once, [] {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get_current = reinterpret_cast<CtxGetCurrentFn>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      g_ctx_get_id = reinterpret_cast<CtxGetIdFn>(fn);
+  });
+  CUcontext ctx = nullptr;
+  unsigned long long id = 0;
+  if (g_ctx_get_current && g_ctx_get_id && g_ctx_get_current(&ctx) == CUDA_SUCCESS && ctx &&
+      g_ctx_get_id(ctx, &id) == CUDA_SUCCESS)
+    return id;
+  return 0;
+}
 
 // Device address of the fixed scratch on the current device.  The array's
-// name is only a host-side stand-in for it, so the address is looked up once
-// per device (with that device current) and kept.
+// name is only a host-side stand-in for it, so the address is looked up with
+// that device current and kept for as long as its context lives.
 metis_status fixed_scratch(void** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices)
     return metis::fail(METIS_ERR_CUDA, "metis_quantize_fp4_noalloc", "no current CUDA device");
+  const unsigned long long id = current_ctx_id();
   std::lock_guard<std::mutex> lock(g_mu);
-  if (!g_scratch_addr[dev]) {
+  CachedAddr& c = g_scratch_addr[dev];
+  if (!c.addr || id == 0 || c.ctx_id != id) {
     void* p = nullptr;
     const cudaError_t e = cudaGetSymbolAddress(&p, g_fixed_scratch);
     if (e != cudaSuccess || !p)
       return metis::fail(METIS_ERR_CUDA, "metis_quantize_fp4_noalloc: cudaGetSymbolAddress", cudaGetErrorString(e));
-    g_scratch_addr[dev] = p;
+    c.addr = p;
+    c.ctx_id = current_ctx_id();   // the lookup created the context if there was none
   }
-  *out = g_scratch_addr[dev];
+  *out = c.addr;
   return METIS_OK;
 }
 

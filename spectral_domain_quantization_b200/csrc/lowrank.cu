@@ -16,6 +16,7 @@
 //   LA[m] = [hi(T1') | lo(T1') | F~_A | F~_A | 0...]
 //   LB[n] = [F~_B    | F~_B    | hi(T2') | lo(T2') | 0...]
 #include "common.cuh"
+#include "fp4_block.cuh"
 #include "lowrank.h"
 
 namespace metis {
@@ -80,15 +81,117 @@ MDEV float t1_value(const LowRankArgs& a, int64_t m, int j) {
   return a.t1raw ? a.t1raw[m * a.t1_ld + j] : 0.f;
 }
 
+// One FP4 block (16 values NVFP4 / 32 MXFP4) of v, in place: v becomes
+// code x block scale (exact in bf16), the tensor scale left out.
+MDEV void requant_block(float* v, int fmt, float s_t) {
+  float dsum;
+  if (fmt == METIS_NVFP4) {
+    float x[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) x[i] = v[i];
+    uint64_t packed;
+    const float d = e4m3_value(quant_block_nv(x, s_t, packed, dsum));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = e2m1_value(static_cast<uint32_t>(packed >> (4 * i)) & 15u) * d;
+  } else {
+    float x[32];
+#pragma unroll
+    for (int i = 0; i < 32; ++i) x[i] = v[i];
+    uint64_t packed[2];
+    const float d = ldexpf(1.f, static_cast<int>(quant_block_mx(x, packed, dsum)) - 127);
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = e2m1_value(static_cast<uint32_t>(packed[i >> 4] >> (4 * (i & 15))) & 15u) * d;
+  }
+}
+
+MDEV float requant_tensor_scale(const LowRankArgs& a, const unsigned* amax) {
+  return a.fmt == METIS_NVFP4 ? nv_tensor_scale(__uint_as_float(*amax)) : 1.f;
+}
+
+MDEV void amax_update(unsigned* amax, float v) {
+  unsigned u = __float_as_uint(fabsf(v));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) u = max(u, __shfl_xor_sync(0xffffffffu, u, o));
+  if ((threadIdx.x & 31) == 0 && u) atomicMax(amax, u);
+}
+
+// T1 = (R_A P_B + F_A S_A (P_A^T P_B)) S_B in float32, element per thread,
+// and (NVFP4) its absolute maximum.
+__global__ void t1_form_kernel(LowRankArgs a) {
+  const float s_fa = tscale(a.fa);
+  const int64_t total = a.M * a.kb;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t end = (total + step - 1) / step * step;   // whole warps take part in the reduction
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < end; t += step) {
+    float v = 0.f;
+    if (t < total) {
+      const int64_t m = t / a.kb;
+      const int j = static_cast<int>(t - m * a.kb);
+      v = t1_value(a, m, j);
+      if (a.ka > 0 && a.cab) {
+        float acc = 0.f;
+        for (int i = 0; i < a.ka; ++i) {
+          const float sa = a.s_a ? a.s_a[i] : 1.f;
+          acc += factor_value(a.fa, i, m) * s_fa * sa * a.cab[i * a.kb + j];
+        }
+        v += acc;
+      }
+      v = v * (a.s_b ? a.s_b[j] : 1.f);
+      a.t1full[t] = v;
+    }
+    if (a.fmt == METIS_NVFP4) amax_update(a.amax1, v);
+  }
+}
+
+// max |T2| with T2 = S_A (P_A^T R_B) (NVFP4).
+__global__ void t2_amax_kernel(LowRankArgs a) {
+  const int64_t total = static_cast<int64_t>(a.ka) * a.N;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  const int64_t end = (total + step - 1) / step * step;
+  for (int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; t < end; t += step) {
+    float v = 0.f;
+    if (t < total) {
+      const int i = static_cast<int>(t / a.N);
+      const int64_t n = t - static_cast<int64_t>(i) * a.N;
+      v = a.t2raw[i * a.t2_ld + n] * (a.s_a ? a.s_a[i] : 1.f);
+    }
+    amax_update(a.amax2, v);
+  }
+}
+
+constexpr int kMaxLowRank = 128;   // k of one operand (checked by the ABI)
+
 // LA: a row per block iteration, a column per thread.
 __global__ void build_la_kernel(LowRankArgs a) {
+  __shared__ float row[kMaxLowRank];
   const float inv_alpha = 1.f / alpha_main(a);
   const float s_fb = tscale(a.fb);
   const float s_fa = tscale(a.fa);
+  const float s_t1 = a.requant_t1 ? requant_tensor_scale(a, a.amax1) : 1.f;
+  const float s_t2 = a.requant_t2 ? requant_tensor_scale(a, a.amax2) : 1.f;
+  const int bs = a.fmt == METIS_MXFP4 ? 32 : 16;
+  const int kbp = (a.kb + bs - 1) / bs * bs;
   for (int64_t m = blockIdx.x; m < a.M; m += gridDim.x) {
+    if (a.requant_t1) {
+      // T1's row in blocks along kb (zero-padded), quantized and dequantized
+      for (int j = threadIdx.x; j < kbp; j += blockDim.x) row[j] = j < a.kb ? a.t1full[m * a.kb + j] : 0.f;
+      __syncthreads();
+      for (int b = threadIdx.x; b < kbp / bs; b += blockDim.x) requant_block(row + b * bs, a.fmt, s_t1);
+      __syncthreads();
+    }
     for (int c = threadIdx.x; c < a.lr_k; c += blockDim.x) {
       __nv_bfloat16 out = __float2bfloat16_rn(0.f);
-      if (c < 2 * a.kb) {
+      if (c < 2 * a.kb && a.requant_t1) {
+        // code x block scale in both chunks; the F_B side carries s_t1
+        out = __float2bfloat16_rn(row[c < a.kb ? c : c - a.kb]);
+      } else if (c < 2 * a.kb + 2 * a.ka && c >= 2 * a.kb && a.requant_t2) {
+        const int cc = c - 2 * a.kb;
+        const int i = cc % a.ka;
+        const float w = factor_value(a.fa, i, m) * s_fa * s_t2 * inv_alpha;
+        __nv_bfloat16 hi, lo;
+        split_hi_lo(w, hi, lo);
+        out = cc < a.ka ? hi : lo;
+      } else if (c < 2 * a.kb) {
         const int j = c < a.kb ? c : c - a.kb;
         float v = t1_value(a, m, j);
         if (a.ka > 0 && a.cab) {
@@ -110,18 +213,43 @@ __global__ void build_la_kernel(LowRankArgs a) {
       }
       a.la[m * a.lr_k + c] = out;
     }
+    if (a.requant_t1) __syncthreads();   // the row buffer is refilled next
   }
 }
 
 // LB: a row per block iteration, a column per thread.
 __global__ void build_lb_kernel(LowRankArgs a) {
+  __shared__ float col[kMaxLowRank];
   const float inv_alpha = 1.f / alpha_main(a);
   const float s_fa = tscale(a.fa);
+  const float s_fb = tscale(a.fb);
+  const float s_t1 = a.requant_t1 ? requant_tensor_scale(a, a.amax1) : 1.f;
+  const float s_t2 = a.requant_t2 ? requant_tensor_scale(a, a.amax2) : 1.f;
+  const int bs = a.fmt == METIS_MXFP4 ? 32 : 16;
+  const int kap = (a.ka + bs - 1) / bs * bs;
   for (int64_t n = blockIdx.x; n < a.N; n += gridDim.x) {
+    if (a.requant_t2) {
+      // column n of T2 = S_A P_A^T R_B in blocks along ka (zero-padded)
+      for (int i = threadIdx.x; i < kap; i += blockDim.x)
+        col[i] = i < a.ka ? a.t2raw[i * a.t2_ld + n] * (a.s_a ? a.s_a[i] : 1.f) : 0.f;
+      __syncthreads();
+      for (int b = threadIdx.x; b < kap / bs; b += blockDim.x) requant_block(col + b * bs, a.fmt, s_t2);
+      __syncthreads();
+    }
     for (int c = threadIdx.x; c < a.lr_k; c += blockDim.x) {
       __nv_bfloat16 out = __float2bfloat16_rn(0.f);
-      if (c < 2 * a.kb) {
+      if (c < 2 * a.kb && a.requant_t1) {
+        // F_B with its tensor scale and T1's, over the main alpha, as hi / lo
+        const float w = factor_value(a.fb, c < a.kb ? c : c - a.kb, n) * s_fb * s_t1 * inv_alpha;
+        __nv_bfloat16 hi, lo;
+        split_hi_lo(w, hi, lo);
+        out = c < a.kb ? hi : lo;
+      } else if (c < 2 * a.kb) {
         out = __float2bfloat16_rn(factor_value(a.fb, c < a.kb ? c : c - a.kb, n));
+      } else if (c < 2 * a.kb + 2 * a.ka && a.requant_t2) {
+        // code x block scale of T2 in both chunks; the F_A side carries s_t2
+        const int cc = c - 2 * a.kb;
+        out = __float2bfloat16_rn(col[cc % a.ka]);
       } else if (c < 2 * a.kb + 2 * a.ka) {
         const int cc = c - 2 * a.kb;
         const int i = cc % a.ka;
@@ -133,6 +261,7 @@ __global__ void build_lb_kernel(LowRankArgs a) {
       }
       a.lb[n * a.lr_k + c] = out;
     }
+    if (a.requant_t2) __syncthreads();   // the column buffer is refilled next
   }
 }
 
@@ -182,6 +311,15 @@ int row_blocks(int64_t rows, int sms) {
 
 void launch_build_lowrank(const LowRankArgs& a, int sms, cudaStream_t s) {
   const int threads = a.lr_k >= 128 ? 128 : 64;
+  if (a.requant_t1 || a.requant_t2) {
+    if (a.fmt == METIS_NVFP4) {
+      if (a.requant_t1) cudaMemsetAsync(a.amax1, 0, sizeof(unsigned), s);
+      if (a.requant_t2) cudaMemsetAsync(a.amax2, 0, sizeof(unsigned), s);
+    }
+    if (a.requant_t1) t1_form_kernel<<<blocks_for(a.M * a.kb, sms), 256, 0, s>>>(a);
+    if (a.requant_t2 && a.fmt == METIS_NVFP4)
+      t2_amax_kernel<<<blocks_for(static_cast<int64_t>(a.ka) * a.N, sms), 256, 0, s>>>(a);
+  }
   build_la_kernel<<<row_blocks(a.M, sms), threads, 0, s>>>(a);
   build_lb_kernel<<<row_blocks(a.N, sms), threads, 0, s>>>(a);
 }

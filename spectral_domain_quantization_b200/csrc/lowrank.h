@@ -42,6 +42,13 @@ struct LowRankArgs {
   const float* ts_rb;
   __nv_bfloat16* la;        // out: M x lr_k
   __nv_bfloat16* lb;        // out: N x lr_k
+  // FP4 re-quantized intermediates: T1 (M x kb) in blocks along kb, T2
+  // (ka x N) in blocks along ka, each with its own NVFP4 tensor scale
+  int requant_t1, requant_t2;
+  int fmt;                  // format of the re-quantization (the product's)
+  float* t1full;            // M x kb: T1 with every term and S_B (requant_t1)
+  unsigned* amax1;          // max |T1| bits (NVFP4), zeroed before the build
+  unsigned* amax2;          // max |T2| bits (NVFP4)
 };
 
 void launch_cab(const FactorView& pa, const FactorView& pb, int64_t K, int ka, int kb, float* cab,

@@ -106,8 +106,11 @@ def test_fp4_tensor_and_operand_layouts_match_the_header():
     assert ctypes.sizeof(T) == 64
     assert [T.fmt.offset, T.outer.offset, T.inner.offset, T.codes.offset, T.scales.offset,
             T.scales_linear.offset, T.tensor_scale.offset, T.inner_sum.offset] == [0, 8, 16, 24, 32, 40, 48, 56]
-    assert ctypes.sizeof(O) == 40
-    assert [O.R.offset, O.k.offset, O.P.offset, O.F.offset, O.S.offset] == [0, 8, 16, 24, 32]
+    assert ctypes.sizeof(O) == 48
+    assert [O.R.offset, O.k.offset, O.P.offset, O.F.offset, O.S.offset, O.flags.offset] == [0, 8, 16, 24, 32, 40]
+    # the flag bit the header defines
+    hdr = open(api.HEADER).read()
+    assert "#define METIS_REQUANT_LOWRANK 1" in hdr and api.REQUANT_LOWRANK == 1
 
 
 def test_split_params_layout_matches_the_header():
@@ -235,6 +238,9 @@ def test_linear_argument_checks_and_workspace_query():
     assert _fwd(X, _operand(nv, N, K, 8, _fake_fp4(nv, 8, N), F), M, N, K)[0] == ERR_SHAPE   # P must be k x K
     assert _fwd(X, _operand(nv, N, K, 200, P, F), M, N, K)[0] == ERR_ARG                     # k above 128
     assert _fwd(X, _operand(nv, N, K, 2), M, N, K)[0] == ERR_ARG        # only k = 1 may omit P and F (ones)
+    bad = _operand(nv, N, K, 8, P, F)
+    bad.flags = 2                                                       # an undefined flag bit
+    assert _fwd(X, bad, M, N, K)[0] == ERR_ARG
     # an all-ones P (the Averis rank-1 form) needs the other operand's inner sums
     ones = _operand(nv, N, K, 1, None, _fake_fp4(nv, 1, N))
     assert _fwd(X, ones, M, N, K)[0] == ERR_NULL
@@ -274,3 +280,4 @@ def test_averis_argument_checks_and_workspace_query():
     assert st == api.OK and 0 < need1 < need
     assert _averis(ws=ctypes.c_void_p(_WS), wsb=need1 - 1,
                    mean_q=_fake_fp4(api.NVFP4, 1, 128))[0] == ERR_WORKSPACE
+

@@ -4,16 +4,20 @@ Some callers cannot hand the library scratch memory (they may not allocate
 where they quantize, or hold no spare device buffer), so this entry point keeps
 its scratch in a fixed array inside the library.  This file checks, through the
 C ABI, that it gives exactly what metis_quantize_fp4 gives, on two calls in a
-row (the second call must not see leftovers of the first), and that a request
-larger than the fixed array is refused.  The file is named so that pytest
-collects it last."""
+row (the second call must not see leftovers of the first), that its bytes are
+the oracle quantizer's on the same float32 values, and that a request larger
+than the fixed array is refused.  The file is named so that pytest collects it
+last."""
 import ctypes
 
 import numpy as np
 import pytest
 import torch
 
+from oracle import fp4
 from spectral_domain_quantization_b200 import api
+
+from gpu_helpers import assert_fp4_equal
 
 pytestmark = pytest.mark.gpu
 
@@ -37,6 +41,8 @@ def test_noalloc_matches_workspace_entry_point_twice():
         got = api.quantize_fp4_noalloc(X, fmt, axis, inner_sum=True)
         torch.cuda.synchronize()
         _same(got, ref)
+        # and directly against the oracle on the bf16 values both sides saw
+        assert_fp4_equal(got, fp4.quantize(X.float().cpu().numpy(), fmt, axis), check_linear=False)
     # a second call on the same inputs as the first (scratch reused)
     x = (rng.standard_normal((1056, 304)) * 3).astype(np.float32)
     X = torch.from_numpy(x).cuda()
