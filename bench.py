@@ -61,6 +61,9 @@ def parse():
                     help="measure the mean + spectral composite split of the Averis-shaped activation instead")
     ap.add_argument("--profile-steps", type=int, default=0,
                     help="run this many eager steps (no graphs, no timing) and exit: the command profiled by ncu")
+    ap.add_argument("--workload", default="layer_4096",
+                    choices=["layer_4096", "averis_32768", "llama3_8b_mlp", "sampled_65536"],
+                    help="the timed step: the single layer (default) or another synthetic workload")
     return ap.parse_args()
 
 
@@ -505,6 +508,398 @@ def run_ours(args, rank, world, local):
     del g_step, g_split, g_quant, g_gemm, g_plain
 
 
+# --------------------------------------------------------------------------
+# the other synthetic workloads (--workload): one step each, the same timing
+# rules; the split / quantize phase is also reported against the HBM peak
+# with its algorithmic bytes (each input byte read and each output byte
+# written once per pass the method needs)
+# --------------------------------------------------------------------------
+
+def _fp4_bytes(rows, cols, fmt):
+    """codes + scale bytes of one FP4 copy of a rows x cols matrix."""
+    return rows * cols // 2 + rows * cols // (32 if fmt == "mx" else 16)
+
+
+class AverisWorkload:
+    """averis_32768: X bf16 32768 x 4096 = 1 mu^T + Z (0.1 % outliers), W bf16
+    4096 x 4096, dY bf16 32768 x 4096.  Step: the Averis split of X and of dY
+    (NVFP4, both block axes), W quantized along K and along N, then Y = X W,
+    dX = dY W^T and dW = X^T dY (bf16 outputs)."""
+
+    name = "averis_32768"
+
+    def __init__(self, dev):
+        import torch
+        from spectral_domain_quantization_b200 import api, inputs
+        self.api = api
+        d = inputs.make("averis_32768")
+        c = d["cfg"]
+        self.M, self.K, self.N = c["M"], c["K"], c["N"]
+        self.host = {k: _pinned_bf16(d[k]) for k in ("X", "W", "dY")}
+        self.dev = {k: v.to(dev) for k, v in self.host.items()}
+        self.Y = torch.empty((self.M, self.N), dtype=torch.bfloat16, device=dev)
+        self.dX = torch.empty((self.M, self.K), dtype=torch.bfloat16, device=dev)
+        self.dW = torch.empty((self.K, self.N), dtype=torch.bfloat16, device=dev)
+        self.data = d
+        M, K, N = self.M, self.K, self.N
+        self.flops = 3 * 2.0 * M * N * K
+        # X and dY: two reads (the column sums, then the residual pass) and
+        # two FP4 copies each; W: amax and quantize reads per axis, two copies
+        self.split_bytes = (2 * (2 * M * K * 2 + 2 * _fp4_bytes(M, K, "nv"))
+                            + 2 * (2 * K * N * 2 + _fp4_bytes(K, N, "nv")))
+        self.config = {"workload": "averis_32768: X bf16 32768x4096 = 1 mu^T + Z, dY bf16 32768x4096, W bf16 "
+                                   "4096x4096; Averis split of X and dY, W plain, NVFP4; forward, dX, dW",
+                       "M": M, "K": K, "N": N, "fmt": "nvfp4"}
+        self.ops = None
+
+    def split(self):
+        api, d = self.api, self.dev
+        self.ops = (api.averis_split(d["X"], "nv"), api.averis_split(d["dY"], "nv"),
+                    api.quantize_fp4(d["W"], "nv", 0), api.quantize_fp4(d["W"], "nv", 1))
+
+    def products(self):
+        api = self.api
+        ax, ady, qw_k, qw_n = self.ops
+        api.linear_fwd(ax.left(), api.Operand(qw_k), self.M, self.N, self.K, Y=self.Y)
+        api.linear_bwd(ady.left(), api.Operand(qw_n), ax.left_t(), ady.right_m(), self.M, self.N, self.K,
+                       out_dtype=self.Y.dtype, dX=self.dX, dW=self.dW)
+
+    def plain(self):
+        """the largest product with plain operands: one launch of the FP4 GEMM kernel"""
+        api = self.api
+        ax, _, qw_k, _ = self.ops
+        api.linear_fwd(api.Operand(ax.R_rows), api.Operand(qw_k), self.M, self.N, self.K, Y=self.Y)
+        return 2.0 * self.M * self.N * self.K, f"gemm_fp4 ({self.M}x{self.N}x{self.K} NVFP4)"
+
+    def outputs(self):
+        return [self.Y, self.dX, self.dW]
+
+    def oracle_sample(self, rows=256):
+        from oracle import averis, fp4, gemm
+        d = self.data
+        t0 = time.perf_counter()
+        out = []
+        for key in ("X", "dY"):
+            x = d[key].f64()
+            mu, _ = averis.split(x)               # the column mean needs every row
+            out.append((x, mu))
+        W = d["W"].f32()
+        qk, qn = fp4.quantize(W, "nv", 0), fp4.quantize(W, "nv", 1)
+        wk, wn = gemm.dense_right(gemm.Operand(qk)), gemm.dense_right(gemm.Operand(qn)).T
+        t_fixed = time.perf_counter() - t0
+        t1 = time.perf_counter()
+        (x, mu), (dy, nu) = out
+        rx = np.float32(x[:rows] - mu)
+        rdy = np.float32(dy[:rows] - nu)
+        xq = fp4.quantize(rx, "nv", 1)
+        dyq = fp4.quantize(rdy, "nv", 1)
+        (xq.dequantize() + mu[None, :]) @ wk
+        (dyq.dequantize() + nu[None, :]) @ wn.T
+        # dW = X^T dY over the sampled rows (its share of the contraction)
+        fp4.quantize(rx, "nv", 0).dequantize() @ fp4.quantize(rdy, "nv", 0).dequantize().T
+        t_rows = time.perf_counter() - t1
+        full = t_fixed + t_rows * (self.M / rows)
+        return full, t_fixed + t_rows, (f"column means of X and dY, W's two FP4 copies once; residuals, their FP4 "
+                                        f"copies and the three products on {rows} of {self.M} rows, scaled "
+                                        f"x{self.M // rows}")
+
+
+class LlamaMlpWorkload:
+    """llama3_8b_mlp (gate projection): W bf16 4096 x 14336 (planted), X bf16
+    16384 x 4096, dY bf16 16384 x 14336.  Step: the spectral split of W, X and
+    dY (k = 64, p = 16, q = 1, NVFP4, residuals along both axes, FP4 factors),
+    then Y = X W, dX = dY W^T and dW = X^T dY (bf16 outputs)."""
+
+    name = "llama3_8b_mlp"
+
+    def __init__(self, dev):
+        import torch
+        from spectral_domain_quantization_b200 import api, inputs
+        self.api = api
+        d = inputs.make("llama3_8b_mlp", keys=("W", "X", "dY"))
+        c = d["cfg"]
+        self.c = c
+        self.M, self.K, self.N, self.k = c["M"], c["K"], c["N"], c["k"]
+        self.host = {k: _pinned_bf16(d[k]) for k in ("W", "X", "dY")}
+        self.dev = {k: v.to(dev) for k, v in self.host.items()}
+        self.Y = torch.empty((self.M, self.N), dtype=torch.bfloat16, device=dev)
+        self.dX = torch.empty((self.M, self.K), dtype=torch.bfloat16, device=dev)
+        self.dW = torch.empty((self.K, self.N), dtype=torch.bfloat16, device=dev)
+        self.data = d
+        M, K, N, k = self.M, self.K, self.N, self.k
+        self.flops = 3 * 2.0 * M * N * K
+
+        def split_bytes(m, n):   # four sketch passes and two residual passes, two FP4 copies, the factors
+            return 6 * m * n * 2 + 2 * _fp4_bytes(m, n, "nv") + (m + n) * k * 4 + _fp4_bytes(k, m + n, "nv")
+        self.split_bytes = split_bytes(K, N) + split_bytes(M, K) + split_bytes(M, N)
+        self.config = {"workload": "llama3_8b_mlp gate projection: W bf16 4096x14336 planted spectrum, X bf16 "
+                                   "16384x4096, dY bf16 16384x14336; split k=64 p=16 q=1 Gaussian of W, X, dY, "
+                                   "NVFP4; forward, dX, dW",
+                       "M": M, "K": K, "N": N, "k": k, "p": c["p"], "power_iters": c["q"], "fmt": "nvfp4"}
+        self.ops = None
+
+    def split(self):
+        api, d, c = self.api, self.dev, self.c
+        args = (self.k, c["p"], c["q"], c["sketch_seed"], "nv")
+        self.ops = tuple(api.split(d[key], *args, rows=True, cols=True) for key in ("W", "X", "dY"))
+
+    def products(self):
+        api = self.api
+        Ws, Xs, Ds = self.ops
+        k = self.k
+        api.linear_fwd(Xs.operand("left"), Ws.operand("right"), self.M, self.N, self.K, Y=self.Y)
+        api.linear_bwd(Ds.operand("left"), api.Operand(Ws.R_rows, k, Ws.V_q, Ws.U_q, Ws.S),
+                       api.Operand(Xs.R_cols, k, Xs.U_q, Xs.V_q, Xs.S), Ds.operand("right"), self.M, self.N,
+                       self.K, out_dtype=self.Y.dtype, dX=self.dX, dW=self.dW)
+
+    def plain(self):
+        api = self.api
+        Ws, Xs, _ = self.ops
+        api.linear_fwd(api.Operand(Xs.R_rows), api.Operand(Ws.R_cols), self.M, self.N, self.K, Y=self.Y)
+        return 2.0 * self.M * self.N * self.K, f"gemm_fp4 ({self.M}x{self.N}x{self.K} NVFP4)"
+
+    def outputs(self):
+        return [self.Y, self.dX, self.dW]
+
+    def oracle_sample(self, rows=64):
+        from oracle import fp4, gemm, split
+        d, c, k = self.data, self.c, self.k
+        t0 = time.perf_counter()
+        res = {}
+        for key in ("W", "X", "dY"):
+            res[key] = split.split(d[key].f64(), k, c["p"], c["q"], c["sketch_seed"])
+        q = lambda a, axis: fp4.quantize(np.float32(a), "nv", axis)
+        w, x, dy = res["W"], res["X"], res["dY"]
+        # W's two dense operands do not depend on the rows
+        wr = gemm.dense_right(gemm.Operand(q(w["R"], 0), k, q(w["U"], 0), q(w["V"], 0), w["S"]))
+        wt = gemm.dense_right(gemm.Operand(q(w["R"], 1), k, q(w["V"], 0), q(w["U"], 0), w["S"]))
+        t_split = time.perf_counter() - t0
+        t1 = time.perf_counter()
+        # the rows' share of each product: forward and dX on `rows` rows of
+        # X / dY, dW on `rows` rows of the contraction over M
+        xl = gemm.Operand(q(x["R"][:rows], 1), k, q(x["V"], 0), q(x["U"][:rows], 0), x["S"])
+        gemm.dense_left(xl) @ wr
+        dl = gemm.Operand(q(dy["R"][:rows], 1), k, q(dy["V"], 0), q(dy["U"][:rows], 0), dy["S"])
+        gemm.dense_left(dl) @ wt
+        xt = gemm.dense_left(gemm.Operand(q(x["R"][:rows], 0), k, q(x["U"][:rows], 0), q(x["V"], 0), x["S"]))
+        dr = gemm.dense_right(gemm.Operand(q(dy["R"][:rows], 0), k, q(dy["U"][:rows], 0), q(dy["V"], 0), dy["S"]))
+        xt @ dr
+        t_rows = time.perf_counter() - t1
+        full = t_split + t_rows * (self.M / rows)
+        return full, t_split + t_rows, (f"splits of W, X and dY and W's dense operands once; FP4 operands and the "
+                                        f"three products on {rows} of {self.M} rows, scaled x{self.M // rows}")
+
+
+class SampledWorkload:
+    """sampled_65536: A bf16 65536 x 4096 with a planted rank-32 spike, W bf16
+    4096 x 4096.  Step: the sampled split of A (2048 rows, sparse-sign sketch
+    with 4 nonzeros, k = 32, p = 16, q = 0, MXFP4, residual along K), W
+    quantized along K, then Y = A W (bf16 output)."""
+
+    name = "sampled_65536"
+
+    def __init__(self, dev):
+        import torch
+        from spectral_domain_quantization_b200 import api, inputs
+        self.api = api
+        d = inputs.make("sampled_65536")
+        c = d["cfg"]
+        self.c = c
+        self.M, self.K, self.N, self.k = c["M"], c["K"], c["N"], c["k"]
+        self.host = {k: _pinned_bf16(d[k]) for k in ("A", "W")}
+        self.dev = {k: v.to(dev) for k, v in self.host.items()}
+        self.Y = torch.empty((self.M, self.N), dtype=torch.bfloat16, device=dev)
+        self.data = d
+        M, K, N, k, s = self.M, self.K, self.N, self.k, c["sample_rows"]
+        self.flops = 2.0 * M * N * K
+        # gather s rows, two passes over them, one pass over A (P = A V_s, the
+        # residual and its FP4 copy), the W copy (one read, codes and scales)
+        self.split_bytes = (s * K * 2 * 3 + M * K * 2 + _fp4_bytes(M, K, "mx") + M * k * 4 * 2
+                            + K * N * 2 + _fp4_bytes(K, N, "mx"))
+        self.config = {"workload": "sampled_65536: A bf16 65536x4096 planted rank-32 spike, W bf16 4096x4096; "
+                                   "2048 sampled rows, sparse-sign sketch (4 nnz), k=32 p=16 q=0, MXFP4; forward",
+                       "M": M, "K": K, "N": N, "k": k, "p": c["p"], "sample_rows": s, "fmt": "mxfp4"}
+        self.ops = None
+
+    def split(self):
+        api, d, c = self.api, self.dev, self.c
+        self.ops = (api.split(d["A"], self.k, c["p"], 0, c["sketch_seed"], "mx", sketch="sparse_sign", nnz=4,
+                              sample_rows=c["sample_rows"], rows=True, cols=False),
+                    api.quantize_fp4(d["W"], "mx", 0))
+
+    def products(self):
+        api = self.api
+        As, qw = self.ops
+        api.linear_fwd(As.operand("left"), api.Operand(qw), self.M, self.N, self.K, Y=self.Y)
+
+    def plain(self):
+        api = self.api
+        As, qw = self.ops
+        api.linear_fwd(api.Operand(As.R_rows), api.Operand(qw), self.M, self.N, self.K, Y=self.Y)
+        return 2.0 * self.M * self.N * self.K, f"gemm_fp4 ({self.M}x{self.N}x{self.K} MXFP4)"
+
+    def outputs(self):
+        return [self.Y]
+
+    def oracle_sample(self, rows=512):
+        from oracle import fp4, gemm, split
+        d, c, k = self.data, self.c, self.k
+        t0 = time.perf_counter()
+        A = d["A"].f64()
+        r = split.split(A, k, c["p"], 0, c["sketch_seed"], kind="sparse_sign", nnz=4, sample_rows=c["sample_rows"])
+        wr = gemm.dense_right(gemm.Operand(fp4.quantize(d["W"].f32(), "mx", 0)))
+        t_fixed = time.perf_counter() - t0
+        t1 = time.perf_counter()
+        q = lambda a, axis: fp4.quantize(np.float32(a), "mx", axis)
+        left = gemm.Operand(q(r["R"][:rows], 1), k, q(r["V"], 0), q(r["U"][:rows], 0), r["S"])
+        gemm.dense_left(left) @ wr
+        t_rows = time.perf_counter() - t1
+        full = t_fixed + t_rows * (self.M / rows)
+        return full, t_fixed + t_rows, (f"sampled split of A and W's FP4 copy once; the residual rows' FP4 copy and "
+                                        f"the product on {rows} of {self.M} rows, scaled x{self.M // rows}")
+
+
+def _pinned_bf16(mat):
+    import torch
+    return torch.from_numpy(mat.data.view(np.int16)).view(torch.bfloat16).pin_memory()
+
+
+def run_workload(args, rank, world, local):
+    """One timed step of a --workload other than the single layer: the
+    split / quantize phase, then the products, captured as one CUDA graph
+    and replayed with L2 flushed before every step."""
+    import torch
+    from spectral_domain_quantization_b200 import api
+
+    assert torch.cuda.is_available(), "bench needs a GPU"
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    if not api.lib().metis_device_supported():
+        raise RuntimeError("metis needs an sm_100 (B200) device")
+    wl = {"averis_32768": AverisWorkload, "llama3_8b_mlp": LlamaMlpWorkload,
+          "sampled_65536": SampledWorkload}[args.workload](dev)
+    flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
+
+    def step():
+        wl.split()
+        wl.products()
+
+    def capture(fn):
+        for _ in range(2):
+            fn()
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            fn()
+        torch.cuda.synchronize()
+        return g
+
+    def time_graph(g, steps, warmup):
+        for _ in range(warmup):
+            flush.fill_(1)
+            g.replay()
+        torch.cuda.synchronize()
+        starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+        for i in range(steps):
+            flush.fill_(1)
+            starts[i].record()
+            g.replay()
+            ends[i].record()
+        torch.cuda.synchronize()
+        return float(np.mean([s.elapsed_time(e) for s, e in zip(starts, ends)]))
+
+    g_step = capture(step)
+    from torch.profiler import ProfilerActivity, profile
+    with profile(activities=[ProfilerActivity.CUDA]) as prof:
+        step()
+        torch.cuda.synchronize()
+    launches = sum(1 for e in prof.events() if e.device_type.name == "CUDA" and "metis" in e.name)
+
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks.start()
+    ms = time_graph(g_step, args.steps, args.warmup)
+    torch.cuda.synchronize()
+    clk = clocks.stop()
+    barrier(world)
+    ms = reduce_max(ms, world)
+
+    g_split = capture(wl.split)
+    ms_split = time_graph(g_split, args.steps, 3)
+    wl.split()
+    g_prod = capture(wl.products)
+    ms_prod = time_graph(g_prod, args.steps, 3)
+    plain_flops, plain_name = wl.plain()
+    g_plain = capture(wl.plain)
+    ms_plain = time_graph(g_plain, args.steps, 3)
+
+    e2e = None
+    if not args.no_e2e:
+        # every step uploads its inputs from pinned host memory and copies its
+        # outputs back, on the compute stream, inside the timed region
+        outs = wl.outputs()
+        out_host = [torch.empty(o.shape, dtype=o.dtype).pin_memory() for o in outs]
+
+        def e2e_step():
+            for k, h in wl.host.items():
+                wl.dev[k].copy_(h, non_blocking=True)
+            g_step.replay()
+            for h, o in zip(out_host, outs):
+                h.copy_(o, non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        barrier(world)
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(args.steps):
+            e2e_step()
+        e1.record()
+        torch.cuda.synchronize()
+        e2e_ms = reduce_max(e0.elapsed_time(e1) / args.steps, world)
+        e2e = {"value": world * wl.flops / (e2e_ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": e2e_ms,
+               "h2d_bytes_per_step": int(sum(h.numel() * h.element_size() for h in wl.host.values())),
+               "d2h_bytes_per_step": int(sum(o.numel() * o.element_size() for o in outs)),
+               "pipelining": "none: uploads, the step and the downloads in order on one stream"}
+
+    hbm, bf16_tf, peak_kind = measured_peaks()
+    fp4_peak = 4.0 * bf16_tf
+    achieved = plain_flops / (ms_plain * 1e-3) / 1e12
+    value = world * wl.flops / (ms * 1e-3) / 1e12
+    cpu = None
+    if rank == 0 and not args.no_cpu_baseline:
+        t, _, desc = wl.oracle_sample()
+        cpu = {"value": wl.flops / t / 1e12, "unit": "TFLOPS", "cores": blas_threads(), "kind": "oracle",
+               "sample": desc, "full_step_ms_extrapolated": t * 1e3}
+    if rank == 0:
+        split_gbs = wl.split_bytes / (ms_split * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "fp4 (e2m1 with nvfp4 / mxfp4 scales; fp32 accumulate)", "data": "synthetic",
+            "config": dict(wl.config, l2="flushed (512 MB write) before every timed step"),
+            "frac_of_fp4_peak": value / world / fp4_peak,
+            "split_quantize_us_per_layer": ms_split * 1e3,
+            "breakdown_us": {"split_quantize": ms_split * 1e3, "products": ms_prod * 1e3,
+                             "fp4_gemm_kernel": ms_plain * 1e3},
+            "hbm": {"split_quantize": {"algorithmic_bytes": wl.split_bytes, "achieved_gbs": split_gbs,
+                                       "peak_gbs": hbm, "frac": split_gbs / hbm, "peak_source": peak_kind}},
+            "roofline": {"kernel": plain_name, "bound": "tensor", "achieved": achieved, "peak": fp4_peak,
+                         "unit": "TFLOP/s", "frac": achieved / fp4_peak,
+                         "peak_source": f"{peak_kind} bf16 {bf16_tf} TFLOP/s x 4 (nominal FP4/bf16 ratio)",
+                         "traffic": None},
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches,
+            "clocks": clk,
+        }
+        print(json.dumps(line), flush=True)
+    del g_step, g_split, g_prod, g_plain
+
+
 def run_profile(args, local):
     """The step, eagerly and untimed: a short launch list for profilers."""
     import torch
@@ -599,6 +994,8 @@ def main():
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
+        elif args.workload != "layer_4096":
+            run_workload(args, rank, world, local)
         else:
             run_ours(args, rank, world, local)
     finally:

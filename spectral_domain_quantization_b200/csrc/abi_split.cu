@@ -8,11 +8,14 @@
 // Enqueued pipeline (all on `stream`, no host synchronisation):
 //   [sample rows -> gather A_s]                      sketch.cu
 //   Omega^T (Philox Gaussian / sparse sign, bf16)    sketch.cu
-//   Y = A Omega                                      skinny_gemm.cu (tcgen05)
+//   Y = A Omega                                      skinny_gemm.cu (tcgen05;
+//                                                    each pass also writes the
+//                                                    operand of the next one
+//                                                    and its Gram partials)
 //   q = 0: Q = orth(Y), two CholeskyQR passes        small_linalg.cu
 //   q >= 1: Y as is, then q x { Q1 = orth(A^T Y); Y = A Q1; Q = orth(Y) },
 //           one CholeskyQR pass each
-//   Z = B^T = A^T Q, C = Z^T Z                       skinny GEMM + Gram
+//   Z = B^T = A^T Q, C = Z^T Z                       skinny pass + Gram
 //   C = W diag(sigma^2) W^T, top k                   core_eig.cu (tridiagonal
 //                                                    reduction, multisection,
 //                                                    twisted factorisation)
@@ -46,7 +49,7 @@ struct SplitPlan {
   int64_t ms;            // rows of the range-finder matrix (m or sample_rows)
   int l, lp, k, kp, kq;  // kq = k padded to 16 (sampled P width); kp = k padded to 64
   int64_t ld_m, ld_n;    // padded lengths (multiples of 8) of transposed operands
-  int split_m, split_n;  // split-K of the A X (rows ms or m) and A^T X passes
+  int cs_m, cs_n;        // K slices (cluster size) of the A X (rows ms) and A^T X passes
   int sampled, fp32;
 };
 
@@ -60,7 +63,6 @@ struct SplitBuffers {
   int32_t* idx = nullptr;
   SelectState* sel = nullptr;
   unsigned* hist = nullptr;
-  float* part = nullptr;             // split partials
   float* Y = nullptr;                // max(m, n) x lp
   float* Q1 = nullptr;               // max(m, n) x lp
   float* Qm = nullptr;               // ms x lp   (range basis)
@@ -100,8 +102,8 @@ SplitPlan make_plan(int64_t m, int64_t n, int dtype, const metis_split_params* p
   p.ld_n = round_up64(n, 8);
   p.fp32 = dtype == METIS_F32;
   const int sms = device_sm_count();
-  p.split_m = skinny_splits(p.ms, n, sms);
-  p.split_n = skinny_splits(n, p.ms, sms);
+  p.cs_m = skinny_cluster(p.ms, n, sms);
+  p.cs_n = skinny_cluster(n, p.ms, sms);
   return p;
 }
 
@@ -124,16 +126,14 @@ SplitBuffers carve(const SplitPlan& p, int64_t lda, Carver& ws) {
       b.af_lo = ws.take<__nv_bfloat16>(static_cast<size_t>(p.m) * lda);
     }
   }
-  const int64_t parts_rows = big;
-  const int splits = p.split_m > p.split_n ? p.split_m : p.split_n;
   const int wmax = p.lp > p.kq ? p.lp : p.kq;
-  b.part = ws.take<float>(static_cast<size_t>(splits) * parts_rows * wmax);
   b.Y = ws.take<float>(static_cast<size_t>(big) * wmax);
   b.Q1 = ws.take<float>(static_cast<size_t>(big) * p.lp);
   b.Qm = ws.take<float>(static_cast<size_t>(p.ms) * p.lp);
   b.Zn = ws.take<float>(static_cast<size_t>(p.n) * p.lp);
   b.qt = ws.take<__nv_bfloat16>(static_cast<size_t>(2 * wmax) * bigld);
-  b.gpart = ws.take<double>(static_cast<size_t>(gram_blocks(big)) * wmax * wmax);
+  const int64_t gblocks = imax64(gram_blocks(big), apply_blocks(big));  // Gram partials per row block
+  b.gpart = ws.take<double>(static_cast<size_t>(gblocks) * wmax * wmax);
   b.G = ws.take<double>(static_cast<size_t>(wmax) * wmax);
   b.eig_ws = reinterpret_cast<double*>(ws.take<uint8_t>(core_eig_workspace(wmax)));
   b.Rinv = ws.take<float>(static_cast<size_t>(p.lp) * p.lp);
@@ -182,8 +182,11 @@ struct Source {             // one matrix seen by the skinny GEMMs (bf16 parts)
   int64_t rows, cols, ld;
 };
 
-metis_status skinny(const Source& a, int mode, const __nv_bfloat16* xt, int64_t ldx, int xparts, int lp, int splits,
-                    float* out, int32_t* dev_status, cudaStream_t s) {
+// One pass over `a` (see skinny_gemm.h): Y = A X (mode 0) or A^T X (mode 1),
+// written as float32 rows (out) and / or as a transposed bf16 hi / lo copy
+// (outT, row stride ldo).
+metis_status skinny(const Source& a, int mode, const __nv_bfloat16* xt, int64_t ldx, int xparts, int lp, int cs,
+                    float* out, __nv_bfloat16* outT, int64_t ldo, int32_t* dev_status, cudaStream_t s) {
   SkinnyCall c{};
   c.mode = mode;
   c.m = a.rows;
@@ -196,19 +199,21 @@ metis_status skinny(const Source& a, int mode, const __nv_bfloat16* xt, int64_t 
   c.ldx = ldx;
   c.xparts = xparts;
   c.lp = lp;
-  c.splits = splits;
+  c.cs = cs;
   c.out = out;
+  c.outT = outT;
+  c.ldo = ldo;
   c.dev_status = dev_status;
   return run_skinny_gemm(c, s);
 }
 
-// CholeskyQR of the split partials of a rows x lp product, `passes` times
-// (2 for the only basis when there is no power iteration; otherwise 1 for
-// every basis: the Gram is float64 from float32 data).  Output: Q
-// (fp32, rows x lp) and Q^T as bf16 hi / lo rows of qt (row stride ldq).
-metis_status cholqr(const SplitBuffers& b, int splits, int64_t rows, int lp, float* Q, int64_t ldq, int passes,
+// CholeskyQR of a rows x lp product the last pass left in b.Y, `passes` times (2 for the only basis
+// when there is no power iteration; otherwise 1 for every basis: the Gram is
+// float64 from float32 data).  Output: Q (fp32, rows x lp) and Q^T as bf16
+// hi / lo rows of qt (row stride ldq).
+metis_status cholqr(const SplitBuffers& b, int64_t rows, int lp, float* Q, int64_t ldq, int passes,
                     cudaStream_t s) {
-  launch_gram(b.part, splits, rows, lp, b.Y, b.gpart, b.G, s);
+  launch_gram(b.Y, rows, lp, b.gpart, b.G, s);
   METIS_TRY(step_status("cholqr gram"));
   const float* in = b.Y;
   for (int pass = 0; pass < passes; ++pass) {
@@ -248,26 +253,25 @@ metis_status cholqr(const SplitBuffers& b, int splits, int64_t rows, int lp, flo
 metis_status range_and_core(const SplitPlan& p, const SplitBuffers& b, const Source& src, int power_iters,
                             int max_iters, int32_t* dev_status, cudaStream_t s) {
   const int lp = p.lp;
-  METIS_TRY(skinny(src, 0, b.omt, p.ld_n, 1, lp, p.split_m, b.part, dev_status, s));
   if (power_iters > 0) {
     // A^T Y0 spans the same space as A^T orth(Y0): Y0 = A Omega goes to the
     // next product as it is (its hi / lo transpose), and the next basis is
     // orthonormalised
-    launch_sum_hilo(b.part, p.split_m, src.rows, lp, b.qt, p.ld_m, s);
-    METIS_TRY(step_status("sketch hi/lo"));
+    METIS_TRY(skinny(src, 0, b.omt, p.ld_n, 1, lp, p.cs_m, nullptr, b.qt, p.ld_m, dev_status, s));
   } else {
-    METIS_TRY(cholqr(b, p.split_m, src.rows, lp, b.Qm, p.ld_m, 2, s));
+    METIS_TRY(skinny(src, 0, b.omt, p.ld_n, 1, lp, p.cs_m, b.Y, nullptr, 0, dev_status, s));
+    METIS_TRY(cholqr(b, src.rows, lp, b.Qm, p.ld_m, 2, s));
   }
   for (int it = 0; it < power_iters; ++it) {
-    METIS_TRY(skinny(src, 1, b.qt, p.ld_m, 2, lp, p.split_n, b.part, dev_status, s));
-    METIS_TRY(cholqr(b, p.split_n, p.n, lp, b.Zn, p.ld_n, 1, s));
-    METIS_TRY(skinny(src, 0, b.qt, p.ld_n, 2, lp, p.split_m, b.part, dev_status, s));
+    METIS_TRY(skinny(src, 1, b.qt, p.ld_m, 2, lp, p.cs_n, b.Y, nullptr, 0, dev_status, s));
+    METIS_TRY(cholqr(b, p.n, lp, b.Zn, p.ld_n, 1, s));
+    METIS_TRY(skinny(src, 0, b.qt, p.ld_n, 2, lp, p.cs_m, b.Y, nullptr, 0, dev_status, s));
     // one pass also for the final basis: the Gram is formed in float64 from
     // float32 data, so a pass leaves |Q^T Q - I| near kappa(Y) 2^-23
-    METIS_TRY(cholqr(b, p.split_m, src.rows, lp, b.Qm, p.ld_m, 1, s));
+    METIS_TRY(cholqr(b, src.rows, lp, b.Qm, p.ld_m, 1, s));
   }
-  METIS_TRY(skinny(src, 1, b.qt, p.ld_m, 2, lp, p.split_n, b.part, dev_status, s));
-  launch_gram(b.part, p.split_n, p.n, lp, b.Zn, b.gpart, b.G, s);
+  METIS_TRY(skinny(src, 1, b.qt, p.ld_m, 2, lp, p.cs_n, b.Zn, nullptr, 0, dev_status, s));
+  launch_gram(b.Zn, p.n, lp, b.gpart, b.G, s);
   METIS_TRY(step_status("core gram"));
   launch_core_eig(b.G, lp, max_iters, b.eval, b.evec, b.eig_ws, dev_status, s);
   return step_status("core eigensolver");
@@ -419,9 +423,8 @@ extern "C" metis_status metis_split(const void* A, int32_t dtype, int64_t m, int
     avs.ldx = p.ld_n;
     launch_apply(avs, s);
     // P = A V_s over all rows, and P^T P
-    const int sp = skinny_splits(m, n, sms);
-    METIS_TRY(skinny(full, 0, b.qt, p.ld_n, 2, p.kq, sp, b.part, dev_status, s));
-    launch_gram(b.part, sp, m, p.kq, b.P, b.gpart, b.G, s);
+    METIS_TRY(skinny(full, 0, b.qt, p.ld_n, 2, p.kq, skinny_cluster(m, n, sms), b.P, nullptr, 0, dev_status, s));
+    launch_gram(b.P, m, p.kq, b.gpart, b.G, s);
     launch_core_eig(b.G, p.kq, prm->max_core_iters, b.eval2, b.evec2, b.eig_ws, dev_status, s);
     launch_factor_mats(b.eval2, b.evec2, p.kq, p.k, b.Mu, b.Mv, S, s);
     ApplyArgs au{};

@@ -107,6 +107,44 @@ MDEV bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort) {
 }
 
 // ---------------------------------------------------------------------------
+// thread-block clusters (distributed shared memory)
+// ---------------------------------------------------------------------------
+
+MDEV uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+
+// Address of the same shared-memory location in CTA `rank` of the cluster.
+MDEV uint32_t map_to_rank(uint32_t smem_addr, uint32_t rank) {
+  uint32_t out;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(out) : "r"(smem_addr), "r"(rank));
+  return out;
+}
+
+// Every thread of every CTA of the cluster arrives; the waits see the other
+// CTAs' shared-memory writes made before their arrival.
+MDEV void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+MDEV float4 ld_cluster_f32x4(uint32_t cluster_addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(cluster_addr)
+               : "memory");
+  return v;
+}
+
+MDEV double2 ld_cluster_f64x2(uint32_t cluster_addr) {
+  double2 v;
+  asm volatile("ld.shared::cluster.v2.f64 {%0, %1}, [%2];" : "=d"(v.x), "=d"(v.y) : "r"(cluster_addr) : "memory");
+  return v;
+}
+
+// ---------------------------------------------------------------------------
 // TMA and bulk copies (global -> shared, completion on an mbarrier)
 // ---------------------------------------------------------------------------
 

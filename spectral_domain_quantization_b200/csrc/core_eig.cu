@@ -306,23 +306,42 @@ MDEV int sturm_count(const double* d, const double* e2, int n, double x) {
     cnt += s != sg;
     sg = s;
   }
-  for (int i = 1; i < n; ++i) {
+  // four steps per pass, their loads issued together ahead of the recurrence
+  // (only the fma on p_{i-1} is on the dependent chain)
+  int i = 1;
+  for (; i + 3 < n; i += 4) {
+    double dd[4], ff[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      dd[u] = d[i + u] - x;
+      ff[u] = e2[i + u - 1];
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const double p = fma(dd[u], pm1, -ff[u] * pm2);
+      const int s = p < 0.0 ? -1 : (p > 0.0 ? 1 : sg);
+      cnt += s != sg;
+      sg = s;
+      pm2 = pm1;
+      pm1 = p;
+    }
+    // scale (p_{i-1}, p_i) by 2^-e, e the exponent of the larger one (a
+    // power of two: the signs, and so the count, are unchanged)
+    const long long bits = __double_as_longlong(fmax(fabs(pm1), fabs(pm2)));
+    const int ex = static_cast<int>((bits >> 52) & 0x7FF) - 1023;
+    if (ex > -1000) {
+      const double sc = __longlong_as_double(static_cast<long long>(1023 - ex) << 52);
+      pm1 *= sc;
+      pm2 *= sc;
+    }
+  }
+  for (; i < n; ++i) {
     const double p = fma(d[i] - x, pm1, -e2[i - 1] * pm2);
     const int s = p < 0.0 ? -1 : (p > 0.0 ? 1 : sg);
     cnt += s != sg;
     sg = s;
     pm2 = pm1;
     pm1 = p;
-    if ((i & 3) == 0) {
-      // scale (p_{i-1}, p_i) by 2^-e, e the exponent of the larger one
-      const long long bits = __double_as_longlong(fmax(fabs(pm1), fabs(pm2)));
-      const int ex = static_cast<int>((bits >> 52) & 0x7FF) - 1023;
-      if (ex > -1000) {
-        const double sc = __longlong_as_double(static_cast<long long>(1023 - ex) << 52);
-        pm1 *= sc;
-        pm2 *= sc;
-      }
-    }
   }
   return cnt;
 }

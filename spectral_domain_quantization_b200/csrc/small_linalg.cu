@@ -22,7 +22,6 @@ namespace metis {
 
 namespace {
 
-constexpr int kRowsPerBlock = 32;
 constexpr double kDropTol = 1e-12;
 
 // Gram partial of a row block held in shared memory (rows x cols floats with
@@ -66,54 +65,30 @@ MDEV void gram_block(const float* ys, int rows, int cols, int ld, double* out) {
   }
 }
 
-// Sum split partials into Y (optional) and the Gram partial of each block.
-// One thread per 4 consecutive columns of one row (blockDim = 32 lp / 4), so
-// every split partial is one 16-byte load and a thread's loads are
-// independent; the sum keeps the split order.
-__global__ void __launch_bounds__(1024) gram_kernel(const float* __restrict__ partial, int splits, int64_t rows,
-                                                    int lp, float* __restrict__ Y, double* __restrict__ gpart,
-                                                    __nv_bfloat16* __restrict__ outT, int64_t ldx) {
-  extern __shared__ float ys[];  // kRowsPerBlock x (lp + 1)
+constexpr int kGramRows = 32;
+
+// Float64 Gram partial of each 32-row block of Y (rows x lp float32, row
+// stride lp): the block staged in shared memory, then 4 x 4 register tiles
+// over the rows in order.  One thread per 4 x 4 tile pair (blockDim covers
+// (lp/4)(lp/4+1)/2 pairs).
+__global__ void __launch_bounds__(1024) gram_kernel(const float* __restrict__ Y, int64_t rows, int lp,
+                                                    double* __restrict__ gpart) {
+  extern __shared__ float ys[];  // kGramRows x (lp + 1)
   const int ld = lp + 1;
   const int q4 = lp / 4;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kRowsPerBlock;
-  const int nr = static_cast<int>(imin64(kRowsPerBlock, rows - r0));
-  const int64_t stride4 = rows * q4;
-  const float4* src = reinterpret_cast<const float4*>(partial);
-  for (int e = threadIdx.x; e < kRowsPerBlock * q4; e += blockDim.x) {
+  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kGramRows;
+  const int nr = static_cast<int>(imin64(kGramRows, rows - r0));
+  for (int e = threadIdx.x; e < kGramRows * q4; e += blockDim.x) {
     const int r = e / q4, c4 = e - r * q4;
-    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-    if (r < nr) {
-      const float4* p = src + (r0 + r) * q4 + c4;
-#pragma unroll 8
-      for (int sp = 0; sp < splits; ++sp) {
-        const float4 x = p[sp * stride4];
-        acc.x += x.x;
-        acc.y += x.y;
-        acc.z += x.z;
-        acc.w += x.w;
-      }
-      if (Y) reinterpret_cast<float4*>(Y)[(r0 + r) * q4 + c4] = acc;
-    }
+    const float4 x = r < nr ? reinterpret_cast<const float4*>(Y)[(r0 + r) * q4 + c4] : make_float4(0.f, 0.f, 0.f, 0.f);
     float* d = ys + r * ld + 4 * c4;
-    d[0] = acc.x;
-    d[1] = acc.y;
-    d[2] = acc.z;
-    d[3] = acc.w;
+    d[0] = x.x;
+    d[1] = x.y;
+    d[2] = x.z;
+    d[3] = x.w;
   }
   __syncthreads();
-  if (outT) {  // transposed bf16 hi / lo copy (rows lp apart), coalesced along the rows
-    for (int e = threadIdx.x; e < kRowsPerBlock * lp; e += blockDim.x) {
-      const int c = e / kRowsPerBlock, r = e - c * kRowsPerBlock;
-      if (r < nr) {
-        const float v = ys[r * ld + c];
-        const __nv_bfloat16 hi = __float2bfloat16_rn(v);
-        outT[static_cast<int64_t>(c) * ldx + r0 + r] = hi;
-        outT[static_cast<int64_t>(lp + c) * ldx + r0 + r] = __float2bfloat16_rn(__fsub_rn(v, __bfloat162float(hi)));
-      }
-    }
-  }
-  if (gpart) gram_block(ys, nr, lp, ld, gpart + static_cast<int64_t>(blockIdx.x) * lp * lp);
+  gram_block(ys, nr, lp, ld, gpart + static_cast<int64_t>(blockIdx.x) * lp * lp);
 }
 
 // Sum of the block partials: a CTA takes 32 consecutive entries (coalesced
@@ -140,7 +115,6 @@ __global__ void __launch_bounds__(256) gram_reduce_kernel(const double* __restri
   }
 }
 
-// Lower-triangle element e (column-major order: column 0 top to bottom, then
 // column 1 ...) of an n x n matrix, packed as (row << 8) | column.
 MDEV int tri_element(int e, int n) {
   const int ntri = n * (n + 1) / 2;
@@ -548,25 +522,16 @@ __global__ void sign_kernel(const float* __restrict__ U, const float* __restrict
 
 }  // namespace
 
-int64_t gram_blocks(int64_t rows) { return (rows + kRowsPerBlock - 1) / kRowsPerBlock; }
-
 int64_t apply_blocks(int64_t rows) { return (rows + kApplyRows - 1) / kApplyRows; }
 
-void launch_gram(const float* partial, int splits, int64_t rows, int lp, float* Y, double* gpart, double* G,
-                 cudaStream_t s) {
-  const int nb = static_cast<int>(gram_blocks(rows));
-  const int threads = (kRowsPerBlock * (lp / 4) + 31) / 32 * 32;  // lp <= 112: at most 896
-  gram_kernel<<<nb, threads, kRowsPerBlock * (lp + 1) * sizeof(float), s>>>(partial, splits, rows, lp, Y, gpart,
-                                                                            nullptr, 0);
-  launch_gram_reduce(gpart, nb, lp, G, s);
-}
+int64_t gram_blocks(int64_t rows) { return (rows + kGramRows - 1) / kGramRows; }
 
-void launch_sum_hilo(const float* partial, int splits, int64_t rows, int lp, __nv_bfloat16* outT, int64_t ldx,
-                     cudaStream_t s) {
+void launch_gram(const float* Y, int64_t rows, int lp, double* gpart, double* G, cudaStream_t s) {
   const int nb = static_cast<int>(gram_blocks(rows));
-  const int threads = (kRowsPerBlock * (lp / 4) + 31) / 32 * 32;
-  gram_kernel<<<nb, threads, kRowsPerBlock * (lp + 1) * sizeof(float), s>>>(partial, splits, rows, lp, nullptr,
-                                                                            nullptr, outT, ldx);
+  const int pairs = (lp / 4) * (lp / 4 + 1) / 2;
+  const int threads = (pairs + 31) / 32 * 32;
+  gram_kernel<<<nb, threads, kGramRows * (lp + 1) * sizeof(float), s>>>(Y, rows, lp, gpart);
+  launch_gram_reduce(gpart, nb, lp, G, s);
 }
 
 void launch_gram_reduce(const double* gpart, int nblocks, int lp, double* G, cudaStream_t s) {

@@ -23,18 +23,14 @@ struct ApplyArgs {
   double* gpart;           // optional [blocks][kout][kout]
 };
 
-int64_t gram_blocks(int64_t rows);
 // row blocks of launch_apply (its Gram partials come one per block)
 int64_t apply_blocks(int64_t rows);
-// Y (optional) = sum of split partials; G = Y^T Y (float64, lp x lp).
-// gpart: gram_blocks(rows) * lp * lp doubles of scratch.
-void launch_gram(const float* partial, int splits, int64_t rows, int lp, float* Y, double* gpart, double* G,
-                 cudaStream_t s);
-// Sum of split partials written only as a transposed bf16 hi / lo copy
-// ([2 lp][ldx]: hi rows 0..lp-1, lo rows lp..2lp-1): the operand of the next
-// skinny product when this basis needs no orthonormalisation.
-void launch_sum_hilo(const float* partial, int splits, int64_t rows, int lp, __nv_bfloat16* outT, int64_t ldx,
-                     cudaStream_t s);
+// G = Y^T Y (float64, lp x lp) of a rows x lp float32 Y (row stride lp):
+// Gram partials of 32-row blocks (gram_blocks(rows) * lp * lp doubles of
+// scratch in gpart), then their sum in block order.
+int64_t gram_blocks(int64_t rows);
+void launch_gram(const float* Y, int64_t rows, int lp, double* gpart, double* G, cudaStream_t s);
+// G = sum of nblocks Gram partials (lp x lp float64 each), in block order.
 void launch_gram_reduce(const double* gpart, int nblocks, int lp, double* G, cudaStream_t s);
 // Rinv (lp x lp float, upper triangular) with G = R^T R, dropped pivots -> 0.
 void launch_cholesky_inv(const double* G, int lp, float* Rinv, cudaStream_t s);

@@ -147,3 +147,108 @@ def test_averis_full_size():
     want = gemm.gemm(gemm.Operand(read_fp4(ax.R_rows), 1, read_fp4(ax.mean_q), "ones", [1.0]),
                      gemm.Operand(read_fp4(qw)), rows=rows)
     assert rel_fro(y.cpu().numpy()[rows], want) < TOL_GEMM
+
+
+def _op(k, qr, P, F, S):
+    """oracle operand from the GPU's own FP4 tensors"""
+    return gemm.Operand(read_fp4(qr), k, read_fp4(P), read_fp4(F), S.cpu().numpy().astype(np.float64))
+
+
+def test_tiny_forward_product():
+    """W fp32 256 x 256 (planted, k = 8, p = 8, q = 1, MXFP4) split, X fp32
+    128 x 256 quantized along K: Y = X W against the oracle's product of the
+    same FP4 operands, and against the oracle's own chain from the inputs."""
+    d = inputs.make("tiny_256")
+    c = d["cfg"]
+    M, K, N, k = c["M"], c["K"], c["N"], c["k"]
+    ws = api.split(to_device(d["W"]), k, c["p"], c["q"], c["sketch_seed"], "mx", rows=False, cols=True)
+    qx = api.quantize_fp4(to_device(d["X"]), "mx", 1)
+    y = api.linear_fwd(api.Operand(qx), ws.operand("right"), M, N, K)
+    torch.cuda.synchronize()
+    assert int(ws.dev_status.cpu()[0]) == 0
+    want = gemm.gemm(gemm.Operand(read_fp4(qx)), _op(k, ws.R_cols, ws.U_q, ws.V_q, ws.S))
+    assert rel_fro(y.cpu().numpy(), want) < TOL_GEMM
+    # the oracle's own chain: its split, its quantization, its product
+    W64 = d["W"].f64()
+    ref = split.split(W64, k, c["p"], c["q"], c["sketch_seed"])
+    rq = fp4.quantize(ref["R"].astype(np.float32), "mx", 0)
+    uq = fp4.quantize(ref["U"].astype(np.float32), "mx", 0)
+    vq = fp4.quantize(ref["V"].astype(np.float32), "mx", 0)
+    chain = gemm.gemm(gemm.Operand(fp4.quantize(d["X"].f32(), "mx", 1)),
+                      gemm.Operand(rq, k, uq, vq, ref["S"]))
+    assert rel_fro(y.cpu().numpy(), chain) < 2e-2
+
+
+def test_layer_benched_call_full_size():
+    """The timed step at its full size: split W 4096 x 4096 (k = 64, p = 16,
+    q = 1, NVFP4, residual along K, FP4 factors), quantize X 8192 x 4096 along
+    K, Y = X W with bf16 output.  The bf16 output is the float32 output of the
+    same product rounded once; the float32 output matches the oracle's product
+    of the same FP4 operands on sampled rows."""
+    d = inputs.make("layer_4096")
+    c = d["cfg"]
+    M, K, N, k = c["M"], c["K"], c["N"], c["k"]
+    ws = api.split(to_device(d["W"]), k, c["p"], c["q"], c["sketch_seed"], "nv", rows=False, cols=True)
+    qx = api.quantize_fp4(to_device(d["X"]), "nv", 1)
+    y16 = api.linear_fwd(api.Operand(qx), ws.operand("right"), M, N, K, out_dtype=torch.bfloat16)
+    y = api.linear_fwd(api.Operand(qx), ws.operand("right"), M, N, K)
+    torch.cuda.synchronize()
+    assert int(ws.dev_status.cpu()[0]) == 0
+    assert torch.equal(y16, y.to(torch.bfloat16))
+    rows = _rows(M, 64, 13)
+    want = gemm.gemm(gemm.Operand(read_fp4(qx)), _op(k, ws.R_cols, ws.U_q, ws.V_q, ws.S), rows=rows)
+    assert rel_fro(y.cpu().numpy()[rows], want) < TOL_GEMM
+
+
+def test_averis_backward_full_size():
+    """X, dY 32768 x 4096 mean-split (NVFP4) along both axes, W 4096 x 4096:
+    dX = dY W^T (contraction over N) and dW = X^T dY (contraction over M) on
+    sampled output rows."""
+    d = inputs.make("averis_32768")
+    c = d["cfg"]
+    M, K, N = c["M"], c["K"], c["N"]
+    ax = api.averis_split(to_device(d["X"]), "nv", rows=False, cols=True)
+    ady = api.averis_split(to_device(d["dY"]), "nv", rows=True, cols=True)
+    qw_n = api.quantize_fp4(to_device(d["W"]), "nv", 1)          # outer K, blocks along N
+    dX, dW = api.linear_bwd(ady.left(), api.Operand(qw_n), ax.left_t(), ady.right_m(), M, N, K)
+    torch.cuda.synchronize()
+    assert int(ax.dev_status.cpu()[0]) == 0 and int(ady.dev_status.cpu()[0]) == 0
+    rows = _rows(M, 64, 14)
+    left = gemm.Operand(read_fp4(ady.R_rows), 1, read_fp4(ady.mean_q), "ones", [1.0])
+    want = gemm.gemm(left, gemm.Operand(read_fp4(qw_n)), rows=rows)
+    assert rel_fro(dX.cpu().numpy()[rows], want) < TOL_GEMM
+    rows_k = _rows(K, 64, 15)
+    left = gemm.Operand(read_fp4(ax.R_cols), 1, "ones", read_fp4(ax.mean_q), [1.0])
+    right = gemm.Operand(read_fp4(ady.R_cols), 1, "ones", read_fp4(ady.mean_q), [1.0])
+    want = gemm.gemm(left, right, rows=rows_k)
+    assert rel_fro(dW.cpu().numpy()[rows_k], want) < TOL_GEMM
+
+
+def test_llama3_mlp_down_projection_full_size():
+    """Down projection: W 14336 x 4096, H 16384 x 14336, dY 16384 x 4096, all
+    split (k = 64, p = 16, q = 1, NVFP4); Y = H W, dH = dY W^T, dW = H^T dY."""
+    d = inputs.make("llama3_8b_mlp", keys=("W_down", "H", "dY_down"))
+    c = d["cfg"]
+    M, K, N, k = c["M"], c["N"], c["K"], c["k"]   # contraction over the 14336 hidden units
+    args = (k, c["p"], c["q"], c["sketch_seed"], "nv")
+    Ws = api.split(to_device(d["W_down"]), *args, rows=True, cols=True, tap=True)
+    Hs = api.split(to_device(d["H"]), *args, rows=True, cols=True, tap=True)
+    Ds = api.split(to_device(d["dY_down"]), *args, rows=True, cols=True, tap=True)
+    torch.cuda.synchronize()
+    for name, res, m in (("W_down", Ws, K), ("H", Hs, M), ("dY_down", Ds, M)):
+        A64 = d[name].f64()
+        ref = split.split(A64, k, c["p"], c["q"], c["sketch_seed"])
+        _check_split_rows(A64, res, ref, _rows(m, 64, 16), subspace=name == "W_down")
+        del A64, ref
+    y = api.linear_fwd(Hs.operand("left"), Ws.operand("right"), M, N, K)
+    dH, dW = api.linear_bwd(Ds.operand("left"), api.Operand(Ws.R_rows, k, Ws.V_q, Ws.U_q, Ws.S),
+                            api.Operand(Hs.R_cols, k, Hs.U_q, Hs.V_q, Hs.S), Ds.operand("right"), M, N, K)
+    torch.cuda.synchronize()
+    rows = _rows(M, 64, 17)
+    want = gemm.gemm(_op(k, Hs.R_rows, Hs.V_q, Hs.U_q, Hs.S), _op(k, Ws.R_cols, Ws.U_q, Ws.V_q, Ws.S), rows=rows)
+    assert rel_fro(y.cpu().numpy()[rows], want) < TOL_GEMM
+    want = gemm.gemm(_op(k, Ds.R_rows, Ds.V_q, Ds.U_q, Ds.S), _op(k, Ws.R_rows, Ws.V_q, Ws.U_q, Ws.S), rows=rows)
+    assert rel_fro(dH.cpu().numpy()[rows], want) < TOL_GEMM
+    rows_k = _rows(K, 64, 18)
+    want = gemm.gemm(_op(k, Hs.R_cols, Hs.U_q, Hs.V_q, Hs.S), _op(k, Ds.R_cols, Ds.U_q, Ds.V_q, Ds.S), rows=rows_k)
+    assert rel_fro(dW.cpu().numpy()[rows_k], want) < TOL_GEMM
