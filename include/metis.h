@@ -370,6 +370,36 @@ METIS_API metis_status averis_split(const void* X, int32_t dtype, int64_t m, int
                           void* workspace, size_t* workspace_bytes, int32_t* dev_status,
                           void* stream);
 
+/*
+ * metis_spectral_scale -- adaptive spectral learning: the gradient G of a
+ * split weight W = U diag(S) V^T + R preconditioned along W's singular
+ * directions.
+ * Source: SII release section 2.4 item 2 (the gradients along the mid and
+ * low singular-value directions are scaled up by an inverse normalisation,
+ * so that long-tail directions keep learning, without amplifying noise);
+ * older Metis abstract item (ii) (adaptive learning rates in the spectral
+ * domain).  The pages give no formula; the reading taken is
+ *   lambda_i = min(S_1 / S_i, cap)   (1 where S_i <= 0),
+ *   G' = (I + U (L - I) U^T) G (I + V (L - I) V^T),  L = diag(sqrt(lambda)),
+ * so the component along u_i v_j^T is scaled by sqrt(lambda_i lambda_j), a
+ * component with one side in a split direction by that side's
+ * sqrt(lambda), and the rest of G (the long tail) is left as it is.
+ *   G, K, N, ldg  device float32 gradient, row-major, 16-byte rows.
+ *   U, S, V       device float32 factors of the split of W (K x k, k, N x k),
+ *                 as metis_split writes them (orthonormal columns, S
+ *                 descending).
+ *   k             1 .. 64.  cap >= 1.
+ *   Gout          device K x N float32 (row stride N, 16-byte aligned); may
+ *                 not alias G.
+ * K and N must be multiples of 32 (METIS_ERR_SHAPE).  The rank-2k update is
+ * formed with bf16 hi / lo tensor-core products, so G' carries a relative
+ * error of about 2^-16 of the update on top of float32 rounding.
+ */
+METIS_API metis_status metis_spectral_scale(const float* G, int64_t K, int64_t N, int64_t ldg,
+                                  const float* U, const float* S, const float* V, int32_t k,
+                                  float cap, float* Gout, void* workspace, size_t* workspace_bytes,
+                                  int32_t* dev_status, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -84,6 +84,8 @@ _SIGS = {
                                 _VP, _SZP, _VP, _VP]),
     "averis_split": (_I32, [_VP, _I32, _I64, _I64, _I64, _I32, _VP, _FP, _FP, _FP, _VP, _VP, _SZP,
                             _VP, _VP]),
+    "metis_spectral_scale": (_I32, [_VP, _I64, _I64, _I64, _VP, _VP, _VP, _I32, ctypes.c_float, _VP, _VP, _SZP,
+                                    _VP, _VP]),
 }
 
 
@@ -484,6 +486,28 @@ def composite_split(A, k, p, q=1, seed=0, fmt="nv", sketch="gaussian", nnz=4, ma
     return CompositeSplit(mean=av.mean, R1=av.R_f32, U=sp.U, S=sp.S, V=sp.V, F32=F32, P32=P32, F_q=F_q,
                           P_q=P_q, S1=S1, R_rows=sp.R_rows, R_cols=sp.R_cols, R2_f32=sp.R_f32, k=k, k1=k1,
                           fmt=sp.fmt, dev_status=dev_status)
+
+
+def spectral_scale(G, U, S, V, cap, out=None, dev_status=None):
+    """Adaptive spectral learning (metis_spectral_scale): G' = P_L G P_R with
+    the gains min(S_1 / S_i, cap) along the split's singular directions.
+    G: K x N float32 CUDA tensor; U (K x k), S (k), V (N x k) from split()."""
+    if G.dim() != 2 or G.stride(1) != 1 or G.dtype != torch.float32:
+        raise ValueError("G must be a row-major float32 2-D tensor")
+    if not (U.is_contiguous() and S.is_contiguous() and V.is_contiguous()):
+        raise ValueError("U, S and V must be contiguous")
+    K, N = G.shape
+    k = U.shape[1]
+    if out is None:
+        out = torch.empty((K, N), dtype=torch.float32, device=G.device)
+    if dev_status is None:
+        dev_status = torch.zeros(1, dtype=torch.int32, device=G.device)
+    _call_with_workspace(
+        lib().metis_spectral_scale,
+        (_ptr(G), K, N, G.stride(0), _ptr(U), _ptr(S), _ptr(V), k,
+         ctypes.c_float(cap), _ptr(out)),
+        (_ptr(dev_status), _stream()), G.device, "metis_spectral_scale")
+    return out
 
 
 def selftest_wait_timeout(limit_ns=1_000_000, device="cuda"):

@@ -346,6 +346,12 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
           }
         }
       }
+      // the residual: using every loaded value here means the shared-memory
+      // reads have returned before the stage is handed back to the producer
+      // (a load whose value is first used after the arrive could still be
+      // reading while the next TMA copy lands in the stage)
+#pragma unroll
+      for (int j = 0; j < 32; ++j) v[j] = __fsub_rn(v[j], __uint_as_float(L[j]));
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[stage]);
       if (++stage == S) {
@@ -360,8 +366,6 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
       const int64_t col0 = static_cast<int64_t>(tn) * kBN + 32 * h;
       if (row0 >= p.m || col0 >= p.n) continue;  // m, n are multiples of 32: whole warp
       const int64_t row = row0 + lane;
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = __fsub_rn(v[j], __uint_as_float(L[j]));
       if (p.mode == 0) {
 #pragma unroll
         for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));

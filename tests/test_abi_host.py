@@ -281,3 +281,21 @@ def test_averis_argument_checks_and_workspace_query():
     assert _averis(ws=ctypes.c_void_p(_WS), wsb=need1 - 1,
                    mean_q=_fake_fp4(api.NVFP4, 1, 128))[0] == ERR_WORKSPACE
 
+
+def _scale(G=_A, K=256, N=128, ldg=128, U=_U, S=_S, V=_V, k=8, cap=4.0, out=0x90000, ws=None, wsb=0):
+    size = ctypes.c_size_t(wsb)
+    st = api.lib().metis_spectral_scale(G, K, N, ldg, U, S, V, k, ctypes.c_float(cap), out, ws, ctypes.byref(size),
+                                        _ST, None)
+    return st, size.value
+
+
+def test_spectral_scale_argument_checks_and_workspace_query():
+    st, need = _scale()
+    assert st == api.OK and need > 0
+    for kw in (dict(G=None), dict(U=None), dict(S=None), dict(V=None), dict(out=None)):
+        assert _scale(**kw)[0] == ERR_NULL
+    assert _scale(k=0)[0] == ERR_ARG and _scale(k=65)[0] == ERR_ARG           # 1 <= k <= 64
+    assert _scale(cap=0.5)[0] == ERR_ARG and _scale(cap=float("nan"))[0] == ERR_ARG
+    assert _scale(K=100)[0] == ERR_SHAPE and _scale(N=96 + 8, ldg=104)[0] == ERR_SHAPE
+    assert _scale(ldg=130)[0] == ERR_ALIGN and _scale(out=0x90004)[0] == ERR_ALIGN
+    assert _scale(ws=ctypes.c_void_p(_WS), wsb=need - 1)[0] == ERR_WORKSPACE
