@@ -21,72 +21,114 @@ namespace metis {
 
 namespace {
 
-constexpr int kColsPerBlock = 64;   // 32 threads x 2 columns
-constexpr int kRowGroups = 8;       // threads per column pair
+constexpr int kColsPerThread = 8;                     // one 16-byte bf16 load (two for f32)
+constexpr int kColsPerBlock = 32 * kColsPerThread;    // a warp spans 256 columns
+constexpr int kRowGroups = 8;                         // warps, interleaved over the rows
+constexpr int kRowUnroll = 4;                         // rows whose loads are in flight together
 
-// Block (col tile, row chunk): 32 x 8 threads; thread (x, y) owns columns
-// c = tile*64 + 2x, 2x+1 and rows r0 + y, r0 + y + 8, ...
-__global__ void colstats_kernel(const void* X, int dtype, int64_t m, int64_t n, int64_t ld, int64_t chunk_rows,
-                                double* psum, float* pmin, float* pmax) {
+// 8 consecutive elements of one row from column c (c + 8 <= n: vector loads).
+MDEV void load8(const void* X, int dtype, int64_t idx, float* v) {
+  if (dtype == METIS_BF16) {
+    const uint4 u = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(X) + idx);
+    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      v[2 * i] = __uint_as_float(w[i] << 16);
+      v[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+    }
+  } else {
+    const float4 a = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(X) + idx);
+    const float4 b = *reinterpret_cast<const float4*>(reinterpret_cast<const float*>(X) + idx + 4);
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+}
+
+// Block (column tile of 256, row chunk): warp w takes rows r0 + w, r0 + w + 8,
+// ...; lane l takes columns tile*256 + 8 l .. + 7 (16-byte loads, a warp
+// reads 512 contiguous bytes of a bf16 row), four rows' loads in flight at a
+// time.  Per column: a float64 sum in row order within the warp, then the
+// warps' sums in warp order; minimum and maximum.
+__global__ void __launch_bounds__(32 * kRowGroups) colstats_kernel(const void* X, int dtype, int64_t m, int64_t n,
+                                                                   int64_t ld, int64_t chunk_rows, double* psum,
+                                                                   float* pmin, float* pmax) {
   __shared__ double ssum[kRowGroups][kColsPerBlock];
   __shared__ float smin[kRowGroups][kColsPerBlock], smax[kRowGroups][kColsPerBlock];
-  const int x = threadIdx.x, y = threadIdx.y;
-  const int64_t c = static_cast<int64_t>(blockIdx.x) * kColsPerBlock + 2 * x;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
+  const int64_t c = static_cast<int64_t>(blockIdx.x) * kColsPerBlock + kColsPerThread * lane;
   const int64_t r0 = static_cast<int64_t>(blockIdx.y) * chunk_rows;
   const int64_t r1 = imin64(m, r0 + chunk_rows);
-  double s0 = 0.0, s1 = 0.0;
-  float mn0 = INFINITY, mn1 = INFINITY, mx0 = -INFINITY, mx1 = -INFINITY;
+  double sm[kColsPerThread];
+  float mn[kColsPerThread], mx[kColsPerThread];
+#pragma unroll
+  for (int j = 0; j < kColsPerThread; ++j) {
+    sm[j] = 0.0;
+    mn[j] = INFINITY;
+    mx[j] = -INFINITY;
+  }
+  const bool full = c + kColsPerThread <= n;
   if (c < n) {
-    const bool two = c + 1 < n;
-    for (int64_t r = r0 + y; r < r1; r += kRowGroups) {
-      float a, b = 0.f;
-      const int64_t idx = r * ld + c;
-      if (two) {
-        if (dtype == METIS_BF16) {
-          const uint32_t u = *reinterpret_cast<const uint32_t*>(reinterpret_cast<const __nv_bfloat16*>(X) + idx);
-          a = __uint_as_float(u << 16);
-          b = __uint_as_float(u & 0xFFFF0000u);
+    int64_t r = r0 + w;
+    for (; r + (kRowUnroll - 1) * kRowGroups < r1; r += kRowUnroll * kRowGroups) {
+      float v[kRowUnroll][kColsPerThread];
+#pragma unroll
+      for (int u = 0; u < kRowUnroll; ++u) {
+        const int64_t idx = (r + u * kRowGroups) * ld + c;
+        if (full) {
+          load8(X, dtype, idx, v[u]);
         } else {
-          const float2 f = *reinterpret_cast<const float2*>(reinterpret_cast<const float*>(X) + idx);
-          a = f.x;
-          b = f.y;
+#pragma unroll
+          for (int j = 0; j < kColsPerThread; ++j) v[u][j] = c + j < n ? load_elem(X, dtype, idx + j) : 0.f;
         }
-      } else {
-        a = load_elem(X, dtype, idx);
       }
-      s0 += a;
-      mn0 = fminf(mn0, a);
-      mx0 = fmaxf(mx0, a);
-      if (two) {
-        s1 += b;
-        mn1 = fminf(mn1, b);
-        mx1 = fmaxf(mx1, b);
+#pragma unroll
+      for (int u = 0; u < kRowUnroll; ++u) {
+#pragma unroll
+        for (int j = 0; j < kColsPerThread; ++j) {
+          sm[j] += v[u][j];
+          mn[j] = fminf(mn[j], v[u][j]);
+          mx[j] = fmaxf(mx[j], v[u][j]);
+        }
+      }
+    }
+    for (; r < r1; r += kRowGroups) {
+      float v[kColsPerThread];
+      const int64_t idx = r * ld + c;
+      if (full) {
+        load8(X, dtype, idx, v);
+      } else {
+#pragma unroll
+        for (int j = 0; j < kColsPerThread; ++j) v[j] = c + j < n ? load_elem(X, dtype, idx + j) : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < kColsPerThread; ++j) {
+        sm[j] += v[j];
+        mn[j] = fminf(mn[j], v[j]);
+        mx[j] = fmaxf(mx[j], v[j]);
       }
     }
   }
-  ssum[y][2 * x] = s0;
-  ssum[y][2 * x + 1] = s1;
-  smin[y][2 * x] = mn0;
-  smin[y][2 * x + 1] = mn1;
-  smax[y][2 * x] = mx0;
-  smax[y][2 * x + 1] = mx1;
+#pragma unroll
+  for (int j = 0; j < kColsPerThread; ++j) {
+    ssum[w][kColsPerThread * lane + j] = sm[j];
+    smin[w][kColsPerThread * lane + j] = mn[j];
+    smax[w][kColsPerThread * lane + j] = mx[j];
+  }
   __syncthreads();
-  const int t = y * 32 + x;
-  if (t < kColsPerBlock) {
-    const int64_t col = static_cast<int64_t>(blockIdx.x) * kColsPerBlock + t;
-    if (col < n) {
-      double s = 0.0;
-      float mn = INFINITY, mx = -INFINITY;
-      for (int g = 0; g < kRowGroups; ++g) {
-        s += ssum[g][t];
-        mn = fminf(mn, smin[g][t]);
-        mx = fmaxf(mx, smax[g][t]);
-      }
-      const int64_t o = static_cast<int64_t>(blockIdx.y) * n + col;
-      psum[o] = s;
-      pmin[o] = mn;
-      pmax[o] = mx;
+  const int t = threadIdx.x;   // one column of the tile
+  const int64_t col = static_cast<int64_t>(blockIdx.x) * kColsPerBlock + t;
+  if (col < n) {
+    double sum = 0.0;
+    float lo = INFINITY, hi = -INFINITY;
+    for (int g = 0; g < kRowGroups; ++g) {
+      sum += ssum[g][t];
+      lo = fminf(lo, smin[g][t]);
+      hi = fmaxf(hi, smax[g][t]);
     }
+    const int64_t o = static_cast<int64_t>(blockIdx.y) * n + col;
+    psum[o] = sum;
+    pmin[o] = lo;
+    pmax[o] = hi;
   }
 }
 
@@ -127,7 +169,7 @@ void launch_colstats(const void* X, int dtype, int64_t m, int64_t n, int64_t ld,
                      float* pmin, float* pmax, float* mean, unsigned* amax_bits, cudaStream_t s) {
   const int64_t nchunks = (m + chunk_rows - 1) / chunk_rows;
   const dim3 grid(static_cast<unsigned>((n + kColsPerBlock - 1) / kColsPerBlock), static_cast<unsigned>(nchunks));
-  colstats_kernel<<<grid, dim3(32, kRowGroups), 0, s>>>(X, dtype, m, n, ld, chunk_rows, psum, pmin, pmax);
+  colstats_kernel<<<grid, 32 * kRowGroups, 0, s>>>(X, dtype, m, n, ld, chunk_rows, psum, pmin, pmax);
   cudaMemsetAsync(amax_bits, 0, sizeof(unsigned), s);
   colstats_finalize_kernel<<<static_cast<unsigned>((n + 255) / 256), 256, 0, s>>>(
       psum, pmin, pmax, static_cast<int>(nchunks), m, n, mean, amax_bits);

@@ -293,6 +293,16 @@ void launch_tridiag(const double* C, int n, double* ws, cudaStream_t s) {
 // 2. one eigenpair per CTA (one warp)
 // ---------------------------------------------------------------------------
 
+// Sign of p as -1 / +1, or `prev` for a zero (bit tests: the fp64 compare
+// unit is far slower than the integer pipe).
+MDEV int sign_or(double p, int prev) {
+  const long long b = __double_as_longlong(p);
+  return (b << 1) == 0 ? prev : (b < 0 ? -1 : 1);
+}
+
+// Biased exponent field of |p|.
+MDEV int exp_field(double p) { return static_cast<int>((__double_as_longlong(p) >> 52) & 0x7FF); }
+
 // Number of eigenvalues of T below x (scaled T: |d|, |e| <= 1): sign changes
 // of the leading principal minors p_{-1} = 1, p_0, ..., p_{n-1}, with
 // p_i = (d_i - x) p_{i-1} - e_{i-1}^2 p_{i-2}; a zero minor takes the sign of
@@ -300,12 +310,8 @@ void launch_tridiag(const double* C, int n, double* ws, cudaStream_t s) {
 // every fourth step (|p| grows at most 5x per step), so nothing overflows.
 MDEV int sturm_count(const double* d, const double* e2, int n, double x) {
   double pm2 = 1.0, pm1 = d[0] - x;
-  int sg = 1, cnt = 0;
-  {
-    const int s = pm1 < 0.0 ? -1 : (pm1 > 0.0 ? 1 : sg);
-    cnt += s != sg;
-    sg = s;
-  }
+  int sg = sign_or(pm1, 1);
+  int cnt = sg != 1;
   // four steps per pass, their loads issued together ahead of the recurrence
   // (only the fma on p_{i-1} is on the dependent chain)
   int i = 1;
@@ -319,16 +325,16 @@ MDEV int sturm_count(const double* d, const double* e2, int n, double x) {
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const double p = fma(dd[u], pm1, -ff[u] * pm2);
-      const int s = p < 0.0 ? -1 : (p > 0.0 ? 1 : sg);
-      cnt += s != sg;
-      sg = s;
+      const int sv = sign_or(p, sg);
+      cnt += sv != sg;
+      sg = sv;
       pm2 = pm1;
       pm1 = p;
     }
     // scale (p_{i-1}, p_i) by 2^-e, e the exponent of the larger one (a
     // power of two: the signs, and so the count, are unchanged)
-    const long long bits = __double_as_longlong(fmax(fabs(pm1), fabs(pm2)));
-    const int ex = static_cast<int>((bits >> 52) & 0x7FF) - 1023;
+    const int ef = max(exp_field(pm1), exp_field(pm2));
+    const int ex = ef - 1023;
     if (ex > -1000) {
       const double sc = __longlong_as_double(static_cast<long long>(1023 - ex) << 52);
       pm1 *= sc;
@@ -337,9 +343,9 @@ MDEV int sturm_count(const double* d, const double* e2, int n, double x) {
   }
   for (; i < n; ++i) {
     const double p = fma(d[i] - x, pm1, -e2[i - 1] * pm2);
-    const int s = p < 0.0 ? -1 : (p > 0.0 ? 1 : sg);
-    cnt += s != sg;
-    sg = s;
+    const int sv = sign_or(p, sg);
+    cnt += sv != sg;
+    sg = sv;
     pm2 = pm1;
     pm1 = p;
   }

@@ -58,14 +58,17 @@ MDEV void nv_enc_table(float s_t, float* tab) {
   }
 }
 
-// quant_block_nv without the per-block reciprocal (taken from nv_enc_table).
-MDEV uint32_t quant_block_nv_tab(const float* v, float s_t, const float* enc_tab, uint64_t& packed) {
+// quant_block_nv without the per-block reciprocal (taken from nv_enc_table);
+// with SUM, the same dequantized sum as quant_block_nv<true>.
+template <bool SUM = false>
+MDEV uint32_t quant_block_nv_tab(const float* v, float s_t, const float* enc_tab, uint64_t& packed, float& dsum) {
   float a = 0.f;
 #pragma unroll
   for (int i = 0; i < 16; ++i) a = fmaxf(a, fabsf(v[i]));
   const float t = __fdiv_rn(__fdiv_rn(a, s_t), 6.f);
   const uint32_t dc = e4m3_code(t);
   packed = 0;
+  dsum = 0.f;
   if (dc == 0u) return dc;  // d(0) = 0 and every other code has d > 0
   const float enc = enc_tab[dc];
   float q[16];
@@ -73,7 +76,16 @@ MDEV uint32_t quant_block_nv_tab(const float* v, float s_t, const float* enc_tab
   for (int i = 0; i < 16; ++i) q[i] = __fmul_rn(v[i], enc);
   const uint32_t w0 = e2m1_pack8(q), w1 = e2m1_pack8(q + 8);
   packed = static_cast<uint64_t>(w0) | (static_cast<uint64_t>(w1) << 32);
+  if (SUM) {
+    const float csum = e2m1_sum8(w0) + e2m1_sum8(w1);
+    dsum = __fmul_rn(csum * e4m3_value(dc), s_t);
+  }
   return dc;
+}
+
+MDEV uint32_t quant_block_nv_tab(const float* v, float s_t, const float* enc_tab, uint64_t& packed) {
+  float unused;
+  return quant_block_nv_tab<false>(v, s_t, enc_tab, packed, unused);
 }
 
 // MXFP4 block of 32.  Returns the E8M0 scale code; writes 32 nibbles to

@@ -127,11 +127,14 @@ __global__ void __launch_bounds__(256) quantize_rows_kernel(QuantParams p) {
   }
 }
 
-// blocks along columns without inner sums (the common case): a grid-stride
-// loop over 32-element units (2 NVFP4 blocks or 1 MXFP4 block); the raw
-// bytes of a thread's next unit are loaded before its current unit is
-// quantized, so every thread keeps a load in flight while it computes.
-template <int FMT, bool BF16>
+// blocks along columns: a grid-stride loop over 32-element units (2 NVFP4
+// blocks or 1 MXFP4 block); the raw bytes of a thread's next unit are loaded
+// before its current unit is quantized, so every thread keeps a load in
+// flight while it computes.  With SUM (rows a multiple of 1024 elements, so a
+// warp's 32 units always lie in one row) the warp adds its units' dequantized
+// sums in a fixed tree order and lane 0 writes one partial per 1024 elements
+// (partial_sums[o][u / 32], ngroups = inner / 1024).
+template <int FMT, bool BF16, bool SUM, bool SUB>
 __global__ void __launch_bounds__(256) quantize_rows_fast_kernel(QuantParams p) {
   constexpr int kU = 32;
   constexpr int kVec = BF16 ? 4 : 8;  // 16-byte words per unit
@@ -157,6 +160,29 @@ __global__ void __launch_bounds__(256) quantize_rows_fast_kernel(QuantParams p) 
     return reinterpret_cast<const uint4*>(X + (o * p.ld + (unit - o * upr) * kU) * esize);
   };
   int64_t t = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
+  // with the grid stride a multiple of the units per row, a thread keeps one
+  // column unit for its whole loop, so its 32 column means are loaded once
+  const bool fixed_u = SUB && stride % upr == 0;
+  float subr[kU];
+  if constexpr (SUB) {
+    if (fixed_u && t < total) {
+      const float* sp = p.sub + (t % upr) * kU;
+      if ((reinterpret_cast<uintptr_t>(p.sub) & 15u) == 0) {
+        const float4* s4 = reinterpret_cast<const float4*>(sp);
+#pragma unroll
+        for (int k = 0; k < kU / 4; ++k) {
+          const float4 f = s4[k];
+          subr[4 * k] = f.x;
+          subr[4 * k + 1] = f.y;
+          subr[4 * k + 2] = f.z;
+          subr[4 * k + 3] = f.w;
+        }
+      } else {
+#pragma unroll
+        for (int j = 0; j < kU; ++j) subr[j] = sp[j];
+      }
+    }
+  }
   uint4 cur[kVec], nxt[kVec];
   if (t < total) {
     const uint4* a = src(t);
@@ -186,9 +212,14 @@ __global__ void __launch_bounds__(256) quantize_rows_fast_kernel(QuantParams p) 
         for (int i = 0; i < 4; ++i) v[4 * k + i] = __uint_as_float(w[i]);
       }
     }
-    if (p.sub) {
+    if constexpr (SUB) {
+      if (fixed_u) {
 #pragma unroll
-      for (int j = 0; j < kU; ++j) v[j] = __fsub_rn(v[j], p.sub[u * kU + j]);
+        for (int j = 0; j < kU; ++j) v[j] = __fsub_rn(v[j], subr[j]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < kU; ++j) v[j] = __fsub_rn(v[j], p.sub[u * kU + j]);
+      }
     }
     if (p.r_tap) {
       float* tp = p.r_tap + o * p.tap_ld + u * kU;
@@ -196,11 +227,13 @@ __global__ void __launch_bounds__(256) quantize_rows_fast_kernel(QuantParams p) 
       for (int j = 0; j < kU; ++j) tp[j] = v[j];
     }
     uint4* dst = reinterpret_cast<uint4*>(p.codes + o * (p.inner / 2) + u * (kU / 2));
-    float ds;
+    float ds = 0.f;
     if (FMT == METIS_NVFP4) {
       uint64_t pk0, pk1;
-      const uint32_t c0 = quant_block_nv_tab(v, s_t, enc_tab, pk0);
-      const uint32_t c1 = quant_block_nv_tab(v + 16, s_t, enc_tab, pk1);
+      float ds0, ds1;
+      const uint32_t c0 = quant_block_nv_tab<SUM>(v, s_t, enc_tab, pk0, ds0);
+      const uint32_t c1 = quant_block_nv_tab<SUM>(v + 16, s_t, enc_tab, pk1, ds1);
+      if (SUM) ds = ds0 + ds1;
       *dst = make_uint4(static_cast<uint32_t>(pk0), static_cast<uint32_t>(pk0 >> 32), static_cast<uint32_t>(pk1),
                         static_cast<uint32_t>(pk1 >> 32));
       *reinterpret_cast<uint16_t*>(p.scales + tc_scale_offset(o, 2 * u, p.scale_cols)) =
@@ -211,70 +244,110 @@ __global__ void __launch_bounds__(256) quantize_rows_fast_kernel(QuantParams p) 
       }
     } else {
       uint64_t pk[2];
-      const uint32_t c0 = quant_block_mx<false>(v, pk, ds);
+      const uint32_t c0 = quant_block_mx<SUM>(v, pk, ds);
       *dst = make_uint4(static_cast<uint32_t>(pk[0]), static_cast<uint32_t>(pk[0] >> 32),
                         static_cast<uint32_t>(pk[1]), static_cast<uint32_t>(pk[1] >> 32));
       p.scales[tc_scale_offset(o, u, p.scale_cols)] = static_cast<uint8_t>(c0);
       if (p.scales_linear) p.scales_linear[o * (p.inner / 32) + u] = static_cast<uint8_t>(c0);
+    }
+    if (SUM) {
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) ds += __shfl_xor_sync(0xFFFFFFFFu, ds, off);
+      if ((threadIdx.x & 31) == 0) p.partial_sums[o * (upr / 32) + u / 32] = ds;
     }
 #pragma unroll
     for (int k = 0; k < kVec; ++k) cur[k] = nxt[k];
   }
 }
 
-// blocks along rows: one CTA per 64-row x 64-column tile of X.  The tile is
-// read with 16-byte row-segment loads into shared memory; then each thread
-// quantizes one block of one column (four threads, or two for MXFP4, cover
-// a column's 64 rows, so their codes form one contiguous 32-byte segment).
+// blocks along rows: CTA (x, y) takes the 64-column strip x of X and a run of
+// consecutive 64-row groups [y G, y G + G).  Each group's 64 x 64 tile goes
+// through shared memory (coalesced 16-byte row loads in, a column per
+// thread group out); the next group's loads are issued into registers before
+// the current tile is quantized, so loads stay in flight while the CTA
+// computes.  Then each thread quantizes one block of one column (four
+// threads, or two for MXFP4, cover a column's 64 rows, so their codes form
+// one contiguous 32-byte segment).  With SUM the column's threads add their
+// blocks' dequantized sums (shuffles, fixed order) and the first keeps a
+// running sum over the run: one partial per column and run
+// (partial_sums[o][y], ngroups = runs).
 constexpr int kColTile = 64;
 
 template <int FMT, bool SUM>
-__global__ void __launch_bounds__(256) quantize_cols_kernel(QuantParams p) {
+__global__ void __launch_bounds__(256) quantize_cols_kernel(QuantParams p, int64_t run) {
   constexpr int kBlk = FMT == METIS_NVFP4 ? 16 : 32;
   constexpr int kPerCol = kColTile / kBlk;  // threads per column
+  constexpr int kSlots = kColTile * (kColTile / 8) / 256;  // 16-byte row segments per thread per tile
   __shared__ float tile[kColTile][kColTile + 1];
-  __shared__ float bsum[kColTile][kPerCol];
+  __shared__ float enc_tab[128];
   const float s_t = tensor_scale_of(p);
   if (FMT == METIS_NVFP4 && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0 && p.tensor_scale)
     *p.tensor_scale = s_t;
+  if (FMT == METIS_NVFP4) nv_enc_table(s_t, enc_tab);
   // p.outer = columns of X, p.inner = rows of X
   const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kColTile;
-  const int64_t g = blockIdx.y;
-  const int64_t r0 = g * kColTile;
-  const int nr = static_cast<int>(imin64(kColTile, p.inner - r0));
   const int nc = static_cast<int>(imin64(kColTile, p.outer - c0));
-  for (int e = threadIdx.x; e < kColTile * (kColTile / 8); e += blockDim.x) {
-    const int r = e >> 3, q = (e & 7) * 8;
-    float v[8];
-    if (r < nr && q + 8 <= nc) {
-      ld8(p.X, p.dtype, (r0 + r) * p.ld + c0 + q, v);
-    } else {
+  const int64_t ngr = (p.inner + kColTile - 1) / kColTile;
+  const int64_t g0 = static_cast<int64_t>(blockIdx.y) * run;
+  const int64_t g1 = imin64(ngr, g0 + run);
+  float raw[kSlots][8];
+  auto fetch = [&](int64_t g) {
+    const int64_t r0 = g * kColTile;
+    const int nr = static_cast<int>(imin64(kColTile, p.inner - r0));
 #pragma unroll
-      for (int j = 0; j < 8; ++j) v[j] = (r < nr && q + j < nc) ? ld1(p.X, p.dtype, (r0 + r) * p.ld + c0 + q + j) : 0.f;
-    }
+    for (int k = 0; k < kSlots; ++k) {
+      const int e = threadIdx.x + 256 * k;
+      const int r = e >> 3, q = (e & 7) * 8;
+      if (r < nr && q + 8 <= nc) {
+        ld8(p.X, p.dtype, (r0 + r) * p.ld + c0 + q, raw[k]);
+      } else {
 #pragma unroll
-    for (int j = 0; j < 8; ++j) {
-      if (p.sub && q + j < nc) v[j] = __fsub_rn(v[j], p.sub[c0 + q + j]);
-      tile[r][q + j] = v[j];
-      if (p.r_tap && r < nr && q + j < nc) p.r_tap[(r0 + r) * p.tap_ld + c0 + q + j] = v[j];
+        for (int j = 0; j < 8; ++j)
+          raw[k][j] = (r < nr && q + j < nc) ? ld1(p.X, p.dtype, (r0 + r) * p.ld + c0 + q + j) : 0.f;
+      }
     }
+  };
+  const int b = threadIdx.x % kPerCol, cc = threadIdx.x / kPerCol;  // this thread's block and column
+  float subc[kSlots][8];  // the column means of this thread's row segments
+#pragma unroll
+  for (int k = 0; k < kSlots; ++k) {
+    const int q = ((threadIdx.x + 256 * k) & 7) * 8;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) subc[k][j] = (p.sub && q + j < nc) ? p.sub[c0 + q + j] : 0.f;
   }
-  __syncthreads();
-  const int nb = nr / kBlk;
-  if (threadIdx.x < kColTile * kPerCol) {
-    const int b = threadIdx.x % kPerCol, cc = threadIdx.x / kPerCol;
-    if (cc < nc && b < nb) {
+  float colsum = 0.f;
+  if (g0 < g1) fetch(g0);
+  for (int64_t g = g0; g < g1; ++g) {
+    const int64_t r0 = g * kColTile;
+    const int nr = static_cast<int>(imin64(kColTile, p.inner - r0));
+    __syncthreads();  // the previous tile has been read (and the encode table is ready)
+#pragma unroll
+    for (int k = 0; k < kSlots; ++k) {
+      const int e = threadIdx.x + 256 * k;
+      const int r = e >> 3, q = (e & 7) * 8;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        float v = raw[k][j];
+        if (p.sub && q + j < nc) v = __fsub_rn(v, subc[k][j]);
+        tile[r][q + j] = v;
+        if (p.r_tap && r < nr && q + j < nc) p.r_tap[(r0 + r) * p.tap_ld + c0 + q + j] = v;
+      }
+    }
+    if (g + 1 < g1) fetch(g + 1);
+    __syncthreads();
+    const int nb = nr / kBlk;
+    float ds = 0.f;
+    if (threadIdx.x < kColTile * kPerCol && cc < nc && b < nb) {
       const int64_t o = c0 + cc;
       float v[kBlk];
 #pragma unroll
       for (int i = 0; i < kBlk; ++i) v[i] = tile[b * kBlk + i][cc];
-      float ds = 0.f;
       uint8_t* dst = p.codes + o * (p.inner / 2) + (r0 + b * kBlk) / 2;
       const int64_t sc_col = (r0 + b * kBlk) / kBlk;
       uint32_t code;
       if (FMT == METIS_NVFP4) {
         uint64_t pk;
-        code = quant_block_nv<SUM>(v, s_t, pk, ds);
+        code = quant_block_nv_tab<SUM>(v, s_t, enc_tab, pk, ds);
         *reinterpret_cast<uint2*>(dst) = make_uint2(static_cast<uint32_t>(pk), static_cast<uint32_t>(pk >> 32));
       } else {
         uint64_t pk[2];
@@ -284,17 +357,15 @@ __global__ void __launch_bounds__(256) quantize_cols_kernel(QuantParams p) {
       }
       p.scales[tc_scale_offset(o, sc_col, p.scale_cols)] = static_cast<uint8_t>(code);
       if (p.scales_linear) p.scales_linear[o * (p.inner / kBlk) + sc_col] = static_cast<uint8_t>(code);
-      if (SUM) bsum[cc][b] = ds;
+    }
+    if (SUM) {
+      // the column's kPerCol threads are adjacent lanes: add their block sums
+#pragma unroll
+      for (int off = 1; off < kPerCol; off <<= 1) ds += __shfl_xor_sync(0xFFFFFFFFu, ds, off);
+      colsum += ds;
     }
   }
-  if (SUM) {
-    __syncthreads();
-    if (threadIdx.x < nc) {
-      float s = 0.f;
-      for (int b = 0; b < nb; ++b) s += bsum[threadIdx.x][b];
-      p.partial_sums[(c0 + threadIdx.x) * p.ngroups + g] = s;
-    }
-  }
+  if (SUM && b == 0 && cc < nc) p.partial_sums[(c0 + cc) * p.ngroups + blockIdx.y] = colsum;
 }
 
 // max |x - sub| over the matrix into *out_bits (float bits, atomicMax).
@@ -353,12 +424,18 @@ __global__ void __launch_bounds__(256) amax_kernel(const void* X, int dtype, int
   }
 }
 
-__global__ void inner_sum_kernel(const float* partial, int64_t outer, int64_t ngroups, float* out) {
-  const int64_t o = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
-  if (o >= outer) return;
+// out[o] = sum of partial[o][0 .. ngroups): a warp per o, lanes strided over
+// the groups (coalesced), then a fixed tree order.
+__global__ void __launch_bounds__(256) inner_sum_kernel(const float* partial, int64_t outer, int64_t ngroups,
+                                                        float* out) {
+  const int64_t o = (blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (o >= outer) return;  // whole warps
   float s = 0.f;
-  for (int64_t g = 0; g < ngroups; ++g) s += partial[o * ngroups + g];
-  out[o] = s;
+  for (int64_t g = lane; g < ngroups; g += 32) s += partial[o * ngroups + g];
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xFFFFFFFFu, s, off);
+  if (lane == 0) out[o] = s;
 }
 
 }  // namespace
@@ -379,34 +456,64 @@ void launch_amax(const void* X, int dtype, int64_t rows, int64_t cols, int64_t l
 }
 
 template <int FMT, bool SUM>
-void launch_quantize_t(const QuantParams& p, int axis, int num_sms, cudaStream_t s) {
-  if (axis == 1 && !SUM) {
+void launch_quantize_t(QuantParams& p, int axis, int num_sms, cudaStream_t s) {
+  if (axis == 1 && (!SUM || p.inner % 1024 == 0)) {
+    if (SUM) p.ngroups = p.inner / 1024;  // one partial per warp of units
     // two or more units per thread, so the prefetch overlaps; no more CTAs
     // than are resident at once (the grid-stride loop is latency-bound, so a
     // second wave would add its full length)
     const int64_t units = p.outer * (p.inner / 32);
-    const void* k = p.dtype == METIS_BF16 ? reinterpret_cast<const void*>(quantize_rows_fast_kernel<FMT, true>)
-                                          : reinterpret_cast<const void*>(quantize_rows_fast_kernel<FMT, false>);
+    const bool bf = p.dtype == METIS_BF16, sub = p.sub != nullptr;
+    const void* k = bf ? (sub ? reinterpret_cast<const void*>(quantize_rows_fast_kernel<FMT, true, SUM, true>)
+                              : reinterpret_cast<const void*>(quantize_rows_fast_kernel<FMT, true, SUM, false>))
+                       : (sub ? reinterpret_cast<const void*>(quantize_rows_fast_kernel<FMT, false, SUM, true>)
+                              : reinterpret_cast<const void*>(quantize_rows_fast_kernel<FMT, false, SUM, false>));
     int per_sm = 0;
     if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, k, 256, 0) != cudaSuccess || per_sm < 1) per_sm = 1;
     int blocks = static_cast<int>(imin64((units + 511) / 512, static_cast<int64_t>(num_sms) * per_sm));
     if (blocks < 1) blocks = 1;
-    if (p.dtype == METIS_BF16)
-      quantize_rows_fast_kernel<FMT, true><<<blocks, 256, 0, s>>>(p);
+    if (p.sub) {
+      // a multiple of upr / gcd(upr, 256) CTAs makes the stride a multiple of
+      // the units per row (each thread then keeps one column unit)
+      int64_t a = p.inner / 32, b = 256;
+      while (b) {
+        const int64_t r = a % b;
+        a = b;
+        b = r;
+      }
+      const int64_t mult = (p.inner / 32) / a;
+      if (mult <= 4 * static_cast<int64_t>(num_sms) * per_sm)
+        blocks = static_cast<int>(imax64(mult, blocks / mult * mult));
+    }
+    if (bf && sub)
+      quantize_rows_fast_kernel<FMT, true, SUM, true><<<blocks, 256, 0, s>>>(p);
+    else if (bf)
+      quantize_rows_fast_kernel<FMT, true, SUM, false><<<blocks, 256, 0, s>>>(p);
+    else if (sub)
+      quantize_rows_fast_kernel<FMT, false, SUM, true><<<blocks, 256, 0, s>>>(p);
     else
-      quantize_rows_fast_kernel<FMT, false><<<blocks, 256, 0, s>>>(p);
+      quantize_rows_fast_kernel<FMT, false, SUM, false><<<blocks, 256, 0, s>>>(p);
   } else if (axis == 1) {
     const int64_t total = p.outer * p.ngroups;
     int blocks = static_cast<int>(imin64((total + 255) / 256, static_cast<int64_t>(num_sms) * 16));
     if (blocks < 1) blocks = 1;
     quantize_rows_kernel<FMT, SUM><<<blocks, 256, 0, s>>>(p);
   } else {
-    const dim3 grid(static_cast<unsigned>((p.outer + kColTile - 1) / kColTile), static_cast<unsigned>(p.ngroups));
-    quantize_cols_kernel<FMT, SUM><<<grid, 256, 0, s>>>(p);
+    // about one wave of CTAs (8 resident per SM), each over a run of row groups
+    const int64_t strips = (p.outer + kColTile - 1) / kColTile;
+    const int64_t ngr = (p.inner + kColTile - 1) / kColTile;
+    int64_t runs = (static_cast<int64_t>(num_sms) * 8 + strips - 1) / strips;
+    runs = runs < 1 ? 1 : (runs > ngr ? ngr : runs);
+    const int64_t run = (ngr + runs - 1) / runs;
+    runs = (ngr + run - 1) / run;
+    if (SUM) p.ngroups = runs;   // one partial per column and run
+    const dim3 grid(static_cast<unsigned>(strips), static_cast<unsigned>(runs));
+    quantize_cols_kernel<FMT, SUM><<<grid, 256, 0, s>>>(p, run);
   }
 }
 
-void launch_quantize(const QuantParams& p, int axis, int num_sms, cudaStream_t s) {
+void launch_quantize(const QuantParams& params, int axis, int num_sms, cudaStream_t s) {
+  QuantParams p = params;  // the launcher may regroup the partial sums
   const bool sum = p.partial_sums != nullptr;
   if (p.fmt == METIS_NVFP4) {
     if (sum)
@@ -420,7 +527,7 @@ void launch_quantize(const QuantParams& p, int axis, int num_sms, cudaStream_t s
       launch_quantize_t<METIS_MXFP4, false>(p, axis, num_sms, s);
   }
   if (p.partial_sums && p.inner_sum) {
-    inner_sum_kernel<<<static_cast<unsigned>((p.outer + 255) / 256), 256, 0, s>>>(
+    inner_sum_kernel<<<static_cast<unsigned>((p.outer * 32 + 255) / 256), 256, 0, s>>>(
         p.partial_sums, p.outer, p.ngroups, p.inner_sum);
   }
 }

@@ -185,61 +185,62 @@ MDEV void inverse_block_row(const double* L, double* X, double* T, int ld, int t
   __syncthreads();
 }
 
-// Warp 0: factor panel K (columns 4K .. 4K+3, rows 4K .. lp-1, held in P
-// as lp x 4) in place: a lane per row (rows r0 + lane + 32 q), the pivot row
-// broadcast by shuffles.  Writes L's columns, 1/sqrt(pivot) and sqrt(pivot).
-MDEV void factor_panel(int K, double* P, double* L, double* invd, double* sqd, const double* diag0, int lp,
-                       int ld, int lane) {
-  const int r0 = kTile * K;
-  double pr[4][kTile];  // rows r0 + lane + 32 q
-#pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int row = r0 + lane + 32 * q;
-#pragma unroll
-    for (int c = 0; c < kTile; ++c) pr[q][c] = row < lp ? P[row * kTile + c] : 0.0;
-  }
-  double rinv[kTile], rsq[kTile];
+// Factor the diagonal tile (K, K), held in registers by its owner (lower
+// triangle valid), in place: column c takes the pivot d = v[c][c], dropped
+// (1/sqrt = 0, the column of L zero) when it falls below kDropTol of its
+// original diagonal; otherwise L[a][c] = v[a][c] / sqrt(d) and the columns
+// right of it take the rank-1 update.  Writes L's diagonal block, 1/sqrt(d)
+// and sqrt(d).
+MDEV void factor_diag(double (&v)[kTile][kTile], int K, double* L, double* invd, double* sqd, const double* diag0,
+                      int ld) {
+  const int o = kTile * K;
 #pragma unroll
   for (int c = 0; c < kTile; ++c) {
-    const int gc = r0 + c;
-    const double d = __shfl_sync(0xFFFFFFFFu, pr[0][c], c);  // row gc lives in lane c, q = 0
-    double prow[kTile];
+    const double d = v[c][c];
+    const bool drop = !(diag0[o + c] > 0.0) || !(d > kDropTol * diag0[o + c]);
+    const double ri = drop ? 0.0 : rsqrt(d);
+    invd[o + c] = ri;
+    sqd[o + c] = d * ri;
+    double l[kTile];
 #pragma unroll
-    for (int cc = 0; cc < kTile; ++cc) prow[cc] = __shfl_sync(0xFFFFFFFFu, pr[0][cc], c);
-    const bool drop = !(diag0[gc] > 0.0) || !(d > kDropTol * diag0[gc]);
-    rinv[c] = drop ? 0.0 : rsqrt(d);
-    rsq[c] = d * rinv[c];
-    const double inv2 = rinv[c] * rinv[c];
+    for (int a = 0; a < kTile; ++a) l[a] = a > c ? v[a][c] * ri : 0.0;
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
-      const int row = r0 + lane + 32 * q;
-      if (row > gc) {
+    for (int a = c + 1; a < kTile; ++a)
 #pragma unroll
-        for (int cc = c + 1; cc < kTile; ++cc) pr[q][cc] = fma(-pr[q][c], prow[cc] * inv2, pr[q][cc]);
-      }
-    }
+      for (int b = c + 1; b <= a; ++b) v[a][b] = fma(-l[a], l[b], v[a][b]);
+#pragma unroll
+    for (int a = 0; a < kTile; ++a) L[(o + a) * ld + o + c] = a == c ? d * ri : l[a];
   }
-  if (lane < kTile) {
-    double ri = rinv[0], rs = rsq[0];
+}
+
+// Rows 4I .. 4I+3 of panel K (the owner's updated tile (I, K), I > K):
+// forward substitution with the panel's diagonal block of L,
+// L[r][c] = (v[r][c] - sum_{c' < c} L[r][c'] L[c][c']) / sqrt(pivot c), into
+// the panel buffer P (lp x 4) and L.
+MDEV void solve_rows(const double (&v)[kTile][kTile], int I, int K, double* P, double* L, const double* invd, int ld) {
+  const int o = kTile * K;
+  double dl[kTile][kTile], ri[kTile];
 #pragma unroll
-    for (int c = 1; c < kTile; ++c) {
-      ri = lane == c ? rinv[c] : ri;
-      rs = lane == c ? rsq[c] : rs;
-    }
-    invd[r0 + lane] = ri;
-    sqd[r0 + lane] = rs;
+  for (int c = 0; c < kTile; ++c) {
+    ri[c] = invd[o + c];
+#pragma unroll
+    for (int cp = 0; cp < c; ++cp) dl[c][cp] = L[(o + c) * ld + o + cp];
   }
 #pragma unroll
-  for (int q = 0; q < 4; ++q) {
-    const int row = r0 + lane + 32 * q;
-    if (row < lp) {
+  for (int a = 0; a < kTile; ++a) {
+    double lr[kTile];
 #pragma unroll
-      for (int c = 0; c < kTile; ++c) {
-        const int gc = r0 + c;
-        const double l = row == gc ? rsq[c] : (row > gc ? pr[q][c] * rinv[c] : 0.0);
-        P[row * kTile + c] = l;
-        L[row * ld + gc] = l;
-      }
+    for (int c = 0; c < kTile; ++c) {
+      double x = v[a][c];
+#pragma unroll
+      for (int cp = 0; cp < c; ++cp) x = fma(-lr[cp], dl[c][cp], x);
+      lr[c] = x * ri[c];
+    }
+    const int row = kTile * I + a;
+#pragma unroll
+    for (int c = 0; c < kTile; ++c) {
+      P[row * kTile + c] = lr[c];
+      L[row * ld + o + c] = lr[c];
     }
   }
 }
@@ -268,11 +269,11 @@ MDEV void panel_update(double (&v)[kTile][kTile], const double* P, int I, int J)
 // G = L L^T (with drops), then Rinv = L^-T (upper triangular, float32).
 //  Cholesky, right-looking by panels of 4 columns with look-ahead: thread
 //  32 + T owns the 4 x 4 tile (I, J), I >= J, of the lower triangle in
-//  registers; panel K sits in shared memory.  Per panel, two barriers:
-//    (1) the tiles of column K + 1 take the rank-4 update of panel K and
-//        write themselves into the next panel buffer;
-//    (2) warp 0 factors panel K + 1 while every other tile right of it
-//        takes the update of panel K.
+//  registers; panel K's columns of L sit in shared memory.  Per panel K + 1,
+//  two barriers:
+//    (A) every tile right of panel K takes its rank-4 update; the owner of
+//        the diagonal tile (K+1, K+1) then factors it at once;
+//    (B) the owners of the tiles below it solve their rows of panel K + 1.
 //  Inverse: X = L^-1 by 16 x 16 blocks (see below).
 __global__ void __launch_bounds__(kSmallThreads, 1) cholesky_inv_kernel(const double* G, int lp, float* Rinv) {
   extern __shared__ double sm[];
@@ -300,31 +301,21 @@ __global__ void __launch_bounds__(kSmallThreads, 1) cholesky_inv_kernel(const do
 #pragma unroll
       for (int a = 0; a < kTile; ++a) diag0[kTile * I + a] = v[a][a];
     }
-    if (J == 0) {
-#pragma unroll
-      for (int a = 0; a < kTile; ++a)
-#pragma unroll
-        for (int b = 0; b < kTile; ++b) pan[(kTile * I + a) * kTile + b] = v[a][b];
-    }
   }
   __syncthreads();
-  if (warp == 0) factor_panel(0, pan, L, invd, sqd, diag0, lp, ld, lane);
+  if (owner && I == 0 && J == 0) factor_diag(v, 0, L, invd, sqd, diag0, ld);
+  __syncthreads();
+  if (owner && J == 0 && I > 0) solve_rows(v, I, 0, pan, L, invd, ld);
   __syncthreads();
   for (int K = 0; K + 1 < nb; ++K) {
     const double* P = pan + (K & 1) * 4 * lp;
     double* Pn = pan + ((K + 1) & 1) * 4 * lp;
-    if (owner && J == K + 1) {
+    if (owner && J > K) {
       panel_update(v, P, I, J);
-#pragma unroll
-      for (int a = 0; a < kTile; ++a)
-#pragma unroll
-        for (int b = 0; b < kTile; ++b) Pn[(kTile * I + a) * kTile + b] = v[a][b];
+      if (I == K + 1 && J == K + 1) factor_diag(v, K + 1, L, invd, sqd, diag0, ld);
     }
     __syncthreads();
-    if (warp == 0)
-      factor_panel(K + 1, Pn, L, invd, sqd, diag0, lp, ld, lane);
-    else if (owner && J > K + 1)
-      panel_update(v, P, I, J);
+    if (owner && J == K + 1 && I > K + 1) solve_rows(v, I, K + 1, Pn, L, invd, ld);
     __syncthreads();
   }
   // X = L^-1 by 16 x 16 blocks: the diagonal blocks are inverted by one warp
