@@ -362,7 +362,10 @@ METIS_API metis_status metis_linear_bwd(const metis_operand* dY_n, const metis_o
  *   R_cols   optional FP4 of the same residual, blocks along m (outer n).
  *   R_f32    optional device m x n float tap.
  * NVFP4 takes the residual's tensor maximum from the column minima and maxima
- * (exact: rounding is monotonic), so X is read twice in total.
+ * (exact: rounding is monotonic), so X is read once for the statistics and
+ * once per requested residual axis.  dev_status (device int32, may be NULL):
+ * a bounded wait of the TMA-fed bf16 kernels that gives up ORs in
+ * METIS_DEV_TIMEOUT.
  */
 METIS_API metis_status averis_split(const void* X, int32_t dtype, int64_t m, int64_t n, int64_t ld,
                           int32_t fmt, float* mean, metis_fp4_tensor* mean_q,

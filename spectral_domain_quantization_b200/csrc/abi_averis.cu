@@ -21,8 +21,7 @@ struct AverisBuffers {
   unsigned* amax;
 };
 
-AverisBuffers carve_averis(int64_t m, int64_t n, int64_t chunk_rows, Carver& ws) {
-  const int64_t nchunks = (m + chunk_rows - 1) / chunk_rows;
+AverisBuffers carve_averis(int64_t nchunks, int64_t n, Carver& ws) {
   AverisBuffers b;
   b.psum = ws.take<double>(static_cast<size_t>(nchunks) * n);
   b.pmin = ws.take<float>(static_cast<size_t>(nchunks) * n);
@@ -38,7 +37,6 @@ extern "C" metis_status averis_split(const void* X, int32_t dtype, int64_t m, in
                                      metis_fp4_tensor* R_cols, float* R_f32, void* workspace,
                                      size_t* workspace_bytes, int32_t* dev_status, void* stream) {
   if (!workspace_bytes || !mean) return METIS_ERR_NULL;
-  (void)dev_status;
   METIS_TRY(validate_dense(X, dtype, m, n, ld));
   if (!valid_fmt(fmt)) return METIS_ERR_ARG;
   if ((reinterpret_cast<uintptr_t>(mean) & 15u) != 0) return METIS_ERR_ALIGN;
@@ -46,11 +44,11 @@ extern "C" metis_status averis_split(const void* X, int32_t dtype, int64_t m, in
   if (R_rows) METIS_TRY(check_fp4(R_rows, m, n, fmt));
   if (R_cols) METIS_TRY(check_fp4(R_cols, n, m, fmt));
   const int sms = device_sm_count();
-  const int64_t chunk_rows = colstats_chunk_rows(m, n, sms);
+  const int64_t nchunks = colstats_chunks(X, dtype, m, n, ld, sms);
   size_t need;
   {
     Carver c(nullptr);
-    carve_averis(m, n, chunk_rows, c);
+    carve_averis(nchunks, n, c);
     need = c.used;
     if (mean_q) need += quantize_workspace(mean_q);
     if (R_rows) need += quantize_workspace(R_rows);
@@ -64,8 +62,8 @@ extern "C" metis_status averis_split(const void* X, int32_t dtype, int64_t m, in
   if (!device_is_sm100()) return METIS_ERR_UNSUPPORTED;
   const cudaStream_t s = static_cast<cudaStream_t>(stream);
   Carver ws(workspace);
-  const AverisBuffers b = carve_averis(m, n, chunk_rows, ws);
-  launch_colstats(X, dtype, m, n, ld, chunk_rows, b.psum, b.pmin, b.pmax, mean, b.amax, s);
+  const AverisBuffers b = carve_averis(nchunks, n, ws);
+  launch_colstats(X, dtype, m, n, ld, sms, b.psum, b.pmin, b.pmax, mean, b.amax, dev_status, s);
   if (mean_q) METIS_TRY(enqueue_quantize(mean, METIS_F32, 1, n, n, 1, nullptr, mean_q, nullptr, nullptr, ws, s));
   bool tapped = false;
   if (R_rows) {

@@ -329,8 +329,18 @@ __host__ __device__ inline float e2m1_value(uint32_t code) {
   return (code & 8u) ? -v : v;
 }
 
-// E4M3 code of t >= 0: round to nearest even, saturating at 448 (0x7E).
+// E4M3 code of t >= 0 by the hardware conversion (round to nearest even,
+// saturating finite values and infinity at 448 = 0x7E): the same code as
+// e4m3_code_ref below for every t >= 0.
 MDEV uint32_t e4m3_code(float t) {
+  uint16_t d;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(d) : "f"(0.f), "f"(t));
+  return d & 0xFFu;
+}
+
+// E4M3 code of t >= 0: round to nearest even, saturating at 448 (0x7E),
+// written out from the format's definition.
+MDEV uint32_t e4m3_code_ref(float t) {
   if (!(t > 0.f)) return 0u;
   if (t >= 464.f) return 0x7Eu;  // half-way to the non-finite 480 and above
   const uint32_t bits = __float_as_uint(t);

@@ -132,10 +132,15 @@ MDEV void tri_step(double (&a)[NH], TriShared<NH>& sh, const EigScratch& S, int 
     const double x0 = cur[j + 1].x;
     double alpha = x0, beta = 0.0, v0 = 0.0;
     if (sg > 0.0) {
-      const double nrm = sqrt(fma(x0, x0, sg));
+      // |x| = s rsqrt(s), s = |x|^2, and beta = 2 / (v0^2 + sg) =
+      // 1 / (|x| (|x| + |x0|)): two reciprocal square roots in place of a
+      // square root and a division on this warp's chain
+      const double s2 = fma(x0, x0, sg);
+      const double nrm = s2 * rsqrt(s2);
       alpha = x0 >= 0.0 ? -nrm : nrm;
-      v0 = x0 - alpha;
-      beta = 2.0 / fma(v0, v0, sg);
+      v0 = x0 - alpha;                                   // sign(x0) (|x0| + |x|)
+      const double r2 = rsqrt(nrm * (nrm + fabs(x0)));
+      beta = r2 * r2;
     }
     if (lane == 0) {
       sh.refl[0] = beta;

@@ -12,12 +12,20 @@ MDEV float nv_tensor_scale(float alpha) {
   return alpha == 0.f ? 1.f : __fdiv_rn(alpha, 2688.f);
 }
 
-// Sum of the 8 E2M1 values packed in w, as a multiple of 0.5 (exact).
+// Sum of the 8 E2M1 values packed in w, as a multiple of 0.5 (exact), in
+// integer arithmetic: a byte permute looks up twice each code's magnitude
+// {0, 1, 2, 3, 4, 6, 8, 12} from an 8-byte table (selected by the code's 3
+// magnitude bits), a second permute turns each sign bit into a +1 / -1 byte,
+// and two signed 4-way byte dot products add the lot (twice the sum).
 MDEV float e2m1_sum8(uint32_t w) {
-  float s = 0.f;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) s += e2m1_value((w >> (4 * i)) & 15u);
-  return s;
+  constexpr uint32_t kMagLo = 0x03020100u, kMagHi = 0x0C080604u, kSign = 0x0000FF01u;
+  const uint32_t mlo = __byte_perm(kMagLo, kMagHi, w & 0x7777u);
+  const uint32_t mhi = __byte_perm(kMagLo, kMagHi, (w >> 16) & 0x7777u);
+  const uint32_t slo = __byte_perm(kSign, 0u, (w >> 3) & 0x1111u);
+  const uint32_t shi = __byte_perm(kSign, 0u, (w >> 19) & 0x1111u);
+  const int twice = __dp4a(static_cast<int>(mhi), static_cast<int>(shi),
+                           __dp4a(static_cast<int>(mlo), static_cast<int>(slo), 0));
+  return static_cast<float>(twice) * 0.5f;
 }
 
 // NVFP4 block of 16.  Returns the E4M3 scale code; writes 16 nibbles to

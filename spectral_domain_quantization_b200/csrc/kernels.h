@@ -34,5 +34,10 @@ void launch_amax(const void* X, int dtype, int64_t rows, int64_t cols, int64_t l
                  unsigned* out_bits, int num_sms, cudaStream_t s);
 // axis 1: blocks along X's columns (outer = rows); axis 0: along rows.
 void launch_quantize(const QuantParams& p, int axis, int num_sms, cudaStream_t s);
+// The TMA-fed quantizer (quantize_tma.cu) for bf16 X: whether it takes this
+// call, and its launch (regroups the partial sums itself).
+bool quantize_tma_ok(const QuantParams& p, int axis, int sms);
+int64_t quantize_tma_groups(const QuantParams& p, int axis, int sms);
+void launch_quantize_tma(QuantParams p, int axis, int sms, int32_t* dev_status, cudaStream_t s);
 
 }  // namespace metis

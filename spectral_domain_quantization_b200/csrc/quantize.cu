@@ -515,6 +515,14 @@ void launch_quantize_t(QuantParams& p, int axis, int num_sms, cudaStream_t s) {
 void launch_quantize(const QuantParams& params, int axis, int num_sms, cudaStream_t s) {
   QuantParams p = params;  // the launcher may regroup the partial sums
   const bool sum = p.partial_sums != nullptr;
+  if (quantize_tma_ok(p, axis, num_sms)) {
+    if (sum) p.ngroups = quantize_tma_groups(p, axis, num_sms);
+    launch_quantize_tma(p, axis, num_sms, nullptr, s);
+    if (p.partial_sums && p.inner_sum)
+      inner_sum_kernel<<<static_cast<unsigned>((p.outer * 32 + 255) / 256), 256, 0, s>>>(
+          p.partial_sums, p.outer, p.ngroups, p.inner_sum);
+    return;
+  }
   if (p.fmt == METIS_NVFP4) {
     if (sum)
       launch_quantize_t<METIS_NVFP4, true>(p, axis, num_sms, s);

@@ -24,10 +24,13 @@ namespace {
 
 constexpr double kDropTol = 1e-12;
 
-// Gram partial of a row block held in shared memory (rows x cols floats with
-// row stride ld, cols a multiple of 4): out[i][j] for all i, j (symmetric).
-// Each thread accumulates a 4 x 4 tile (16 independent float64 chains).
-MDEV void gram_block(const float* ys, int rows, int cols, int ld, double* out) {
+// Gram partial of a row block held in shared memory (rows x cols values of
+// type T with row stride ld, cols a multiple of 4): the upper 4 x 4 tiles
+// (bi <= bj), tile p written as 16 contiguous doubles out[16 p + 4 x + y] =
+// sum_r Y[r][4 bi + x] Y[r][4 bj + y], p counting the pairs bi-major.  Each
+// thread accumulates one tile (16 independent float64 chains).
+template <typename T>
+MDEV void gram_block(const T* ys, int rows, int cols, int ld, double* out) {
   const int nb = cols / 4;
   const int npairs = nb * (nb + 1) / 2;
   for (int pidx = threadIdx.x; pidx < npairs; pidx += blockDim.x) {
@@ -43,7 +46,7 @@ MDEV void gram_block(const float* ys, int rows, int cols, int ld, double* out) {
 #pragma unroll
       for (int y = 0; y < 4; ++y) acc[x][y] = 0.0;
     for (int r = 0; r < rows; ++r) {
-      const float* row = ys + r * ld;
+      const T* row = ys + r * ld;
       double a[4], b[4];
 #pragma unroll
       for (int x = 0; x < 4; ++x) {
@@ -55,25 +58,23 @@ MDEV void gram_block(const float* ys, int rows, int cols, int ld, double* out) {
 #pragma unroll
         for (int y = 0; y < 4; ++y) acc[x][y] = fma(a[x], b[y], acc[x][y]);
     }
+    double* o = out + 16 * pidx;
 #pragma unroll
     for (int x = 0; x < 4; ++x)
 #pragma unroll
-      for (int y = 0; y < 4; ++y) {
-        out[(4 * bi + x) * cols + 4 * bj + y] = acc[x][y];
-        out[(4 * bj + y) * cols + 4 * bi + x] = acc[x][y];
-      }
+      for (int y = 0; y < 4; ++y) o[4 * x + y] = acc[x][y];
   }
 }
 
 constexpr int kGramRows = 32;
 
 // Float64 Gram partial of each 32-row block of Y (rows x lp float32, row
-// stride lp): the block staged in shared memory, then 4 x 4 register tiles
-// over the rows in order.  One thread per 4 x 4 tile pair (blockDim covers
-// (lp/4)(lp/4+1)/2 pairs).
+// stride lp): the block staged in shared memory as float64 (each value
+// converted once), then 4 x 4 register tiles over the rows in order.  One
+// thread per 4 x 4 tile pair (blockDim covers (lp/4)(lp/4+1)/2 pairs).
 __global__ void __launch_bounds__(1024) gram_kernel(const float* __restrict__ Y, int64_t rows, int lp,
                                                     double* __restrict__ gpart) {
-  extern __shared__ float ys[];  // kGramRows x (lp + 1)
+  extern __shared__ double ys[];  // kGramRows x (lp + 1)
   const int ld = lp + 1;
   const int q4 = lp / 4;
   const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kGramRows;
@@ -81,7 +82,7 @@ __global__ void __launch_bounds__(1024) gram_kernel(const float* __restrict__ Y,
   for (int e = threadIdx.x; e < kGramRows * q4; e += blockDim.x) {
     const int r = e / q4, c4 = e - r * q4;
     const float4 x = r < nr ? reinterpret_cast<const float4*>(Y)[(r0 + r) * q4 + c4] : make_float4(0.f, 0.f, 0.f, 0.f);
-    float* d = ys + r * ld + 4 * c4;
+    double* d = ys + r * ld + 4 * c4;
     d[0] = x.x;
     d[1] = x.y;
     d[2] = x.z;
@@ -91,27 +92,39 @@ __global__ void __launch_bounds__(1024) gram_kernel(const float* __restrict__ Y,
   gram_block(ys, nr, lp, ld, gpart + static_cast<int64_t>(blockIdx.x) * lp * lp);
 }
 
-// Sum of the block partials: a CTA takes 32 consecutive entries (coalesced
-// 256-byte rows of each partial); its 8 warps take every 8th block, then the
-// 8 partial sums are added in warp order (deterministic).
+// Sum of the block partials (packed upper tiles, block stride lp^2): a CTA
+// takes 32 consecutive packed entries (coalesced 256-byte runs of each
+// partial); its 8 warps take every 8th block, the 8 sums are added in warp
+// order (deterministic), and each entry goes to G[i][j] and G[j][i].
 constexpr int kReduceGroups = 8;
-__global__ void __launch_bounds__(256) gram_reduce_kernel(const double* __restrict__ gpart, int nblocks, int n2,
+__global__ void __launch_bounds__(256) gram_reduce_kernel(const double* __restrict__ gpart, int nblocks, int lp,
                                                           double* __restrict__ G) {
   __shared__ double part[kReduceGroups][32];
   const int lane = threadIdx.x & 31, grp = threadIdx.x >> 5;
+  const int nb = lp / 4;
+  const int npk = 8 * nb * (nb + 1);   // packed entries: 16 per tile pair
   const int e = blockIdx.x * 32 + lane;
+  const int64_t stride = static_cast<int64_t>(lp) * lp;
   double s = 0.0;
-  if (e < n2) {
+  if (e < npk) {
 #pragma unroll 8
-    for (int b = grp; b < nblocks; b += kReduceGroups) s += gpart[static_cast<int64_t>(b) * n2 + e];
+    for (int b = grp; b < nblocks; b += kReduceGroups) s += gpart[static_cast<int64_t>(b) * stride + e];
   }
   part[grp][lane] = s;
   __syncthreads();
-  if (grp == 0 && e < n2) {
+  if (grp == 0 && e < npk) {
     double t = 0.0;
 #pragma unroll
     for (int g = 0; g < kReduceGroups; ++g) t += part[g][lane];
-    G[e] = t;
+    int pidx = e >> 4, bi = 0;
+    while (pidx >= nb - bi) {
+      pidx -= nb - bi;
+      ++bi;
+    }
+    const int bj = bi + pidx, x = (e >> 2) & 3, y = e & 3;
+    const int i = 4 * bi + x, j = 4 * bj + y;
+    G[i * lp + j] = t;
+    G[j * lp + i] = t;
   }
 }
 
@@ -434,7 +447,7 @@ __global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) {
       }
     }
   }
-  if (a.gpart) gram_block(Out, nr, a.kout, a.kout + 1, a.gpart + static_cast<int64_t>(blockIdx.x) * a.kout * a.kout);
+  if (a.gpart) gram_block<float>(Out, nr, a.kout, a.kout + 1, a.gpart + static_cast<int64_t>(blockIdx.x) * a.kout * a.kout);
 }
 
 // Factor matrices from the sorted eigen-decomposition of the core Gram:
@@ -521,13 +534,14 @@ void launch_gram(const float* Y, int64_t rows, int lp, double* gpart, double* G,
   const int nb = static_cast<int>(gram_blocks(rows));
   const int pairs = (lp / 4) * (lp / 4 + 1) / 2;
   const int threads = (pairs + 31) / 32 * 32;
-  gram_kernel<<<nb, threads, kGramRows * (lp + 1) * sizeof(float), s>>>(Y, rows, lp, gpart);
+  gram_kernel<<<nb, threads, kGramRows * (lp + 1) * sizeof(double), s>>>(Y, rows, lp, gpart);
   launch_gram_reduce(gpart, nb, lp, G, s);
 }
 
 void launch_gram_reduce(const double* gpart, int nblocks, int lp, double* G, cudaStream_t s) {
-  const int n2 = lp * lp;
-  gram_reduce_kernel<<<(n2 + 31) / 32, 32 * kReduceGroups, 0, s>>>(gpart, nblocks, n2, G);
+  const int nb = lp / 4;
+  const int npk = 8 * nb * (nb + 1);
+  gram_reduce_kernel<<<(npk + 31) / 32, 32 * kReduceGroups, 0, s>>>(gpart, nblocks, lp, G);
 }
 
 void launch_cholesky_inv(const double* G, int lp, float* Rinv, cudaStream_t s) {
