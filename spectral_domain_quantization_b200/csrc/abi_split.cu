@@ -394,7 +394,8 @@ extern "C" metis_status metis_split(const void* A, int32_t dtype, int64_t m, int
     au.kout = p.k;
     au.out = U;
     au.out_ld = p.k;
-    launch_apply(au, s);
+    au.bmax = b.bmax;   // U's column maxima per 32-row block, for the sign convention
+    au.bidx = b.bidx;
     ApplyArgs av{};
     av.in = b.Zn;
     av.rows = n;
@@ -404,7 +405,7 @@ extern "C" metis_status metis_split(const void* A, int32_t dtype, int64_t m, int
     av.kout = p.k;
     av.out = V;
     av.out_ld = p.k;
-    launch_apply(av, s);
+    launch_apply2(au, av, s);
   } else {
     // V_s = Z W_k / sigma (n x k, stored with width kq and as bf16 hi/lo^T)
     cudaMemsetAsync(b.Vs, 0, static_cast<size_t>(n) * p.kq * sizeof(float), s);
@@ -436,7 +437,8 @@ extern "C" metis_status metis_split(const void* A, int32_t dtype, int64_t m, int
     au.kout = p.k;
     au.out = U;
     au.out_ld = p.k;
-    launch_apply(au, s);
+    au.bmax = b.bmax;
+    au.bidx = b.bidx;
     ApplyArgs av{};
     av.in = b.Vs;
     av.rows = n;
@@ -446,10 +448,10 @@ extern "C" metis_status metis_split(const void* A, int32_t dtype, int64_t m, int
     av.kout = p.k;
     av.out = V;
     av.out_ld = p.k;
-    launch_apply(av, s);
+    launch_apply2(au, av, s);
   }
   METIS_TRY(step_status("factors"));
-  launch_signs(U, m, V, n, p.k, b.bmax, b.bidx, b.sign, sms, s);
+  launch_signs_from_blocks(U, m, V, n, p.k, b.bmax, b.bidx, b.sign, s);
   METIS_TRY(step_status("signs"));
   const bool residual = R_rows || R_cols || R_f32;
   cudaMemsetAsync(b.amax, 0, 3 * sizeof(unsigned), s);  // [0] |U|, [1] |V|, [2] |R|

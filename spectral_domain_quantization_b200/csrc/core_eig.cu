@@ -13,8 +13,8 @@
 //      symmetric tridiagonal T (diagonal d, off-diagonal e), keeping the
 //      reflectors; A's rows held in registers by thread pairs, two barriers
 //      per column.
-//   2. core_vector_kernel (one CTA of one warp per eigenvalue): the
-//      eigenvalue by multisection on Sturm counts (32 points per round, the
+//   2. core_vector_kernel (one CTA of four warps per eigenvalue): the
+//      eigenvalue by multisection on Sturm counts (128 points per round, the
 //      counts from the division-free determinant recurrence with power-of-two
 //      rescaling), then its eigenvector from the twisted factorization of
 //      T - lambda I (the twist at the smallest |gamma_r|), normalised and
@@ -357,18 +357,65 @@ MDEV int sturm_count(const double* d, const double* e2, int n, double x) {
   return cnt;
 }
 
-__global__ void __launch_bounds__(32) core_vector_kernel(int n, double* ws, int max_rounds, int32_t* dev_status) {
+constexpr int kVecWarps = 4;   // warps per eigenvalue CTA
+constexpr int kWY = 8;         // reflectors per block of the back-transformation
+constexpr int kMaxBlocks = (kMaxN + kWY - 1) / kWY;
+
+// T of the block of reflectors H_j0 ... H_j0+b-1 (columns v_j of V, the j-th
+// row of Vs), as in LAPACK's larft (forward, columnwise): H_j0 ... = I -
+// V T V^T with T upper triangular, T[i][i] = beta_i and T[0:i, i] = -beta_i
+// T[0:i, 0:i] (V[:, 0:i]^T v_i).  One warp; lanes stride the vector entries.
+MDEV void wy_block(const double* Vs, const double* bs, int n, int j0, int b, double (*T)[kWY]) {
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) T[0][0] = bs[j0];
+  __syncwarp();
+  for (int i = 1; i < b; ++i) {
+    const double* vi = Vs + (j0 + i) * n;
+    double dot[kWY];
+#pragma unroll
+    for (int c = 0; c < kWY; ++c) dot[c] = 0.0;
+    for (int t = lane; t < n; t += 32) {
+      const double x = vi[t];
+#pragma unroll
+      for (int c = 0; c < kWY; ++c)
+        if (c < i) dot[c] = fma(Vs[(j0 + c) * n + t], x, dot[c]);
+    }
+#pragma unroll
+    for (int c = 0; c < kWY; ++c)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) dot[c] += __shfl_xor_sync(0xFFFFFFFFu, dot[c], o);
+    const double beta = bs[j0 + i];
+    if (lane < i) {
+      double y = 0.0;   // (T[0:i, 0:i] dot)[lane], upper triangular: columns lane .. i-1
+#pragma unroll
+      for (int c = 0; c < kWY; ++c)
+        if (c >= lane && c < i) y = fma(T[lane][c], dot[c], y);
+      T[lane][i] = -beta * y;
+    }
+    if (lane == 0) T[i][i] = beta;
+    __syncwarp();
+  }
+}
+
+__global__ void __launch_bounds__(32 * kVecWarps) core_vector_kernel(int n, double* ws, int max_rounds,
+                                                                     int32_t* dev_status) {
   __shared__ double d[kMaxN], e[kMaxN], e2[kMaxN], dp[kMaxN], dm[kMaxN], lp[kMaxN], um[kMaxN], z[kMaxN];
   __shared__ __align__(16) double bs[kMaxN];
   extern __shared__ __align__(16) double Vs[];  // n x n reflectors
   __shared__ uint64_t vbar;
   __shared__ int vabort;
+  __shared__ double interval[2];                // the Gershgorin interval, by warp 0
+  __shared__ int scaled;                        // T != 0 (the multisection runs)
+  __shared__ unsigned masks[2][kVecWarps];      // per round parity: each warp's ballot
+  __shared__ double part[2][kVecWarps][kWY];    // per block parity: each warp's partial dot products
+  __shared__ double Tw[kMaxBlocks][kWY][kWY];    // T of each block of kWY reflectors
   const EigScratch S = scratch(ws, n);
-  const int lane = threadIdx.x, idx = blockIdx.x;  // eigenvalue idx in ascending order
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int idx = blockIdx.x;  // eigenvalue idx in ascending order
   // the reflectors and their betas come in by one bulk copy each, started
   // now so that they land while the eigenvalue is found
   const uint32_t vbytes = static_cast<uint32_t>(n) * n * sizeof(double);
-  if (lane == 0) {
+  if (tid == 0) {
     vabort = 0;
     mbar_init(&vbar, 1);
     fence_barrier_init();
@@ -376,187 +423,242 @@ __global__ void __launch_bounds__(32) core_vector_kernel(int n, double* ws, int 
     bulk_load(Vs, S.V, vbytes, &vbar);
     bulk_load(bs, S.beta, static_cast<uint32_t>(n) * sizeof(double), &vbar);
   }
-  __syncwarp();
-  // scale T by a power of two so that |d|, |e| <= 1
-  double mx = 0.0;
-  for (int i = lane; i < n; i += 32) {
-    mx = fmax(mx, fabs(S.d[i]));
-    if (i + 1 < n) mx = fmax(mx, fabs(S.e[i]));
-  }
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-  if (mx == 0.0) {  // T = 0: every unit vector is an eigenvector
-    for (int i = lane; i < n; i += 32) z[i] = i == idx ? 1.0 : 0.0;
-  }
   int ex = 0;
-  double lam = 0.0;
-  if (mx > 0.0) {
-    frexp(mx, &ex);  // mx < 2^ex
+  if (warp == 0) {
+    // scale T by a power of two so that |d|, |e| <= 1
+    double mx = 0.0;
     for (int i = lane; i < n; i += 32) {
-      d[i] = ldexp(S.d[i], -ex);
-      const double ei = i + 1 < n ? ldexp(S.e[i], -ex) : 0.0;
-      e[i] = ei;
-      e2[i] = ei * ei;
-    }
-    __syncwarp();
-    // Gershgorin interval
-    double lo = 1e300, hi = -1e300;
-    for (int i = lane; i < n; i += 32) {
-      const double r = fabs(e[i]) + (i > 0 ? fabs(e[i - 1]) : 0.0);
-      lo = fmin(lo, d[i] - r);
-      hi = fmax(hi, d[i] + r);
+      mx = fmax(mx, fabs(S.d[i]));
+      if (i + 1 < n) mx = fmax(mx, fabs(S.e[i]));
     }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      lo = fmin(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
-      hi = fmax(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
+    for (int o = 16; o > 0; o >>= 1) mx = fmax(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+    if (mx == 0.0) {  // T = 0: every unit vector is an eigenvector
+      for (int i = lane; i < n; i += 32) z[i] = i == idx ? 1.0 : 0.0;
+    } else {
+      frexp(mx, &ex);  // mx < 2^ex
+      for (int i = lane; i < n; i += 32) {
+        d[i] = ldexp(S.d[i], -ex);
+        const double ei = i + 1 < n ? ldexp(S.e[i], -ex) : 0.0;
+        e[i] = ei;
+        e2[i] = ei * ei;
+      }
+      __syncwarp();
+      // Gershgorin interval
+      double lo = 1e300, hi = -1e300;
+      for (int i = lane; i < n; i += 32) {
+        const double r = fabs(e[i]) + (i > 0 ? fabs(e[i - 1]) : 0.0);
+        lo = fmin(lo, d[i] - r);
+        hi = fmax(hi, d[i] + r);
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        lo = fmin(lo, __shfl_xor_sync(0xFFFFFFFFu, lo, o));
+        hi = fmax(hi, __shfl_xor_sync(0xFFFFFFFFu, hi, o));
+      }
+      if (lane == 0) {
+        interval[0] = lo - 1e-12;
+        interval[1] = hi + 1e-12;
+      }
     }
-    lo -= 1e-12;
-    hi += 1e-12;
-    // multisection: the smallest x with count(x) > idx
+    if (lane == 0) scaled = mx > 0.0;
+  }
+  __syncthreads();
+  double lam = 0.0;   // found by warp 0 (thread 0 writes it with warp 0's exponent ex)
+  if (scaled) {
+    // multisection over all warps: point t = 32 w + l (0 .. 127) sits at
+    // lo + (hi - lo) (t + 1) / 129, rising with t; the smallest point with
+    // count > idx bounds the eigenvalue.  Every thread updates (lo, hi) from
+    // the four ballots by the same float operations, so they stay equal.
+    constexpr int kPoints = 32 * kVecWarps;
+    double lo = interval[0], hi = interval[1];
     bool done = false;
     for (int round = 0; round < max_rounds; ++round) {
       if (hi - lo <= 0x1p-50 * fmax(fabs(lo), fabs(hi)) + 0x1p-60) {
         done = true;
         break;
       }
-      const double x = lo + (hi - lo) * (static_cast<double>(lane + 1) / 33.0);
+      const double w = hi - lo;
+      const double x = lo + w * (static_cast<double>(tid + 1) / (kPoints + 1));
       const int c = sturm_count(d, e2, n, x);
       const unsigned mask = __ballot_sync(0xFFFFFFFFu, c > idx);
-      const double x_prev = __shfl_up_sync(0xFFFFFFFFu, x, 1);
-      if (mask) {
-        const int f = __ffs(mask) - 1;
-        const double nlo = f > 0 ? __shfl_sync(0xFFFFFFFFu, x_prev, f) : lo;
-        hi = __shfl_sync(0xFFFFFFFFu, x, f);
-        lo = nlo;
-      } else {
-        lo = __shfl_sync(0xFFFFFFFFu, x, 31);
-      }
-    }
-    if (!done && lane == 0) report(dev_status, METIS_DEV_NUMERIC);
-    lam = 0.5 * (lo + hi);
-    // twisted factorisation of T - lam I: lane 0 runs the top-down LDL^T
-    // recurrence, lane 1 the bottom-up UDU^T one, in lockstep (one
-    // instruction stream, per-lane indices)
-    const double pivmin = 0x1p-100;
-    if (lane < 2) {
-      const bool up = lane == 1;
-      double* Dst = up ? dm : dp;
-      double* Lst = up ? um : lp;
-      double D = (up ? d[n - 1] : d[0]) - lam;
-      for (int st = 0; st + 1 < n; ++st) {
-        const int ie = up ? n - 2 - st : st;      // e index of this step
-        const int inext = up ? n - 2 - st : st + 1;
-        const double ee = e[ie], dn = d[inext];
-        if (fabs(D) < pivmin) D = D < 0.0 ? -pivmin : pivmin;
-        Dst[up ? n - 1 - st : st] = D;
-        const double l = ee / D;
-        Lst[ie] = l;
-        D = (dn - lam) - l * ee;
-      }
-      Dst[up ? 0 : n - 1] = D;
-    }
-    __syncwarp();
-    // twist index r: the smallest |gamma_r| = |D+_r + D-_r - (d_r - lam)|
-    // (the lowest r on ties)
-    double best = 1e308;
-    int r = n;
-    for (int i = lane; i < n; i += 32) {
-      const double g = fabs(dp[i] + dm[i] - (d[i] - lam));
-      if (g < best) {
-        best = g;
-        r = i;
-      }
-    }
+      if (lane == 0) masks[round & 1][warp] = mask;
+      __syncthreads();
+      int f = kPoints;  // the first point with count > idx
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const double ob = __shfl_xor_sync(0xFFFFFFFFu, best, o);
-      const int orr = __shfl_xor_sync(0xFFFFFFFFu, r, o);
-      if (ob < best || (ob == best && orr < r)) {
-        best = ob;
-        r = orr;
+      for (int q = kVecWarps - 1; q >= 0; --q) {
+        const unsigned mq = masks[round & 1][q];
+        if (mq) f = 32 * q + __ffs(mq) - 1;
       }
+      const double nlo = f > 0 ? lo + w * (static_cast<double>(f) / (kPoints + 1)) : lo;
+      if (f < kPoints) hi = lo + w * (static_cast<double>(f + 1) / (kPoints + 1));
+      lo = nlo;
     }
-    if (r >= n) r = 0;  // no finite gamma (a non-finite input): any in-range twist
-    // z_r = 1; lane 0 walks up, lane 1 walks down, in lockstep (each
-    // rescales its own side by 1e-150 if it grows past 1e150; the sides are
-    // reconciled after)
-    int sc = 0;
-    if (lane < 2) {
-      const bool up = lane == 0;
-      const double* mul = up ? lp : um;
-      const int steps = up ? r : n - 1 - r;
-      const int smax = r > n - 1 - r ? r : n - 1 - r;
-      double zc = 1.0;
-      for (int st = 0; st < smax; ++st) {
-        if (st < steps) {
-          const int i = up ? r - 1 - st : r + st;      // multiplier index
-          const int dst = up ? r - 1 - st : r + 1 + st;
-          zc = -mul[i] * zc;
-          z[dst] = zc;
-          if (fabs(zc) > 1e150) {
-            const int q0 = up ? dst : r + 1, q1 = up ? r - 1 : dst;
-            for (int q = q0; q <= q1; ++q) z[q] *= 1e-150;
-            zc *= 1e-150;
-            ++sc;
+    if (!done && tid == 0) report(dev_status, METIS_DEV_NUMERIC);
+    if (warp != 0) {
+      // the other warps form the back-transformation's block factors now
+      if (mbar_wait(&vbar, 0, &vabort))
+        for (int k = warp - 1; k * kWY < n - 2; k += kVecWarps - 1)
+          wy_block(Vs, bs, n, k * kWY, min(kWY, n - 2 - k * kWY), Tw[k]);
+    }
+    if (warp == 0) {
+      lam = 0.5 * (lo + hi);
+      // twisted factorisation of T - lam I: lane 0 runs the top-down LDL^T
+      // recurrence, lane 1 the bottom-up UDU^T one, in lockstep (one
+      // instruction stream, per-lane indices)
+      const double pivmin = 0x1p-100;
+      if (lane < 2) {
+        const bool up = lane == 1;
+        double* Dst = up ? dm : dp;
+        double* Lst = up ? um : lp;
+        double D = (up ? d[n - 1] : d[0]) - lam;
+        for (int st = 0; st + 1 < n; ++st) {
+          const int ie = up ? n - 2 - st : st;      // e index of this step
+          const int inext = up ? n - 2 - st : st + 1;
+          const double ee = e[ie], dn = d[inext];
+          if (fabs(D) < pivmin) D = D < 0.0 ? -pivmin : pivmin;
+          Dst[up ? n - 1 - st : st] = D;
+          const double l = ee / D;
+          Lst[ie] = l;
+          D = (dn - lam) - l * ee;
+        }
+        Dst[up ? 0 : n - 1] = D;
+      }
+      __syncwarp();
+      // twist index r: the smallest |gamma_r| = |D+_r + D-_r - (d_r - lam)|
+      // (the lowest r on ties)
+      double best = 1e308;
+      int r = n;
+      for (int i = lane; i < n; i += 32) {
+        const double g = fabs(dp[i] + dm[i] - (d[i] - lam));
+        if (g < best) {
+          best = g;
+          r = i;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        const double ob = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+        const int orr = __shfl_xor_sync(0xFFFFFFFFu, r, o);
+        if (ob < best || (ob == best && orr < r)) {
+          best = ob;
+          r = orr;
+        }
+      }
+      if (r >= n) r = 0;  // no finite gamma (a non-finite input): any in-range twist
+      // z_r = 1; lane 0 walks up, lane 1 walks down, in lockstep (each
+      // rescales its own side by 1e-150 if it grows past 1e150; the sides are
+      // reconciled after)
+      int sc = 0;
+      if (lane < 2) {
+        const bool up = lane == 0;
+        const double* mul = up ? lp : um;
+        const int steps = up ? r : n - 1 - r;
+        const int smax = r > n - 1 - r ? r : n - 1 - r;
+        double zc = 1.0;
+        for (int st = 0; st < smax; ++st) {
+          if (st < steps) {
+            const int i = up ? r - 1 - st : r + st;      // multiplier index
+            const int dst = up ? r - 1 - st : r + 1 + st;
+            zc = -mul[i] * zc;
+            z[dst] = zc;
+            if (fabs(zc) > 1e150) {
+              const int q0 = up ? dst : r + 1, q1 = up ? r - 1 : dst;
+              for (int q = q0; q <= q1; ++q) z[q] *= 1e-150;
+              zc *= 1e-150;
+              ++sc;
+            }
           }
         }
       }
+      const int s0 = __shfl_sync(0xFFFFFFFFu, sc, 0), s1 = __shfl_sync(0xFFFFFFFFu, sc, 1);
+      __syncwarp();
+      if (lane == 0) {
+        const int smax = s0 > s1 ? s0 : s1;
+        double f = 1.0;
+        for (int k = 0; k < smax; ++k) f *= 1e-150;
+        z[r] = f;
+        for (int k = s0; k < smax; ++k)
+          for (int q = 0; q < r; ++q) z[q] *= 1e-150;
+        for (int k = s1; k < smax; ++k)
+          for (int q = r + 1; q < n; ++q) z[q] *= 1e-150;
+      }
     }
-    const int s0 = __shfl_sync(0xFFFFFFFFu, sc, 0), s1 = __shfl_sync(0xFFFFFFFFu, sc, 1);
-    __syncwarp();
-    if (lane == 0) {
-      const int smax = s0 > s1 ? s0 : s1;
-      double f = 1.0;
-      for (int k = 0; k < smax; ++k) f *= 1e-150;
-      z[r] = f;
-      for (int k = s0; k < smax; ++k)
-        for (int q = 0; q < r; ++q) z[q] *= 1e-150;
-      for (int k = s1; k < smax; ++k)
-        for (int q = r + 1; q < n; ++q) z[q] *= 1e-150;
-    }
-  }  // mx > 0
-  __syncwarp();
+  }
+  __syncthreads();
   // x = H_0 H_1 ... H_{n-3} z, the reflectors staged in shared memory;
-  // lane l holds entries l, l + 32, l + 64, l + 96
+  // thread t holds entry t (n <= 128); each reflector's dot product is a
+  // warp reduction, then the four warp sums in warp order
   const bool landed = mbar_wait(&vbar, 0, &vabort);  // bounded wait
-  if (!__all_sync(0xFFFFFFFFu, landed)) {
-    if (lane == 0) {
+  if (!__syncthreads_and(landed)) {
+    if (tid == 0) {
       report(dev_status, METIS_DEV_TIMEOUT);
-      // the copies were issued by this warp: give them a bounded time to land
+      // the copies were issued by this CTA: give them a bounded time to land
       const uint64_t t0 = global_timer_ns();
       while (!mbar_try_wait(&vbar, 0) && global_timer_ns() - t0 < 100000000ull) {
       }
     }
-    __syncwarp();
+    __syncthreads();
     return;
   }
-  double xv[4];
-#pragma unroll
-  for (int q = 0; q < 4; ++q) xv[q] = lane + 32 * q < n ? z[lane + 32 * q] : 0.0;
-  for (int j = n - 3; j >= 0; --j) {
-    const double* vj = Vs + j * n;
-    double c = 0.0;
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (lane + 32 * q < n) c = fma(vj[lane + 32 * q], xv[q], c);
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
-    c *= bs[j];
-#pragma unroll
-    for (int q = 0; q < 4; ++q)
-      if (lane + 32 * q < n) xv[q] = fma(-c, vj[lane + 32 * q], xv[q]);
+  const bool mine = tid < n;
+  double xv = mine ? z[tid] : 0.0;
+  if (!scaled) {
+    // T = 0 (no multisection ran): the block factors are still needed
+    if (warp != 0)
+      for (int k = warp - 1; k * kWY < n - 2; k += kVecWarps - 1)
+        wy_block(Vs, bs, n, k * kWY, min(kWY, n - 2 - k * kWY), Tw[k]);
+    __syncthreads();
   }
-  double nrm = 0.0;
+  // x = B_0 B_1 ... z with B_k = I - V_k T_k V_k^T (blocks of kWY
+  // reflectors), the last block first: per block one reduction of kWY dot
+  // products (warp sums, then the four warps in warp order)
+  const int nrefl = n - 2;
+  int par = 0;
+  for (int k = (nrefl - 1) / kWY; k >= 0 && nrefl > 0; --k, par ^= 1) {
+    const int j0 = k * kWY, b = min(kWY, nrefl - j0);
+    double vt[kWY], w[kWY];
 #pragma unroll
-  for (int q = 0; q < 4; ++q) nrm = fma(xv[q], xv[q], nrm);
+    for (int i = 0; i < kWY; ++i) {
+      vt[i] = (mine && i < b) ? Vs[(j0 + i) * n + tid] : 0.0;
+      w[i] = vt[i] * xv;
+    }
+#pragma unroll
+    for (int i = 0; i < kWY; ++i)
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) w[i] += __shfl_xor_sync(0xFFFFFFFFu, w[i], o);
+    if (lane < kWY) {
+      double wl = w[0];
+#pragma unroll
+      for (int i = 1; i < kWY; ++i) wl = lane == i ? w[i] : wl;
+      part[par][warp][lane] = wl;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < kWY; ++i) w[i] = (part[par][0][i] + part[par][1][i]) + (part[par][2][i] + part[par][3][i]);
+    // y = T w (upper triangular), then x -= V y
+    double upd = 0.0;
+#pragma unroll
+    for (int i = 0; i < kWY; ++i) {
+      if (i < b) {
+        double y = 0.0;
+#pragma unroll
+        for (int c = 0; c < kWY; ++c)
+          if (c >= i && c < b) y = fma(Tw[k][i][c], w[c], y);
+        upd = fma(vt[i], y, upd);
+      }
+    }
+    xv -= upd;
+  }
+  double nrm = xv * xv;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) nrm += __shfl_xor_sync(0xFFFFFFFFu, nrm, o);
+  if (lane == 0) part[par][warp][0] = nrm;
+  __syncthreads();
+  nrm = (part[par][0][0] + part[par][1][0]) + (part[par][2][0] + part[par][3][0]);
   const double inv = 1.0 / sqrt(nrm);
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-    if (lane + 32 * q < n) S.X[(lane + 32 * q) * n + idx] = xv[q] * inv;
-  if (lane == 0) S.lam[idx] = ldexp(lam, ex);
+  if (mine) S.X[tid * n + idx] = xv * inv;
+  if (tid == 0) S.lam[idx] = ldexp(lam, ex);
 }
 
 // ---------------------------------------------------------------------------
@@ -682,7 +784,7 @@ void launch_core_eig(double* C, int n, int max_iters, double* eval, float* evec,
   else launch_tridiag<56>(C, n, ws, s);
   const size_t vsmem = static_cast<size_t>(n) * n * sizeof(double);
   if (!ensure_smem(reinterpret_cast<const void*>(core_vector_kernel), vsmem)) return;
-  core_vector_kernel<<<n, 32, vsmem, s>>>(n, ws, max_iters, dev_status);
+  core_vector_kernel<<<n, 32 * kVecWarps, vsmem, s>>>(n, ws, max_iters, dev_status);
   core_finish_kernel<<<1, 1024, 0, s>>>(n, ws, eval, evec);
 }
 

@@ -45,6 +45,7 @@ MDEV void gram_block(const T* ys, int rows, int cols, int ld, double* out) {
     for (int x = 0; x < 4; ++x)
 #pragma unroll
       for (int y = 0; y < 4; ++y) acc[x][y] = 0.0;
+#pragma unroll 4
     for (int r = 0; r < rows; ++r) {
       const T* row = ys + r * ld;
       double a[4], b[4];
@@ -144,6 +145,11 @@ MDEV int tri_element(int e, int n) {
 
 constexpr int kSmallThreads = 512;
 constexpr int kTile = 4;  // register tile edge and panel width of the Cholesky
+// Panel buffer layout: tile row I (rows 4I .. 4I+3, 4 columns: 16 doubles)
+// starts at double 18 I.  The 16-byte skew puts the same word of consecutive
+// tile rows in different bank groups: the warps' 16-byte reads of their own
+// tile rows then run at the minimum 4 wavefronts instead of up to 32.
+constexpr int kPanStride = 18;
 
 // Block row BI of X = L^-1 (16 x 16 blocks, o = 16 BI), after blocks
 // 0 .. BI-1 of X and the diagonal block X(BI, BI) are known:
@@ -252,7 +258,7 @@ MDEV void solve_rows(const double (&v)[kTile][kTile], int I, int K, double* P, d
     const int row = kTile * I + a;
 #pragma unroll
     for (int c = 0; c < kTile; ++c) {
-      P[row * kTile + c] = lr[c];
+      P[I * kPanStride + a * kTile + c] = lr[c];
       L[row * ld + o + c] = lr[c];
     }
   }
@@ -261,12 +267,17 @@ MDEV void solve_rows(const double (&v)[kTile][kTile], int I, int K, double* P, d
 // Rank-4 update of the register tile (I, J) with panel P: v -= L(I, K) L(J, K)^T.
 MDEV void panel_update(double (&v)[kTile][kTile], const double* P, int I, int J) {
   double li[kTile][kTile], lj[kTile][kTile];
+  const double2* pi = reinterpret_cast<const double2*>(P + I * kPanStride);
+  const double2* pj = reinterpret_cast<const double2*>(P + J * kPanStride);
 #pragma unroll
   for (int a = 0; a < kTile; ++a)
 #pragma unroll
-    for (int c = 0; c < kTile; ++c) {
-      li[a][c] = P[(kTile * I + a) * kTile + c];
-      lj[a][c] = P[(kTile * J + a) * kTile + c];
+    for (int c = 0; c < kTile; c += 2) {
+      const double2 x = pi[a * 2 + c / 2], y = pj[a * 2 + c / 2];
+      li[a][c] = x.x;
+      li[a][c + 1] = x.y;
+      lj[a][c] = y.x;
+      lj[a][c + 1] = y.y;
     }
 #pragma unroll
   for (int a = 0; a < kTile; ++a)
@@ -291,8 +302,9 @@ MDEV void panel_update(double (&v)[kTile][kTile], const double* P, int I, int J)
 __global__ void __launch_bounds__(kSmallThreads, 1) cholesky_inv_kernel(const double* G, int lp, float* Rinv) {
   extern __shared__ double sm[];
   const int ld = lp + 1;
-  double* pan = sm;               // 2 x lp x 4: panel buffers
-  double* invd = pan + 8 * lp;    // lp: 1/sqrt(pivot) (0 when dropped)
+  double* pan = sm;               // 2 panel buffers of (lp / 4) x kPanStride
+  const int pan_size = (lp / kTile) * kPanStride;
+  double* invd = pan + 2 * pan_size;  // lp: 1/sqrt(pivot) (0 when dropped)
   double* sqd = invd + lp;        // lp: sqrt(pivot) (0 when dropped)
   double* diag0 = sqd + lp;       // lp: the original diagonal (drop rule)
   double* L = diag0 + lp;         // lp x ld: final L
@@ -321,8 +333,8 @@ __global__ void __launch_bounds__(kSmallThreads, 1) cholesky_inv_kernel(const do
   if (owner && J == 0 && I > 0) solve_rows(v, I, 0, pan, L, invd, ld);
   __syncthreads();
   for (int K = 0; K + 1 < nb; ++K) {
-    const double* P = pan + (K & 1) * 4 * lp;
-    double* Pn = pan + ((K + 1) & 1) * 4 * lp;
+    const double* P = pan + (K & 1) * pan_size;
+    double* Pn = pan + ((K + 1) & 1) * pan_size;
     if (owner && J > K) {
       panel_update(v, P, I, J);
       if (I == K + 1 && J == K + 1) factor_diag(v, K + 1, L, invd, sqd, diag0, ld);
@@ -372,13 +384,14 @@ constexpr int kApplyRows = 32;
 
 // out = in (rows x kin) * M (kin x kout).  32 rows per CTA, 256 threads, each
 // thread a 4-row x 4-column register tile (4 consecutive columns).  Optional fp32 out,
-// transposed bf16 hi/lo copy, Gram partial of the output block.
-__global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) {
+// transposed bf16 hi/lo copy, Gram partial of the output block, and per
+// column the block's largest |out| with its first row (the sign convention).
+MDEV void apply_block(const ApplyArgs& a, int64_t blk) {
   extern __shared__ float smf[];
   float* Ms = smf;                                   // kin x kout
   float* In = Ms + a.kin * a.kout;                   // kApplyRows x (kin + 1)
   float* Out = In + kApplyRows * (a.kin + 1);        // kApplyRows x (kout + 1)
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kApplyRows;
+  const int64_t r0 = blk * kApplyRows;
   const int nr = static_cast<int>(imin64(kApplyRows, a.rows - r0));
   {
     const float4* M4 = reinterpret_cast<const float4*>(a.M);
@@ -447,7 +460,32 @@ __global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) {
       }
     }
   }
-  if (a.gpart) gram_block<float>(Out, nr, a.kout, a.kout + 1, a.gpart + static_cast<int64_t>(blockIdx.x) * a.kout * a.kout);
+  if (a.gpart) gram_block<float>(Out, nr, a.kout, a.kout + 1, a.gpart + blk * a.kout * a.kout);
+  if (a.bmax && threadIdx.x < a.kout) {
+    // rows in order, strictly larger wins (the lowest row on ties); a NaN
+    // never wins, so a column of NaNs keeps -1 and the block's first row
+    const int j = threadIdx.x;
+    float best = -1.f;
+    int64_t bi = r0;
+    for (int r = 0; r < nr; ++r) {
+      const float v = fabsf(Out[r * (a.kout + 1) + j]);
+      if (v > best) {
+        best = v;
+        bi = r0 + r;
+      }
+    }
+    a.bmax[blk * a.kout + j] = best;
+    a.bidx[blk * a.kout + j] = bi;
+  }
+}
+
+__global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) { apply_block(a, blockIdx.x); }
+
+__global__ void __launch_bounds__(256) apply2_kernel(ApplyArgs a, ApplyArgs b, int64_t blocks_a) {
+  if (blockIdx.x < blocks_a)
+    apply_block(a, blockIdx.x);
+  else
+    apply_block(b, blockIdx.x - blocks_a);
 }
 
 // Factor matrices from the sorted eigen-decomposition of the core Gram:
@@ -467,28 +505,7 @@ __global__ void factor_mats_kernel(const double* eval, const float* evec, int lp
   if (i == 0) S[j] = static_cast<float>(sigma);
 }
 
-// Per block of kSignRows rows: for each column, the largest |U| and its lowest
-// row index.
-constexpr int kSignRows = 32;
-__global__ void colmax_kernel(const float* __restrict__ U, int64_t rows, int k, float* bmax, int64_t* bidx) {
-  const int j = threadIdx.x;
-  if (j >= k) return;
-  const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kSignRows;
-  float v[kSignRows];
-#pragma unroll
-  for (int r = 0; r < kSignRows; ++r) v[r] = r0 + r < rows ? fabsf(U[(r0 + r) * k + j]) : -1.f;
-  float best = -1.f;
-  int64_t bi = r0;
-#pragma unroll
-  for (int r = 0; r < kSignRows; ++r) {
-    if (v[r] > best) {
-      best = v[r];
-      bi = r0 + r;
-    }
-  }
-  bmax[static_cast<int64_t>(blockIdx.x) * k + j] = best;
-  bidx[static_cast<int64_t>(blockIdx.x) * k + j] = bi;
-}
+constexpr int kSignRows = kApplyRows;  // the sign convention's row blocks are the apply kernel's
 
 // One warp per column: lanes take every 32nd block, then a shuffle reduction
 // keeps the largest |U| (the lowest block, hence the lowest row, on ties).
@@ -546,16 +563,29 @@ void launch_gram_reduce(const double* gpart, int nblocks, int lp, double* G, cud
 
 void launch_cholesky_inv(const double* G, int lp, float* Rinv, cudaStream_t s) {
   // panels x2, invd, sqd, diag0, L, X, T
-  const size_t smem = ((2 * static_cast<size_t>(lp) + 16) * (lp + 1) + 11 * lp) * sizeof(double);
+  const size_t smem = ((2 * static_cast<size_t>(lp) + 16) * (lp + 1) + 2 * (lp / kTile) * kPanStride + 3 * lp) *
+                      sizeof(double);
   if (!ensure_smem(reinterpret_cast<const void*>(cholesky_inv_kernel), smem)) return;
   cholesky_inv_kernel<<<1, kSmallThreads, smem, s>>>(G, lp, Rinv);
 }
 
+size_t apply_smem(const ApplyArgs& a) {
+  return (static_cast<size_t>(a.kin) * a.kout + kApplyRows * (a.kin + 1) + kApplyRows * (a.kout + 1)) *
+         sizeof(float);
+}
+
 void launch_apply(const ApplyArgs& a, cudaStream_t s) {
-  const size_t smem = (static_cast<size_t>(a.kin) * a.kout + kApplyRows * (a.kin + 1) +
-                       kApplyRows * (a.kout + 1)) * sizeof(float);
+  const size_t smem = apply_smem(a);
   if (!ensure_smem(reinterpret_cast<const void*>(apply_kernel), smem)) return;
   apply_kernel<<<static_cast<unsigned>(apply_blocks(a.rows)), 256, smem, s>>>(a);
+}
+
+void launch_apply2(const ApplyArgs& a, const ApplyArgs& b, cudaStream_t s) {
+  const size_t sa = apply_smem(a), sb = apply_smem(b);
+  const size_t smem = sa > sb ? sa : sb;
+  if (!ensure_smem(reinterpret_cast<const void*>(apply2_kernel), smem)) return;
+  const int64_t na = apply_blocks(a.rows), nb = apply_blocks(b.rows);
+  apply2_kernel<<<static_cast<unsigned>(na + nb), 256, smem, s>>>(a, b, na);
 }
 
 void launch_factor_mats(const double* eval, const float* evec, int lp, int k, float* Mu, float* Mv, float* S,
@@ -565,11 +595,12 @@ void launch_factor_mats(const double* eval, const float* evec, int lp, int k, fl
 
 int64_t sign_blocks(int64_t rows) { return (rows + kSignRows - 1) / kSignRows; }
 
-void launch_signs(float* U, int64_t m, float* V, int64_t n, int k, float* bmax, int64_t* bidx, float* sign, int sms,
-                  cudaStream_t s) {
-  const int nb = static_cast<int>(sign_blocks(m));
-  colmax_kernel<<<nb, 128, 0, s>>>(U, m, k, bmax, bidx);
-  sign_kernel<<<k, 32, 0, s>>>(U, bmax, bidx, nb, k, sign);
+void launch_signs_from_blocks(float* U, int64_t m, float* V, int64_t n, int k, const float* bmax,
+                              const int64_t* bidx, float* sign, cudaStream_t s) {
+  (void)V;
+  (void)n;
+  sign_kernel<<<k, 32, 0, s>>>(U, bmax, bidx, static_cast<int>(sign_blocks(m)), k, sign);
 }
+
 
 }  // namespace metis

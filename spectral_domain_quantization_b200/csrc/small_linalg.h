@@ -21,6 +21,8 @@ struct ApplyArgs {
   int lpT;
   int64_t ldx;
   double* gpart;           // optional [blocks][kout][kout]
+  float* bmax;             // optional [blocks][kout]: max |out| of each 32-row block's columns
+  int64_t* bidx;           // with bmax: the first row holding it
 };
 
 // row blocks of launch_apply (its Gram partials come one per block)
@@ -35,6 +37,13 @@ void launch_gram_reduce(const double* gpart, int nblocks, int lp, double* G, cud
 // Rinv (lp x lp float, upper triangular) with G = R^T R, dropped pivots -> 0.
 void launch_cholesky_inv(const double* G, int lp, float* Rinv, cudaStream_t s);
 void launch_apply(const ApplyArgs& a, cudaStream_t s);
+// Two independent products in one launch (blocks of a first, then of b).
+void launch_apply2(const ApplyArgs& a, const ApplyArgs& b, cudaStream_t s);
+// sign[j] = the sign that makes the largest-|.| entry (lowest row on ties)
+// of column j of U positive (applied by launch_factor_finish), from U's
+// column maxima per 32-row block that its apply wrote (bmax / bidx).
+void launch_signs_from_blocks(float* U, int64_t m, float* V, int64_t n, int k, const float* bmax,
+                              const int64_t* bidx, float* sign, cudaStream_t s);
 // Symmetric eigen-decomposition of C (n x n float64, n <= 112, a multiple of
 // 16), eigenvalues descending in eval, evec[i * n + j] = component i of
 // eigenvector j (core_eig.cu).  ws: core_eig_workspace(n) bytes of scratch;
@@ -46,9 +55,5 @@ void launch_core_eig(double* C, int n, int max_iters, double* eval, float* evec,
 void launch_factor_mats(const double* eval, const float* evec, int lp, int k, float* Mu, float* Mv, float* S,
                         cudaStream_t s);
 int64_t sign_blocks(int64_t rows);
-// sign[j] = the sign that makes the largest-|.| entry (lowest row on ties)
-// of column j of U positive (applied by launch_factor_finish).
-void launch_signs(float* U, int64_t m, float* V, int64_t n, int k, float* bmax, int64_t* bidx, float* sign, int sms,
-                  cudaStream_t s);
 
 }  // namespace metis
