@@ -230,6 +230,7 @@ MDEV void tri_step(double (&a)[NH], TriShared<NH>& sh, const EigScratch& S, int 
 // One CTA of round32(2 n) + 32 threads, n <= 2 NH.
 template <int NH>
 __global__ void __launch_bounds__(4 * NH + 32, 1) core_tridiag_kernel(const double* C, int n, double* ws) {
+  pdl_prologue();
   __shared__ TriShared<NH> sh;
   const EigScratch S = scratch(ws, n);
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -291,7 +292,7 @@ __global__ void __launch_bounds__(4 * NH + 32, 1) core_tridiag_kernel(const doub
 template <int NH>
 void launch_tridiag(const double* C, int n, double* ws, cudaStream_t s) {
   const int threads = (2 * n + 31) / 32 * 32 + 32;
-  core_tridiag_kernel<NH><<<1, threads, 0, s>>>(C, n, ws);
+  launch_pdl(core_tridiag_kernel<NH>, dim3(1), dim3(threads), 0, s, C, n, ws);
 }
 
 // ---------------------------------------------------------------------------
@@ -358,47 +359,10 @@ MDEV int sturm_count(const double* d, const double* e2, int n, double x) {
 }
 
 constexpr int kVecWarps = 4;   // warps per eigenvalue CTA
-constexpr int kWY = 8;         // reflectors per block of the back-transformation
-constexpr int kMaxBlocks = (kMaxN + kWY - 1) / kWY;
-
-// T of the block of reflectors H_j0 ... H_j0+b-1 (columns v_j of V, the j-th
-// row of Vs), as in LAPACK's larft (forward, columnwise): H_j0 ... = I -
-// V T V^T with T upper triangular, T[i][i] = beta_i and T[0:i, i] = -beta_i
-// T[0:i, 0:i] (V[:, 0:i]^T v_i).  One warp; lanes stride the vector entries.
-MDEV void wy_block(const double* Vs, const double* bs, int n, int j0, int b, double (*T)[kWY]) {
-  const int lane = threadIdx.x & 31;
-  if (lane == 0) T[0][0] = bs[j0];
-  __syncwarp();
-  for (int i = 1; i < b; ++i) {
-    const double* vi = Vs + (j0 + i) * n;
-    double dot[kWY];
-#pragma unroll
-    for (int c = 0; c < kWY; ++c) dot[c] = 0.0;
-    for (int t = lane; t < n; t += 32) {
-      const double x = vi[t];
-#pragma unroll
-      for (int c = 0; c < kWY; ++c)
-        if (c < i) dot[c] = fma(Vs[(j0 + c) * n + t], x, dot[c]);
-    }
-#pragma unroll
-    for (int c = 0; c < kWY; ++c)
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) dot[c] += __shfl_xor_sync(0xFFFFFFFFu, dot[c], o);
-    const double beta = bs[j0 + i];
-    if (lane < i) {
-      double y = 0.0;   // (T[0:i, 0:i] dot)[lane], upper triangular: columns lane .. i-1
-#pragma unroll
-      for (int c = 0; c < kWY; ++c)
-        if (c >= lane && c < i) y = fma(T[lane][c], dot[c], y);
-      T[lane][i] = -beta * y;
-    }
-    if (lane == 0) T[i][i] = beta;
-    __syncwarp();
-  }
-}
 
 __global__ void __launch_bounds__(32 * kVecWarps) core_vector_kernel(int n, double* ws, int max_rounds,
                                                                      int32_t* dev_status) {
+  pdl_prologue();
   __shared__ double d[kMaxN], e[kMaxN], e2[kMaxN], dp[kMaxN], dm[kMaxN], lp[kMaxN], um[kMaxN], z[kMaxN];
   __shared__ __align__(16) double bs[kMaxN];
   extern __shared__ __align__(16) double Vs[];  // n x n reflectors
@@ -407,8 +371,7 @@ __global__ void __launch_bounds__(32 * kVecWarps) core_vector_kernel(int n, doub
   __shared__ double interval[2];                // the Gershgorin interval, by warp 0
   __shared__ int scaled;                        // T != 0 (the multisection runs)
   __shared__ unsigned masks[2][kVecWarps];      // per round parity: each warp's ballot
-  __shared__ double part[2][kVecWarps][kWY];    // per block parity: each warp's partial dot products
-  __shared__ double Tw[kMaxBlocks][kWY][kWY];    // T of each block of kWY reflectors
+  __shared__ double part[2][kVecWarps];         // per step parity: each warp's partial dot product
   const EigScratch S = scratch(ws, n);
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int idx = blockIdx.x;  // eigenvalue idx in ascending order
@@ -495,12 +458,6 @@ __global__ void __launch_bounds__(32 * kVecWarps) core_vector_kernel(int n, doub
       lo = nlo;
     }
     if (!done && tid == 0) report(dev_status, METIS_DEV_NUMERIC);
-    if (warp != 0) {
-      // the other warps form the back-transformation's block factors now
-      if (mbar_wait(&vbar, 0, &vabort))
-        for (int k = warp - 1; k * kWY < n - 2; k += kVecWarps - 1)
-          wy_block(Vs, bs, n, k * kWY, min(kWY, n - 2 - k * kWY), Tw[k]);
-    }
     if (warp == 0) {
       lam = 0.5 * (lo + hi);
       // twisted factorisation of T - lam I: lane 0 runs the top-down LDL^T
@@ -508,19 +465,26 @@ __global__ void __launch_bounds__(32 * kVecWarps) core_vector_kernel(int n, doub
       // instruction stream, per-lane indices)
       const double pivmin = 0x1p-100;
       if (lane < 2) {
+        // the chain per step is one reciprocal and one fma: the pivot guard
+        // reads the exponent bits (|D| < 2^-100), the multiplier l = e / D
+        // and D' = (d - lam) - e^2 / D come from 1 / D, and the loads and
+        // stores (restrict: the arrays do not overlap) leave the chain
         const bool up = lane == 1;
-        double* Dst = up ? dm : dp;
-        double* Lst = up ? um : lp;
-        double D = (up ? d[n - 1] : d[0]) - lam;
+        double* __restrict__ Dst = up ? dm : dp;
+        double* __restrict__ Lst = up ? um : lp;
+        const double* __restrict__ dd = d;
+        const double* __restrict__ ev = e;
+        const double* __restrict__ ev2 = e2;
+        double D = (up ? dd[n - 1] : dd[0]) - lam;
         for (int st = 0; st + 1 < n; ++st) {
           const int ie = up ? n - 2 - st : st;      // e index of this step
           const int inext = up ? n - 2 - st : st + 1;
-          const double ee = e[ie], dn = d[inext];
-          if (fabs(D) < pivmin) D = D < 0.0 ? -pivmin : pivmin;
+          const double ee = ev[ie], ee2 = ev2[ie], dn = dd[inext] - lam;
+          if (exp_field(D) < 1023 - 100) D = __double_as_longlong(D) < 0 ? -pivmin : pivmin;
           Dst[up ? n - 1 - st : st] = D;
-          const double l = ee / D;
-          Lst[ie] = l;
-          D = (dn - lam) - l * ee;
+          const double rD = 1.0 / D;
+          Lst[ie] = ee * rD;
+          D = fma(-ee2, rD, dn);
         }
         Dst[up ? 0 : n - 1] = D;
       }
@@ -547,12 +511,15 @@ __global__ void __launch_bounds__(32 * kVecWarps) core_vector_kernel(int n, doub
       }
       if (r >= n) r = 0;  // no finite gamma (a non-finite input): any in-range twist
       // z_r = 1; lane 0 walks up, lane 1 walks down, in lockstep (each
-      // rescales its own side by 1e-150 if it grows past 1e150; the sides are
-      // reconciled after)
+      // rescales its own side by 1e-150 once |z| reaches 2^499 (about
+      // 1.6e150; read from the exponent bits); the sides are reconciled
+      // after).  restrict: the multipliers and z do not overlap, so the
+      // multiplier loads leave the chain.
       int sc = 0;
       if (lane < 2) {
         const bool up = lane == 0;
-        const double* mul = up ? lp : um;
+        const double* __restrict__ mul = up ? lp : um;
+        double* __restrict__ zz = z;
         const int steps = up ? r : n - 1 - r;
         const int smax = r > n - 1 - r ? r : n - 1 - r;
         double zc = 1.0;
@@ -561,10 +528,10 @@ __global__ void __launch_bounds__(32 * kVecWarps) core_vector_kernel(int n, doub
             const int i = up ? r - 1 - st : r + st;      // multiplier index
             const int dst = up ? r - 1 - st : r + 1 + st;
             zc = -mul[i] * zc;
-            z[dst] = zc;
-            if (fabs(zc) > 1e150) {
+            zz[dst] = zc;
+            if (exp_field(zc) > 1023 + 498) {
               const int q0 = up ? dst : r + 1, q1 = up ? r - 1 : dst;
-              for (int q = q0; q <= q1; ++q) z[q] *= 1e-150;
+              for (int q = q0; q <= q1; ++q) zz[q] *= 1e-150;   // through zz: the one name for z here
               zc *= 1e-150;
               ++sc;
             }
@@ -603,59 +570,23 @@ __global__ void __launch_bounds__(32 * kVecWarps) core_vector_kernel(int n, doub
   }
   const bool mine = tid < n;
   double xv = mine ? z[tid] : 0.0;
-  if (!scaled) {
-    // T = 0 (no multisection ran): the block factors are still needed
-    if (warp != 0)
-      for (int k = warp - 1; k * kWY < n - 2; k += kVecWarps - 1)
-        wy_block(Vs, bs, n, k * kWY, min(kWY, n - 2 - k * kWY), Tw[k]);
-    __syncthreads();
-  }
-  // x = B_0 B_1 ... z with B_k = I - V_k T_k V_k^T (blocks of kWY
-  // reflectors), the last block first: per block one reduction of kWY dot
-  // products (warp sums, then the four warps in warp order)
-  const int nrefl = n - 2;
   int par = 0;
-  for (int k = (nrefl - 1) / kWY; k >= 0 && nrefl > 0; --k, par ^= 1) {
-    const int j0 = k * kWY, b = min(kWY, nrefl - j0);
-    double vt[kWY], w[kWY];
+  for (int j = n - 3; j >= 0; --j, par ^= 1) {
+    const double vt = mine ? Vs[j * n + tid] : 0.0;
+    double c = vt * xv;
 #pragma unroll
-    for (int i = 0; i < kWY; ++i) {
-      vt[i] = (mine && i < b) ? Vs[(j0 + i) * n + tid] : 0.0;
-      w[i] = vt[i] * xv;
-    }
-#pragma unroll
-    for (int i = 0; i < kWY; ++i)
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) w[i] += __shfl_xor_sync(0xFFFFFFFFu, w[i], o);
-    if (lane < kWY) {
-      double wl = w[0];
-#pragma unroll
-      for (int i = 1; i < kWY; ++i) wl = lane == i ? w[i] : wl;
-      part[par][warp][lane] = wl;
-    }
+    for (int o = 16; o > 0; o >>= 1) c += __shfl_xor_sync(0xFFFFFFFFu, c, o);
+    if (lane == 0) part[par][warp] = c;
     __syncthreads();
-#pragma unroll
-    for (int i = 0; i < kWY; ++i) w[i] = (part[par][0][i] + part[par][1][i]) + (part[par][2][i] + part[par][3][i]);
-    // y = T w (upper triangular), then x -= V y
-    double upd = 0.0;
-#pragma unroll
-    for (int i = 0; i < kWY; ++i) {
-      if (i < b) {
-        double y = 0.0;
-#pragma unroll
-        for (int c = 0; c < kWY; ++c)
-          if (c >= i && c < b) y = fma(Tw[k][i][c], w[c], y);
-        upd = fma(vt[i], y, upd);
-      }
-    }
-    xv -= upd;
+    c = ((part[par][0] + part[par][1]) + (part[par][2] + part[par][3])) * bs[j];
+    xv = fma(-c, vt, xv);
   }
   double nrm = xv * xv;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) nrm += __shfl_xor_sync(0xFFFFFFFFu, nrm, o);
-  if (lane == 0) part[par][warp][0] = nrm;
+  if (lane == 0) part[par][warp] = nrm;
   __syncthreads();
-  nrm = (part[par][0][0] + part[par][1][0]) + (part[par][2][0] + part[par][3][0]);
+  nrm = (part[par][0] + part[par][1]) + (part[par][2] + part[par][3]);
   const double inv = 1.0 / sqrt(nrm);
   if (mine) S.X[tid * n + idx] = xv * inv;
   if (tid == 0) S.lam[idx] = ldexp(lam, ex);
@@ -700,6 +631,7 @@ MDEV double warp_norm(const double* v, int n) {
 }
 
 __global__ void __launch_bounds__(1024) core_finish_kernel(int n, double* ws, double* eval, float* evec) {
+  pdl_prologue();
   __shared__ double lam[kMaxN];
   const EigScratch S = scratch(ws, n);
   double* X = S.X;
@@ -784,8 +716,8 @@ void launch_core_eig(double* C, int n, int max_iters, double* eval, float* evec,
   else launch_tridiag<56>(C, n, ws, s);
   const size_t vsmem = static_cast<size_t>(n) * n * sizeof(double);
   if (!ensure_smem(reinterpret_cast<const void*>(core_vector_kernel), vsmem)) return;
-  core_vector_kernel<<<n, 32 * kVecWarps, vsmem, s>>>(n, ws, max_iters, dev_status);
-  core_finish_kernel<<<1, 1024, 0, s>>>(n, ws, eval, evec);
+  launch_pdl(core_vector_kernel, dim3(n), dim3(32 * kVecWarps), vsmem, s, n, ws, max_iters, dev_status);
+  launch_pdl(core_finish_kernel, dim3(1), dim3(1024), 0, s, n, ws, eval, evec);
 }
 
 }  // namespace metis
