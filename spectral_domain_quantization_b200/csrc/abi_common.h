@@ -30,25 +30,6 @@ inline size_t dtype_size(int dt) { return dt == METIS_BF16 ? 2 : 4; }
 inline bool valid_dtype(int dt) { return dt == METIS_BF16 || dt == METIS_F32; }
 inline bool valid_fmt(int f) { return f == METIS_MXFP4 || f == METIS_NVFP4; }
 
-// Launch `kernel` on `s` with programmatic stream serialization: it may
-// begin while the stream's previous kernel finishes and must call pdl_wait
-// (common.cuh) before it reads anything that kernel wrote.
-template <typename... KArgs, typename... Args>
-cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s,
-                       Args&&... args) {
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = grid;
-  cfg.blockDim = block;
-  cfg.dynamicSmemBytes = smem;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, kernel, static_cast<KArgs>(args)...);
-}
-
 // Number of SMs of the current device (cached per device).
 int device_sm_count();
 // 1 when the current device is compute capability 10.x.

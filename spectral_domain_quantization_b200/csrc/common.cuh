@@ -72,19 +72,6 @@ MDEV void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
-// Programmatic dependent launch.  A kernel launched with launch_pdl may
-// start while the kernel before it in the stream finishes: it lets its own
-// dependents launch (pdl_launch_dependents) and then, before its first global
-// access, waits for the previous kernel to complete with its writes visible
-// (pdl_wait).  Both are no-ops in a kernel launched the ordinary way.
-MDEV void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-MDEV void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-// Both, at the top of a kernel.
-MDEV void pdl_prologue() {
-  pdl_launch_dependents();
-  pdl_wait();
-}
-
 MDEV bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(

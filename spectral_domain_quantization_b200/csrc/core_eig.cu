@@ -230,7 +230,6 @@ MDEV void tri_step(double (&a)[NH], TriShared<NH>& sh, const EigScratch& S, int 
 // One CTA of round32(2 n) + 32 threads, n <= 2 NH.
 template <int NH>
 __global__ void __launch_bounds__(4 * NH + 32, 1) core_tridiag_kernel(const double* C, int n, double* ws) {
-  pdl_prologue();
   __shared__ TriShared<NH> sh;
   const EigScratch S = scratch(ws, n);
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -292,7 +291,7 @@ __global__ void __launch_bounds__(4 * NH + 32, 1) core_tridiag_kernel(const doub
 template <int NH>
 void launch_tridiag(const double* C, int n, double* ws, cudaStream_t s) {
   const int threads = (2 * n + 31) / 32 * 32 + 32;
-  launch_pdl(core_tridiag_kernel<NH>, dim3(1), dim3(threads), 0, s, C, n, ws);
+  core_tridiag_kernel<NH><<<1, threads, 0, s>>>(C, n, ws);
 }
 
 // ---------------------------------------------------------------------------
@@ -362,7 +361,6 @@ constexpr int kVecWarps = 4;   // warps per eigenvalue CTA
 
 __global__ void __launch_bounds__(32 * kVecWarps) core_vector_kernel(int n, double* ws, int max_rounds,
                                                                      int32_t* dev_status) {
-  pdl_prologue();
   __shared__ double d[kMaxN], e[kMaxN], e2[kMaxN], dp[kMaxN], dm[kMaxN], lp[kMaxN], um[kMaxN], z[kMaxN];
   __shared__ __align__(16) double bs[kMaxN];
   extern __shared__ __align__(16) double Vs[];  // n x n reflectors
@@ -631,7 +629,6 @@ MDEV double warp_norm(const double* v, int n) {
 }
 
 __global__ void __launch_bounds__(1024) core_finish_kernel(int n, double* ws, double* eval, float* evec) {
-  pdl_prologue();
   __shared__ double lam[kMaxN];
   const EigScratch S = scratch(ws, n);
   double* X = S.X;
@@ -716,8 +713,8 @@ void launch_core_eig(double* C, int n, int max_iters, double* eval, float* evec,
   else launch_tridiag<56>(C, n, ws, s);
   const size_t vsmem = static_cast<size_t>(n) * n * sizeof(double);
   if (!ensure_smem(reinterpret_cast<const void*>(core_vector_kernel), vsmem)) return;
-  launch_pdl(core_vector_kernel, dim3(n), dim3(32 * kVecWarps), vsmem, s, n, ws, max_iters, dev_status);
-  launch_pdl(core_finish_kernel, dim3(1), dim3(1024), 0, s, n, ws, eval, evec);
+  core_vector_kernel<<<n, 32 * kVecWarps, vsmem, s>>>(n, ws, max_iters, dev_status);
+  core_finish_kernel<<<1, 1024, 0, s>>>(n, ws, eval, evec);
 }
 
 }  // namespace metis

@@ -129,7 +129,6 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
                                                                      const __grid_constant__ CUtensorMap tmWhi,
                                                                      const __grid_constant__ CUtensorMap tmWlo,
                                                                      const __grid_constant__ CUtensorMap tmA) {
-  pdl_prologue();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const Layout lo = layout(p.kp, p.dtype);
@@ -414,7 +413,6 @@ __global__ void __launch_bounds__(256) factor_finish_kernel(float* U, int64_t m,
                                                             __nv_bfloat16* u_hi, __nv_bfloat16* u_lo,
                                                             __nv_bfloat16* w_hi, __nv_bfloat16* w_lo,
                                                             unsigned* amax) {
-  pdl_prologue();
   // thread (c, ry): column c of rows ry, ry + blockDim.y, ... of this CTA's
   // share (U's rows first, then V's); one atomic per CTA and matrix
   __shared__ float red[2][32];
@@ -494,7 +492,7 @@ void launch_factor_finish(float* U, int64_t m, float* V, int64_t n, int k, const
   const dim3 block(cols, 256 / cols);
   int64_t grid = (m + n + block.y - 1) / block.y;
   if (grid > 2 * sms) grid = 2 * sms;  // a few atomics per matrix, not one per warp
-  launch_pdl(factor_finish_kernel, dim3(static_cast<unsigned>(grid)), block, 0, s, U, m, V, n, k, sign, S, kp, u_hi, u_lo, w_hi,
+  factor_finish_kernel<<<static_cast<unsigned>(grid), block, 0, s>>>(U, m, V, n, k, sign, S, kp, u_hi, u_lo, w_hi,
                                                                      w_lo, amax);
 }
 
@@ -512,7 +510,7 @@ metis_status run_residual_quant(const ResidualParams& p, const ResidualOperands&
   const int sms = device_sm_count();
   const int64_t per = (tiles + sms - 1) / sms;
   const unsigned grid = static_cast<unsigned>((tiles + per - 1) / per);
-  launch_pdl(residual_quant_kernel, dim3(grid), dim3(kThreads), lo.total, s, p, uh, ul, wh, wl, ta);
+  residual_quant_kernel<<<grid, kThreads, lo.total, s>>>(p, uh, ul, wh, wl, ta);
   const cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return fail(METIS_ERR_CUDA, "residual_quant launch", cudaGetErrorString(e));
   return METIS_OK;

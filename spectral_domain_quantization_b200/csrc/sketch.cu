@@ -10,7 +10,6 @@
 //
 // The sketch is written transposed, Omega^T (lp x n, bf16, rows l..lp-1 zero),
 // which is the K-major operand layout the sketch GEMM wants.
-#include "abi_common.h"
 #include "common.cuh"
 #include "sketch.h"
 
@@ -36,7 +35,6 @@ MDEV uint4 philox(uint4 c, uint32_t k0, uint32_t k1) {
 
 // One thread per (row i, column pair c): Box-Muller in float64, rounded to bf16.
 __global__ void gaussian_omega_kernel(int64_t n, int l, uint64_t seed, __nv_bfloat16* omt, int64_t ldo) {
-  pdl_prologue();
   const int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x;
   const int c = blockIdx.y;
   if (i >= n) return;
@@ -198,7 +196,7 @@ void launch_gaussian_omega(int64_t n, int l, int lp, uint64_t seed, __nv_bfloat1
                            cudaStream_t s) {
   cudaMemsetAsync(omt, 0, static_cast<size_t>(lp) * ldo * 2, s);
   const dim3 grid(static_cast<unsigned>((n + 255) / 256), static_cast<unsigned>((l + 1) / 2));
-  launch_pdl(gaussian_omega_kernel, dim3(grid), dim3(256), 0, s, n, l, seed, omt, ldo);
+  gaussian_omega_kernel<<<grid, 256, 0, s>>>(n, l, seed, omt, ldo);
 }
 
 void launch_sparse_sign(int64_t n, int l, int lp, int nnz, uint64_t seed, __nv_bfloat16* omt, int64_t ldo,

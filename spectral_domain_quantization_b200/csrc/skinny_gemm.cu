@@ -72,7 +72,6 @@ __host__ __device__ inline SkinnySmem skinny_smem(int aparts, int nmma, int lp, 
 __global__ void __launch_bounds__(128) skinny_gemm_kernel(const SkinnyParams p, const __grid_constant__ CUtensorMap tmA0,
                                                           const __grid_constant__ CUtensorMap tmA1,
                                                           const __grid_constant__ CUtensorMap tmX) {
-  pdl_prologue();
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int cs = p.cs;
@@ -338,15 +337,13 @@ metis_status run_skinny_gemm(const SkinnyCall& c, cudaStream_t s) {
   cfg.blockDim = dim3(128);
   cfg.dynamicSmemBytes = static_cast<size_t>(L.total);
   cfg.stream = s;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = 1;
-  attr[0].val.clusterDim.y = static_cast<unsigned>(c.cs);
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;   // see pdl_prologue
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
+  cudaLaunchAttribute attr;
+  attr.id = cudaLaunchAttributeClusterDimension;
+  attr.val.clusterDim.x = 1;
+  attr.val.clusterDim.y = static_cast<unsigned>(c.cs);
+  attr.val.clusterDim.z = 1;
+  cfg.attrs = &attr;
+  cfg.numAttrs = 1;
   const cudaError_t e = cudaLaunchKernelEx(&cfg, skinny_gemm_kernel, p, ma0, ma1, mx);
   if (e != cudaSuccess) return fail(METIS_ERR_CUDA, "skinny_gemm launch", cudaGetErrorString(e));
   return METIS_OK;

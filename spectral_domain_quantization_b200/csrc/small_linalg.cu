@@ -75,7 +75,6 @@ constexpr int kGramRows = 32;
 // thread per 4 x 4 tile pair (blockDim covers (lp/4)(lp/4+1)/2 pairs).
 __global__ void __launch_bounds__(1024) gram_kernel(const float* __restrict__ Y, int64_t rows, int lp,
                                                     double* __restrict__ gpart) {
-  pdl_prologue();
   extern __shared__ double ys[];  // kGramRows x (lp + 1)
   const int ld = lp + 1;
   const int q4 = lp / 4;
@@ -101,7 +100,6 @@ __global__ void __launch_bounds__(1024) gram_kernel(const float* __restrict__ Y,
 constexpr int kReduceGroups = 8;
 __global__ void __launch_bounds__(256) gram_reduce_kernel(const double* __restrict__ gpart, int nblocks, int lp,
                                                           double* __restrict__ G) {
-  pdl_prologue();
   __shared__ double part[kReduceGroups][32];
   const int lane = threadIdx.x & 31, grp = threadIdx.x >> 5;
   const int nb = lp / 4;
@@ -302,7 +300,6 @@ MDEV void panel_update(double (&v)[kTile][kTile], const double* P, int I, int J)
 //    (B) the owners of the tiles below it solve their rows of panel K + 1.
 //  Inverse: X = L^-1 by 16 x 16 blocks (see below).
 __global__ void __launch_bounds__(kSmallThreads, 1) cholesky_inv_kernel(const double* G, int lp, float* Rinv) {
-  pdl_prologue();
   extern __shared__ double sm[];
   const int ld = lp + 1;
   double* pan = sm;               // 2 panel buffers of (lp / 4) x kPanStride
@@ -482,13 +479,9 @@ MDEV void apply_block(const ApplyArgs& a, int64_t blk) {
   }
 }
 
-__global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) {
-  pdl_prologue();
-  apply_block(a, blockIdx.x);
-}
+__global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) { apply_block(a, blockIdx.x); }
 
 __global__ void __launch_bounds__(256) apply2_kernel(ApplyArgs a, ApplyArgs b, int64_t blocks_a) {
-  pdl_prologue();
   if (blockIdx.x < blocks_a)
     apply_block(a, blockIdx.x);
   else
@@ -500,7 +493,6 @@ __global__ void __launch_bounds__(256) apply2_kernel(ApplyArgs a, ApplyArgs b, i
 // S = sigma_k.
 __global__ void factor_mats_kernel(const double* eval, const float* evec, int lp, int k, float* Mu, float* Mv,
                                    float* S) {
-  pdl_prologue();
   // block i, thread j: entry (i, j) of Mu and Mv
   const int i = blockIdx.x, j = threadIdx.x;
   if (j >= k) return;
@@ -519,7 +511,6 @@ constexpr int kSignRows = kApplyRows;  // the sign convention's row blocks are t
 // keeps the largest |U| (the lowest block, hence the lowest row, on ties).
 __global__ void sign_kernel(const float* __restrict__ U, const float* __restrict__ bmax,
                             const int64_t* __restrict__ bidx, int nblocks, int k, float* sign) {
-  pdl_prologue();
   const int j = blockIdx.x, lane = threadIdx.x;
   // below every block maximum (colmax reports -1 for a block with no value
   // above -1, e.g. NaN entries), so each lane with a block picks one and the
@@ -560,14 +551,14 @@ void launch_gram(const float* Y, int64_t rows, int lp, double* gpart, double* G,
   const int nb = static_cast<int>(gram_blocks(rows));
   const int pairs = (lp / 4) * (lp / 4 + 1) / 2;
   const int threads = (pairs + 31) / 32 * 32;
-  launch_pdl(gram_kernel, dim3(nb), dim3(threads), kGramRows * (lp + 1) * sizeof(double), s, Y, rows, lp, gpart);
+  gram_kernel<<<nb, threads, kGramRows * (lp + 1) * sizeof(double), s>>>(Y, rows, lp, gpart);
   launch_gram_reduce(gpart, nb, lp, G, s);
 }
 
 void launch_gram_reduce(const double* gpart, int nblocks, int lp, double* G, cudaStream_t s) {
   const int nb = lp / 4;
   const int npk = 8 * nb * (nb + 1);
-  launch_pdl(gram_reduce_kernel, dim3((npk + 31) / 32), dim3(32 * kReduceGroups), 0, s, gpart, nblocks, lp, G);
+  gram_reduce_kernel<<<(npk + 31) / 32, 32 * kReduceGroups, 0, s>>>(gpart, nblocks, lp, G);
 }
 
 void launch_cholesky_inv(const double* G, int lp, float* Rinv, cudaStream_t s) {
@@ -575,7 +566,7 @@ void launch_cholesky_inv(const double* G, int lp, float* Rinv, cudaStream_t s) {
   const size_t smem = ((2 * static_cast<size_t>(lp) + 16) * (lp + 1) + 2 * (lp / kTile) * kPanStride + 3 * lp) *
                       sizeof(double);
   if (!ensure_smem(reinterpret_cast<const void*>(cholesky_inv_kernel), smem)) return;
-  launch_pdl(cholesky_inv_kernel, dim3(1), dim3(kSmallThreads), smem, s, G, lp, Rinv);
+  cholesky_inv_kernel<<<1, kSmallThreads, smem, s>>>(G, lp, Rinv);
 }
 
 size_t apply_smem(const ApplyArgs& a) {
@@ -586,7 +577,7 @@ size_t apply_smem(const ApplyArgs& a) {
 void launch_apply(const ApplyArgs& a, cudaStream_t s) {
   const size_t smem = apply_smem(a);
   if (!ensure_smem(reinterpret_cast<const void*>(apply_kernel), smem)) return;
-  launch_pdl(apply_kernel, dim3(static_cast<unsigned>(apply_blocks(a.rows))), dim3(256), smem, s, a);
+  apply_kernel<<<static_cast<unsigned>(apply_blocks(a.rows)), 256, smem, s>>>(a);
 }
 
 void launch_apply2(const ApplyArgs& a, const ApplyArgs& b, cudaStream_t s) {
@@ -594,12 +585,12 @@ void launch_apply2(const ApplyArgs& a, const ApplyArgs& b, cudaStream_t s) {
   const size_t smem = sa > sb ? sa : sb;
   if (!ensure_smem(reinterpret_cast<const void*>(apply2_kernel), smem)) return;
   const int64_t na = apply_blocks(a.rows), nb = apply_blocks(b.rows);
-  launch_pdl(apply2_kernel, dim3(static_cast<unsigned>(na + nb)), dim3(256), smem, s, a, b, na);
+  apply2_kernel<<<static_cast<unsigned>(na + nb), 256, smem, s>>>(a, b, na);
 }
 
 void launch_factor_mats(const double* eval, const float* evec, int lp, int k, float* Mu, float* Mv, float* S,
                         cudaStream_t s) {
-  launch_pdl(factor_mats_kernel, dim3(lp), dim3((k + 31) / 32 * 32), 0, s, eval, evec, lp, k, Mu, Mv, S);
+  factor_mats_kernel<<<lp, (k + 31) / 32 * 32, 0, s>>>(eval, evec, lp, k, Mu, Mv, S);
 }
 
 int64_t sign_blocks(int64_t rows) { return (rows + kSignRows - 1) / kSignRows; }
@@ -608,7 +599,7 @@ void launch_signs_from_blocks(float* U, int64_t m, float* V, int64_t n, int k, c
                               const int64_t* bidx, float* sign, cudaStream_t s) {
   (void)V;
   (void)n;
-  launch_pdl(sign_kernel, dim3(k), dim3(32), 0, s, U, bmax, bidx, static_cast<int>(sign_blocks(m)), k, sign);
+  sign_kernel<<<k, 32, 0, s>>>(U, bmax, bidx, static_cast<int>(sign_blocks(m)), k, sign);
 }
 
 
