@@ -759,6 +759,10 @@ class SampledWorkload:
                                         f"the product on {rows} of {self.M} rows, scaled x{self.M // rows}")
 
 
+WORKLOADS = {"averis_32768": AverisWorkload, "llama3_8b_mlp": LlamaMlpWorkload,
+             "sampled_65536": SampledWorkload}
+
+
 def _pinned_bf16(mat):
     import torch
     return torch.from_numpy(mat.data.view(np.int16)).view(torch.bfloat16).pin_memory()
@@ -776,8 +780,7 @@ def run_workload(args, rank, world, local):
     torch.cuda.set_device(dev)
     if not api.lib().metis_device_supported():
         raise RuntimeError("metis needs an sm_100 (B200) device")
-    wl = {"averis_32768": AverisWorkload, "llama3_8b_mlp": LlamaMlpWorkload,
-          "sampled_65536": SampledWorkload}[args.workload](dev)
+    wl = WORKLOADS[args.workload](dev)
     flush = torch.empty(512 << 20, dtype=torch.uint8, device=dev)
 
     def step():
@@ -901,11 +904,20 @@ def run_workload(args, rank, world, local):
 
 
 def run_profile(args, local):
-    """The step, eagerly and untimed: a short launch list for profilers."""
+    """The step, eagerly and untimed: a short launch list for profilers
+    (the single-layer step, or the --workload step)."""
     import torch
     from spectral_domain_quantization_b200 import api, inputs
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
+    if args.workload != "layer_4096":
+        wl = WORKLOADS[args.workload](dev)
+        for _ in range(args.profile_steps):
+            wl.split()
+            wl.products()
+        torch.cuda.synchronize()
+        print(json.dumps({"profile_steps": args.profile_steps, "workload": args.workload}), flush=True)
+        return
     data = inputs.make("layer_4096")
     W = torch.from_numpy(data["W"].data.view(np.int16)).view(torch.bfloat16).to(dev)
     X = torch.from_numpy(data["X"].data.view(np.int16)).view(torch.bfloat16).to(dev)

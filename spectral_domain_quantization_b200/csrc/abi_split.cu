@@ -50,6 +50,7 @@ struct SplitPlan {
   int l, lp, k, kp, kq;  // kq = k padded to 16 (sampled P width); kp = k padded to 64
   int64_t ld_m, ld_n;    // padded lengths (multiples of 8) of transposed operands
   int cs_m, cs_n;        // K slices (cluster size) of the A X (rows ms) and A^T X passes
+  int cs_m2;             // the A X passes with a two-part (hi / lo) X
   int sampled, fp32;
 };
 
@@ -102,8 +103,13 @@ SplitPlan make_plan(int64_t m, int64_t n, int dtype, const metis_split_params* p
   p.ld_n = round_up64(n, 8);
   p.fp32 = dtype == METIS_F32;
   const int sms = device_sm_count();
+  // passes whose X has two parts (hi / lo; every pass but the sketch's) run
+  // fastest with at most 4 K slices per tile (measured: 12.8 against 13.9 us
+  // on 4096 x 4096 at 8 slices)
   p.cs_m = skinny_cluster(p.ms, n, sms);
+  p.cs_m2 = p.cs_m > 4 ? 4 : p.cs_m;
   p.cs_n = skinny_cluster(n, p.ms, sms);
+  if (p.cs_n > 4) p.cs_n = 4;
   return p;
 }
 
@@ -265,7 +271,7 @@ metis_status range_and_core(const SplitPlan& p, const SplitBuffers& b, const Sou
   for (int it = 0; it < power_iters; ++it) {
     METIS_TRY(skinny(src, 1, b.qt, p.ld_m, 2, lp, p.cs_n, b.Y, nullptr, 0, dev_status, s));
     METIS_TRY(cholqr(b, p.n, lp, b.Zn, p.ld_n, 1, s));
-    METIS_TRY(skinny(src, 0, b.qt, p.ld_n, 2, lp, p.cs_m, b.Y, nullptr, 0, dev_status, s));
+    METIS_TRY(skinny(src, 0, b.qt, p.ld_n, 2, lp, p.cs_m2, b.Y, nullptr, 0, dev_status, s));
     // one pass also for the final basis: the Gram is formed in float64 from
     // float32 data, so a pass leaves |Q^T Q - I| near kappa(Y) 2^-23
     METIS_TRY(cholqr(b, src.rows, lp, b.Qm, p.ld_m, 1, s));

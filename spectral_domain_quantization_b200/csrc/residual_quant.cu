@@ -7,15 +7,19 @@
 // feature list (MXFP4 / NVFP4).
 //
 // Persistent, warp-specialized kernel; one CTA per SM walks a contiguous run
-// of 128 x 64 tiles of A in row-band order:
+// of 128 x BN tiles of A in row-band order (BN = 128 where two stages of that
+// width fit in shared memory, else 64; a wider tile halves the MMA
+// instructions per output, and the MMA warp's issue rate is what bounds the
+// pass):
 //   warp 0      TMA producer: the band's rows of U (hi, lo; reloaded only
-//               when the band changes) and, per tile, the 64 rows of
-//               W = V diag(S) (hi, lo) and the 128 x 64 tile of A, into a ring
+//               when the band changes) and, per tile, the BN rows of
+//               W = V diag(S) (hi, lo) and the 128 x BN tile of A, into a ring
 //               of shared-memory stages;
 //   warp 1      TMEM owner and MMA issuer: U_hi W_hi + U_hi W_lo + U_lo W_hi as
-//               kind::f16 MMAs (M 128, N 64) into one of four TMEM
+//               kind::f16 MMAs (M 128, N BN) into one of four TMEM
 //               accumulators, so L = U S V^T to ~2^-16 relative;
-//   warps 2-9   epilogue, 32 rows x 32 columns each: L from TMEM, A from the
+//   warps 2-9   epilogue, 32 rows x 32 columns per chunk (BN / 64 chunks
+//               each): L from TMEM, A from the
 //               swizzled stage, R = fl32(a - l); then either the tensor
 //               maximum of |R| (the NVFP4 pre-pass) or the FP4 codes: blocks
 //               along n straight from registers, blocks along m through a
@@ -92,16 +96,15 @@ MDEV void emit(const float* v, int n, int fmt, float s_t, const float* enc_tab, 
 
 
 constexpr int kBM = 128;         // tile rows (one band)
-constexpr int kBN = 64;          // tile columns
-constexpr int kAccBufs = 4;      // TMEM accumulators of kBN columns
-constexpr int kTmemCols = kAccBufs * kBN;
+constexpr int kAccBufs = 4;      // TMEM accumulators of BN columns
 constexpr int kEpiWarps = 8;
 constexpr int kThreads = 32 * (2 + kEpiWarps);
-constexpr int kMaxStages = 4;
+constexpr int kMaxStages = 6;
 constexpr int kSmemLimit = 232448;  // opt-in shared memory per CTA on sm_100
 constexpr int kTransposeBytes = kEpiWarps * 32 * 33 * 4;
 
 struct Layout {
+  int bn;           // tile columns: 128, or 64 where two such stages do not fit
   int chunks;       // kp / 64
   int u_bytes;      // U hi + lo
   int w_bytes;      // per stage: W hi + lo
@@ -110,17 +113,25 @@ struct Layout {
   int total;        // dynamic shared memory including 1024 B of alignment slack
 };
 
-__host__ __device__ inline Layout layout(int kp, int dtype) {
+// `transpose`: the column-axis codes need the per-warp transpose buffer;
+// without them its space goes to more stages.
+__host__ __device__ inline Layout layout_bn(int kp, int dtype, bool transpose, int bn) {
   Layout l{};
+  l.bn = bn;
   l.chunks = kp / 64;
   l.u_bytes = 2 * l.chunks * kBM * 128;
-  l.w_bytes = 2 * l.chunks * kBN * 128;
-  l.a_bytes = kBM * kBN * (dtype == METIS_BF16 ? 2 : 4);
-  const int fixed = 1024 + l.u_bytes + kTransposeBytes + 1024;  // barriers 256 B, encode table 512 B
+  l.w_bytes = 2 * l.chunks * bn * 128;
+  l.a_bytes = kBM * bn * (dtype == METIS_BF16 ? 2 : 4);
+  const int fixed = 1024 + l.u_bytes + (transpose ? kTransposeBytes : 0) + 1024;  // barriers 256 B, encode table 512 B
   int st = (kSmemLimit - fixed) / (l.w_bytes + l.a_bytes);
   l.stages = st > kMaxStages ? kMaxStages : st;
   l.total = fixed + l.stages * (l.w_bytes + l.a_bytes);
   return l;
+}
+
+__host__ __device__ inline Layout layout(int kp, int dtype, bool transpose) {
+  const Layout wide = layout_bn(kp, dtype, transpose, 128);
+  return wide.stages >= 2 ? wide : layout_bn(kp, dtype, transpose, 64);
 }
 
 __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const ResidualParams p,
@@ -131,14 +142,15 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
                                                                      const __grid_constant__ CUtensorMap tmA) {
   extern __shared__ __align__(1024) uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  const Layout lo = layout(p.kp, p.dtype);
+  const bool transpose = p.c_codes != nullptr;
+  const Layout lo = layout(p.kp, p.dtype, transpose);
   const int S = lo.stages;
   uint8_t* sUhi = smem;
   uint8_t* sUlo = sUhi + lo.u_bytes / 2;
   uint8_t* sStage = smem + lo.u_bytes;
   const int stage_bytes = lo.w_bytes + lo.a_bytes;
   float* tstage = reinterpret_cast<float*>(sStage + S * stage_bytes);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(tstage) + kTransposeBytes);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<uint8_t*>(tstage) + (transpose ? kTransposeBytes : 0));
   uint64_t* full = bars;                           // [kMaxStages]
   uint64_t* empty = full + kMaxStages;             // [kMaxStages]
   uint64_t* acc_full = empty + kMaxStages;         // [kAccBufs]
@@ -172,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
     prefetch_tensormap(&tmA);
   }
   if (warp == 1) {
-    tmem_alloc(tmem_sh, kTmemCols);
+    tmem_alloc(tmem_sh, static_cast<uint32_t>(kAccBufs * lo.bn));
     tmem_relinquish();
   }
   if (p.mode == 1 && p.fmt == METIS_NVFP4) nv_enc_table(nv_tensor_scale(__uint_as_float(*p.amax_bits)), enc_tab);
@@ -182,7 +194,8 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
   const uint32_t tmem = *tmem_sh;
 
   // this CTA's contiguous run of tiles, in row-band order
-  const int nt = static_cast<int>((p.n + kBN - 1) / kBN);
+  const int bn = lo.bn;
+  const int nt = static_cast<int>((p.n + bn - 1) / bn);
   const int total = static_cast<int>((p.m + kBM - 1) / kBM) * nt;
   const int per = (total + gridDim.x - 1) / gridDim.x;
   const int t0 = blockIdx.x * per;
@@ -214,15 +227,13 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
         uint8_t* sA = sW + lo.w_bytes;
         mbar_arrive_expect_tx(&full[stage], stage_bytes);
         for (int c = 0; c < lo.chunks; ++c) {
-          tma_load_2d(sW + c * kBN * 128, &tmWhi, &full[stage], 64 * c, tn * kBN);
-          tma_load_2d(sW + (lo.chunks + c) * kBN * 128, &tmWlo, &full[stage], 64 * c, tn * kBN);
+          tma_load_2d(sW + c * bn * 128, &tmWhi, &full[stage], 64 * c, tn * bn);
+          tma_load_2d(sW + (lo.chunks + c) * bn * 128, &tmWlo, &full[stage], 64 * c, tn * bn);
         }
-        if (f32) {
-          tma_load_2d(sA, &tmA, &full[stage], tn * kBN, tm * kBM);
-          tma_load_2d(sA + kBM * 128, &tmA, &full[stage], tn * kBN + 32, tm * kBM);
-        } else {
-          tma_load_2d(sA, &tmA, &full[stage], tn * kBN, tm * kBM);
-        }
+        // A: boxes of 128 bytes per row (32 float32 or 64 bf16 columns)
+        const int box_cols = f32 ? 32 : 64;
+        for (int b = 0; b < bn / box_cols; ++b)
+          tma_load_2d(sA + b * kBM * 128, &tmA, &full[stage], tn * bn + box_cols * b, tm * kBM);
         ++issued;
         if (++stage == S) {
           stage = 0;
@@ -248,7 +259,7 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
     if (lane == 0) {
       int stage = 0, acc = 0, bands = 0, cur_tm = -1;
       uint32_t ph = 0, aph = 0;
-      const uint32_t idesc = idesc_bf16(kBM, kBN, false, false);
+      const uint32_t idesc = idesc_bf16(kBM, bn, false, false);
       for (int t = t0; t < t1; ++t) {
         const int tm = t / nt;
         if (tm != cur_tm) {
@@ -261,13 +272,13 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
         if (!mbar_wait(&full[stage], ph, abort_flag)) break;
         tc_fence_after();
         uint8_t* sW = sStage + stage * stage_bytes;
-        const uint32_t d = tmem + static_cast<uint32_t>(acc * kBN);
+        const uint32_t d = tmem + static_cast<uint32_t>(acc * bn);
         uint32_t accumulate = 0;
         for (int c = 0; c < lo.chunks; ++c) {
           const uint64_t uh = make_sdesc(smem_u32(sUhi + c * kBM * 128), 16, 1024, kSwizzle128B);
           const uint64_t ul = make_sdesc(smem_u32(sUlo + c * kBM * 128), 16, 1024, kSwizzle128B);
-          const uint64_t wh = make_sdesc(smem_u32(sW + c * kBN * 128), 16, 1024, kSwizzle128B);
-          const uint64_t wl = make_sdesc(smem_u32(sW + (lo.chunks + c) * kBN * 128), 16, 1024, kSwizzle128B);
+          const uint64_t wh = make_sdesc(smem_u32(sW + c * bn * 128), 16, 1024, kSwizzle128B);
+          const uint64_t wl = make_sdesc(smem_u32(sW + (lo.chunks + c) * bn * 128), 16, 1024, kSwizzle128B);
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
             const uint64_t o = static_cast<uint64_t>(2 * j);  // 32 bytes of K per step
@@ -297,7 +308,7 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
   } else {
     // ------------------------------------------------------------ epilogue
     const int q = warp & 3;             // TMEM lane quadrant: rows 32 q .. 32 q + 31
-    const int h = (warp - 2) >> 2;      // columns 32 h .. 32 h + 31 of the tile
+    const int h = (warp - 2) >> 2;      // chunk parity: columns 32 h .. (and 32 (h + 2) .. for BN = 128)
     float* my_t = tstage + (warp - 2) * 32 * 33;
     float s_t = 1.f;
     if (p.mode == 1 && p.fmt == METIS_NVFP4) s_t = nv_tensor_scale(__uint_as_float(*p.amax_bits));
@@ -308,50 +319,63 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
     float amax = 0.f;
     int stage = 0, acc = 0;
     uint32_t ph = 0, aph = 0;
+    const int nc = bn / 64;             // 32-column chunks of this warp: h, h + 2 (BN = 128)
     for (int t = t0; t < t1; ++t) {
       const int tm = t / nt, tn = t - tm * nt;
       if (!mbar_wait(&acc_full[acc], aph, abort_flag)) break;
       tc_fence_after();
-      uint32_t L[32];
-      tmem_ld16(tmem + (static_cast<uint32_t>(32 * q) << 16) + acc * kBN + 32 * h, L);
-      tmem_ld16(tmem + (static_cast<uint32_t>(32 * q) << 16) + acc * kBN + 32 * h + 16, L + 16);
+      uint32_t L[2][32];
+#pragma unroll
+      for (int cc = 0; cc < 2; ++cc) {
+        if (cc < nc) {
+          const uint32_t col = static_cast<uint32_t>(acc * bn + 32 * (h + 2 * cc));
+          tmem_ld16(tmem + (static_cast<uint32_t>(32 * q) << 16) + col, L[cc]);
+          tmem_ld16(tmem + (static_cast<uint32_t>(32 * q) << 16) + col + 16, L[cc] + 16);
+        }
+      }
       tmem_ld_wait();
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
       if (!mbar_wait(&full[stage], ph, abort_flag)) break;  // the A tile has landed
       const int r = 32 * q + lane;                          // row within the tile
-      const uint8_t* arow = sStage + stage * stage_bytes + lo.w_bytes + r * 128;
-      float v[32];
-      if (f32) {
-        const uint8_t* base = arow + h * kBM * 128;  // box h holds columns 32 h ..
+      const uint8_t* sA = sStage + stage * stage_bytes + lo.w_bytes;
+      float v[2][32];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const float4 f = *reinterpret_cast<const float4*>(base + ((j ^ (r & 7)) << 4));
-          v[4 * j] = f.x;
-          v[4 * j + 1] = f.y;
-          v[4 * j + 2] = f.z;
-          v[4 * j + 3] = f.w;
-        }
-      } else {
+      for (int cc = 0; cc < 2; ++cc) {
+        if (cc >= nc) continue;
+        const int ch = h + 2 * cc;                          // columns 32 ch .. 32 ch + 31
+        if (f32) {
+          const uint8_t* base = sA + ch * kBM * 128 + r * 128;  // box ch holds columns 32 ch ..
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int j = 4 * h + jj;
-          const uint4 u = *reinterpret_cast<const uint4*>(arow + ((j ^ (r & 7)) << 4));
-          const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+          for (int j = 0; j < 8; ++j) {
+            const float4 f = *reinterpret_cast<const float4*>(base + ((j ^ (r & 7)) << 4));
+            v[cc][4 * j] = f.x;
+            v[cc][4 * j + 1] = f.y;
+            v[cc][4 * j + 2] = f.z;
+            v[cc][4 * j + 3] = f.w;
+          }
+        } else {
+          const uint8_t* base = sA + (ch >> 1) * kBM * 128 + r * 128;  // box ch / 2 holds columns 64 (ch / 2) ..
 #pragma unroll
-          for (int i = 0; i < 4; ++i) {
-            v[8 * jj + 2 * i] = __uint_as_float(w[i] << 16);
-            v[8 * jj + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+          for (int jj = 0; jj < 4; ++jj) {
+            const int j = 4 * (ch & 1) + jj;
+            const uint4 u = *reinterpret_cast<const uint4*>(base + ((j ^ (r & 7)) << 4));
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              v[cc][8 * jj + 2 * i] = __uint_as_float(w[i] << 16);
+              v[cc][8 * jj + 2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+            }
           }
         }
-      }
-      // the residual: using every loaded value here means the shared-memory
-      // reads have returned before the stage is handed back to the producer
-      // (a load whose value is first used after the arrive could still be
-      // reading while the next TMA copy lands in the stage)
+        // the residual: using every loaded value before the stage is handed
+        // back means the shared-memory reads have returned (a load whose
+        // value is first used after the arrive could still be reading while
+        // the next TMA copy lands in the stage)
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = __fsub_rn(v[j], __uint_as_float(L[j]));
+        for (int j = 0; j < 32; ++j) v[cc][j] = __fsub_rn(v[cc][j], __uint_as_float(L[cc][j]));
+      }
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[stage]);
       if (++stage == S) {
@@ -363,30 +387,35 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
         aph ^= 1u;
       }
       const int64_t row0 = static_cast<int64_t>(tm) * kBM + 32 * q;
-      const int64_t col0 = static_cast<int64_t>(tn) * kBN + 32 * h;
-      if (row0 >= p.m || col0 >= p.n) continue;  // m, n are multiples of 32: whole warp
       const int64_t row = row0 + lane;
-      if (p.mode == 0) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(v[j]));
-        continue;
-      }
-      if (p.r_tap) {
-        float* tp = p.r_tap + row * p.n + col0;
+      for (int cc = 0; cc < 2; ++cc) {
+        if (cc >= nc) continue;
+        const int64_t col0 = static_cast<int64_t>(tn) * bn + 32 * (h + 2 * cc);
+        if (row0 >= p.m || col0 >= p.n) continue;  // m, n are multiples of 32: whole warp
+        const float* vc = v[cc];
+        if (p.mode == 0) {
 #pragma unroll
-        for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4*>(tp + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
-      }
-      if (p.r_codes) emit(v, 32, p.fmt, s_t, enc_tab, p.r_codes, p.r_scales, p.r_scale_cols, p.n, row, col0);
-      if (p.c_codes) {
-        // the warp's 32 rows x 32 columns, transposed through shared memory
+          for (int j = 0; j < 32; ++j) amax = fmaxf(amax, fabsf(vc[j]));
+          continue;
+        }
+        if (p.r_tap) {
+          float* tp = p.r_tap + row * p.n + col0;
 #pragma unroll
-        for (int j = 0; j < 32; ++j) my_t[lane * 33 + j] = v[j];
-        __syncwarp();
-        float col[32];
+          for (int j = 0; j < 32; j += 4) *reinterpret_cast<float4*>(tp + j) = make_float4(vc[j], vc[j + 1], vc[j + 2], vc[j + 3]);
+        }
+        if (p.r_codes) emit(vc, 32, p.fmt, s_t, enc_tab, p.r_codes, p.r_scales, p.r_scale_cols, p.n, row, col0);
+        if (p.c_codes) {
+          // the warp's 32 rows x 32 columns, transposed through shared memory
 #pragma unroll
-        for (int i = 0; i < 32; ++i) col[i] = my_t[i * 33 + lane];
-        __syncwarp();
-        emit(col, 32, p.fmt, s_t, enc_tab, p.c_codes, p.c_scales, p.c_scale_cols, p.m, col0 + lane, row0);
+          for (int j = 0; j < 32; ++j) my_t[lane * 33 + j] = vc[j];
+          __syncwarp();
+          float col[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) col[i] = my_t[i * 33 + lane];
+          __syncwarp();
+          emit(col, 32, p.fmt, s_t, enc_tab, p.c_codes, p.c_scales, p.c_scale_cols, p.m, col0 + lane, row0);
+        }
       }
     }
     if (p.mode == 0) {
@@ -398,7 +427,7 @@ __global__ void __launch_bounds__(kThreads, 1) residual_quant_kernel(const Resid
   __syncthreads();
   if (warp == 1) {
     tc_fence_after();
-    tmem_dealloc(tmem, kTmemCols);
+    tmem_dealloc(tmem, static_cast<uint32_t>(kAccBufs * lo.bn));
   }
   if (threadIdx.x == 0 && *abort_flag) report(p.dev_status, METIS_DEV_TIMEOUT);
 }
@@ -497,16 +526,16 @@ void launch_factor_finish(float* U, int64_t m, float* V, int64_t n, int k, const
 }
 
 metis_status run_residual_quant(const ResidualParams& p, const ResidualOperands& o, cudaStream_t s) {
+  const Layout lo = layout(p.kp, p.dtype, p.c_codes != nullptr);
   CUtensorMap uh, ul, wh, wl, ta;
   if (map_kmajor(&uh, o.u_hi, p.m, p.kp, kBM) != CUDA_SUCCESS || map_kmajor(&ul, o.u_lo, p.m, p.kp, kBM) != CUDA_SUCCESS ||
-      map_kmajor(&wh, o.w_hi, p.n, p.kp, kBN) != CUDA_SUCCESS || map_kmajor(&wl, o.w_lo, p.n, p.kp, kBN) != CUDA_SUCCESS ||
+      map_kmajor(&wh, o.w_hi, p.n, p.kp, lo.bn) != CUDA_SUCCESS || map_kmajor(&wl, o.w_lo, p.n, p.kp, lo.bn) != CUDA_SUCCESS ||
       map_a(&ta, p) != CUDA_SUCCESS)
     return fail(METIS_ERR_CUDA, "residual tensor map");
-  const Layout lo = layout(p.kp, p.dtype);
   if (lo.stages < 2) return fail(METIS_ERR_SHAPE, "residual", "factor rank too large for the shared-memory stages");
   if (!ensure_smem(reinterpret_cast<const void*>(residual_quant_kernel), lo.total))
     return fail(METIS_ERR_CUDA, "residual shared-memory attribute");
-  const int64_t tiles = ((p.m + kBM - 1) / kBM) * ((p.n + kBN - 1) / kBN);
+  const int64_t tiles = ((p.m + kBM - 1) / kBM) * ((p.n + lo.bn - 1) / lo.bn);
   const int sms = device_sm_count();
   const int64_t per = (tiles + sms - 1) / sms;
   const unsigned grid = static_cast<unsigned>((tiles + per - 1) / per);
