@@ -108,13 +108,13 @@ ProductPlan plan(const metis_operand* A, const metis_operand* B, int64_t M, int6
 // Workspace of one product; with ws.base == NULL only sizes are summed.
 struct ProductBuffers {
   __nv_bfloat16 *la = nullptr, *lb = nullptr;
-  float *t1 = nullptr, *t1p = nullptr, *t2 = nullptr, *t2p = nullptr, *cab = nullptr;
+  float *t1 = nullptr, *t1p = nullptr, *t2 = nullptr, *t2p = nullptr, *cab = nullptr, *cabp = nullptr;
   float* t1full = nullptr;      // re-quantized T1: its float32 values
   unsigned* amax = nullptr;     // [2]: max |T1|, max |T2| (NVFP4)
 };
 
 ProductBuffers carve(const ProductPlan& p, const metis_operand* A, const metis_operand* B, int64_t M,
-                     int64_t N, Carver& ws) {
+                     int64_t N, int64_t K, Carver& ws) {
   ProductBuffers b;
   if (!p.lr_k) return b;
   b.la = ws.take<__nv_bfloat16>(static_cast<size_t>(M) * p.lr_k);
@@ -127,7 +127,10 @@ ProductBuffers carve(const ProductPlan& p, const metis_operand* A, const metis_o
     b.t2 = ws.take<float>(static_cast<size_t>(p.ka) * N);
     if (p.s2 > 1) b.t2p = ws.take<float>(static_cast<size_t>(p.s2) * p.ka * N);
   }
-  if (p.ka && p.kb) b.cab = ws.take<float>(static_cast<size_t>(p.ka) * p.kb);
+  if (p.ka && p.kb) {
+    b.cab = ws.take<float>(static_cast<size_t>(p.ka) * p.kb);
+    b.cabp = ws.take<float>(static_cast<size_t>(cab_parts(K, device_sm_count())) * p.ka * p.kb);
+  }
   if (p.kb && (B->flags & METIS_REQUANT_LOWRANK)) b.t1full = ws.take<float>(static_cast<size_t>(M) * p.kb);
   if ((p.kb && (B->flags & METIS_REQUANT_LOWRANK)) || (p.ka && (A->flags & METIS_REQUANT_LOWRANK)))
     b.amax = ws.take<unsigned>(2);
@@ -152,7 +155,7 @@ metis_status enqueue_product(const metis_operand* A, const metis_operand* B, int
                              void* C, int c_dtype, int64_t ldc, Carver& ws, int32_t* dev_status,
                              cudaStream_t s) {
   const ProductPlan p = plan(A, B, M, N, K);
-  const ProductBuffers b = carve(p, A, B, M, N, ws);
+  const ProductBuffers b = carve(p, A, B, M, N, K, ws);
   if (!ws.base) return METIS_OK;
   const int sms = device_sm_count();
   LowRankArgs la{};
@@ -222,7 +225,8 @@ metis_status enqueue_product(const metis_operand* A, const metis_operand* B, int
     }
     if (p.ka && p.kb) {
       // an all-ones P contributes 1 at every position of the contraction
-      launch_cab(view_of(A->P), view_of(B->P), K, p.ka, p.kb, b.cab, s);
+      if (!launch_cab(view_of(A->P), view_of(B->P), K, p.ka, p.kb, b.cabp, b.cab, sms, s))
+        return fail(METIS_ERR_CUDA, "low-rank core product shared-memory attribute");
       la.cab = b.cab;
     }
     launch_build_lowrank(la, sms, s);
@@ -241,7 +245,7 @@ metis_status enqueue_product(const metis_operand* A, const metis_operand* B, int
 
 size_t product_workspace(const metis_operand* A, const metis_operand* B, int64_t M, int64_t N, int64_t K) {
   Carver c(nullptr);
-  carve(plan(A, B, M, N, K), A, B, M, N, c);
+  carve(plan(A, B, M, N, K), A, B, M, N, K, c);
   return c.used;
 }
 

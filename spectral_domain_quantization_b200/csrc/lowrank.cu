@@ -15,6 +15,7 @@
 // bf16 (<= 6 significant bits); fp32 T1/T2 enter as a bf16 hi/lo pair:
 //   LA[m] = [hi(T1') | lo(T1') | F~_A | F~_A | 0...]
 //   LB[n] = [F~_B    | F~_B    | hi(T2') | lo(T2') | 0...]
+#include "abi_common.h"
 #include "common.cuh"
 #include "fp4_block.cuh"
 #include "lowrank.h"
@@ -22,6 +23,8 @@
 namespace metis {
 
 namespace {
+
+constexpr int kMaxLowRank = 128;   // k of one operand (checked by the ABI)
 
 // Dequantized value of factor element (row i of `outer`, position l of
 // `inner`) without the NVFP4 tensor scale.
@@ -39,19 +42,89 @@ MDEV float tscale(const FactorView& f) {
   return (f.ones || f.fmt != METIS_NVFP4 || !f.tensor_scale) ? 1.f : *f.tensor_scale;
 }
 
-// Cab[i][j] = sum_l P^_A[i][l] P^_B[j][l] (with tensor scales), one block per (i, j).
-__global__ void cab_kernel(FactorView pa, FactorView pb, int64_t K, int kb, float* cab) {
-  const int i = blockIdx.y, j = blockIdx.x;
-  float s = 0.f;
-  for (int64_t l = threadIdx.x; l < K; l += blockDim.x) s += factor_value(pa, i, l) * factor_value(pb, j, l);
-  __shared__ float red[256];
-  red[threadIdx.x] = s;
-  __syncthreads();
-  for (int w = blockDim.x / 2; w > 0; w >>= 1) {
-    if (threadIdx.x < w) red[threadIdx.x] += red[threadIdx.x + w];
+// Cab[i][j] = sum_l P^_A[i][l] P^_B[j][l] (with tensor scales), a ka x kb
+// product over the whole contraction.  Each CTA takes a run of positions,
+// decodes both factors 64 positions at a time into shared memory (each
+// value once, as float: exact) and accumulates 4 x 4 output tiles in
+// registers; its partial goes to part[cta][i][j], and cab_reduce_kernel adds
+// the partials in CTA order (deterministic) and applies the tensor scales.
+constexpr int kCabStep = 64;     // positions decoded per round
+constexpr int kCabThreads = 256;
+
+__host__ __device__ inline int cab_pad(int k) { return (k + 3) / 4 * 4; }
+__host__ __device__ inline int cab_stride(int k) { return cab_pad(k) + 4; }   // 16-byte rows, spread banks
+
+__global__ void __launch_bounds__(kCabThreads) cab_part_kernel(FactorView pa, FactorView pb, int64_t K, int ka,
+                                                               int kb, int64_t per_cta, float* part) {
+  extern __shared__ float cab_sm[];
+  const int sa = cab_stride(ka), sb = cab_stride(kb);
+  float* A = cab_sm;                      // [kCabStep][sa]: A[l][i] = P^_A[i][l0 + l]
+  float* B = A + kCabStep * sa;           // [kCabStep][sb]
+  const int nib = cab_pad(ka) / 4, njb = cab_pad(kb) / 4, ntiles = nib * njb;
+  const int64_t l0 = static_cast<int64_t>(blockIdx.x) * per_cta;
+  const int64_t l1 = l0 + per_cta < K ? l0 + per_cta : K;
+  constexpr int kMaxTiles = (kMaxLowRank / 4) * (kMaxLowRank / 4) / kCabThreads;
+  float acc[kMaxTiles][4][4];
+#pragma unroll
+  for (int t = 0; t < kMaxTiles; ++t)
+#pragma unroll
+    for (int x = 0; x < 4; ++x)
+#pragma unroll
+      for (int y = 0; y < 4; ++y) acc[t][x][y] = 0.f;
+  for (int64_t base = l0; base < l1; base += kCabStep) {
+    __syncthreads();   // the previous round's values are consumed
+    for (int e = threadIdx.x; e < kCabStep * (cab_pad(ka) + cab_pad(kb)); e += kCabThreads) {
+      const int l = e % kCabStep, r = e / kCabStep;
+      const int64_t pos = base + l;
+      const bool isa = r < cab_pad(ka);
+      const int row = isa ? r : r - cab_pad(ka);
+      const int lim = isa ? ka : kb;
+      const float v = (row < lim && pos < l1) ? factor_value(isa ? pa : pb, row, pos) : 0.f;
+      (isa ? A + l * sa : B + l * sb)[row] = v;
+    }
     __syncthreads();
+#pragma unroll
+    for (int t = 0; t < kMaxTiles; ++t) {
+      const int tile = threadIdx.x + t * kCabThreads;
+      if (tile < ntiles) {
+        const int ib = tile % nib, jb = tile / nib;
+#pragma unroll 4
+        for (int l = 0; l < kCabStep; ++l) {
+          const float4 x = *reinterpret_cast<const float4*>(A + l * sa + 4 * ib);
+          const float4 y = *reinterpret_cast<const float4*>(B + l * sb + 4 * jb);
+          const float xv[4] = {x.x, x.y, x.z, x.w}, yv[4] = {y.x, y.y, y.z, y.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u)
+#pragma unroll
+            for (int w = 0; w < 4; ++w) acc[t][u][w] = fmaf(xv[u], yv[w], acc[t][u][w]);
+        }
+      }
+    }
   }
-  if (threadIdx.x == 0) cab[i * kb + j] = red[0] * tscale(pa) * tscale(pb);
+  float* out = part + static_cast<int64_t>(blockIdx.x) * ka * kb;
+#pragma unroll
+  for (int t = 0; t < kMaxTiles; ++t) {
+    const int tile = threadIdx.x + t * kCabThreads;
+    if (tile < ntiles) {
+      const int ib = tile % nib, jb = tile / nib;
+#pragma unroll
+      for (int u = 0; u < 4; ++u)
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          const int i = 4 * ib + u, j = 4 * jb + w;
+          if (i < ka && j < kb) out[i * kb + j] = acc[t][u][w];
+        }
+    }
+  }
+}
+
+__global__ void cab_reduce_kernel(FactorView pa, FactorView pb, int ka, int kb, int nparts, const float* part,
+                                  float* cab) {
+  const int e = blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= ka * kb) return;
+  float s = 0.f;
+  for (int c = 0; c < nparts; ++c) s += part[static_cast<int64_t>(c) * ka * kb + e];
+  cab[e] = s * tscale(pa) * tscale(pb);
 }
 
 MDEV void split_hi_lo(float x, __nv_bfloat16& hi, __nv_bfloat16& lo) {
@@ -159,11 +232,12 @@ __global__ void t2_amax_kernel(LowRankArgs a) {
   }
 }
 
-constexpr int kMaxLowRank = 128;   // k of one operand (checked by the ABI)
-
-// LA: a row per block iteration, a column per thread.
+// LA: a row per block iteration.  F_A's ka values at the row are decoded
+// once into shared memory, T1's kb values (with the C_ab term) formed once,
+// then the lr_k bf16 columns written a column per thread.
 __global__ void build_la_kernel(LowRankArgs a) {
-  __shared__ float row[kMaxLowRank];
+  __shared__ float row[kMaxLowRank];   // T1's row: re-quantized, or scaled for the hi / lo split
+  __shared__ float far[kMaxLowRank];   // F_A at the row, without its tensor scale
   const float inv_alpha = 1.f / alpha_main(a);
   const float s_fb = tscale(a.fb);
   const float s_fa = tscale(a.fa);
@@ -172,48 +246,55 @@ __global__ void build_la_kernel(LowRankArgs a) {
   const int bs = a.fmt == METIS_MXFP4 ? 32 : 16;
   const int kbp = (a.kb + bs - 1) / bs * bs;
   for (int64_t m = blockIdx.x; m < a.M; m += gridDim.x) {
-    if (a.requant_t1) {
-      // T1's row in blocks along kb (zero-padded), quantized and dequantized
+    for (int i = threadIdx.x; i < a.ka; i += blockDim.x) far[i] = factor_value(a.fa, i, m);
+    // T1's row in blocks along kb (zero-padded), quantized and dequantized
+    if (a.requant_t1)
       for (int j = threadIdx.x; j < kbp; j += blockDim.x) row[j] = j < a.kb ? a.t1full[m * a.kb + j] : 0.f;
-      __syncthreads();
+    __syncthreads();
+    if (a.requant_t1) {
       for (int b = threadIdx.x; b < kbp / bs; b += blockDim.x) requant_block(row + b * bs, a.fmt, s_t1);
-      __syncthreads();
-    }
-    for (int c = threadIdx.x; c < a.lr_k; c += blockDim.x) {
-      __nv_bfloat16 out = __float2bfloat16_rn(0.f);
-      if (c < 2 * a.kb && a.requant_t1) {
-        // code x block scale in both chunks; the F_B side carries s_t1
-        out = __float2bfloat16_rn(row[c < a.kb ? c : c - a.kb]);
-      } else if (c < 2 * a.kb + 2 * a.ka && c >= 2 * a.kb && a.requant_t2) {
-        const int cc = c - 2 * a.kb;
-        const int i = cc % a.ka;
-        const float w = factor_value(a.fa, i, m) * s_fa * s_t2 * inv_alpha;
-        __nv_bfloat16 hi, lo;
-        split_hi_lo(w, hi, lo);
-        out = cc < a.ka ? hi : lo;
-      } else if (c < 2 * a.kb) {
-        const int j = c < a.kb ? c : c - a.kb;
+    } else {
+      for (int j = threadIdx.x; j < a.kb; j += blockDim.x) {
         float v = t1_value(a, m, j);
         if (a.ka > 0 && a.cab) {
           float acc = 0.f;
           for (int i = 0; i < a.ka; ++i) {
             const float sa = a.s_a ? a.s_a[i] : 1.f;
-            acc += factor_value(a.fa, i, m) * s_fa * sa * a.cab[i * a.kb + j];
+            acc += far[i] * s_fa * sa * a.cab[i * a.kb + j];
           }
           v += acc;
         }
         const float sb = a.s_b ? a.s_b[j] : 1.f;
-        v = v * sb * s_fb * inv_alpha;
-        __nv_bfloat16 hi, lo;
-        split_hi_lo(v, hi, lo);
-        out = c < a.kb ? hi : lo;
+        row[j] = v * sb * s_fb * inv_alpha;
+      }
+    }
+    __syncthreads();
+    for (int c = threadIdx.x; c < a.lr_k; c += blockDim.x) {
+      __nv_bfloat16 out = __float2bfloat16_rn(0.f);
+      if (c < 2 * a.kb) {
+        const float v = row[c < a.kb ? c : c - a.kb];
+        if (a.requant_t1) {
+          // code x block scale in both chunks; the F_B side carries s_t1
+          out = __float2bfloat16_rn(v);
+        } else {
+          __nv_bfloat16 hi, lo;
+          split_hi_lo(v, hi, lo);
+          out = c < a.kb ? hi : lo;
+        }
       } else if (c < 2 * a.kb + 2 * a.ka) {
-        const int i = (c - 2 * a.kb) % a.ka;
-        out = __float2bfloat16_rn(factor_value(a.fa, i, m));
+        const int cc = c - 2 * a.kb;
+        const int i = cc % a.ka;
+        if (a.requant_t2) {
+          __nv_bfloat16 hi, lo;
+          split_hi_lo(far[i] * s_fa * s_t2 * inv_alpha, hi, lo);
+          out = cc < a.ka ? hi : lo;
+        } else {
+          out = __float2bfloat16_rn(far[i]);
+        }
       }
       a.la[m * a.lr_k + c] = out;
     }
-    if (a.requant_t1) __syncthreads();   // the row buffer is refilled next
+    __syncthreads();   // row and far are refilled next
   }
 }
 
@@ -299,9 +380,21 @@ int blocks_for(int64_t n, int sms) {
 
 }  // namespace
 
-void launch_cab(const FactorView& pa, const FactorView& pb, int64_t K, int ka, int kb, float* cab,
-                cudaStream_t s) {
-  cab_kernel<<<dim3(kb, ka), 256, 0, s>>>(pa, pb, K, kb, cab);
+int cab_parts(int64_t K, int sms) {
+  const int64_t steps = (K + kCabStep - 1) / kCabStep;
+  return static_cast<int>(steps < 2 * sms ? steps : 2 * sms);
+}
+
+bool launch_cab(const FactorView& pa, const FactorView& pb, int64_t K, int ka, int kb, float* part, float* cab,
+                int sms, cudaStream_t s) {
+  const int nparts = cab_parts(K, sms);
+  const int64_t steps = (K + kCabStep - 1) / kCabStep;
+  const int64_t per_cta = (steps + nparts - 1) / nparts * kCabStep;
+  const int smem = kCabStep * (cab_stride(ka) + cab_stride(kb)) * static_cast<int>(sizeof(float));
+  if (!ensure_smem(reinterpret_cast<const void*>(cab_part_kernel), static_cast<size_t>(smem))) return false;
+  cab_part_kernel<<<nparts, kCabThreads, smem, s>>>(pa, pb, K, ka, kb, per_cta, part);
+  cab_reduce_kernel<<<(ka * kb + 255) / 256, 256, 0, s>>>(pa, pb, ka, kb, nparts, part, cab);
+  return true;
 }
 
 int row_blocks(int64_t rows, int sms) {

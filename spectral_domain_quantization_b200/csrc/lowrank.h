@@ -51,8 +51,13 @@ struct LowRankArgs {
   unsigned* amax2;          // max |T2| bits (NVFP4)
 };
 
-void launch_cab(const FactorView& pa, const FactorView& pb, int64_t K, int ka, int kb, float* cab,
-                cudaStream_t s);
+// Cab = P^_A P^_B^T (ka x kb, tensor scales applied) over the contraction
+// of length K: cab_parts(K, sms) partial products (part: that many ka x kb
+// floats of scratch), then their sum in a fixed order.  False when the
+// kernel's shared memory cannot be granted (nothing is launched).
+int cab_parts(int64_t K, int sms);
+bool launch_cab(const FactorView& pa, const FactorView& pb, int64_t K, int ka, int kb, float* part, float* cab,
+                int sms, cudaStream_t s);
 void launch_build_lowrank(const LowRankArgs& a, int sms, cudaStream_t s);
 // hi / lo bf16 operands [rows][kp] of deq(U_q) (m rows) and deq(V_q) diag(S)
 // (n rows) for the error-compensated residual (fu: U_q, fv: V_q, k factors).

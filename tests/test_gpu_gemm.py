@@ -137,6 +137,41 @@ def test_both_split_product(fmt):
     assert rel_fro(y.cpu().numpy(), want) < TOL
 
 
+@pytest.mark.parametrize("fmt,K", [("nv", 1536), ("mx", 20480)])
+def test_both_split_core_product(fmt, K):
+    # P_A and P_B share their first 13 columns, so C_ab = P_A^T P_B is O(1)
+    # and the F_A S_A C_ab S_B F_B^T term carries most of C; an odd
+    # ka = 13 next to the largest kb = 128, and at K = 20480 each partial of
+    # C_ab covers two rounds of 64 positions
+    M, N, ka, kb = 256, 384, 13, 128
+    P = (_rand((K, kb), 61) / np.sqrt(K)).astype(np.float32)
+    Fa = (_rand((M, 16), 62) / np.sqrt(M)).astype(np.float32)
+    # the 13 leading columns are quantized as strided views (row stride 16
+    # and 128 floats keeps 16-byte rows)
+    qPa = api.quantize_fp4(torch.from_numpy(P).cuda()[:, :ka], fmt, 0)
+    qFa = api.quantize_fp4(torch.from_numpy(Fa).cuda()[:, :ka], fmt, 0)
+    rPa, rFa = fp4.quantize(P[:, :ka], fmt, 0), fp4.quantize(Fa[:, :ka], fmt, 0)
+    torch.cuda.synchronize()
+    assert_fp4_equal(qPa, rPa, check_linear=False)
+    assert_fp4_equal(qFa, rFa, check_linear=False)
+    qPb, rPb = _q(P, fmt, 0)
+    qFb, rFb = _q((_rand((N, kb), 63) / np.sqrt(N)).astype(np.float32), fmt, 0)
+    Sa = np.linspace(8, 1, ka).astype(np.float32)
+    Sb = np.linspace(6, 1, kb).astype(np.float32)
+    qra, rra = _q(_rand((M, K), 64, 0.02), fmt, 1)
+    qrb, rrb = _q(_rand((K, N), 65, 0.02), fmt, 0)
+    y = api.linear_fwd(api.Operand(qra, ka, qPa, qFa, torch.from_numpy(Sa).cuda()),
+                       api.Operand(qrb, kb, qPb, qFb, torch.from_numpy(Sb).cuda()), M, N, K)
+    torch.cuda.synchronize()
+    A = gemm.Operand(rra, ka, rPa, rFa, Sa)
+    B = gemm.Operand(rrb, kb, rPb, rFb, Sb)
+    want = gemm.gemm(A, B)
+    # the core term is most of the product
+    core = gemm.gemm(gemm.Operand(rra), gemm.Operand(rrb))
+    assert np.linalg.norm(want - core) > 2 * np.linalg.norm(core)
+    assert rel_fro(y.cpu().numpy(), want) < TOL
+
+
 def test_both_split_long_contraction():
     # K = 14336 (56 K tiles) with few output tiles: the low-rank products run
     # split-K with a split count that does not divide the K tiles evenly

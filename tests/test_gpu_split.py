@@ -96,6 +96,18 @@ def test_split_power_iterations(q):
     _check(A64, res, split.split(A64, 16, 16, q, 5), "nv")
 
 
+@pytest.mark.parametrize("q", [0, 1])
+def test_split_eight_slice_sketch(q):
+    # W 2048 x 4096: the sketch pass runs 8 K slices per 128-row tile (each
+    # CTA of the cluster finishes 16 rows); the 4096-row passes run 4 slices
+    d = inputs.make("layer_4096", scale=dict(K=2048, N=4096, M=128))
+    A = to_device(d["W"])
+    res = api.split(A, 16, 16, q, 2, "nv", tap=True)
+    torch.cuda.synchronize()
+    A64 = d["W"].f64()
+    _check(A64, res, split.split(A64, 16, 16, q, 2), "nv")
+
+
 def test_split_sampled_sparse_sign():
     # the sampled-activation recipe at 4096 x 512: 256 rows, sparse sign (4), k=32, p=16
     d = inputs.make("sampled_65536", scale=dict(M=4096, K=512))
@@ -163,3 +175,61 @@ def test_split_compensated_residual(fmt):
     err_c = rel_fro(low + read_fp4(comp.R_rows).dequantize(), A64)
     err_p = rel_fro(low + read_fp4(plain.R_rows).dequantize(), A64)
     assert err_c < err_p
+
+
+@pytest.mark.parametrize("q", [0, 1])
+def test_split_wide_spectrum(q):
+    # singular values over six decades: sigma_i = 10^(-6 i / 31) for the top
+    # 32 and a tail from 1e-7 down (2^(-1/16) apart).  How far down the GPU
+    # resolves sigma is set by its arithmetic, not by the core solver (the
+    # float64 Gram eigen-decomposition resolves about sqrt(eps64) sigma_1):
+    #  q = 0: the products that form Y, Q and Z (bf16 hi / lo parts on the
+    #    tensor cores) carry a backward error of order 2^-16 |A|;
+    #  q = 1: the first basis is orthonormalised from A^T A Omega directly,
+    #    whose float64 Gram spans sigma^4, so directions below
+    #    eps64^(1/4) sigma_1 ~ 1.2e-4 sigma_1 are lost to its rounding.
+    # Each sigma_i then moves by at most that floor (Weyl's inequality) and
+    # each singular vector turns by at most floor / gap_i (Wedin's theorem);
+    # the test takes eps = 4 x 2^-16 sigma_1 (q = 0) and 2 x eps64^(1/4)
+    # sigma_1 (q = 1).
+    rng = np.random.default_rng(19)
+    m, n, k, p = 384, 256, 32, 16
+    Ul, _ = np.linalg.qr(rng.standard_normal((m, n)))
+    Vr, _ = np.linalg.qr(rng.standard_normal((n, n)))
+    s = np.r_[10.0 ** (-6.0 * np.arange(k) / (k - 1)), 1e-7 * 2.0 ** (-np.arange(n - k) / 16.0)]
+    A = ((Ul * s) @ Vr.T).astype(np.float32)
+    A64 = A.astype(np.float64)
+    res = api.split(torch.from_numpy(A).cuda(), k, p, q, 3, "nv", tap=True)
+    torch.cuda.synchronize()
+    assert int(res.dev_status.cpu()[0]) == 0
+    ref = split.split(A64, k, p, q, 3)
+    U = res.U.cpu().numpy().astype(np.float64)
+    S = res.S.cpu().numpy().astype(np.float64)
+    V = res.V.cpu().numpy().astype(np.float64)
+    R = res.R_f32.cpu().numpy()
+    assert all(np.all(np.isfinite(x)) for x in (U, S, V, R))
+    assert np.all(S >= 0) and np.all(np.diff(S) <= 0)
+    s_full = np.linalg.svd(A64, compute_uv=False)
+    eps = (2.0 ** -14 if q == 0 else 2.0 * np.finfo(np.float64).eps ** 0.25) * s_full[0]
+    dev = np.abs(S - ref["S"])
+    assert dev.max() <= eps, (dev.max() / s_full[0], np.argmax(dev))
+    # the well-resolved values (sigma_i >= 1e-2 sigma_1) to the split tolerance
+    big = ref["S"] >= 1e-2 * s_full[0]
+    assert np.max(dev[big] / ref["S"][big]) < 2e-3
+    gap = np.minimum(s_full[:k] - s_full[1:k + 1], np.r_[np.inf, s_full[:k - 1] - s_full[1:k]])
+    for j in range(k):
+        tol = 2.0 * eps / gap[j]
+        if tol > 0.1:
+            continue
+        for F, Fr in ((U, ref["U"]), (V, ref["V"])):
+            e = min(np.linalg.norm(F[:, j] - Fr[:, j]), np.linalg.norm(F[:, j] + Fr[:, j]))
+            assert e <= tol, (j, e, tol)
+    L = (U * S) @ V.T
+    assert rel_fro(L, (ref["U"] * ref["S"]) @ ref["V"].T) < TOL
+    # the residual is the tail (|R| ~ 3e-7 |A|): the tap equals A - U S V^T of
+    # the GPU's own factors to the products' rounding, relative to |A|
+    assert np.linalg.norm(R.astype(np.float64) - (A64 - L)) / np.linalg.norm(A64) < 1e-5
+    assert np.linalg.norm(R) / np.linalg.norm(A64) < 4 * eps / s_full[0] * np.sqrt(k)
+    assert_fp4_equal(res.U_q, fp4.quantize(res.U.cpu().numpy(), "nv", 0), check_linear=False)
+    assert_fp4_equal(res.V_q, fp4.quantize(res.V.cpu().numpy(), "nv", 0), check_linear=False)
+    assert_fp4_equal(res.R_rows, fp4.quantize(R, "nv", 1), check_linear=False)
