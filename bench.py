@@ -35,11 +35,19 @@ sys.path.insert(0, ROOT)
 
 M, K, N = 8192, 4096, 4096
 RANK_K, OVERSAMPLE, POWER_ITERS, SEED = 64, 16, 1, 0
+# algorithmic bytes of the split of W (four passes of the range finder and two
+# residual passes over W, the NVFP4 copy of R, the float32 factors and their
+# FP4 copies) and of X's NVFP4 quantization (the amax pass and the quantizing
+# pass over X, its codes and scales): each byte the method must move, once
+# per pass
+SPLIT_W_BYTES = (6 * K * N * 2 + (K * N // 2 + K * N // 16) + (K + N) * RANK_K * 4
+                 + (K + N) * RANK_K // 2 + (K + N) * RANK_K // 16)
+QUANT_X_BYTES = 2 * M * K * 2 + M * K // 2 + M * K // 16
 FLOPS = 2.0 * M * N * K
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
 # the plain-operand FP4 GEMM, from one ncu capture of the current kernel; to
 # be set to None whenever the kernel changes after that capture.
-GEMM_NCU_DRAM_BYTES = 34.673920e6 + 18.095104e6
+GEMM_NCU_DRAM_BYTES = 30.669824e6 + 18.200832e6
 METRIC = "FP4 split-linear eff. TFLOPS & % of FP4 peak; split+quantize us/layer"
 CONFIG = {"workload": "layer_4096: W bf16 4096x4096 planted spectrum + X bf16 8192x4096, "
                       "split k=64 p=16 q=1 Gaussian, NVFP4, forward",
@@ -494,6 +502,9 @@ def run_ours(args, rank, world, local):
             "split_quantize_us_per_layer": (ms_split + ms_quant) * 1e3,
             "breakdown_us": {"split_W": ms_split * 1e3, "quantize_X": ms_quant * 1e3,
                              "linear_fwd": ms_gemm * 1e3, "fp4_gemm_kernel": ms_plain * 1e3},
+            "hbm": {name: {"algorithmic_bytes": nbytes, "achieved_gbs": nbytes / (t * 1e-3) / 1e9,
+                           "peak_gbs": hbm, "frac": nbytes / (t * 1e-3) / 1e9 / hbm, "peak_source": peak_kind}
+                    for name, nbytes, t in (("split_W", SPLIT_W_BYTES, ms_split), ("quantize_X", QUANT_X_BYTES, ms_quant))},
             "roofline": {"kernel": "gemm_fp4_kernel<256,4,1> (8192x4096x4096 NVFP4)", "bound": "tensor",
                          "achieved": achieved, "peak": fp4_peak, "unit": "TFLOP/s", "frac": achieved / fp4_peak,
                          "peak_source": f"{peak_kind} bf16 {bf16_tf} TFLOP/s x 4 (nominal FP4/bf16 ratio)",
