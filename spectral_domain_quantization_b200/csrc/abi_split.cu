@@ -72,7 +72,7 @@ struct SplitBuffers {
   double* gpart = nullptr;
   double* G = nullptr;
   double* eig_ws = nullptr;          // core eigensolver scratch
-  float* Rinv = nullptr;
+  float* Lt = nullptr;     // the Cholesky factor, column by column (launch_cholesky)
   double* eval = nullptr;
   float* evec = nullptr;
   float* Mu = nullptr;
@@ -142,7 +142,7 @@ SplitBuffers carve(const SplitPlan& p, int64_t lda, Carver& ws) {
   b.gpart = ws.take<double>(static_cast<size_t>(gblocks) * wmax * wmax);
   b.G = ws.take<double>(static_cast<size_t>(wmax) * wmax);
   b.eig_ws = reinterpret_cast<double*>(ws.take<uint8_t>(core_eig_workspace(wmax)));
-  b.Rinv = ws.take<float>(static_cast<size_t>(p.lp) * p.lp);
+  b.Lt = ws.take<float>(static_cast<size_t>(p.lp) * p.lp);
   b.eval = ws.take<double>(p.lp);
   b.evec = ws.take<float>(static_cast<size_t>(p.lp) * p.lp);
   b.Mu = ws.take<float>(static_cast<size_t>(p.lp) * p.k);
@@ -224,16 +224,15 @@ metis_status cholqr(const SplitBuffers& b, int64_t rows, int lp, float* Q, int64
   const float* in = b.Y;
   for (int pass = 0; pass < passes; ++pass) {
     const bool last = pass == passes - 1;
-    launch_cholesky_inv(b.G, lp, b.Rinv, s);
+    if (!launch_cholesky(b.G, lp, b.Lt, s)) return fail(METIS_ERR_CUDA, "cholqr cholesky shared memory");
     METIS_TRY(step_status("cholqr cholesky"));
     ApplyArgs a{};
     a.in = in;
     a.rows = rows;
     a.kin = lp;
     a.in_ld = lp;
-    a.M = b.Rinv;
+    a.M = b.Lt;
     a.kout = lp;
-    a.upper = 1;
     a.out = last ? Q : b.Q1;
     a.out_ld = lp;
     if (last) {
@@ -243,8 +242,8 @@ metis_status cholqr(const SplitBuffers& b, int64_t rows, int lp, float* Q, int64
     } else {
       a.gpart = b.gpart;
     }
-    launch_apply(a, s);
-    METIS_TRY(step_status("cholqr apply"));
+    if (!launch_solve(a, s)) return fail(METIS_ERR_CUDA, "cholqr solve");
+    METIS_TRY(step_status("cholqr solve"));
     if (!last) {
       launch_gram_reduce(b.gpart, static_cast<int>(apply_blocks(rows)), lp, b.G, s);
       METIS_TRY(step_status("cholqr gram reduce"));

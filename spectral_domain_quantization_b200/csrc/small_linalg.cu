@@ -1,5 +1,5 @@
 // Small dense linear algebra of the randomized split (l = k + p <= 112):
-// Gram matrices, Cholesky with rank drop and triangular inverse (CholeskyQR),
+// Gram matrices, Cholesky with rank drop and forward substitution (CholeskyQR),
 // row-block products, factor assembly and the sign convention.  The core's
 // eigen-decomposition lives in core_eig.cu.
 //
@@ -8,8 +8,8 @@
 // item (i) (random embedding separates dominant from long-tail parts).
 //
 // Numerics: Gram matrices are accumulated in float64 from float32 rows;
-// Cholesky and the triangular inverse run in float64 in one CTA; tall row
-// blocks are multiplied in float32.
+// the Cholesky factor runs in float64 in one CTA; tall row blocks are
+// multiplied (or solved against the factor) in float32.
 //   * CholeskyQR: G = Y^T Y = L L^T, Q = Y L^-T.  A pivot that falls below
 //     1e-12 of its original diagonal (a numerically dependent sketch column,
 //     e.g. for an exactly low-rank input) is dropped: that column of Q
@@ -151,59 +151,6 @@ constexpr int kTile = 4;  // register tile edge and panel width of the Cholesky
 // tile rows then run at the minimum 4 wavefronts instead of up to 32.
 constexpr int kPanStride = 18;
 
-// Block row BI of X = L^-1 (16 x 16 blocks, o = 16 BI), after blocks
-// 0 .. BI-1 of X and the diagonal block X(BI, BI) are known:
-//   T = L(BI, 0:BI) X(0:BI, 0:BI)   and   X(BI, 0:BI) = -X(BI, BI) T.
-// Thread t < 256 owns row r = t / 16 of the block row and the columns
-// c0 + 16 u (c0 = t % 16, u < BI): 16 lanes read 16 consecutive entries of
-// an X row (no bank conflicts).  Only the lower block triangle of X is
-// read: row block mb of the sum meets column blocks u <= mb (the diagonal
-// blocks hold zeros above their diagonal).  Two accumulators per column
-// (even and odd m) halve the dependent chains.
-template <int BI>
-MDEV void inverse_block_row(const double* L, double* X, double* T, int ld, int t) {
-  constexpr int o = 16 * BI;
-  const int r = t >> 4, c0 = t & 15;
-  if (t < 256) {
-    double e[BI], f[BI];
-#pragma unroll
-    for (int u = 0; u < BI; ++u) e[u] = f[u] = 0.0;
-    const double* Lr = L + (o + r) * ld;
-#pragma unroll
-    for (int mb = 0; mb < BI; ++mb) {
-#pragma unroll 4
-      for (int mm = 0; mm < 16; mm += 2) {
-        const int m = 16 * mb + mm;
-        const double l0 = Lr[m], l1 = Lr[m + 1];
-        const double* X0 = X + m * ld + c0;
-        const double* X1 = X0 + ld;
-#pragma unroll
-        for (int u = 0; u <= mb; ++u) {
-          e[u] = fma(l0, X0[16 * u], e[u]);
-          f[u] = fma(l1, X1[16 * u], f[u]);
-        }
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < BI; ++u) T[r * ld + c0 + 16 * u] = e[u] + f[u];
-  }
-  __syncthreads();
-  if (t < 256) {
-    double acc[BI];
-#pragma unroll
-    for (int u = 0; u < BI; ++u) acc[u] = 0.0;
-    const double* Xr = X + (o + r) * ld + o;
-    for (int q = 0; q <= r; ++q) {
-      const double x = Xr[q];
-#pragma unroll
-      for (int u = 0; u < BI; ++u) acc[u] = fma(x, T[q * ld + c0 + 16 * u], acc[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < BI; ++u) X[(o + r) * ld + c0 + 16 * u] = -acc[u];
-  }
-  __syncthreads();
-}
-
 // Factor the diagonal tile (K, K), held in registers by its owner (lower
 // triangle valid), in place: column c takes the pivot d = v[c][c], dropped
 // (1/sqrt = 0, the column of L zero) when it falls below kDropTol of its
@@ -290,7 +237,7 @@ MDEV void panel_update(double (&v)[kTile][kTile], const double* P, int I, int J)
     }
 }
 
-// G = L L^T (with drops), then Rinv = L^-T (upper triangular, float32).
+// G = L L^T (with drops), written column by column for solve_kernel.
 //  Cholesky, right-looking by panels of 4 columns with look-ahead: thread
 //  32 + T owns the 4 x 4 tile (I, J), I >= J, of the lower triangle in
 //  registers; panel K's columns of L sit in shared memory.  Per panel K + 1,
@@ -298,8 +245,12 @@ MDEV void panel_update(double (&v)[kTile][kTile], const double* P, int I, int J)
 //    (A) every tile right of panel K takes its rank-4 update; the owner of
 //        the diagonal tile (K+1, K+1) then factors it at once;
 //    (B) the owners of the tiles below it solve their rows of panel K + 1.
-//  Inverse: X = L^-1 by 16 x 16 blocks (see below).
-__global__ void __launch_bounds__(kSmallThreads, 1) cholesky_inv_kernel(const double* G, int lp, float* Rinv) {
+//  The float64 factor is then written as float32 column by column, the
+//  diagonal as the reciprocal pivots: Lt[i][i] = 1 / L[i][i] (0 for a
+//  dropped pivot), Lt[i][m] = L[m][i] for m > i, 0 above.  (An explicit
+//  inverse by 16 x 16 blocks took a third of this kernel's time, more than
+//  the forward substitution that replaces it costs in solve_kernel.)
+__global__ void __launch_bounds__(kSmallThreads, 1) cholesky_kernel(const double* G, int lp, float* Lt) {
   extern __shared__ double sm[];
   const int ld = lp + 1;
   double* pan = sm;               // 2 panel buffers of (lp / 4) x kPanStride
@@ -343,41 +294,9 @@ __global__ void __launch_bounds__(kSmallThreads, 1) cholesky_inv_kernel(const do
     if (owner && J == K + 1 && I > K + 1) solve_rows(v, I, K + 1, Pn, L, invd, ld);
     __syncthreads();
   }
-  // X = L^-1 by 16 x 16 blocks: the diagonal blocks are inverted by one warp
-  // each (a lane per column, forward substitution), then block row bi is
-  //   T = sum_{k < bi} L(bi, k) X(k, j)   and   X(bi, j) = -X(bi, bi) T
-  // for all j < bi at once (two barriers per block row).
-  double* X = L + lp * ld;        // lp x ld
-  double* T = X + lp * ld;        // 16 x ld
-  const int nb16 = lp / 16;
-  if (warp < nb16 && lane < 16) {
-    const int o = 16 * warp, j = lane;
-    double x[16];
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      double sum = 0.0;
-#pragma unroll
-      for (int m = 0; m < i; ++m)
-        if (m >= j) sum += L[(o + i) * ld + o + m] * x[m];
-      x[i] = i < j ? 0.0 : (i == j ? invd[o + i] : -sum * invd[o + i]);
-      X[(o + i) * ld + o + j] = x[i];
-    }
-  }
-  __syncthreads();
-  for (int bi = 1; bi < nb16; ++bi) {
-    switch (bi) {
-      case 1: inverse_block_row<1>(L, X, T, ld, t); break;
-      case 2: inverse_block_row<2>(L, X, T, ld, t); break;
-      case 3: inverse_block_row<3>(L, X, T, ld, t); break;
-      case 4: inverse_block_row<4>(L, X, T, ld, t); break;
-      case 5: inverse_block_row<5>(L, X, T, ld, t); break;
-      default: inverse_block_row<6>(L, X, T, ld, t); break;
-    }
-  }
-  // Rinv[c][r] = X[r][c] (upper triangular): a warp per column c, lanes
-  // along r (coalesced stores)
-  for (int c = warp; c < lp; c += kSmallThreads / 32)
-    for (int r = lane; r < lp; r += 32) Rinv[c * lp + r] = r >= c ? static_cast<float>(X[r * ld + c]) : 0.f;
+  for (int i = warp; i < lp; i += kSmallThreads / 32)
+    for (int m = lane; m < lp; m += 32)
+      Lt[i * lp + m] = m > i ? static_cast<float>(L[m * ld + i]) : (m == i ? static_cast<float>(invd[i]) : 0.f);
 }
 
 constexpr int kApplyRows = 32;
@@ -386,6 +305,8 @@ constexpr int kApplyRows = 32;
 // thread a 4-row x 4-column register tile (4 consecutive columns).  Optional fp32 out,
 // transposed bf16 hi/lo copy, Gram partial of the output block, and per
 // column the block's largest |out| with its first row (the sign convention).
+MDEV void apply_store(const ApplyArgs& a, int64_t blk, int64_t r0, int nr, const float* Out);
+
 MDEV void apply_block(const ApplyArgs& a, int64_t blk) {
   extern __shared__ float smf[];
   float* Ms = smf;                                   // kin x kout
@@ -445,6 +366,13 @@ MDEV void apply_block(const ApplyArgs& a, int64_t blk) {
       for (int u = 0; u < 4; ++u) Out[(4 * rg + i) * (a.kout + 1) + 4 * cg + u] = acc[i][u];
   }
   __syncthreads();
+  apply_store(a, blk, r0, nr, Out);
+}
+
+// The stores of one 32-row block from its result rows in shared memory
+// (Out, row stride kout + 1): fp32 rows, the bf16 hi / lo transpose, the
+// Gram partial and the per-column block maxima, each where requested.
+MDEV void apply_store(const ApplyArgs& a, int64_t blk, int64_t r0, int nr, const float* Out) {
   for (int e = threadIdx.x; e < kApplyRows * a.kout; e += blockDim.x) {
     if (a.out) {
       const int r = e / a.kout, c = e - r * a.kout;  // column fastest: coalesced rows
@@ -480,6 +408,66 @@ MDEV void apply_block(const ApplyArgs& a, int64_t blk) {
 }
 
 __global__ void __launch_bounds__(256) apply_kernel(ApplyArgs a) { apply_block(a, blockIdx.x); }
+
+// out = in L^-T for the lower-triangular Cholesky factor L (KIN x KIN), by
+// forward substitution row by row: L q^T = y^T, q_i = (y_i - sum_{m<i}
+// L[i][m] q_m) / L[i][i].  M holds L column by column with the reciprocal
+// pivots on the diagonal: M[i][i] = 1 / L[i][i] (0 for a dropped pivot, so
+// that column of the result is 0), M[i][m] = L[m][i] below it.  A thread
+// takes one row of the 32-row block, its KIN running values in registers
+// (right-looking: once q_i is known, every later value takes its term).
+template <int KIN>
+__global__ void __launch_bounds__(256) solve_kernel(ApplyArgs a) {
+  extern __shared__ float smf[];
+  float* Ms = smf;                                   // KIN x KIN
+  float* In = Ms + KIN * KIN;                        // kApplyRows x (KIN + 1)
+  float* Out = In + kApplyRows * (KIN + 1);          // kApplyRows x (KIN + 1)
+  const int64_t blk = blockIdx.x;
+  const int64_t r0 = blk * kApplyRows;
+  const int nr = static_cast<int>(imin64(kApplyRows, a.rows - r0));
+  {
+    const float4* M4 = reinterpret_cast<const float4*>(a.M);
+    float4* Ms4 = reinterpret_cast<float4*>(Ms);
+#pragma unroll 4
+    for (int e = threadIdx.x; e < KIN * KIN / 4; e += blockDim.x) Ms4[e] = M4[e];
+    constexpr int q4 = KIN / 4;
+    for (int e = threadIdx.x; e < kApplyRows * q4; e += blockDim.x) {
+      const int r = e / q4, c4 = e - r * q4;
+      const float4 x = r < nr ? *reinterpret_cast<const float4*>(a.in + (r0 + r) * a.in_ld + 4 * c4)
+                              : make_float4(0.f, 0.f, 0.f, 0.f);
+      float* d = In + r * (KIN + 1) + 4 * c4;
+      d[0] = x.x;
+      d[1] = x.y;
+      d[2] = x.z;
+      d[3] = x.w;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x < kApplyRows) {
+    const int r = threadIdx.x;
+    float acc[KIN];
+#pragma unroll
+    for (int c = 0; c < KIN; ++c) acc[c] = In[r * (KIN + 1) + c];
+#pragma unroll
+    for (int i = 0; i < KIN; ++i) {
+      const float* col = Ms + i * KIN;
+      const float q = acc[i] * col[i];
+      acc[i] = q;
+#pragma unroll
+      for (int m4 = (i + 1) / 4; m4 < KIN / 4; ++m4) {
+        const float4 l = reinterpret_cast<const float4*>(col)[m4];
+        if (4 * m4 + 0 > i) acc[4 * m4 + 0] = fmaf(-l.x, q, acc[4 * m4 + 0]);
+        if (4 * m4 + 1 > i) acc[4 * m4 + 1] = fmaf(-l.y, q, acc[4 * m4 + 1]);
+        if (4 * m4 + 2 > i) acc[4 * m4 + 2] = fmaf(-l.z, q, acc[4 * m4 + 2]);
+        if (4 * m4 + 3 > i) acc[4 * m4 + 3] = fmaf(-l.w, q, acc[4 * m4 + 3]);
+      }
+    }
+#pragma unroll
+    for (int c = 0; c < KIN; ++c) Out[r * (KIN + 1) + c] = acc[c];
+  }
+  __syncthreads();
+  apply_store(a, blk, r0, nr, Out);
+}
 
 __global__ void __launch_bounds__(256) apply2_kernel(ApplyArgs a, ApplyArgs b, int64_t blocks_a) {
   if (blockIdx.x < blocks_a)
@@ -561,17 +549,39 @@ void launch_gram_reduce(const double* gpart, int nblocks, int lp, double* G, cud
   gram_reduce_kernel<<<(npk + 31) / 32, 32 * kReduceGroups, 0, s>>>(gpart, nblocks, lp, G);
 }
 
-void launch_cholesky_inv(const double* G, int lp, float* Rinv, cudaStream_t s) {
-  // panels x2, invd, sqd, diag0, L, X, T
-  const size_t smem = ((2 * static_cast<size_t>(lp) + 16) * (lp + 1) + 2 * (lp / kTile) * kPanStride + 3 * lp) *
-                      sizeof(double);
-  if (!ensure_smem(reinterpret_cast<const void*>(cholesky_inv_kernel), smem)) return;
-  cholesky_inv_kernel<<<1, kSmallThreads, smem, s>>>(G, lp, Rinv);
+bool launch_cholesky(const double* G, int lp, float* Lt, cudaStream_t s) {
+  // panels x2, invd, sqd, diag0, L
+  const size_t smem = (static_cast<size_t>(lp) * (lp + 1) + 2 * (lp / kTile) * kPanStride + 3 * lp) * sizeof(double);
+  if (!ensure_smem(reinterpret_cast<const void*>(cholesky_kernel), smem)) return false;
+  cholesky_kernel<<<1, kSmallThreads, smem, s>>>(G, lp, Lt);
+  return true;
 }
 
 size_t apply_smem(const ApplyArgs& a) {
   return (static_cast<size_t>(a.kin) * a.kout + kApplyRows * (a.kin + 1) + kApplyRows * (a.kout + 1)) *
          sizeof(float);
+}
+
+template <int KIN>
+bool launch_solve_t(const ApplyArgs& a, cudaStream_t s) {
+  const size_t smem = (static_cast<size_t>(KIN) * KIN + 2 * kApplyRows * (KIN + 1)) * sizeof(float);
+  if (!ensure_smem(reinterpret_cast<const void*>(solve_kernel<KIN>), smem)) return false;
+  solve_kernel<KIN><<<static_cast<unsigned>(apply_blocks(a.rows)), 256, smem, s>>>(a);
+  return true;
+}
+
+bool launch_solve(const ApplyArgs& a, cudaStream_t s) {
+  if (a.kin != a.kout) return false;
+  switch (a.kin) {
+    case 16: return launch_solve_t<16>(a, s);
+    case 32: return launch_solve_t<32>(a, s);
+    case 48: return launch_solve_t<48>(a, s);
+    case 64: return launch_solve_t<64>(a, s);
+    case 80: return launch_solve_t<80>(a, s);
+    case 96: return launch_solve_t<96>(a, s);
+    case 112: return launch_solve_t<112>(a, s);
+    default: return false;
+  }
 }
 
 void launch_apply(const ApplyArgs& a, cudaStream_t s) {

@@ -14,7 +14,6 @@ struct ApplyArgs {
   int64_t in_ld;
   const float* M;          // kin x kout, row-major
   int kout;
-  int upper;               // M upper triangular (only j <= c terms)
   float* out;              // optional rows x kout, row stride out_ld
   int64_t out_ld;
   __nv_bfloat16* outT;     // optional [2*lpT][ldx]: hi rows 0..kout-1, lo rows lpT..
@@ -27,6 +26,11 @@ struct ApplyArgs {
 
 // row blocks of launch_apply (its Gram partials come one per block)
 int64_t apply_blocks(int64_t rows);
+// out = in L^-T by forward substitution (M = Lt from launch_cholesky, kin =
+// kout = lp, a multiple of 16 up to 112), with the same optional stores as
+// launch_apply.  False when the width is not supported or the shared memory
+// cannot be granted (nothing is launched).
+bool launch_solve(const ApplyArgs& a, cudaStream_t s);
 // G = Y^T Y (float64, lp x lp) of a rows x lp float32 Y (row stride lp):
 // Gram partials of 32-row blocks (gram_blocks(rows) * lp * lp doubles of
 // scratch in gpart), then their sum in block order.
@@ -34,8 +38,11 @@ int64_t gram_blocks(int64_t rows);
 void launch_gram(const float* Y, int64_t rows, int lp, double* gpart, double* G, cudaStream_t s);
 // G = sum of nblocks Gram partials (lp x lp float64 each), in block order.
 void launch_gram_reduce(const double* gpart, int nblocks, int lp, double* G, cudaStream_t s);
-// Rinv (lp x lp float, upper triangular) with G = R^T R, dropped pivots -> 0.
-void launch_cholesky_inv(const double* G, int lp, float* Rinv, cudaStream_t s);
+// Cholesky factor of G = L L^T (lp x lp float64; a pivot below 1e-12 of
+// its original diagonal is dropped), for launch_solve: Lt (lp x lp float)
+// holds L column by column, Lt[i][i] = 1 / L[i][i] (0 for a dropped pivot) and Lt[i][m] =
+// L[m][i] for m > i.  False when the shared memory cannot be granted.
+bool launch_cholesky(const double* G, int lp, float* Lt, cudaStream_t s);
 void launch_apply(const ApplyArgs& a, cudaStream_t s);
 // Two independent products in one launch (blocks of a first, then of b).
 void launch_apply2(const ApplyArgs& a, const ApplyArgs& b, cudaStream_t s);
