@@ -47,7 +47,7 @@ FLOPS = 2.0 * M * N * K
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
 # the plain-operand FP4 GEMM, from one ncu capture of the current kernel; to
 # be set to None whenever the kernel changes after that capture.
-GEMM_NCU_DRAM_BYTES = 30.669824e6 + 18.200832e6
+GEMM_NCU_DRAM_BYTES = 31.770880e6 + 18.906880e6
 METRIC = "FP4 split-linear eff. TFLOPS & % of FP4 peak; split+quantize us/layer"
 CONFIG = {"workload": "layer_4096: W bf16 4096x4096 planted spectrum + X bf16 8192x4096, "
                       "split k=64 p=16 q=1 Gaussian, NVFP4, forward",

@@ -41,6 +41,9 @@ namespace metis {
 namespace {
 
 constexpr int kThreads = 320;
+// gemm_fp4_kernel adds one warp that only copies the scale factors into TMEM
+constexpr int kSfWarp = 10;
+constexpr int kThreadsMain = 32 * (kSfWarp + 1);
 constexpr int kEpiWarps = 8;
 
 template <int BN, int STAGES>
@@ -64,7 +67,7 @@ MDEV bool wait_ns(uint64_t* bar, uint32_t parity, uint64_t ns) {
 // BN: MMA N; STAGES: shared-memory ring depth; CTAS: CTAs per SM (2 halves
 // the TMEM allocation and lets one CTA's epilogue overlap the other's MMAs).
 template <int BN, int STAGES, int CTAS>
-__global__ void __launch_bounds__(kThreads, CTAS)
+__global__ void __launch_bounds__(kThreadsMain, CTAS)
     gemm_fp4_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmLA,
                     const __grid_constant__ CUtensorMap tmLB) {
@@ -76,7 +79,8 @@ __global__ void __launch_bounds__(kThreads, CTAS)
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 1;
-  uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(acc_empty + 1);
+  uint64_t* sf_ready = acc_empty + 1;   // per stage: its scale factors are in TMEM
+  uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(sf_ready + kStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_sh + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -94,6 +98,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
+      mbar_init(&sf_ready[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, kEpiWarps);
@@ -185,6 +190,7 @@ __global__ void __launch_bounds__(kThreads, CTAS)
       int stage = 0;
       uint32_t phase = 0;
       uint32_t acc_phase = 0;
+      uint32_t sf_phase = 0;   // bit s: parity of sf_ready[s]'s next phase
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         const int split = t % p.splits;
@@ -200,22 +206,21 @@ __global__ void __launch_bounds__(kThreads, CTAS)
         uint32_t accumulate = 0;
         for (int it = kt0; it < kt1 + nlr; ++it) {
           if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+          // an FP4 stage's scale factors are copied into TMEM by the scale
+          // warp; sf_ready[s] completes once per FP4 use of stage s (the
+          // low-rank chunks have none), so its parity is kept per stage
+          if (it < kt1) {
+            if (!mbar_wait(&sf_ready[stage], (sf_phase >> stage) & 1u, abort_flag)) { ok = false; break; }
+            sf_phase ^= 1u << stage;
+          }
           tc_fence_after();
           uint8_t* sA = smem + stage * S::kStage;
           uint8_t* sB = sA + S::kA;
           const uint64_t adesc = make_sdesc(smem_u32(sA), 16, 1024, kSwizzle128B);
           const uint64_t bdesc = make_sdesc(smem_u32(sB), 16, 1024, kSwizzle128B);
           if (it < kt1) {
-            uint8_t* sSFA = sB + S::kB;
-            uint8_t* sSFB = sSFA + S::kSFA;
             const uint32_t sfa_t = tmem + kSfBase + stage * sf_stage_cols;
             const uint32_t sfb_t = sfa_t + sfa_cols + sfb_off;
-            for (int a = 0; a < atoms_per_kt; ++a) {
-              tc_cp_32x128b_warpx4(sfa_t + 4 * a, make_sdesc(smem_u32(sSFA + 512 * a), 0, 128, kSwizzleNone));
-              for (int h = 0; h < kBHalves; ++h)
-                tc_cp_32x128b_warpx4(sfb_t - sfb_off + 4 * kBHalves * a + 4 * h,
-                                     make_sdesc(smem_u32(sSFB + 2048 * h + 512 * a), 0, 128, kSwizzleNone));
-            }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const uint64_t koff = static_cast<uint64_t>((j * 32) >> 4);
@@ -250,6 +255,54 @@ __global__ void __launch_bounds__(kThreads, CTAS)
         tc_commit(acc_full);
         wait_ns(acc_full, acc_phase, 100000000ull);
       }
+    }
+    __syncwarp();
+  } else if (warp == kSfWarp) {
+    // ------------------------------------------------------------ scale copies
+    // Each FP4 stage's scale factors go from shared memory into that stage's
+    // own TMEM columns (tcgen05.cp 32x128b.warpx4), committed to sf_ready;
+    // the MMA issuer waits for them, so copies of later stages are issued
+    // while the MMAs of earlier ones run.  A stage's columns are rewritten
+    // only after its smem was refilled, i.e. after the MMAs that read the
+    // previous contents completed.
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int last = -1;
+      uint32_t last_phase = 0;
+      uint32_t sf_phase = 0;   // bit s: parity of sf_ready[s]'s next phase
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        const int split = t % p.splits;
+        const int tn = (t / p.splits) / tiles_m;
+        const uint32_t sfb_off = BN == 64 ? 2u * (tn & 1) : 0u;
+        const int kt0 = split * kt_per_split;
+        const int kt1 = min(p.num_kt, kt0 + kt_per_split);
+        const int nlr = (split == p.splits - 1) ? p.lr_chunks : 0;
+        for (int it = kt0; it < kt1 + nlr; ++it) {
+          if (it < kt1) {
+            if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+            tc_fence_after();
+            uint8_t* sSFA = smem + stage * S::kStage + S::kA + S::kB;
+            uint8_t* sSFB = sSFA + S::kSFA;
+            const uint32_t sfa_t = tmem + kSfBase + stage * sf_stage_cols;
+            const uint32_t sfb_t = sfa_t + sfa_cols + sfb_off;
+            for (int a = 0; a < atoms_per_kt; ++a) {
+              tc_cp_32x128b_warpx4(sfa_t + 4 * a, make_sdesc(smem_u32(sSFA + 512 * a), 0, 128, kSwizzleNone));
+              for (int h = 0; h < kBHalves; ++h)
+                tc_cp_32x128b_warpx4(sfb_t - sfb_off + 4 * kBHalves * a + 4 * h,
+                                     make_sdesc(smem_u32(sSFB + 2048 * h + 512 * a), 0, 128, kSwizzleNone));
+            }
+            tc_commit(&sf_ready[stage]);
+            last = stage;
+            last_phase = (sf_phase >> stage) & 1u;
+            sf_phase ^= 1u << stage;
+          }
+          if (++stage == kStages) { stage = 0; phase ^= 1u; }
+        }
+      }
+      // copies still in flight land before the TMEM is freed
+      if (last >= 0) wait_ns(&sf_ready[last], last_phase, 100000000ull);
     }
     __syncwarp();
   } else {
@@ -702,7 +755,7 @@ cudaError_t launch_bn(const GemmParams& p, const CUtensorMap& a, const CUtensorM
     return cudaErrorInvalidValue;
   const int slots = device_sm_count() * CTAS;
   const int grid = tiles < slots ? tiles : slots;
-  gemm_fp4_kernel<BN, STAGES, CTAS><<<grid, kThreads, bytes, s>>>(p, a, b, la, lb);
+  gemm_fp4_kernel<BN, STAGES, CTAS><<<grid, kThreadsMain, bytes, s>>>(p, a, b, la, lb);
   return cudaGetLastError();
 }
 
