@@ -85,7 +85,8 @@ __global__ void __launch_bounds__(kThreadsMain, CTAS)
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* sf_ready = acc_empty + 1;   // per stage: its scale factors are in TMEM
-  uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(sf_ready + kStages);
+  uint64_t* sf_full = sf_ready + kStages;  // per stage: its scale bytes are in shared memory
+  uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(sf_full + kStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_sh + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -104,6 +105,7 @@ __global__ void __launch_bounds__(kThreadsMain, CTAS)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
       mbar_init(&sf_ready[s], 1);
+      mbar_init(&sf_full[s], 1);
     }
     mbar_init(acc_full, 1);
     mbar_init(acc_empty, kEpiWarps);
@@ -138,6 +140,8 @@ __global__ void __launch_bounds__(kThreadsMain, CTAS)
       int stage = 0;
       uint32_t phase = 0;
       int issued = 0;
+      uint32_t sf_phase = 0;   // bit s: parity of sf_full[s]'s next phase
+      uint32_t sf_last = 0;    // bit s: the last load into stage s carried scales
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         const int split = t % p.splits;
@@ -157,23 +161,31 @@ __global__ void __launch_bounds__(kThreadsMain, CTAS)
             const int kt = it;
             const uint32_t sf_bytes = 512u * atoms_per_kt;
             const bool second = kBHalves == 2 && (2 * tn + 1) * 128 < p.sfb_rows;
-            const uint32_t bytes = S::kA + S::kB + sf_bytes * (1 + (kBHalves == 2 ? (second ? 2 : 1) : 1));
-            mbar_arrive_expect_tx(&full[stage], bytes);
+            // the operands complete on full[stage] (MMA warp), the scale
+            // chunks on sf_full[stage] (scale warp), which is armed only
+            // for FP4 steps, so its phases count exactly the steps the scale
+            // warp serves
+            const uint32_t sbytes = sf_bytes * (1 + (kBHalves == 2 ? (second ? 2 : 1) : 1));
+            mbar_arrive_expect_tx(&full[stage], S::kA + S::kB);
+            mbar_arrive_expect_tx(&sf_full[stage], sbytes);
             tma_load_2d(sA, &tmA, &full[stage], kt * 128, tm * 128);
             tma_load_2d(sB, &tmB, &full[stage], kt * 128, tn * BN);
             bulk_load(sSFA, p.sfa + (static_cast<int64_t>(tm) * p.sfa_chunks + kt * atoms_per_kt) * 512,
-                      sf_bytes, &full[stage]);
+                      sf_bytes, &sf_full[stage]);
             const int nb0 = kBHalves == 2 ? 2 * tn : tn * BN / 128;
             bulk_load(sSFB, p.sfb + (static_cast<int64_t>(nb0) * p.sfb_chunks + kt * atoms_per_kt) * 512,
-                      sf_bytes, &full[stage]);
+                      sf_bytes, &sf_full[stage]);
             if (kBHalves == 2 && second)
               bulk_load(sSFB + 2048, p.sfb + (static_cast<int64_t>(nb0 + 1) * p.sfb_chunks + kt * atoms_per_kt) * 512,
-                        sf_bytes, &full[stage]);
+                        sf_bytes, &sf_full[stage]);
+            sf_phase ^= 1u << stage;
+            sf_last |= 1u << stage;
           } else {
             const int c = it - kt1;
             mbar_arrive_expect_tx(&full[stage], S::kA + S::kB);
             tma_load_2d(sA, &tmLA, &full[stage], c * 64, tm * 128);
             tma_load_2d(sB, &tmLB, &full[stage], c * 64, tn * BN);
+            sf_last &= ~(1u << stage);
           }
           ++issued;
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -186,6 +198,9 @@ __global__ void __launch_bounds__(kThreadsMain, CTAS)
         for (int i = 0; i < min(issued, kStages); ++i) {
           if (--s < 0) { s = kStages - 1; ph ^= 1u; }
           wait_ns(&full[s], ph, 100000000ull);
+          // sf_phase holds the parity after the last arming: the phase in
+          // flight has the other one
+          if ((sf_last >> s) & 1u) wait_ns(&sf_full[s], ((sf_phase >> s) & 1u) ^ 1u, 100000000ull);
         }
       }
     }
@@ -275,7 +290,7 @@ __global__ void __launch_bounds__(kThreadsMain, CTAS)
       uint32_t phase = 0;
       int last = -1;
       uint32_t last_phase = 0;
-      uint32_t sf_phase = 0;   // bit s: parity of sf_ready[s]'s next phase
+      uint32_t sf_phase = 0;   // bit s: parity of sf_ready[s]'s and sf_full[s]'s next phase
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         const int split = t % p.splits;
@@ -286,7 +301,7 @@ __global__ void __launch_bounds__(kThreadsMain, CTAS)
         const int nlr = (split == p.splits - 1) ? p.lr_chunks : 0;
         for (int it = kt0; it < kt1 + nlr; ++it) {
           if (it < kt1) {
-            if (!mbar_wait(&full[stage], phase, abort_flag)) { ok = false; break; }
+            if (!mbar_wait(&sf_full[stage], (sf_phase >> stage) & 1u, abort_flag)) { ok = false; break; }
             tc_fence_after();
             uint8_t* sSFA = smem + stage * S::kStage + S::kA + S::kB;
             uint8_t* sSFB = sSFA + S::kSFA;

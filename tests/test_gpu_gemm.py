@@ -172,6 +172,29 @@ def test_both_split_core_product(fmt, K):
     assert rel_fro(y.cpu().numpy(), want) < TOL
 
 
+def test_both_split_many_tiles_per_cta():
+    # both operands split at rank 64: four low-rank chunks, as many as the
+    # 128x256 kernel's ring has stages, and about two tiles per CTA, so the
+    # scale copies of a tile's first K step follow a full round of low-rank
+    # stages; the low-rank part carries most of C
+    fmt = "nv"
+    M, N, K, k = 4096, 2048, 1024, 64
+    P = (_rand((K, k), 71) / np.sqrt(K)).astype(np.float32)
+    qPa, rPa = _q(P, fmt, 0)
+    qPb, rPb = qPa, rPa
+    qFa, rFa = _q((_rand((M, k), 72) / np.sqrt(M)).astype(np.float32), fmt, 0)
+    qFb, rFb = _q((_rand((N, k), 73) / np.sqrt(N)).astype(np.float32), fmt, 0)
+    Sa = np.linspace(8, 1, k).astype(np.float32)
+    Sb = np.linspace(6, 1, k).astype(np.float32)
+    qra, rra = _q(_rand((M, K), 74, 0.05), fmt, 1)
+    qrb, rrb = _q(_rand((K, N), 75, 0.05), fmt, 0)
+    y = api.linear_fwd(api.Operand(qra, k, qPa, qFa, torch.from_numpy(Sa).cuda()),
+                       api.Operand(qrb, k, qPb, qFb, torch.from_numpy(Sb).cuda()), M, N, K)
+    torch.cuda.synchronize()
+    want = gemm.gemm(gemm.Operand(rra, k, rPa, rFa, Sa), gemm.Operand(rrb, k, rPb, rFb, Sb))
+    assert rel_fro(y.cpu().numpy(), want) < TOL
+
+
 def test_both_split_long_contraction():
     # K = 14336 (56 K tiles) with few output tiles: the low-rank products run
     # split-K with a split count that does not divide the K tiles evenly
