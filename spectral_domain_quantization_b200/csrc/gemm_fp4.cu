@@ -16,8 +16,10 @@
 // Design (one persistent CTA per SM, 352 threads, warp-specialized):
 //   warp 0      TMA producer: per 256-element K tile loads the A tile
 //               (128 rows x 128 B) and B tile (BN rows x 128 B) with 128-byte
-//               swizzle, and the matching 512-byte scale chunks with bulk
-//               copies, into a 4-stage shared-memory ring.
+//               swizzle (completing on the stage's operand barrier), and the
+//               matching 512-byte scale chunks with bulk copies (completing
+//               on the stage's scale barrier, armed only for FP4 steps), into
+//               a 4-stage shared-memory ring.
 //   warp 1      TMEM allocator + MMA issuer: waits for a stage's operands and
 //               its scale factors, issues four K=64 block-scaled MMAs
 //               (kind::mxf4 / mxf4nvf4), then kind::f16 MMAs for the low-rank
@@ -25,11 +27,14 @@
 //   warps 2-9   epilogue: drain the 128 x BN fp32 accumulator from TMEM into
 //               registers, release it, scale and store (fp32 or bf16), or
 //               store raw partial sums for split-K.
-//   warp 10     scale copies: each stage's scale chunks into that stage's own
-//               TMEM columns (tcgen05.cp 32x128b.warpx4), committed to a
-//               per-stage barrier; issued by the MMA warp itself, the copies
-//               sat in front of every stage's MMAs (125.7 against 107.6 us on
-//               8192 x 4096 x 4096 NVFP4).
+//   warp 10     scale copies: waits for a stage's scale chunks, copies them
+//               into that stage's own TMEM columns (tcgen05.cp
+//               32x128b.warpx4) and commits them to a per-stage barrier the
+//               MMA warp waits on; issued by the MMA warp itself, the copies
+//               sat in front of every stage's MMAs (125.7 against 105.3 us on
+//               8192 x 4096 x 4096 NVFP4).  Both scale barriers count FP4
+//               steps only, so the low-rank steps the scale warp skips never
+//               let a parity wait pass a phase early.
 // Every wait is bounded (METIS_DEV_TIMEOUT) and the kernel always frees its
 // TMEM.  Shared memory per stage: A 16 KB + B BN*128 B + scales 6 KB.
 //
