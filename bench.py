@@ -45,9 +45,10 @@ SPLIT_W_BYTES = (6 * K * N * 2 + (K * N // 2 + K * N // 16) + (K + N) * RANK_K *
 QUANT_X_BYTES = 2 * M * K * 2 + M * K // 2 + M * K // 16
 FLOPS = 2.0 * M * N * K
 # DRAM bytes (dram__bytes_read.sum + dram__bytes_write.sum) of one launch of
-# the plain-operand FP4 GEMM, from one ncu capture of the current kernel; to
-# be set to None whenever the kernel changes after that capture.
-GEMM_NCU_DRAM_BYTES = 31.770880e6 + 18.906880e6
+# the plain-operand FP4 GEMM, from one ncu capture of the current kernel; None
+# whenever the kernel changed after that capture (the last capture, 50.7 MB,
+# predates the separate scale barrier).
+GEMM_NCU_DRAM_BYTES = None
 METRIC = "FP4 split-linear eff. TFLOPS & % of FP4 peak; split+quantize us/layer"
 CONFIG = {"workload": "layer_4096: W bf16 4096x4096 planted spectrum + X bf16 8192x4096, "
                       "split k=64 p=16 q=1 Gaussian, NVFP4, forward",
