@@ -38,8 +38,9 @@
 // Every wait is bounded (METIS_DEV_TIMEOUT) and the kernel always frees its
 // TMEM.  Shared memory per stage: A 16 KB + B BN*128 B + scales 6 KB.
 //
-// A second kernel, gemm_fp4_wide_kernel, runs the same pipeline on a
-// 256 x 192 tile (two 128-row M halves sharing one B tile, three stages);
+// A second kernel, gemm_fp4_wide_kernel, runs the same pipeline (scale warp
+// included) on a 256 x 192 tile (two 128-row M halves sharing one B tile,
+// three stages, two TMEM scale slots);
 // run_gemm_fp4 picks it for unsplit products when its rounds of tiles over
 // the SMs cost less than the 128 x 256 tile's.
 #include "abi_common.h"
@@ -50,10 +51,9 @@ namespace metis {
 
 namespace {
 
-constexpr int kThreads = 320;
-// gemm_fp4_kernel adds one warp that only copies the scale factors into TMEM
+// warps 0-1 producer and MMA issuer, 2-9 epilogue, 10 the scale copies
 constexpr int kSfWarp = 10;
-constexpr int kThreadsMain = 32 * (kSfWarp + 1);
+constexpr int kThreads = 32 * (kSfWarp + 1);
 constexpr int kEpiWarps = 8;
 
 template <int BN, int STAGES>
@@ -77,7 +77,7 @@ MDEV bool wait_ns(uint64_t* bar, uint32_t parity, uint64_t ns) {
 // BN: MMA N; STAGES: shared-memory ring depth; CTAS: CTAs per SM (2 halves
 // the TMEM allocation and lets one CTA's epilogue overlap the other's MMAs).
 template <int BN, int STAGES, int CTAS>
-__global__ void __launch_bounds__(kThreadsMain, CTAS)
+__global__ void __launch_bounds__(kThreads, CTAS)
     gemm_fp4_kernel(const GemmParams p, const __grid_constant__ CUtensorMap tmA,
                     const __grid_constant__ CUtensorMap tmB, const __grid_constant__ CUtensorMap tmLA,
                     const __grid_constant__ CUtensorMap tmLB) {
@@ -420,8 +420,8 @@ __global__ void __launch_bounds__(kThreadsMain, CTAS)
 // Wide tile: two 128-row M halves share one 192-row B tile (256 x 192 per
 // CTA).  Per flop it moves 22 % fewer operand bytes from L2 than a 128 x 256
 // tile and issues fewer scale copies.  TMEM: the two halves' accumulators in
-// columns 0-383 and the scale factors in two 64-column slots; a slot is
-// refilled only after the commit of the stage that last read it.  B's scale
+// columns 0-383 and the scale factors in two 64-column slots; the scale warp
+// refills a slot only after the commit of the K step that last read it.  B's scale
 // chunks come from the 128-row chunk at or below the tile's first row: a tile
 // that starts 64 rows into a chunk (odd tn) reads them two TMEM columns
 // further.  Rows past M and columns past N are computed on zero-filled (TMA)
@@ -452,8 +452,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* empty = full + kStages;
   uint64_t* acc_full = empty + kStages;
   uint64_t* acc_empty = acc_full + 1;
-  uint64_t* sf_free = acc_empty + 1;     // [2]
-  uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(sf_free + 2);
+  uint64_t* sf_free = acc_empty + 1;     // [2]: the MMAs that read a slot have retired
+  uint64_t* sf_ready = sf_free + 2;      // [2]: a slot holds the next K step's scales
+  uint64_t* sf_full = sf_ready + 2;      // per stage: its scale bytes are in shared memory
+  uint32_t* tmem_base_sh = reinterpret_cast<uint32_t*>(sf_full + kStages);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_base_sh + 1);
 
   const int warp = threadIdx.x >> 5;
@@ -470,6 +472,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(acc_empty, kEpiWarps);
     mbar_init(&sf_free[0], 1);
     mbar_init(&sf_free[1], 1);
+    mbar_init(&sf_ready[0], 1);
+    mbar_init(&sf_ready[1], 1);
+    for (int s = 0; s < kStages; ++s) mbar_init(&sf_full[s], 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -500,6 +505,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     if (lane == 0) {
       int stage = 0, issued = 0;
       uint32_t phase = 0;
+      uint32_t sf_phase = 0;   // bit s: parity of sf_full[s]'s next phase
+      uint32_t sf_last = 0;    // bit s: the last load into stage s carried scales
       bool ok = true;
       for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
         const int tm = t % tiles_m, tn = t / tiles_m;
@@ -517,27 +524,33 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (it < p.num_kt) {
             const int kt = it;
             const uint32_t sf_bytes = 512u * atoms_per_kt;
-            const uint32_t bytes = 2 * S::kA + S::kB + sf_bytes * ((half1 ? 2 : 1) + (second ? 2 : 1));
-            mbar_arrive_expect_tx(&full[stage], bytes);
+            // operands on full[stage] (MMA warp), scale chunks on sf_full[stage]
+            // (scale warp), armed only for FP4 steps
+            const uint32_t sbytes = sf_bytes * ((half1 ? 2 : 1) + (second ? 2 : 1));
+            mbar_arrive_expect_tx(&full[stage], 2 * S::kA + S::kB);
+            mbar_arrive_expect_tx(&sf_full[stage], sbytes);
             tma_load_2d(sA0, &tmA, &full[stage], kt * 128, 256 * tm);
             tma_load_2d(sA1, &tmA, &full[stage], kt * 128, 256 * tm + 128);
             tma_load_2d(sB, &tmB, &full[stage], kt * 128, tn * BN);
             bulk_load(sSFA0, p.sfa + (static_cast<int64_t>(2 * tm) * p.sfa_chunks + kt * atoms_per_kt) * 512, sf_bytes,
-                      &full[stage]);
+                      &sf_full[stage]);
             if (half1)
               bulk_load(sSFA1, p.sfa + (static_cast<int64_t>(2 * tm + 1) * p.sfa_chunks + kt * atoms_per_kt) * 512,
-                        sf_bytes, &full[stage]);
+                        sf_bytes, &sf_full[stage]);
             bulk_load(sSFB, p.sfb + (static_cast<int64_t>(nb0) * p.sfb_chunks + kt * atoms_per_kt) * 512, sf_bytes,
-                      &full[stage]);
+                      &sf_full[stage]);
             if (second)
               bulk_load(sSFB + 2048, p.sfb + (static_cast<int64_t>(nb0 + 1) * p.sfb_chunks + kt * atoms_per_kt) * 512,
-                        sf_bytes, &full[stage]);
+                        sf_bytes, &sf_full[stage]);
+            sf_phase ^= 1u << stage;
+            sf_last |= 1u << stage;
           } else {
             const int c = it - p.num_kt;
             mbar_arrive_expect_tx(&full[stage], 2 * S::kA + S::kB);
             tma_load_2d(sA0, &tmLA, &full[stage], c * 64, 256 * tm);
             tma_load_2d(sA1, &tmLA, &full[stage], c * 64, 256 * tm + 128);
             tma_load_2d(sB, &tmLB, &full[stage], c * 64, tn * BN);
+            sf_last &= ~(1u << stage);
           }
           ++issued;
           if (++stage == kStages) { stage = 0; phase ^= 1u; }
@@ -550,6 +563,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int i = 0; i < min(issued, kStages); ++i) {
           if (--s < 0) { s = kStages - 1; ph ^= 1u; }
           wait_ns(&full[s], ph, 100000000ull);
+          if ((sf_last >> s) & 1u) wait_ns(&sf_full[s], ((sf_phase >> s) & 1u) ^ 1u, 100000000ull);
         }
       }
     }
@@ -577,23 +591,11 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bd = make_sdesc(smem_u32(sB), 16, 1024, kSwizzle128B);
           if (it < p.num_kt) {
             const int slot = g & 1;
-            if (g >= 2) {
-              // the MMAs that last read this slot (stage g - 2) have retired
-              if (!mbar_wait(&sf_free[slot], static_cast<uint32_t>((g >> 1) - 1) & 1u, abort_flag)) { ok = false; break; }
-              tc_fence_after();
-            }
-            uint8_t* sSFA0 = sB + S::kB;
-            uint8_t* sSFA1 = sSFA0 + S::kSFA;
-            uint8_t* sSFB = sSFA1 + S::kSFA;
+            // the scale warp has copied this K step's scales into the slot
+            if (!mbar_wait(&sf_ready[slot], static_cast<uint32_t>(g >> 1) & 1u, abort_flag)) { ok = false; break; }
+            tc_fence_after();
             const uint32_t sf = tmem + kSfBase + slot * kSlotCols;
             const uint32_t sfa0 = sf, sfa1 = sf + 16, sfb = sf + 32;
-            for (int a = 0; a < atoms_per_kt; ++a) {
-              tc_cp_32x128b_warpx4(sfa0 + 4 * a, make_sdesc(smem_u32(sSFA0 + 512 * a), 0, 128, kSwizzleNone));
-              tc_cp_32x128b_warpx4(sfa1 + 4 * a, make_sdesc(smem_u32(sSFA1 + 512 * a), 0, 128, kSwizzleNone));
-              for (int h = 0; h < 2; ++h)
-                tc_cp_32x128b_warpx4(sfb + 8 * a + 4 * h,
-                                     make_sdesc(smem_u32(sSFB + 2048 * h + 512 * a), 0, 128, kSwizzleNone));
-            }
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               const uint64_t koff = static_cast<uint64_t>((j * 32) >> 4);
@@ -634,6 +636,49 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_commit(acc_full);
         wait_ns(acc_full, acc_phase, 100000000ull);
       }
+    }
+    __syncwarp();
+  } else if (warp == kSfWarp) {
+    // ------------------------------------------------------------ scale copies
+    // K step g's scales go into slot g & 1 once the MMAs of step g - 2 (the
+    // slot's last readers) have retired and the step's scale chunks are in
+    // shared memory (sf_full, counted in FP4 steps only), committed to
+    // sf_ready[slot]; the copies of step g + 1 run while the MMAs of step g
+    // are issued.
+    if (lane == 0) {
+      int stage = 0, g = 0;
+      uint32_t sf_phase = 0;   // bit s: parity of sf_full[s]'s next phase
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        for (int it = 0; it < nk; ++it) {
+          if (it < p.num_kt) {
+            const int slot = g & 1;
+            if (g >= 2) {
+              if (!mbar_wait(&sf_free[slot], static_cast<uint32_t>((g >> 1) - 1) & 1u, abort_flag)) { ok = false; break; }
+            }
+            if (!mbar_wait(&sf_full[stage], (sf_phase >> stage) & 1u, abort_flag)) { ok = false; break; }
+            sf_phase ^= 1u << stage;
+            tc_fence_after();
+            uint8_t* sSFA0 = smem + stage * S::kStage + 2 * S::kA + S::kB;
+            uint8_t* sSFA1 = sSFA0 + S::kSFA;
+            uint8_t* sSFB = sSFA1 + S::kSFA;
+            const uint32_t sf = tmem + kSfBase + slot * kSlotCols;
+            const uint32_t sfa0 = sf, sfa1 = sf + 16, sfb = sf + 32;
+            for (int a = 0; a < atoms_per_kt; ++a) {
+              tc_cp_32x128b_warpx4(sfa0 + 4 * a, make_sdesc(smem_u32(sSFA0 + 512 * a), 0, 128, kSwizzleNone));
+              tc_cp_32x128b_warpx4(sfa1 + 4 * a, make_sdesc(smem_u32(sSFA1 + 512 * a), 0, 128, kSwizzleNone));
+              for (int h = 0; h < 2; ++h)
+                tc_cp_32x128b_warpx4(sfb + 8 * a + 4 * h,
+                                     make_sdesc(smem_u32(sSFB + 2048 * h + 512 * a), 0, 128, kSwizzleNone));
+            }
+            tc_commit(&sf_ready[slot]);
+            ++g;
+          }
+          if (++stage == kStages) stage = 0;
+        }
+      }
+      // copies still in flight land before the TMEM is freed
+      if (g >= 1) wait_ns(&sf_ready[(g - 1) & 1], static_cast<uint32_t>((g - 1) >> 1) & 1u, 100000000ull);
     }
     __syncwarp();
   } else {
@@ -780,7 +825,7 @@ cudaError_t launch_bn(const GemmParams& p, const CUtensorMap& a, const CUtensorM
     return cudaErrorInvalidValue;
   const int slots = device_sm_count() * CTAS;
   const int grid = tiles < slots ? tiles : slots;
-  gemm_fp4_kernel<BN, STAGES, CTAS><<<grid, kThreadsMain, bytes, s>>>(p, a, b, la, lb);
+  gemm_fp4_kernel<BN, STAGES, CTAS><<<grid, kThreads, bytes, s>>>(p, a, b, la, lb);
   return cudaGetLastError();
 }
 
