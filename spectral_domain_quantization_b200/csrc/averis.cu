@@ -144,6 +144,7 @@ __global__ void __launch_bounds__(32 * kRowGroups, 3) colstats_kernel(const void
 constexpr int kStatTile = 64;
 constexpr int kStatConsumers = 8;
 constexpr int kStatStages = 12;           // 96 KB of stages: two CTAs per SM
+static_assert((2 * kStatStages) % kStatConsumers == 0, "a stage's rounds must alternate between at most two warps");
 
 struct StatArgs {
   int64_t m, n, strips, runs, run_tiles, ntiles;
@@ -228,6 +229,13 @@ __global__ void __launch_bounds__(32 * (kStatConsumers + 1), 2) colstats_tma_ker
       }
       if (++turn == kStatConsumers) turn = 0;
       if (!mine) continue;
+      // Stage s's rounds alternate between this warp and at most one other
+      // (2 x the stage count is a multiple of the consumer warps), so the
+      // round before this one may be the other warp's and its load may still
+      // be in flight, when a parity wait on full[s] would pass a phase early.
+      // Its consumption on empty[s] comes first: at once for the first round
+      // and for a round this warp consumed itself.
+      if (!mbar_wait(&empty[s], sph ^ 1u, abort_flag)) break;
       if (!mbar_wait(&full[s], sph, abort_flag)) break;
       const uint8_t* tile = ring + s * kStageBytes;
       const int nr = static_cast<int>(imin64(16, a.m - (g * kStatTile + 16 * r)));  // rows of this lane in X

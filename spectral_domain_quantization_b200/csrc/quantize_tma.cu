@@ -171,6 +171,13 @@ __global__ void __launch_bounds__(kQThreads, ctas_per_sm(AXIS)) quantize_tma_ker
         }
         if (++turn == kConsumers) turn = 0;
         if (!mine) continue;
+        // Stage s's rounds alternate between this warp and at most one other
+        // (2 x the stage count is a multiple of the consumer warps), so the
+        // round before this one may be the other warp's and its load may still
+        // be in flight, when a parity wait on full[s] would pass a phase early.
+        // Its consumption on empty[s] comes first: at once for the first round
+        // and for a round this warp consumed itself.
+        if (!mbar_wait(&empty[s], sph ^ 1u, abort_flag)) break;
         if (!mbar_wait(&full[s], sph, abort_flag)) break;
         const uint8_t* tile = ring + s * a.stage_bytes;
 #pragma unroll 1
@@ -264,6 +271,13 @@ __global__ void __launch_bounds__(kQThreads, ctas_per_sm(AXIS)) quantize_tma_ker
         }
         if (++turn == kConsumers) turn = 0;
         if (!mine) continue;
+        // Stage s's rounds alternate between this warp and at most one other
+        // (2 x the stage count is a multiple of the consumer warps), so the
+        // round before this one may be the other warp's and its load may still
+        // be in flight, when a parity wait on full[s] would pass a phase early.
+        // Its consumption on empty[s] comes first: at once for the first round
+        // and for a round this warp consumed itself.
+        if (!mbar_wait(&empty[s], sph ^ 1u, abort_flag)) break;
         if (!mbar_wait(&full[s], sph, abort_flag)) break;
         const uint8_t* tile = ring + s * a.stage_bytes;
         const int64_t rb = g * kTileRows + kBlk * b;        // the block's first X row
@@ -397,6 +411,11 @@ void launch_quantize_tma(QuantParams p, int axis, int sms, int32_t* dev_status, 
   a.strip_cols = (axis == 0 && mx) ? 128 : 64;
   a.stage_bytes = kTileRows * a.strip_cols * 2;
   a.stages = ring_bytes(axis) / a.stage_bytes;
+  // the consumers' waits assume a stage's rounds alternate between at most two warps
+  if ((2 * a.stages) % kConsumers != 0) {
+    fail(METIS_ERR_ARG, "quantize ring stages");
+    return;
+  }
   a.strips = (a.n + a.strip_cols - 1) / a.strip_cols;
   a.ntiles = (a.m + kTileRows - 1) / kTileRows;
   // about four items per CTA slot (two CTAs per SM) for balance
